@@ -1,0 +1,465 @@
+/*
+ * dla_oracle.c -- plain, slow, token-by-token fp64 CPU oracle of the
+ * Dynamic Linear Attention (DLA) forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library.  It shares
+ * no code, header, table or helper with the CUDA library and neither side
+ * imports the other.
+ *
+ * What it computes (per (batch, head) stream, in fp64; f32 and bf16 inputs are
+ * widened exactly):
+ *
+ *   - per-token state v_t phi(k_t)^T with phi = elu + 1
+ *       ("Dynamic Linear Attention | Chlience Paper Archive", section 5.1,
+ *        the per-token state s_t; stored transposed as [d_v][d_k]);
+ *   - token score r_t = 1 - cos(k_t, k_{t-1}) on the raw keys, r_0 = 0, and a
+ *     token joins the open segment only when r_t < tau and r_{t-1} < tau
+ *       (ai-feeds.com "Dynamic Linear Attention" summary, section
+ *        "信息感知的动态状态合并": two consecutive low-information tokens are
+ *        merged; Chlience section 5.1: b_t = 1 opens a new state, b_t = 0 adds
+ *        s_t to the current state);
+ *   - a time-ordered cache of at most C states (open one included); when a
+ *     boundary seals the open state and C states are sealed, the adjacent
+ *     sealed pair with the smallest Ward loss
+ *         n_i n_j / (n_i + n_j) * || mu_i - mu_j ||^2,   mu = z / n,
+ *     z = sum of phi(k), is merged into the left one (earlier timestamp kept),
+ *     ties to the leftmost pair
+ *       (Chlience section 5.2, capacity-bounded memory and the merge update
+ *        S <- S + S', n <- n + n'; ai-feeds "容量受限的内存建模": adjacent
+ *        pair with least merge loss, merged state keeps the earlier timestamp;
+ *        Chlience Corollary 1: the Ward term is the within-block scatter);
+ *   - readout o_t = sum_i lambda_{t,i} S_i phi(q_t) over the states present at
+ *     t (after the merge at t, open state including token t), with
+ *     lambda_{t,i} = softmax_i( phi(q_t) . mu_i / sqrt(d_k) )
+ *       (Chlience section 5.3, reading from bounded states).
+ *
+ * The fixed-bucket policy (Chlience section 2 and section 5.4, Log-Linear
+ * Attention's Fenwick buckets) keeps a binary-counter list of blocks over
+ * [0, t-1]; token t reads the blocks plus {t} with the same softmax, then {t}
+ * is pushed and the two newest blocks are merged while their sizes are equal.
+ *
+ * Readings where the pages are silent (applied identically by the CUDA path):
+ *   r_0 = 0 (no predecessor); a zero-norm key gives cos = 0 (r = 1);
+ *   "below tau" is strict; C counts the open state, so a merge fires only at a
+ *   boundary when C sealed states exist; order within a token is
+ *   decide -> merge -> add v phi(k)^T -> read out.
+ *
+ * Arithmetic order (fixed so that r_t is bit-identical on both sides): dot
+ * products and squared norms are summed sequentially over the index, with no
+ * fused multiply-add (build with -ffp-contract=off), and
+ * cos = dot / (sqrt(|a|^2) * sqrt(|b|^2)).  z is summed token by token.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_F32 0
+#define OR_BF16 1
+#define OR_F64 2
+
+#define OR_POLICY_DLA 0
+#define OR_POLICY_FENWICK 1
+
+typedef struct {
+  double *S; /* [dv][dk] sum of v phi(k)^T */
+  double *z; /* [dk] sum of phi(k) */
+  int64_t n;
+  int64_t ts;
+} ostate;
+
+typedef struct {
+  int nsealed;
+  int cap_sealed;
+  ostate *sealed; /* time order */
+  int has_open;
+  ostate open;
+  double *prev_k;
+  double prev_r;
+  int64_t t;
+} ohead;
+
+typedef struct {
+  int nheads, dk, dv, C, policy, want_S;
+  ohead *heads;
+} oracle;
+
+static double widen(const void *p, int dtype, size_t i) {
+  if (dtype == OR_F32) return (double)((const float *)p)[i];
+  if (dtype == OR_F64) return ((const double *)p)[i];
+  uint32_t b = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+  float f;
+  memcpy(&f, &b, sizeof f);
+  return (double)f;
+}
+
+/* phi = elu + 1: x + 1 for x > 0, exp(x) for x <= 0. */
+static double phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+
+static void st_alloc(ostate *s, int dk, int dv, int want_S) {
+  s->S = want_S ? (double *)calloc((size_t)dv * dk, sizeof(double)) : NULL;
+  s->z = (double *)calloc((size_t)dk, sizeof(double));
+  s->n = 0;
+  s->ts = 0;
+}
+
+static void st_zero(ostate *s, int dk, int dv) {
+  if (s->S) memset(s->S, 0, sizeof(double) * (size_t)dv * dk);
+  memset(s->z, 0, sizeof(double) * (size_t)dk);
+  s->n = 0;
+  s->ts = 0;
+}
+
+static void st_copy(ostate *dst, const ostate *src, int dk, int dv) {
+  if (dst->S && src->S) memcpy(dst->S, src->S, sizeof(double) * (size_t)dv * dk);
+  memcpy(dst->z, src->z, sizeof(double) * (size_t)dk);
+  dst->n = src->n;
+  dst->ts = src->ts;
+}
+
+/* left <- left + right (S, z, n); left keeps its timestamp. */
+static void st_absorb(ostate *left, const ostate *right, int dk, int dv) {
+  if (left->S && right->S)
+    for (size_t i = 0; i < (size_t)dv * dk; i++) left->S[i] = left->S[i] + right->S[i];
+  for (int i = 0; i < dk; i++) left->z[i] = left->z[i] + right->z[i];
+  left->n = left->n + right->n;
+}
+
+/* Ward loss n_a n_b / (n_a + n_b) * sum_i (z_a[i]/n_a - z_b[i]/n_b)^2. */
+static double ward(const ostate *a, const ostate *b, int dk) {
+  double na = (double)a->n, nb = (double)b->n;
+  double f = (na * nb) / (na + nb);
+  double s = 0.0;
+  for (int i = 0; i < dk; i++) {
+    double diff = a->z[i] / na - b->z[i] / nb;
+    s = s + diff * diff;
+  }
+  return f * s;
+}
+
+/* r = 1 - cos(a, b); zero norm gives cos = 0. */
+static double score(const double *a, const double *b, int dk) {
+  double dot = 0.0, na = 0.0, nb = 0.0;
+  for (int i = 0; i < dk; i++) dot = dot + a[i] * b[i];
+  for (int i = 0; i < dk; i++) na = na + a[i] * a[i];
+  for (int i = 0; i < dk; i++) nb = nb + b[i] * b[i];
+  if (na == 0.0 || nb == 0.0) return 1.0;
+  return 1.0 - dot / (sqrt(na) * sqrt(nb));
+}
+
+oracle *dla_oracle_new(int nheads, int dk, int dv, int C, int policy, int want_S) {
+  oracle *o = (oracle *)calloc(1, sizeof(oracle));
+  o->nheads = nheads;
+  o->dk = dk;
+  o->dv = dv;
+  o->C = C;
+  o->policy = policy;
+  o->want_S = want_S;
+  o->heads = (ohead *)calloc((size_t)nheads, sizeof(ohead));
+  int cap = policy == OR_POLICY_DLA ? C : 64;
+  for (int h = 0; h < nheads; h++) {
+    ohead *hd = &o->heads[h];
+    hd->cap_sealed = cap;
+    hd->sealed = (ostate *)calloc((size_t)cap, sizeof(ostate));
+    for (int i = 0; i < cap; i++) st_alloc(&hd->sealed[i], dk, dv, want_S);
+    st_alloc(&hd->open, dk, dv, want_S);
+    hd->prev_k = (double *)calloc((size_t)dk, sizeof(double));
+  }
+  return o;
+}
+
+void dla_oracle_free(oracle *o) {
+  if (!o) return;
+  for (int h = 0; h < o->nheads; h++) {
+    ohead *hd = &o->heads[h];
+    for (int i = 0; i < hd->cap_sealed; i++) {
+      free(hd->sealed[i].S);
+      free(hd->sealed[i].z);
+    }
+    free(hd->sealed);
+    free(hd->open.S);
+    free(hd->open.z);
+    free(hd->prev_k);
+  }
+  free(o->heads);
+  free(o);
+}
+
+typedef struct {
+  oracle *o;
+  int head_lo, head_hi, T;
+  double tau;
+  int dtype;
+  const void *q, *k, *v; /* [nrun][T][d] */
+  double *out;           /* [nrun][T][dv] or NULL */
+  uint8_t *boundary;     /* [nrun][T] or NULL */
+  int32_t *merge_t, *merge_i, *merge_count; /* [nrun][cap], [nrun] */
+  int cap;
+  int32_t *live; /* [nrun][T] live states read by token t, or NULL */
+  double *margins; /* [nrun][3]: min |r - tau|, min Ward relative gap, #exact ties */
+  int next;        /* work counter */
+  pthread_mutex_t mu;
+} job;
+
+static void record_merge(job *J, int r, int64_t t, int i) {
+  int32_t c = J->merge_count[r];
+  if (c < J->cap) {
+    J->merge_t[(size_t)r * J->cap + c] = (int32_t)t;
+    J->merge_i[(size_t)r * J->cap + c] = i;
+  }
+  J->merge_count[r] = c + 1;
+}
+
+/* Readout: lambda = softmax(phi(q).mu/sqrt(dk)) over states; o = sum lambda S p. */
+static void readout(const oracle *o, ostate *const *st, int m, const double *p, double *out) {
+  int dk = o->dk, dv = o->dv;
+  double *a = (double *)malloc(sizeof(double) * (size_t)m);
+  double amax = -INFINITY;
+  for (int i = 0; i < m; i++) {
+    double dot = 0.0;
+    for (int c = 0; c < dk; c++) {
+      double mu = st[i]->z[c] / (double)st[i]->n;
+      dot = dot + p[c] * mu;
+    }
+    a[i] = dot / sqrt((double)dk);
+    if (a[i] > amax) amax = a[i];
+  }
+  double den = 0.0;
+  for (int i = 0; i < m; i++) {
+    a[i] = exp(a[i] - amax);
+    den = den + a[i];
+  }
+  for (int r = 0; r < dv; r++) out[r] = 0.0;
+  for (int i = 0; i < m; i++) {
+    double lam = a[i] / den;
+    for (int r = 0; r < dv; r++) {
+      double acc = 0.0;
+      for (int c = 0; c < dk; c++) acc = acc + st[i]->S[(size_t)r * dk + c] * p[c];
+      out[r] = out[r] + lam * acc;
+    }
+  }
+  free(a);
+}
+
+static void run_head_dla(job *J, int r) {
+  oracle *o = J->o;
+  int dk = o->dk, dv = o->dv, C = o->C, T = J->T;
+  ohead *hd = &o->heads[J->head_lo + r];
+  double *kk = (double *)malloc(sizeof(double) * dk);
+  double *u = (double *)malloc(sizeof(double) * dk);
+  double *p = (double *)malloc(sizeof(double) * dk);
+  double *vv = (double *)malloc(sizeof(double) * dv);
+  ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(C + 1));
+  double min_rm = INFINITY, min_gap = INFINITY, ties = 0.0;
+  for (int tl = 0; tl < T; tl++) {
+    size_t base = ((size_t)r * T + tl) * dk;
+    for (int c = 0; c < dk; c++) kk[c] = widen(J->k, J->dtype, base + c);
+    for (int c = 0; c < dk; c++) u[c] = phi(kk[c]);
+    double rt = hd->t == 0 ? 0.0 : score(kk, hd->prev_k, dk);
+    if (hd->t > 0) {
+      double mrg = fabs(rt - J->tau);
+      if (mrg < min_rm) min_rm = mrg;
+    }
+    int join = hd->t > 0 && rt < J->tau && hd->prev_r < J->tau;
+    if (J->boundary) J->boundary[(size_t)r * T + tl] = (uint8_t)(!join);
+    if (!join) {
+      if (hd->has_open) {
+        st_copy(&hd->sealed[hd->nsealed], &hd->open, dk, dv);
+        hd->nsealed++;
+      }
+      if (hd->nsealed == C) {
+        int best = 0;
+        double bl = ward(&hd->sealed[0], &hd->sealed[1], dk);
+        double second = INFINITY;
+        for (int i = 1; i < C - 1; i++) {
+          double l = ward(&hd->sealed[i], &hd->sealed[i + 1], dk);
+          if (l < bl) {
+            second = bl;
+            bl = l;
+            best = i;
+          } else if (l < second) {
+            second = l;
+          }
+        }
+        if (second == bl) ties += 1.0;
+        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;
+        st_absorb(&hd->sealed[best], &hd->sealed[best + 1], dk, dv);
+        /* drop best+1: rotate its buffers to the end of the list */
+        ostate tmp = hd->sealed[best + 1];
+        for (int i = best + 1; i < hd->nsealed - 1; i++) hd->sealed[i] = hd->sealed[i + 1];
+        hd->sealed[hd->nsealed - 1] = tmp;
+        hd->nsealed--;
+        record_merge(J, r, hd->t, best);
+      }
+      st_zero(&hd->open, dk, dv);
+      hd->open.ts = hd->t;
+      hd->has_open = 1;
+    }
+    if (J->out) {
+      size_t vb = ((size_t)r * T + tl) * dv;
+      for (int c = 0; c < dv; c++) vv[c] = widen(J->v, J->dtype, vb + c);
+      for (int a = 0; a < dv; a++)
+        for (int c = 0; c < dk; c++)
+          hd->open.S[(size_t)a * dk + c] = hd->open.S[(size_t)a * dk + c] + vv[a] * u[c];
+    }
+    for (int c = 0; c < dk; c++) hd->open.z[c] = hd->open.z[c] + u[c];
+    hd->open.n = hd->open.n + 1;
+    int m = 0;
+    for (int i = 0; i < hd->nsealed; i++) lst[m++] = &hd->sealed[i];
+    lst[m++] = &hd->open;
+    if (J->live) J->live[(size_t)r * T + tl] = m;
+    if (J->out) {
+      for (int c = 0; c < dk; c++) p[c] = phi(widen(J->q, J->dtype, base + c));
+      readout(o, lst, m, p, J->out + ((size_t)r * T + tl) * dv);
+    }
+    for (int c = 0; c < dk; c++) hd->prev_k[c] = kk[c];
+    hd->prev_r = rt;
+    hd->t = hd->t + 1;
+  }
+  if (J->margins) {
+    double *mg = J->margins + (size_t)r * 3;
+    if (min_rm < mg[0]) mg[0] = min_rm;
+    if (min_gap < mg[1]) mg[1] = min_gap;
+    mg[2] += ties;
+  }
+  free(kk);
+  free(u);
+  free(p);
+  free(vv);
+  free(lst);
+}
+
+static void run_head_fenwick(job *J, int r) {
+  oracle *o = J->o;
+  int dk = o->dk, dv = o->dv, T = J->T;
+  ohead *hd = &o->heads[J->head_lo + r];
+  double *u = (double *)malloc(sizeof(double) * dk);
+  double *p = (double *)malloc(sizeof(double) * dk);
+  double *vv = (double *)malloc(sizeof(double) * dv);
+  ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(hd->cap_sealed + 1));
+  for (int tl = 0; tl < T; tl++) {
+    size_t base = ((size_t)r * T + tl) * dk;
+    for (int c = 0; c < dk; c++) u[c] = phi(widen(J->k, J->dtype, base + c));
+    if (J->boundary) J->boundary[(size_t)r * T + tl] = 1;
+    /* {t} is the open bucket; {t-1} was pushed and carried at the end of t-1. */
+    st_zero(&hd->open, dk, dv);
+    hd->open.ts = hd->t;
+    hd->has_open = 1;
+    if (J->out) {
+      size_t vb = ((size_t)r * T + tl) * dv;
+      for (int c = 0; c < dv; c++) vv[c] = widen(J->v, J->dtype, vb + c);
+      for (int a = 0; a < dv; a++)
+        for (int c = 0; c < dk; c++) hd->open.S[(size_t)a * dk + c] = vv[a] * u[c];
+    }
+    for (int c = 0; c < dk; c++) hd->open.z[c] = u[c];
+    hd->open.n = 1;
+    int m = 0;
+    for (int i = 0; i < hd->nsealed; i++) lst[m++] = &hd->sealed[i];
+    lst[m++] = &hd->open;
+    if (J->live) J->live[(size_t)r * T + tl] = m;
+    if (J->out) {
+      for (int c = 0; c < dk; c++) p[c] = phi(widen(J->q, J->dtype, base + c));
+      readout(o, lst, m, p, J->out + ((size_t)r * T + tl) * dv);
+    }
+    /* push {t}; carry while the two newest blocks have equal size.  The
+     * merged buckets are first read by token t+1, so the trace records t+1. */
+    st_copy(&hd->sealed[hd->nsealed], &hd->open, dk, dv);
+    hd->nsealed++;
+    while (hd->nsealed >= 2 && hd->sealed[hd->nsealed - 1].n == hd->sealed[hd->nsealed - 2].n) {
+      int left = hd->nsealed - 2;
+      st_absorb(&hd->sealed[left], &hd->sealed[left + 1], dk, dv);
+      hd->nsealed--;
+      record_merge(J, r, hd->t + 1, left);
+    }
+    hd->t = hd->t + 1;
+  }
+  free(u);
+  free(p);
+  free(vv);
+  free(lst);
+}
+
+static void *worker(void *arg) {
+  job *J = (job *)arg;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    int r = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (r >= J->head_hi - J->head_lo) break;
+    if (J->o->policy == OR_POLICY_DLA) run_head_dla(J, r);
+    else run_head_fenwick(J, r);
+  }
+  return NULL;
+}
+
+/* Run T tokens for heads [head_lo, head_hi).  Inputs are [nrun][T][d] in
+ * `dtype`; outputs (all optional) are indexed by the run-local head r.
+ * `out` needs the oracle created with want_S = 1.  Returns 0 on success. */
+int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+                   const void *q, const void *k, const void *v, double *out,
+                   uint8_t *boundary, int32_t *merge_t, int32_t *merge_i,
+                   int32_t *merge_count, int cap, int32_t *live, double *margins,
+                   int nthreads) {
+  if (!o || head_lo < 0 || head_hi > o->nheads || head_lo > head_hi || T < 0) return 1;
+  if (out && (!o->want_S || !q || !v)) return 2;
+  if (!k) return 3;
+  job J;
+  memset(&J, 0, sizeof J);
+  J.o = o;
+  J.head_lo = head_lo;
+  J.head_hi = head_hi;
+  J.T = T;
+  J.tau = tau;
+  J.dtype = dtype;
+  J.q = q;
+  J.k = k;
+  J.v = v;
+  J.out = out;
+  J.boundary = boundary;
+  J.merge_t = merge_t;
+  J.merge_i = merge_i;
+  J.merge_count = merge_count;
+  J.cap = cap;
+  J.live = live;
+  J.margins = margins;
+  int nrun = head_hi - head_lo;
+  int32_t *mc_local = NULL;
+  if (!merge_count) {
+    mc_local = (int32_t *)calloc((size_t)(nrun > 0 ? nrun : 1), sizeof(int32_t));
+    J.merge_count = mc_local;
+    J.cap = 0;
+  }
+  pthread_mutex_init(&J.mu, NULL);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > nrun) nthreads = nrun > 0 ? nrun : 1;
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  for (int i = 0; i < nthreads; i++) pthread_create(&th[i], NULL, worker, &J);
+  for (int i = 0; i < nthreads; i++) pthread_join(th[i], NULL);
+  free(th);
+  pthread_mutex_destroy(&J.mu);
+  free(mc_local);
+  return 0;
+}
+
+/* Live states of one head in time order (sealed..., open).  Returns m and
+ * fills up to `maxm` entries: S [m][dv][dk] (if non-NULL and kept), z
+ * [m][dk], n [m], ts [m]; plus prev_r and t. */
+int dla_oracle_state(const oracle *o, int head, int maxm, double *S, double *z, int64_t *n,
+                     int64_t *ts, double *prev_r, int64_t *t) {
+  if (!o || head < 0 || head >= o->nheads) return -1;
+  const ohead *hd = &o->heads[head];
+  int m = hd->nsealed + (hd->has_open ? 1 : 0);
+  int dk = o->dk, dv = o->dv;
+  for (int i = 0; i < m && i < maxm; i++) {
+    const ostate *s = i < hd->nsealed ? &hd->sealed[i] : &hd->open;
+    if (S && s->S) memcpy(S + (size_t)i * dv * dk, s->S, sizeof(double) * (size_t)dv * dk);
+    if (z) memcpy(z + (size_t)i * dk, s->z, sizeof(double) * (size_t)dk);
+    if (n) n[i] = s->n;
+    if (ts) ts[i] = s->ts;
+  }
+  if (prev_r) *prev_r = hd->prev_r;
+  if (t) *t = hd->t;
+  return m;
+}
