@@ -1,0 +1,258 @@
+// dla_api.cu -- host side of the libdla C ABI: argument checks, cache and
+// workspace layout, and the per-window launch sequence.
+#include <string.h>
+
+#include "dla_internal.cuh"
+
+namespace dla {
+
+int simt_tile_rows();
+
+namespace {
+
+constexpr size_t ALIGN = 256;
+
+size_t align_up(size_t x) { return (x + ALIGN - 1) / ALIGN * ALIGN; }
+
+// Sequential carve-up of a device buffer (or a dry run for size queries).
+struct Carver {
+  char *base;
+  size_t off = 0;
+  template <typename T>
+  T *take(size_t count) {
+    T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+bool d_ok(int32_t d) { return d == 32 || d == 64 || d == 128; }
+
+void carve_cache(Carver &cv, dla_cache &c) {
+  const size_t u = (size_t)c.N * c.H;
+  c.S = cv.take<float>(u * c.C * c.d_v * c.d_k);
+  c.z = cv.take<double>(u * c.C * c.d_k);
+  c.n = cv.take<int64_t>(u * c.C);
+  c.ts = cv.take<int64_t>(u * c.C);
+  c.pair_loss = cv.take<double>(u * c.C);
+  c.order = cv.take<int32_t>(u * c.C);
+  c.m = cv.take<int32_t>(u);
+  c.prev_k = cv.take<float>(u * c.d_k);
+  c.prev_r = cv.take<double>(u);
+  c.t = cv.take<int64_t>(u);
+}
+
+Dims make_dims(const dla_config &cfg, int policy) {
+  Dims dm{};
+  dm.heads = cfg.B * cfg.H;
+  dm.T = cfg.T;
+  dm.M = simt_tile_rows();
+  dm.D = cfg.d_k;
+  dm.C = policy == DLA_POLICY_DYNAMIC ? cfg.C : 64;
+  int W = cfg.window > 0 ? cfg.window : 2048;
+  W = (W + dm.M - 1) / dm.M * dm.M;
+  const int Tr = (cfg.T + dm.M - 1) / dm.M * dm.M;
+  if (Tr > 0 && W > Tr) W = Tr;
+  if (W < dm.M) W = dm.M;
+  dm.W = W;
+  dm.tiles = W / dm.M;
+  dm.amax = dm.C;
+  const int per_tile = dm.C < 2 * dm.M + 1 ? dm.C : 2 * dm.M + 1;
+  dm.vmax = dm.C + dm.tiles * per_tile;
+  dm.opsmax = 3 * W + dm.tiles + 1 + dm.vmax + 8;
+  dm.vbytes = dm.D * dm.D * (int)sizeof(float);
+  return dm;
+}
+
+void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
+  const size_t h = dm.heads;
+  pl.r = cv.take<double>(h * dm.W);
+  pl.b = cv.take<uint8_t>(h * dm.W);
+  pl.seg_start = cv.take<int32_t>(h * (dm.W + 1));
+  pl.nseg = cv.take<int32_t>(h);
+  pl.z_end = cv.take<double>(h * dm.W * dm.D);
+  pl.z_tile = cv.take<double>(h * dm.tiles * dm.D);
+  pl.ops = cv.take<int4>(h * dm.opsmax);
+  pl.nops = cv.take<int32_t>(h);
+  pl.tile_m0 = cv.take<int32_t>(h * dm.tiles);
+  pl.tile_atoms = cv.take<int32_t>(h * dm.tiles * dm.amax);
+  pl.tile_nev = cv.take<int32_t>(h * dm.tiles);
+  pl.tile_ev_off = cv.take<int32_t>(h * dm.tiles * dm.M);
+  pl.tile_ev_mrg = cv.take<int32_t>(h * dm.tiles * dm.M);
+  pl.ver_mu = cv.take<float>(h * dm.vmax * dm.D);
+  pl.ver_n = cv.take<float>(h * dm.vmax);
+  pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
+  pl.slot_ver = cv.take<int32_t>(h * dm.C);
+}
+
+bool cfg_ok(const dla_config *cfg, int policy) {
+  if (!cfg) return false;
+  if (cfg->B <= 0 || cfg->H <= 0 || cfg->T < 0) return false;
+  if (cfg->in_dtype != DLA_F32 && cfg->in_dtype != DLA_BF16) return false;
+  if (cfg->window < 0) return false;
+  (void)policy;
+  return true;
+}
+
+dla_status shape_ok(const dla_config *cfg, int policy) {
+  if (cfg->d_k != cfg->d_v || !d_ok(cfg->d_k)) return DLA_ERR_UNSUPPORTED;
+  if (policy == DLA_POLICY_DYNAMIC && (cfg->C < 2 || cfg->C > 128)) return DLA_ERR_UNSUPPORTED;
+  return DLA_OK;
+}
+
+}  // namespace
+}  // namespace dla
+
+using namespace dla;
+
+extern "C" {
+
+const char *dla_status_string(dla_status s) {
+  switch (s) {
+    case DLA_OK: return "ok";
+    case DLA_ERR_INVALID_ARG: return "invalid argument";
+    case DLA_ERR_UNSUPPORTED: return "unsupported shape (need d_k == d_v in {32, 64, 128}, 2 <= C <= 128)";
+    case DLA_ERR_CUDA: return "CUDA launch failed";
+    case DLA_ERR_TRACE_OVERFLOW: return "more merges than the trace capacity";
+    case DLA_ERR_WORKSPACE: return "workspace smaller than dla_workspace_bytes()";
+    case DLA_ERR_INVARIANT: return "device invariant violated";
+  }
+  return "unknown status";
+}
+
+size_t dla_cache_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {
+  if (N <= 0 || H <= 0 || C <= 0 || d_k <= 0 || d_v <= 0) return 0;
+  dla_cache c{};
+  c.N = N;
+  c.H = H;
+  c.C = C;
+  c.d_k = d_k;
+  c.d_v = d_v;
+  Carver cv{nullptr};
+  carve_cache(cv, c);
+  return cv.off;
+}
+
+dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int32_t d_k,
+                          int32_t d_v, void *dev_base, size_t bytes, void *stream) {
+  if (!cache || !dev_base) return DLA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(dev_base) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  const size_t need = dla_cache_bytes(N, H, C, d_k, d_v);
+  if (need == 0) return DLA_ERR_INVALID_ARG;
+  if (bytes < need) return DLA_ERR_WORKSPACE;
+  if (d_k != d_v || !d_ok(d_k) || C < 2 || C > 128) return DLA_ERR_UNSUPPORTED;
+  dla_cache c{};
+  c.N = N;
+  c.H = H;
+  c.C = C;
+  c.d_k = d_k;
+  c.d_v = d_v;
+  Carver cv{static_cast<char *>(dev_base)};
+  carve_cache(cv, c);
+  if (cudaMemsetAsync(dev_base, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DLA_ERR_CUDA;
+  *cache = c;
+  return DLA_OK;
+}
+
+size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
+  if (!cfg_ok(cfg, policy) || shape_ok(cfg, policy) != DLA_OK) return 0;
+  const Dims dm = make_dims(*cfg, policy);
+  Plan pl{};
+  Carver cv{nullptr};
+  carve_plan(cv, dm, pl);
+  return cv.off;
+}
+
+dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, const void *v,
+                       void *o, const dla_cache *cache, const dla_trace *trace, void *ws,
+                       size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg, DLA_POLICY_DYNAMIC) || !cache) return DLA_ERR_INVALID_ARG;
+  const dla_status sh = shape_ok(cfg, DLA_POLICY_DYNAMIC);
+  if (sh != DLA_OK) return sh;
+  if (cache->N != cfg->B || cache->H != cfg->H || cache->C != cfg->C || cache->d_k != cfg->d_k ||
+      cache->d_v != cfg->d_v)
+    return DLA_ERR_INVALID_ARG;
+  if (cfg->T == 0) return DLA_OK;
+  if (!q || !k || !v || !o || !ws) return DLA_ERR_INVALID_ARG;
+  if (trace && (!trace->boundary || !trace->merge_t || !trace->merge_i || !trace->merge_count ||
+                trace->cap < 0))
+    return DLA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
+  Plan pl{};
+  Carver cv{static_cast<char *>(ws)};
+  carve_plan(cv, dm, pl);
+  if (cv.off > ws_bytes) return DLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CallArgs ca{};
+  ca.q = q;
+  ca.k = k;
+  ca.v = v;
+  ca.o = o;
+  ca.in_dtype = cfg->in_dtype;
+  ca.tau = cfg->tau;
+  ca.cache = *cache;
+  if (trace) {
+    ca.trace = *trace;
+    if (cudaMemsetAsync(trace->merge_count, 0, sizeof(int32_t) * dm.heads, s) != cudaSuccess)
+      return DLA_ERR_CUDA;
+  } else {
+    memset(&ca.trace, 0, sizeof ca.trace);
+  }
+  ca.dev_status = dev_status;
+  for (int w0 = 0; w0 < cfg->T; w0 += dm.W) {
+    ca.w0 = w0;
+    ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
+    if (launch_decide(dm, pl, ca, DLA_POLICY_DYNAMIC, s) != cudaSuccess) return DLA_ERR_CUDA;
+    if (launch_materialize(dm, pl, ca, s) != cudaSuccess) return DLA_ERR_CUDA;
+    if (launch_readout_simt(dm, pl, ca, s) != cudaSuccess) return DLA_ERR_CUDA;
+  }
+  return DLA_OK;
+}
+
+size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {
+  (void)N;
+  (void)H;
+  (void)C;
+  (void)d_k;
+  (void)d_v;
+  return 0;
+}
+
+dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype, const void *q,
+                           const void *k, const void *v, void *o, uint8_t *boundary,
+                           int32_t *merge_i, void *ws, size_t ws_bytes, int32_t *dev_status,
+                           void *stream) {
+  (void)cache;
+  (void)tau;
+  (void)in_dtype;
+  (void)q;
+  (void)k;
+  (void)v;
+  (void)o;
+  (void)boundary;
+  (void)merge_i;
+  (void)ws;
+  (void)ws_bytes;
+  (void)dev_status;
+  (void)stream;
+  return DLA_ERR_UNSUPPORTED;
+}
+
+dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,
+                                    const void *v, void *o, void *ws, size_t ws_bytes,
+                                    int32_t *dev_status, void *stream) {
+  (void)cfg;
+  (void)q;
+  (void)k;
+  (void)v;
+  (void)o;
+  (void)ws;
+  (void)ws_bytes;
+  (void)dev_status;
+  (void)stream;
+  return DLA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+// dla_internal.cuh -- data structures shared by the libdla kernels.
+//
+// A prefill call is processed in windows of W tokens.  For each window the
+// decision kernels (score, segment scan, segment sums, capacity-merge engine)
+// turn the keys into a *plan*:
+//   - an op list per head that the materializer executes in time order on the
+//     fp32 slot states of the cache (ZERO / ADD tokens / MERGE / SHADOW);
+//   - per readout tile (M tokens): the states present just before the tile
+//     ("atoms", as frozen versions written by SHADOW ops) and the in-tile
+//     boundaries with their merges.
+// The readout kernels then treat every tile independently.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dla.h"
+
+namespace dla {
+
+enum OpCode : int32_t { OP_ZERO = 0, OP_ADD = 1, OP_MERGE = 2, OP_SHADOW = 3 };
+
+// Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
+// pair at that time-order position, <= -2 merge the two newest sealed states
+// (-code - 1) times (binary-counter carries of the fixed policy).
+constexpr int32_t EV_NO_MERGE = -1;
+
+struct Dims {
+  int32_t heads;   // B * H streams in the call
+  int32_t T;       // tokens in the call
+  int32_t W;       // window length (multiple of M)
+  int32_t M;       // readout tile rows
+  int32_t tiles;   // W / M
+  int32_t D;       // d_k == d_v
+  int32_t C;       // cache capacity (slots)
+  int32_t amax;    // max atoms per tile
+  int32_t vmax;    // max versions per head per window
+  int32_t opsmax;  // max ops per head per window
+  int32_t vbytes;  // bytes of one version's S
+};
+
+// Per-window plan, every array strided by head.
+struct Plan {
+  double *r;           // [heads][W] scores
+  uint8_t *b;          // [heads][W] boundary flags
+  int32_t *seg_start;  // [heads][W + 1] window-local first token of each piece
+  int32_t *nseg;       // [heads]
+  double *z_end;       // [heads][W][D] phi(k) sum of each piece's state at its end
+  double *z_tile;      // [heads][tiles][D] open state's phi(k) sum before each tile
+  int4 *ops;           // [heads][opsmax]
+  int32_t *nops;       // [heads]
+  int32_t *tile_m0;    // [heads][tiles]
+  int32_t *tile_atoms; // [heads][tiles][amax] version ids
+  int32_t *tile_nev;   // [heads][tiles]
+  int32_t *tile_ev_off;// [heads][tiles][M] boundary offset inside the tile
+  int32_t *tile_ev_mrg;// [heads][tiles][M] merge code (see EV_NO_MERGE)
+  float *ver_mu;       // [heads][vmax][D] mean phi(k) of each version
+  float *ver_n;        // [heads][vmax] token count of each version
+  void *ver_S;         // [heads][vmax] versions (fp32 [D][D] or bf16 tiled)
+  int32_t *slot_ver;   // [heads][C] engine scratch
+};
+
+struct CallArgs {
+  const void *q, *k, *v;
+  void *o;
+  int32_t in_dtype;
+  int32_t w0;         // first token of the window inside the call
+  int32_t Tw;         // tokens in this window
+  float tau;
+  dla_cache cache;
+  dla_trace trace;    // boundary == NULL when no trace
+  int32_t *dev_status;
+};
+
+__device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+__device__ __forceinline__ float load_in(const void *p, int32_t dtype, size_t i) {
+  if (dtype == DLA_F32) return static_cast<const float *>(p)[i];
+  uint32_t b = static_cast<uint32_t>(static_cast<const uint16_t *>(p)[i]) << 16;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ void store_out(void *p, int32_t dtype, size_t i, float x) {
+  if (dtype == DLA_F32) {
+    static_cast<float *>(p)[i] = x;
+  } else {
+    // round to nearest even
+    uint32_t u = __float_as_uint(x);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    static_cast<uint16_t *>(p)[i] = static_cast<uint16_t>(u >> 16);
+  }
+}
+
+// phi = elu + 1 in fp64 (decision summaries) and fp32 (states, readout).
+__device__ __forceinline__ double phi64(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+__device__ __forceinline__ float phi32(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
+
+// Host launchers (one per kernel file).
+cudaError_t launch_decide(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
+                          cudaStream_t s);
+cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
+                               cudaStream_t s);
+cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
+                                cudaStream_t s);
+cudaError_t launch_cache_reset(const dla_cache &c, cudaStream_t s);
+cudaError_t launch_decode(const dla_cache &c, float tau, int32_t in_dtype, const void *q,
+                          const void *k, const void *v, void *o, uint8_t *boundary,
+                          int32_t *merge_i, void *ws, int32_t *dev_status, cudaStream_t s);
+size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C, int32_t D);
+
+}  // namespace dla

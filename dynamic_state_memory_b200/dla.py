@@ -1,0 +1,231 @@
+"""Thin ctypes binding of libdla.so (argument marshalling only).
+
+Every step of the DLA path runs in the library's CUDA kernels; PyTorch only
+provides device memory and streams.  Importing this module fails loudly when
+the library is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdla.so")
+
+DLA_OK = 0
+DLA_F32, DLA_BF16 = 0, 1
+DLA_POLICY_DYNAMIC, DLA_POLICY_FENWICK = 0, 1
+STATUS_NAMES = {0: "DLA_OK", 1: "DLA_ERR_INVALID_ARG", 2: "DLA_ERR_UNSUPPORTED", 3: "DLA_ERR_CUDA",
+                4: "DLA_ERR_TRACE_OVERFLOW", 5: "DLA_ERR_WORKSPACE", 6: "DLA_ERR_INVARIANT"}
+
+c_i32, c_f32, c_vp, c_size = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class dla_config(ctypes.Structure):
+    _fields_ = [("B", c_i32), ("H", c_i32), ("T", c_i32), ("d_k", c_i32), ("d_v", c_i32),
+                ("C", c_i32), ("tau", c_f32), ("in_dtype", c_i32), ("window", c_i32)]
+
+
+class dla_cache(ctypes.Structure):
+    _fields_ = [("N", c_i32), ("H", c_i32), ("C", c_i32), ("d_k", c_i32), ("d_v", c_i32),
+                ("S", c_vp), ("z", c_vp), ("n", c_vp), ("ts", c_vp), ("pair_loss", c_vp),
+                ("order", c_vp), ("m", c_vp), ("prev_k", c_vp), ("prev_r", c_vp), ("t", c_vp)]
+
+
+class dla_trace(ctypes.Structure):
+    _fields_ = [("boundary", c_vp), ("merge_t", c_vp), ("merge_i", c_vp),
+                ("merge_count", c_vp), ("cap", c_i32)]
+
+
+class DlaError(RuntimeError):
+    def __init__(self, code, where=""):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({status_string(code)})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libdla.so not built at {LIB_PATH}; run dynamic_state_memory_b200/build.py")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.POINTER
+_lib.dla_status_string.restype = ctypes.c_char_p
+_lib.dla_status_string.argtypes = [c_i32]
+_lib.dla_cache_bytes.restype = c_size
+_lib.dla_cache_bytes.argtypes = [c_i32] * 5
+_lib.dla_cache_init.restype = c_i32
+_lib.dla_cache_init.argtypes = [_P(dla_cache), c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_size, c_vp]
+_lib.dla_workspace_bytes.restype = c_size
+_lib.dla_workspace_bytes.argtypes = [_P(dla_config), c_i32]
+_lib.dla_prefill.restype = c_i32
+_lib.dla_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_cache), _P(dla_trace),
+                             c_vp, c_size, c_vp, c_vp]
+_lib.dla_decode_workspace_bytes.restype = c_size
+_lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
+_lib.dla_decode_step.restype = c_i32
+_lib.dla_decode_step.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                 c_vp, c_size, c_vp, c_vp]
+_lib.dla_fixed_policy_prefill.restype = c_i32
+_lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, c_vp, c_size,
+                                          c_vp, c_vp]
+
+EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
+           "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
+           "dla_fixed_policy_prefill"]
+
+
+def status_string(code: int) -> str:
+    return _lib.dla_status_string(int(code)).decode()
+
+
+def _check(code, where):
+    if code != DLA_OK:
+        raise DlaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DLA_F32
+    if t.dtype == torch.bfloat16:
+        return DLA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ---- raw C entry points (same names, argument marshalling only) -----------
+
+def dla_cache_bytes(N, H, C, d_k, d_v) -> int:
+    return int(_lib.dla_cache_bytes(N, H, C, d_k, d_v))
+
+
+def dla_cache_init(cache: dla_cache, N, H, C, d_k, d_v, base: torch.Tensor, stream=None):
+    _check(_lib.dla_cache_init(ctypes.byref(cache), N, H, C, d_k, d_v, _ptr(base),
+                               base.numel() * base.element_size(), _stream(stream)),
+           "dla_cache_init")
+
+
+def dla_workspace_bytes(cfg: dla_config, policy=DLA_POLICY_DYNAMIC) -> int:
+    return int(_lib.dla_workspace_bytes(ctypes.byref(cfg), policy))
+
+
+def dla_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, stream=None):
+    tr = ctypes.byref(trace) if trace is not None else None
+    _check(_lib.dla_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                            ctypes.byref(cache), tr, _ptr(ws),
+                            0 if ws is None else ws.numel(), _ptr(dev_status), _stream(stream)),
+           "dla_prefill")
+
+
+def dla_decode_workspace_bytes(N, H, C, d_k, d_v) -> int:
+    return int(_lib.dla_decode_workspace_bytes(N, H, C, d_k, d_v))
+
+
+def dla_decode_step(cache, tau, in_dtype, q, k, v, o, boundary, merge_i, ws, dev_status,
+                    stream=None):
+    _check(_lib.dla_decode_step(ctypes.byref(cache), float(tau), int(in_dtype), _ptr(q), _ptr(k),
+                                _ptr(v), _ptr(o), _ptr(boundary), _ptr(merge_i), _ptr(ws),
+                                0 if ws is None else ws.numel(), _ptr(dev_status),
+                                _stream(stream)),
+           "dla_decode_step")
+
+
+def dla_fixed_policy_prefill(cfg, q, k, v, o, ws, dev_status, stream=None):
+    _check(_lib.dla_fixed_policy_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                         _ptr(ws), 0 if ws is None else ws.numel(),
+                                         _ptr(dev_status), _stream(stream)),
+           "dla_fixed_policy_prefill")
+
+
+# ---- convenience layer ------------------------------------------------------
+
+class Cache:
+    """A DLA state cache in one torch uint8 buffer (256-byte aligned)."""
+
+    def __init__(self, N, H, C, d, device="cuda", stream=None):
+        self.N, self.H, self.C, self.d = N, H, C, d
+        nbytes = dla_cache_bytes(N, H, C, d, d)
+        if nbytes == 0:
+            raise DlaError(1, "dla_cache_bytes")
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.base = self.buf[off:off + nbytes]
+        self.c = dla_cache()
+        dla_cache_init(self.c, N, H, C, d, d, self.base, stream)
+
+    def _view(self, name, dtype, shape):
+        off = getattr(self.c, name) - self.base.data_ptr()
+        n = 1
+        for s in shape:
+            n *= s
+        nb = n * torch.empty((), dtype=dtype).element_size()
+        return self.base[off:off + nb].view(dtype).view(*shape)
+
+    def views(self):
+        N, H, C, d = self.N, self.H, self.C, self.d
+        return dict(S=self._view("S", torch.float32, (N, H, C, d, d)),
+                    z=self._view("z", torch.float64, (N, H, C, d)),
+                    n=self._view("n", torch.int64, (N, H, C)),
+                    ts=self._view("ts", torch.int64, (N, H, C)),
+                    pair_loss=self._view("pair_loss", torch.float64, (N, H, C)),
+                    order=self._view("order", torch.int32, (N, H, C)),
+                    m=self._view("m", torch.int32, (N, H)),
+                    prev_k=self._view("prev_k", torch.float32, (N, H, d)),
+                    prev_r=self._view("prev_r", torch.float64, (N, H)),
+                    t=self._view("t", torch.int64, (N, H)))
+
+
+def make_config(B, H, T, d, C, tau, dtype_code, window=0) -> dla_config:
+    return dla_config(B, H, T, d, d, C, float(tau), dtype_code, window)
+
+
+class Trace:
+    def __init__(self, heads, T, cap, device="cuda"):
+        self.boundary = torch.zeros(heads, max(T, 1), dtype=torch.uint8, device=device)
+        self.merge_t = torch.zeros(heads, max(cap, 1), dtype=torch.int32, device=device)
+        self.merge_i = torch.zeros_like(self.merge_t)
+        self.merge_count = torch.zeros(heads, dtype=torch.int32, device=device)
+        self.c = dla_trace(self.boundary.data_ptr(), self.merge_t.data_ptr(),
+                           self.merge_i.data_ptr(), self.merge_count.data_ptr(), cap)
+
+    def merges(self):
+        mc = self.merge_count.cpu().tolist()
+        mt = self.merge_t.cpu()
+        mi = self.merge_i.cpu()
+        cap = self.c.cap
+        return [list(zip(mt[h, :min(c, cap)].tolist(), mi[h, :min(c, cap)].tolist()))
+                for h, c in enumerate(mc)]
+
+
+def check_device_status(dev_status: torch.Tensor, where: str):
+    code = int(dev_status.item())
+    if code != DLA_OK:
+        raise DlaError(code, where + " (device)")
+
+
+def prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, cap=None, window=0,
+            stream=None, sync=True):
+    """o = DLA prefill of q, k, v [B, H, T, d] (fp32 or bf16 CUDA tensors)."""
+    B, H, T, d = k.shape
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    cfg = make_config(B, H, T, d, cache.C, tau, _dtype_code(k), window)
+    ws = torch.empty(max(dla_workspace_bytes(cfg), 1), dtype=torch.uint8, device=k.device)
+    o = torch.empty_like(q)
+    tr = Trace(B * H, T, T + 1 if cap is None else cap, k.device) if trace else None
+    st = torch.zeros(1, dtype=torch.int32, device=k.device)
+    dla_prefill(cfg, q, k, v, o, cache.c, None if tr is None else tr.c, ws, st, stream)
+    if sync:
+        torch.cuda.synchronize()
+        check_device_status(st, "dla_prefill")
+    return o, tr

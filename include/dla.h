@@ -1,0 +1,153 @@
+/*
+ * dla.h -- C ABI of libdla.so, the B200 (sm_100a) Dynamic Linear Attention
+ * (DLA) forward.
+ *
+ * The method ("Dynamic Linear Attention | Chlience Paper Archive", sections
+ * 5.1-5.3; ai-feeds.com "Dynamic Linear Attention" summary, section 方法):
+ * each token writes v_t phi(k_t)^T into the open segment state; a token joins
+ * the open segment only when its score r_t = 1 - cos(k_t, k_{t-1}) and its
+ * predecessor's are both below tau, otherwise it opens a new state; at most C
+ * states (open one included) are kept in time order by merging the adjacent
+ * sealed pair with the smallest Ward loss n_i n_j/(n_i+n_j) |mu_i - mu_j|^2
+ * (mu = mean phi(k), leftmost on ties, merged state keeps the earlier
+ * timestamp); the output is o_t = sum_i lambda_{t,i} S_i phi(q_t) with
+ * lambda_{t,i} = softmax_i(phi(q_t) . mu_i / sqrt(d_k)).  phi = elu + 1.
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory; the
+ *     library allocates no device memory and keeps no global state.
+ *   - Every call is enqueued on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream) and returns without synchronising.
+ *   - Argument errors are returned synchronously (nothing is enqueued).
+ *   - Errors found on the device (trace overflow, broken invariant) are
+ *     written to *dev_status (a device int32 the caller zeroes beforehand and
+ *     reads after synchronising); the first error code wins.
+ *   - Calls are reentrant; concurrent calls must not share a cache, trace,
+ *     workspace or dev_status.
+ *   - Layouts are row-major with the last index fastest.  q, k, v are
+ *     [B][H][T][d]; o is [B][H][T][d_v] in the input dtype (fp32 accumulation).
+ */
+#ifndef DLA_H_
+#define DLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DLA_OK = 0,
+  DLA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, mismatched shapes */
+  DLA_ERR_UNSUPPORTED = 2,     /* d_k != d_v, d not in {32, 64, 128}, C < 2 */
+  DLA_ERR_CUDA = 3,            /* a CUDA launch failed (see cudaGetLastError) */
+  DLA_ERR_TRACE_OVERFLOW = 4,  /* device: more merges than dla_trace.cap */
+  DLA_ERR_WORKSPACE = 5,       /* ws_bytes smaller than the size query */
+  DLA_ERR_INVARIANT = 6        /* device: a cache invariant was violated */
+} dla_status;
+
+typedef enum { DLA_F32 = 0, DLA_BF16 = 1 } dla_dtype;
+
+typedef enum { DLA_POLICY_DYNAMIC = 0, DLA_POLICY_FENWICK = 1 } dla_policy;
+
+/* One prefill call.  d_k == d_v in {32, 64, 128}.  C >= 2 is the cache
+ * capacity (ignored by the fixed policy).  `window` = tokens per internal
+ * window (multiple of 128; 0 = library default); it changes memory use and
+ * speed, never results. */
+typedef struct {
+  int32_t B, H, T, d_k, d_v, C;
+  float tau;
+  int32_t in_dtype; /* dla_dtype of q, k, v and o */
+  int32_t window;
+} dla_config;
+
+/* The DLA state cache of N sequences x H heads (device memory, caller-owned,
+ * laid out by dla_cache_init inside one buffer).  It is the capacity-bounded
+ * memory M = {(S_i, n_i, ...)} of Chlience section 5.2; prefill leaves it
+ * ready for decode and a prefill on a non-empty cache continues the sequence.
+ * States live in slots; `order` lists the live slots in time order, the last
+ * one being the open state.  Per (n, h) = u:
+ *   S         float  [u][C][d_v][d_k]  slot states sum v phi(k)^T (fp32)
+ *   z         double [u][C][d_k]       slot sums of phi(k) (fp64, decisions)
+ *   n, ts     int64  [u][C]            token count and first token of a slot
+ *   pair_loss double [u][C]            Ward loss of sealed pair (p, p+1)
+ *   order     int32  [u][C]            time-order position -> slot
+ *   m         int32  [u]               live states (open one included)
+ *   prev_k    float  [u][d_k]          last key, for the next score
+ *   prev_r    double [u]               last score
+ *   t         int64  [u]               tokens seen                          */
+typedef struct {
+  int32_t N, H, C, d_k, d_v;
+  float *S;
+  double *z;
+  int64_t *n, *ts;
+  double *pair_loss;
+  int32_t *order;
+  int32_t *m;
+  float *prev_k;
+  double *prev_r;
+  int64_t *t;
+} dla_cache;
+
+/* Optional decision trace of one prefill call (device memory):
+ *   boundary    uint8 [B*H][T]   1 where token t opened a state
+ *   merge_t     int32 [B*H][cap] global token index of each merge
+ *   merge_i     int32 [B*H][cap] 0-based time-order position of the merged
+ *                                pair's left member among sealed states
+ *   merge_count int32 [B*H]      merges (may exceed cap: overflow status)  */
+typedef struct {
+  uint8_t *boundary;
+  int32_t *merge_t, *merge_i, *merge_count;
+  int32_t cap;
+} dla_trace;
+
+/* Bytes of device memory a cache of this shape needs (256-byte aligned). */
+size_t dla_cache_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v);
+
+/* Lay out a cache in [dev_base, dev_base + bytes) and reset it to the empty
+ * state (m = 0, t = 0, prev_r = 0, S = 0) with kernels on `stream`.
+ * dev_base must be 256-byte aligned. */
+dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int32_t d_k,
+                          int32_t d_v, void *dev_base, size_t bytes, void *stream);
+
+/* Workspace bytes for dla_prefill (policy = DLA_POLICY_DYNAMIC) or
+ * dla_fixed_policy_prefill (DLA_POLICY_FENWICK) with this config. */
+size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy);
+
+/* DLA prefill of T tokens for B x H streams, continuing `cache` (required,
+ * B == cache->N, H == cache->H, same C, d).  Writes o [B][H][T][d_v] and,
+ * when `trace` is non-NULL, the decision trace.  ws: device workspace of at
+ * least dla_workspace_bytes(cfg, DLA_POLICY_DYNAMIC) bytes. */
+dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, const void *v,
+                       void *o, const dla_cache *cache, const dla_trace *trace, void *ws,
+                       size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Workspace bytes for dla_decode_step on a cache of this shape. */
+size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v);
+
+/* One token for each of the N x H streams of `cache`: decision, any capacity
+ * merge, state write and readout; equivalent to dla_prefill with T = 1.
+ * q, k, v [N][H][d] and o [N][H][d_v] in `in_dtype`.  Optional outputs:
+ * boundary [N][H] (uint8) and merge_i [N][H] (int32, -1 = no merge). */
+dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype,
+                           const void *q, const void *k, const void *v, void *o,
+                           uint8_t *boundary, int32_t *merge_i, void *ws, size_t ws_bytes,
+                           int32_t *dev_status, void *stream);
+
+/* The Log-Linear-style fixed policy through the same engine (Chlience
+ * section 2 and section 5.4): token t reads the Fenwick blocks of [0, t-1]
+ * (one per set bit of t) plus {t}, with the same softmax over block means.
+ * Starts every stream at t = 0; cfg->C and cfg->tau are ignored. */
+dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,
+                                    const void *v, void *o, void *ws, size_t ws_bytes,
+                                    int32_t *dev_status, void *stream);
+
+/* Static description of a status code. */
+const char *dla_status_string(dla_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLA_H_ */
