@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Throughput of the DLA hot path on B200, one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  prefill workloads: dla_cache_init + dla_prefill of B x H x T tokens
+  decode workload:   one dla_decode_step of N x H streams (cache pre-filled)
+Timing: CUDA events on the launching stream around exactly K steps after W
+warm-up steps, barrier + synchronize on both sides, max over ranks.  Inputs
+are larger than L2 (126 MB) so no flush is needed between steps.
+The kernel-level roofline uses events the library records around each of
+its launches in the timed region (dla_profile).
+Under torchrun every rank runs an independent replica (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "DLA prefill Mtok/s and decode steps/s at C=64,d=128; % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        smax = max(r["smax"] for r in rows)
+        load = [r["sm"] for r in rows if r["sm"] > 0.3 * smax] or [r["sm"] for r in rows]
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- inputs ----
+
+def _gen_head(args):
+    from dynamic_state_memory_b200 import synth
+    wl, b, h = args
+    st = synth.HeadStream(wl["seed"], b, h, **wl)
+    cast = synth.to_bf16_bits if wl["dtype"] == "bf16" else (lambda x: x)
+    return b, h, cast(st.q), cast(st.k), cast(st.v)
+
+
+def make_inputs(wl, rank=0):
+    """Host q, k, v [B, H, T, d] of a workload (rank offsets the seed)."""
+    from concurrent.futures import ProcessPoolExecutor
+    import multiprocessing as mp
+    wl = dict(wl, seed=wl["seed"] + 7919 * rank)
+    B, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
+    npdt = np.uint16 if wl["dtype"] == "bf16" else np.float32
+    q = np.empty((B, H, T, d), dtype=npdt)
+    k = np.empty_like(q)
+    v = np.empty_like(q)
+    jobs = [(wl, b, h) for b in range(B) for h in range(H)]
+    workers = min(len(jobs), max(1, len(os.sched_getaffinity(0))))
+    if B * H * T * d < 4_000_000 or workers == 1:
+        res = map(_gen_head, jobs)
+        for b, h, qq, kk, vv in res:
+            q[b, h], k[b, h], v[b, h] = qq, kk, vv
+    else:
+        with ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+            for b, h, qq, kk, vv in ex.map(_gen_head, jobs, chunksize=4):
+                q[b, h], k[b, h], v[b, h] = qq, kk, vv
+    return q, k, v
+
+
+def to_torch(x, dtype, device):
+    import torch
+    if dtype == "bf16":
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(x).to(device)
+
+
+# ------------------------------------------------------------ prefill arm ----
+
+def prefill_flops(trace_live_sum, heads_tokens, d):
+    """Readout FLOPs: sum_t 2 m_t d^2 + 2 m_t d; plus the state build 2 d^2/token."""
+    readout = 2.0 * trace_live_sum * d * d + 2.0 * trace_live_sum * d
+    build = 2.0 * heads_tokens * d * d
+    return readout, build
+
+
+def bench_prefill(args, wl, rank, world, local_rank):
+    import torch
+    from dynamic_state_memory_b200 import dla
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    peaks, peaks_kind = load_peaks()
+    q_h, k_h, v_h = make_inputs(wl, rank)
+    B, H, T, d, C = wl["B"], wl["H"], wl["T"], wl["d"], wl["C"]
+    dt = wl["dtype"]
+    q, k, v = (to_torch(x, dt, dev) for x in (q_h, k_h, v_h))
+    cache = dla.Cache(B, H, C, d, device=dev)
+    prof = dla.Profiler(cap=4096)
+    dcode = dla.DLA_BF16 if dt == "bf16" else dla.DLA_F32
+    cfg = dla.make_config(B, H, T, d, C, wl["tau"], dcode, args.window, prof.p)
+    ws = torch.empty(dla.dla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # one traced run (untimed) to count live states for the FLOP model
+    tr = dla.Trace(B * H, T, T + 1, dev)
+    dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
+    dla.dla_prefill(cfg, q, k, v, o, cache.c, tr.c, ws, st, stream)
+    torch.cuda.synchronize(dev)
+    dla.check_device_status(st, "dla_prefill")
+    bnd = tr.boundary.cpu().numpy()
+    mt = tr.merge_t.cpu().numpy()
+    mc = tr.merge_count.cpu().numpy()
+    live_sum = 0
+    for h in range(B * H):
+        m = np.cumsum(bnd[h].astype(np.int64))
+        merges_at = np.zeros(T, dtype=np.int64)
+        np.add.at(merges_at, mt[h, :mc[h]], 1)
+        m = m - np.cumsum(merges_at)
+        live_sum += int(m.sum())
+    readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
+
+    def step():
+        dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
+        dla.dla_prefill(cfg, q, k, v, o, cache.c, None, ws, st, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    prof.reset()
+    clk = ClockSampler(local_rank)
+    if rank == 0:
+        clk.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = clk.stop() if rank == 0 else None
+    dla.check_device_status(st, "dla_prefill")
+    ms = e0.elapsed_time(e1)
+    ms_max = reduce_max(ms, world, dev)
+    launches = prof.p.count
+    kt = prof.times_ms()
+
+    # end to end through the public API with host buffers
+    pin = [torch.from_numpy(x.view(np.int16) if dt == "bf16" else x).pin_memory()
+           for x in (q_h, k_h, v_h)]
+    o_host = torch.empty(o.shape, dtype=torch.int16 if dt == "bf16" else torch.float32).pin_memory()
+
+    def e2e_step():
+        for hsrc, ddst in zip(pin, (q, k, v)):
+            ddst.view(hsrc.dtype).copy_(hsrc, non_blocking=True)
+        step()
+        o_host.copy_(o.view(o_host.dtype), non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    e2e_steps = max(1, args.steps // 2)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, world, dev)
+    in_bytes = sum(x.nbytes for x in (q_h, k_h, v_h))
+    out_bytes = o_host.numel() * o_host.element_size()
+
+    if rank != 0:
+        return None
+    ms_step = ms_max / args.steps
+    tokens = B * T * world
+    value = tokens / (ms_step * 1e-3) / 1e6
+    # dominant kernel
+    tot = {kname: sum(v_) for kname, v_ in kt.items()}
+    dom = max(tot, key=tot.get)
+    per_launch_ms = statistics.mean(kt[dom])
+    n_launch = len(kt[dom])
+    steps_recorded = args.steps
+    if dom == "readout":
+        flops_per_launch = readout_flops / (n_launch / steps_recorded)
+        if args.path == "simt":
+            bound, unit = "alu", "TFLOP/s"
+            peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock (derived)"
+        else:
+            bound, unit = "tensor", "TFLOP/s"
+            peak = peaks.get("bf16_tflops_sustained", 1371.4)
+            peak_note = f"bf16 dense, {peaks_kind} sustained"
+        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
+    else:
+        bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
+        achieved = float("nan")
+    roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": peak_note, "launch_ms": round(per_launch_ms, 4),
+            "launches": n_launch,
+            "kernel_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()}}
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(wl, q_h, k_h, v_h)
+    e2e_val = tokens / (e2e_ms * 1e-3) / 1e6
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if args.path == "simt" else "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "H": H, "T": T, "d": d, "C": C,
+                   "tau": wl["tau"], "input_dtype": dt, "path": args.path,
+                   "l2": "inputs larger than L2 (q+k+v %d MiB), no flush" % (in_bytes >> 20),
+                   "flops_per_step": readout_flops + build_flops,
+                   "mean_live_states": round(live_sum / (B * H * T), 2)},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 4), "unit": "Mtok/s", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": out_bytes},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+
+
+def cpu_baseline_prefill(wl, q, k, v, target_s=15.0):
+    """The oracle as it stands on a bounded sample of the same workload."""
+    from oracle import oracle as O
+    cores = O.cores()
+    B, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
+    heads = min(B * H, cores)
+    Ts = min(T, 256)
+    t_used = 0.0
+    while True:
+        qs = q.reshape(B * H, T, d)[:heads, :Ts]
+        ks = k.reshape(B * H, T, d)[:heads, :Ts]
+        vs = v.reshape(B * H, T, d)[:heads, :Ts]
+        orc = O.Oracle(heads, d, d, wl["C"])
+        t0 = time.perf_counter()
+        orc.run(ks, qs, vs, tau=wl["tau"], dtype=wl["dtype"], nthreads=cores)
+        t_used = time.perf_counter() - t0
+        if t_used > target_s / 4 or Ts >= T:
+            break
+        Ts = min(T, Ts * 4)
+    head_tokens_s = heads * Ts / t_used
+    return {"value": round(head_tokens_s / H / 1e6, 6), "unit": "Mtok/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{heads} heads x first {Ts} tokens of the workload, full per-token work; "
+                      f"Mtok/s = head-tokens/s / H ({t_used:.1f} s)"}
+
+
+# ------------------------------------------------------------ reference arm ----
+
+def bench_reference(args, wl):
+    from oracle import oracle as O
+    cores = O.cores()
+    q, k, v = make_inputs(dict(wl, B=1, H=min(wl["H"], cores)))
+    B, H, T, d = 1, q.shape[1], wl["T"], wl["d"]
+    Ts = min(T, args.ref_tokens)
+    times = []
+    for i in range(args.warmup + args.steps):
+        orc = O.Oracle(H, d, d, wl["C"])
+        t0 = time.perf_counter()
+        orc.run(k[0, :, :Ts], q[0, :, :Ts], v[0, :, :Ts], tau=wl["tau"], dtype=wl["dtype"],
+                nthreads=cores)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    val = H * Ts / mean / wl["H"] / 1e6
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "Mtok/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(mean * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "B": wl["B"], "H": wl["H"], "T": wl["T"],
+                       "d": d, "C": wl["C"], "tau": wl["tau"]},
+            "cpu_baseline": {"value": round(val, 6), "unit": "Mtok/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{H} heads x first {Ts} tokens per step; Mtok/s = "
+                                       "head-tokens/s / H"},
+            "e2e": {"value": round(val, 6), "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ plumbing ----
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x, world, dev):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_t8192")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--window", type=int, default=0)
+    ap.add_argument("--path", default="simt")
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--B", type=int, default=0, help="override the batch (profiling runs)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    from dynamic_state_memory_b200 import synth
+    wl = dict(synth.WORKLOADS[args.workload])
+    if args.B:
+        wl["B"] = args.B
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(bench_reference(args, wl)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    res = bench_prefill(args, wl, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -423,13 +423,25 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
 
 }  // namespace
 
-cudaError_t launch_decide(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
-                          cudaStream_t s) {
-  dim3 g1((ca.Tw + 255) / 256, dm.heads);
-  k_score<<<g1, 256, 0, s>>>(dm, pl, ca, policy);
+cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
+                         cudaStream_t s) {
+  dim3 g((ca.Tw + 255) / 256, dm.heads);
+  k_score<<<g, 256, 0, s>>>(dm, pl, ca, policy);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   k_segscan<<<dm.heads, 1024, 0, s>>>(dm, pl, ca);
-  dim3 g3(64, dm.heads);
-  k_segsum<<<g3, dm.D, 0, s>>>(dm, pl, ca);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  dim3 g(64, dm.heads);
+  k_segsum<<<g, dm.D, 0, s>>>(dm, pl, ca);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   k_engine<<<dm.heads, 32, 0, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }

@@ -204,9 +204,20 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   for (int w0 = 0; w0 < cfg->T; w0 += dm.W) {
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
-    if (launch_decide(dm, pl, ca, DLA_POLICY_DYNAMIC, s) != cudaSuccess) return DLA_ERR_CUDA;
-    if (launch_materialize(dm, pl, ca, s) != cudaSuccess) return DLA_ERR_CUDA;
-    if (launch_readout_simt(dm, pl, ca, s) != cudaSuccess) return DLA_ERR_CUDA;
+    dla_profile *pf = cfg->profile;
+    cudaError_t e;
+    { ProfScope ps(pf, DLA_K_SCORE, s); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_SEGSCAN, s); e = launch_segscan(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_SEGSUM, s); e = launch_segsum(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_engine(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_READOUT, s); e = launch_readout_simt(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
   }
   return DLA_OK;
 }
@@ -223,7 +234,8 @@ size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, 
 dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype, const void *q,
                            const void *k, const void *v, void *o, uint8_t *boundary,
                            int32_t *merge_i, void *ws, size_t ws_bytes, int32_t *dev_status,
-                           void *stream) {
+                           void *stream, dla_profile *profile) {
+  (void)profile;
   (void)cache;
   (void)tau;
   (void)in_dtype;

@@ -98,16 +98,32 @@ __device__ __forceinline__ double phi64(double x) { return x > 0.0 ? x + 1.0 : e
 __device__ __forceinline__ float phi32(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
 
 // Host launchers (one per kernel file).
-cudaError_t launch_decide(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
-                          cudaStream_t s);
+cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
+                         cudaStream_t s);
+cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s);
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s);
-cudaError_t launch_cache_reset(const dla_cache &c, cudaStream_t s);
-cudaError_t launch_decode(const dla_cache &c, float tau, int32_t in_dtype, const void *q,
-                          const void *k, const void *v, void *o, uint8_t *boundary,
-                          int32_t *merge_i, void *ws, int32_t *dev_status, cudaStream_t s);
-size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C, int32_t D);
+
+// Records a dla_profile event pair around one launch.
+struct ProfScope {
+  dla_profile *p;
+  int idx;
+  cudaStream_t s;
+  ProfScope(dla_profile *prof, int kind, cudaStream_t st) : p(prof), idx(-1), s(st) {
+    if (p && p->count < p->cap && p->begin && p->end) {
+      idx = p->count;
+      if (p->kind) p->kind[idx] = kind;
+      cudaEventRecord(static_cast<cudaEvent_t>(p->begin[idx]), s);
+    }
+    if (p) p->count++;
+  }
+  ~ProfScope() {
+    if (idx >= 0) cudaEventRecord(static_cast<cudaEvent_t>(p->end[idx]), s);
+  }
+};
 
 }  // namespace dla

@@ -23,9 +23,15 @@ STATUS_NAMES = {0: "DLA_OK", 1: "DLA_ERR_INVALID_ARG", 2: "DLA_ERR_UNSUPPORTED",
 c_i32, c_f32, c_vp, c_size = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
 
+class dla_profile(ctypes.Structure):
+    _fields_ = [("begin", ctypes.POINTER(c_vp)), ("end", ctypes.POINTER(c_vp)),
+                ("kind", ctypes.POINTER(c_i32)), ("cap", c_i32), ("count", c_i32)]
+
+
 class dla_config(ctypes.Structure):
     _fields_ = [("B", c_i32), ("H", c_i32), ("T", c_i32), ("d_k", c_i32), ("d_v", c_i32),
-                ("C", c_i32), ("tau", c_f32), ("in_dtype", c_i32), ("window", c_i32)]
+                ("C", c_i32), ("tau", c_f32), ("in_dtype", c_i32), ("window", c_i32),
+                ("profile", ctypes.POINTER(dla_profile))]
 
 
 class dla_cache(ctypes.Structure):
@@ -65,7 +71,7 @@ _lib.dla_decode_workspace_bytes.restype = c_size
 _lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
 _lib.dla_decode_step.restype = c_i32
 _lib.dla_decode_step.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
-                                 c_vp, c_size, c_vp, c_vp]
+                                 c_vp, c_size, c_vp, c_vp, _P(dla_profile)]
 _lib.dla_fixed_policy_prefill.restype = c_i32
 _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, c_vp, c_size,
                                           c_vp, c_vp]
@@ -131,11 +137,12 @@ def dla_decode_workspace_bytes(N, H, C, d_k, d_v) -> int:
 
 
 def dla_decode_step(cache, tau, in_dtype, q, k, v, o, boundary, merge_i, ws, dev_status,
-                    stream=None):
+                    stream=None, profile=None):
     _check(_lib.dla_decode_step(ctypes.byref(cache), float(tau), int(in_dtype), _ptr(q), _ptr(k),
                                 _ptr(v), _ptr(o), _ptr(boundary), _ptr(merge_i), _ptr(ws),
                                 0 if ws is None else ws.numel(), _ptr(dev_status),
-                                _stream(stream)),
+                                _stream(stream),
+                                None if profile is None else ctypes.byref(profile)),
            "dla_decode_step")
 
 
@@ -184,8 +191,43 @@ class Cache:
                     t=self._view("t", torch.int64, (N, H)))
 
 
-def make_config(B, H, T, d, C, tau, dtype_code, window=0) -> dla_config:
-    return dla_config(B, H, T, d, d, C, float(tau), dtype_code, window)
+def make_config(B, H, T, d, C, tau, dtype_code, window=0, profile=None) -> dla_config:
+    cfg = dla_config(B, H, T, d, d, C, float(tau), dtype_code, window)
+    if profile is not None:
+        cfg.profile = ctypes.pointer(profile)
+    return cfg
+
+
+class Profiler:
+    """Caller-owned CUDA events the library records around each launch."""
+
+    KINDS = ["score", "segscan", "segsum", "engine", "materialize", "readout",
+             "decode_decide", "decode_stream"]
+
+    def __init__(self, cap=4096):
+        self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(cap)]
+        for b, e in self.events:      # force creation of the underlying cudaEvent_t
+            b.record()
+            e.record()
+        torch.cuda.synchronize()
+        self._b = (c_vp * cap)(*[b.cuda_event for b, _ in self.events])
+        self._e = (c_vp * cap)(*[e.cuda_event for _, e in self.events])
+        self._k = (c_i32 * cap)()
+        self.p = dla_profile(ctypes.cast(self._b, ctypes.POINTER(c_vp)),
+                             ctypes.cast(self._e, ctypes.POINTER(c_vp)),
+                             ctypes.cast(self._k, ctypes.POINTER(c_i32)), cap, 0)
+
+    def reset(self):
+        self.p.count = 0
+
+    def times_ms(self):
+        """{kind: [ms per recorded launch]} (call after synchronising)."""
+        out = {}
+        for i in range(min(self.p.count, self.p.cap)):
+            b, e = self.events[i]
+            out.setdefault(self.KINDS[self._k[i]], []).append(b.elapsed_time(e))
+        return out
 
 
 class Trace:
@@ -213,13 +255,13 @@ def check_device_status(dev_status: torch.Tensor, where: str):
 
 
 def prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, cap=None, window=0,
-            stream=None, sync=True):
+            stream=None, sync=True, profile=None):
     """o = DLA prefill of q, k, v [B, H, T, d] (fp32 or bf16 CUDA tensors)."""
     B, H, T, d = k.shape
     for t in (q, k, v):
         if not t.is_cuda or not t.is_contiguous() or t.shape != k.shape or t.dtype != k.dtype:
             raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
-    cfg = make_config(B, H, T, d, cache.C, tau, _dtype_code(k), window)
+    cfg = make_config(B, H, T, d, cache.C, tau, _dtype_code(k), window, profile)
     ws = torch.empty(max(dla_workspace_bytes(cfg), 1), dtype=torch.uint8, device=k.device)
     o = torch.empty_like(q)
     tr = Trace(B * H, T, T + 1 if cap is None else cap, k.device) if trace else None

@@ -51,6 +51,29 @@ typedef enum { DLA_F32 = 0, DLA_BF16 = 1 } dla_dtype;
 
 typedef enum { DLA_POLICY_DYNAMIC = 0, DLA_POLICY_FENWICK = 1 } dla_policy;
 
+/* Kernel kinds reported through dla_profile. */
+typedef enum {
+  DLA_K_SCORE = 0,       /* score + boundary scan */
+  DLA_K_SEGSCAN = 1,     /* window piece scan */
+  DLA_K_SEGSUM = 2,      /* fp64 piece sums of phi(k) */
+  DLA_K_ENGINE = 3,      /* capacity-merge engine / bucket planner */
+  DLA_K_MATERIALIZE = 4, /* state build, merges and versions */
+  DLA_K_READOUT = 5,     /* multi-state readout */
+  DLA_K_DECODE_DECIDE = 6,
+  DLA_K_DECODE_STREAM = 7
+} dla_kernel_kind;
+
+/* Optional timing hook (host memory, caller-owned).  When non-NULL, the
+ * library records begin[i] / end[i] (cudaEvent_t handles created by the
+ * caller) on the launch stream around the i-th kernel it launches, stores its
+ * dla_kernel_kind in kind[i] and advances `count`; launches past `cap` are not
+ * recorded.  It adds two event records per launch and changes no result. */
+typedef struct {
+  void **begin, **end;
+  int32_t *kind;
+  int32_t cap, count;
+} dla_profile;
+
 /* One prefill call.  d_k == d_v in {32, 64, 128}.  C >= 2 is the cache
  * capacity (ignored by the fixed policy).  `window` = tokens per internal
  * window (multiple of 128; 0 = library default); it changes memory use and
@@ -60,6 +83,7 @@ typedef struct {
   float tau;
   int32_t in_dtype; /* dla_dtype of q, k, v and o */
   int32_t window;
+  dla_profile *profile; /* optional timing hook, NULL in normal use */
 } dla_config;
 
 /* The DLA state cache of N sequences x H heads (device memory, caller-owned,
@@ -129,11 +153,12 @@ size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, 
 /* One token for each of the N x H streams of `cache`: decision, any capacity
  * merge, state write and readout; equivalent to dla_prefill with T = 1.
  * q, k, v [N][H][d] and o [N][H][d_v] in `in_dtype`.  Optional outputs:
- * boundary [N][H] (uint8) and merge_i [N][H] (int32, -1 = no merge). */
+ * boundary [N][H] (uint8) and merge_i [N][H] (int32, -1 = no merge).
+ * profile: optional timing hook (NULL in normal use). */
 dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype,
                            const void *q, const void *k, const void *v, void *o,
                            uint8_t *boundary, int32_t *merge_i, void *ws, size_t ws_bytes,
-                           int32_t *dev_status, void *stream);
+                           int32_t *dev_status, void *stream, dla_profile *profile);
 
 /* The Log-Linear-style fixed policy through the same engine (Chlience
  * section 2 and section 5.4): token t reads the Fenwick blocks of [0, t-1]
