@@ -319,6 +319,163 @@ def cpu_baseline_prefill(wl, q, k, v, target_s=15.0):
                       f"Mtok/s = head-tokens/s / H ({t_used:.1f} s)"}
 
 
+# ------------------------------------------------------------- decode arm ----
+
+def _gen_decode_head(args):
+    from dynamic_state_memory_b200 import synth
+    wl, n, h, steps = args
+    st = synth.HeadStream(wl["seed"], n, h, **wl)
+    q, k, v = st.decode_steps(steps, wl["switch_p"])
+    c = synth.to_bf16_bits
+    return n, h, c(st.q), c(st.k), c(st.v), c(q), c(k), c(v)
+
+
+def make_decode_inputs(wl, steps, rank=0):
+    from concurrent.futures import ProcessPoolExecutor
+    import multiprocessing as mp
+    wl = dict(wl, seed=wl["seed"] + 7919 * rank)
+    N, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
+    pre = [np.empty((N, H, T, d), dtype=np.uint16) for _ in range(3)]
+    stp = [np.empty((steps, N, H, d), dtype=np.uint16) for _ in range(3)]
+    jobs = [(wl, n, h, steps) for n in range(N) for h in range(H)]
+    workers = min(len(jobs), max(1, len(os.sched_getaffinity(0))))
+    with ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+        for n, h, pq, pk, pv, sq, sk, sv in ex.map(_gen_decode_head, jobs, chunksize=16):
+            pre[0][n, h], pre[1][n, h], pre[2][n, h] = pq, pk, pv
+            stp[0][:, n, h], stp[1][:, n, h], stp[2][:, n, h] = sq, sk, sv
+    return pre, stp
+
+
+def bench_decode(args, wl, rank, world, local_rank):
+    import torch
+    from dynamic_state_memory_b200 import dla
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    peaks, peaks_kind = load_peaks()
+    N, H, T, d, C, tau = wl["B"], wl["H"], wl["T"], wl["d"], wl["C"], wl["tau"]
+    nsteps = args.warmup + args.steps
+    pre_h, stp_h = make_decode_inputs(wl, nsteps, rank)
+    cache = dla.Cache(N, H, C, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    # pre-fill every stream's cache with a T-token prefill, in sequence chunks
+    chunk = 8
+    cfg = dla.make_config(chunk, H, T, d, C, tau, dla.DLA_BF16, 1024)
+    ws = torch.empty(dla.dla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    for n0 in range(0, N, chunk):
+        qq, kk, vv = (to_torch(np.ascontiguousarray(x[n0:n0 + chunk]), "bf16", dev) for x in pre_h)
+        o = torch.empty_like(qq)
+        dla.dla_prefill(cfg, qq, kk, vv, o, cache.sub(n0, n0 + chunk), None, ws, st, stream)
+    torch.cuda.synchronize(dev)
+    dla.check_device_status(st, "prefill of the decode cache")
+    del ws, o, qq, kk, vv
+    sq, sk, sv = (to_torch(x, "bf16", dev) for x in stp_h)
+    dec = dla.Decoder(cache, dev)
+    prof = dla.Profiler(cap=4 * nsteps + 16)
+    o = torch.empty(N, H, d, dtype=torch.bfloat16, device=dev)
+    for i in range(args.warmup):
+        dec.step(sq[i], sk[i], sv[i], tau, o, stream)
+    torch.cuda.synchronize(dev)
+    m_before = int(cache.views()["m"].sum())
+    prof.reset()
+    clk = ClockSampler(local_rank)
+    if rank == 0:
+        clk.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.warmup, nsteps):
+        dec.step(sq[i], sk[i], sv[i], tau, o, stream, prof.p)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = clk.stop() if rank == 0 else None
+    dla.check_device_status(dec.status, "dla_decode_step")
+    m_after = int(cache.views()["m"].sum())
+    ms = reduce_max(e0.elapsed_time(e1), world, dev)
+    kt = prof.times_ms()
+    launches = prof.p.count
+    # end to end: host q, k, v per step, o back to the host
+    hq, hk, hv = (torch.from_numpy(x.view(np.int16)).pin_memory() for x in stp_h)
+    dq, dk_, dv = (torch.empty(N, H, d, dtype=torch.int16, device=dev) for _ in range(3))
+    ho = torch.empty(N, H, d, dtype=torch.int16).pin_memory()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    f0.record(stream)
+    e2e_steps = min(args.steps, 8)
+    for i in range(e2e_steps):
+        j = args.warmup + i
+        dq.copy_(hq[j], non_blocking=True)
+        dk_.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dec.step(dq.view(torch.bfloat16), dk_.view(torch.bfloat16), dv.view(torch.bfloat16), tau,
+                 o, stream)
+        ho.copy_(o.view(torch.int16), non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, world, dev)
+    if rank != 0:
+        return None
+    ms_step = ms / args.steps
+    value = world * 1000.0 / ms_step
+    tot = {kk: sum(vv) for kk, vv in kt.items()}
+    stream_ms = statistics.mean(kt["decode_stream"])
+    live = 0.5 * (m_before + m_after)
+    state_bytes = live * d * d * 4
+    achieved = state_bytes / (stream_ms * 1e-3) / 1e9
+    peak = peaks.get("hbm_gbs", 6540.8)
+    roof = {"kernel": "decode_stream", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peaks_kind} copy bandwidth",
+            "algorithmic_bytes_per_launch": state_bytes, "launch_ms": round(stream_ms, 4),
+            "launches": len(kt["decode_stream"]),
+            "kernel_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()}}
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_decode(wl, pre_h, stp_h)
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "N": N, "H": H, "prefill_T": T, "d": d, "C": C,
+                   "tau": tau, "input_dtype": "bf16", "state_dtype": "f32",
+                   "mean_live_states": round(live / (N * H), 2),
+                   "l2": "state cache %d GiB >> L2, no flush" % (cache.base.numel() >> 30)},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": round(world * 1000.0 / e2e_ms, 3), "unit": "steps/s",
+                "h2d_bytes_per_step": 3 * N * H * d * 2, "d2h_bytes_per_step": N * H * d * 2},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+
+
+def cpu_baseline_decode(wl, pre, stp, prefill_tokens=4096, steps=8):
+    """Oracle: 16 streams pre-filled on the workload's tokens, then timed steps."""
+    from oracle import oracle as O
+    cores = O.cores()
+    N, H, d = wl["B"], wl["H"], wl["d"]
+    U = min(16, N * H)
+    Tp = min(prefill_tokens, wl["T"])
+    k = pre[1].reshape(N * H, -1, d)[:U, :Tp]
+    q = pre[0].reshape(N * H, -1, d)[:U, :Tp]
+    v = pre[2].reshape(N * H, -1, d)[:U, :Tp]
+    orc = O.Oracle(U, d, d, wl["C"])
+    orc.run(k, q, v, tau=wl["tau"], dtype="bf16", nthreads=cores)
+    sk = stp[1].reshape(stp[1].shape[0], N * H, d)
+    sq = stp[0].reshape(stp[0].shape[0], N * H, d)
+    sv = stp[2].reshape(stp[2].shape[0], N * H, d)
+    t0 = time.perf_counter()
+    n = min(steps, sk.shape[0])
+    for i in range(n):
+        orc.run(np.ascontiguousarray(sk[i, :U, None]), np.ascontiguousarray(sq[i, :U, None]),
+                np.ascontiguousarray(sv[i, :U, None]), tau=wl["tau"], dtype="bf16",
+                nthreads=cores)
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(1.0 / (dt * (N * H) / U), 6), "unit": "steps/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{U} streams pre-filled with {Tp} tokens (untimed), {n} timed steps; "
+                      f"steps/s extrapolated to {N * H} streams"}
+
+
 # ------------------------------------------------------------ reference arm ----
 
 def bench_reference(args, wl):
@@ -399,7 +556,10 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-    res = bench_prefill(args, wl, rank, world, local_rank)
+    if args.workload.startswith("decode"):
+        res = bench_decode(args, wl, rank, world, local_rank)
+    else:
+        res = bench_prefill(args, wl, rank, world, local_rank)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

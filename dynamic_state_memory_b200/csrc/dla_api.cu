@@ -223,33 +223,35 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
 }
 
 size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {
-  (void)N;
-  (void)H;
-  (void)C;
-  (void)d_k;
-  (void)d_v;
-  return 0;
+  if (N <= 0 || H <= 0 || C < 2 || C > 128 || d_k != d_v || !d_ok(d_k)) return 0;
+  return decode_ws_bytes(N, H, C);
 }
 
 dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype, const void *q,
                            const void *k, const void *v, void *o, uint8_t *boundary,
                            int32_t *merge_i, void *ws, size_t ws_bytes, int32_t *dev_status,
                            void *stream, dla_profile *profile) {
-  (void)profile;
-  (void)cache;
-  (void)tau;
-  (void)in_dtype;
-  (void)q;
-  (void)k;
-  (void)v;
-  (void)o;
-  (void)boundary;
-  (void)merge_i;
-  (void)ws;
-  (void)ws_bytes;
-  (void)dev_status;
-  (void)stream;
-  return DLA_ERR_UNSUPPORTED;
+  if (!cache || !q || !k || !v || !o || !ws) return DLA_ERR_INVALID_ARG;
+  if (in_dtype != DLA_F32 && in_dtype != DLA_BF16) return DLA_ERR_INVALID_ARG;
+  if (!cache->S || !cache->z || !cache->order || !cache->m) return DLA_ERR_INVALID_ARG;
+  const size_t need = dla_decode_workspace_bytes(cache->N, cache->H, cache->C, cache->d_k,
+                                                 cache->d_v);
+  if (need == 0) return DLA_ERR_UNSUPPORTED;
+  if (ws_bytes < need) return DLA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    ProfScope ps(profile, DLA_K_DECODE_DECIDE, s);
+    e = launch_decode_decide(*cache, tau, in_dtype, q, k, ws, boundary, merge_i, dev_status, s);
+  }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  {
+    ProfScope ps(profile, DLA_K_DECODE_STREAM, s);
+    e = launch_decode_stream(*cache, in_dtype, q, k, v, o, ws, s);
+  }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  return DLA_OK;
 }
 
 dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,

@@ -107,6 +107,12 @@ cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &c
                                cudaStream_t s);
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s);
+cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,
+                                 const void *k, void *ws, uint8_t *boundary, int32_t *merge_i,
+                                 int32_t *dev_status, cudaStream_t s);
+cudaError_t launch_decode_stream(const dla_cache &cc, int32_t dt, const void *q, const void *k,
+                                 const void *v, void *o, void *ws, cudaStream_t s);
+size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C);
 
 // Records a dla_profile event pair around one launch.
 struct ProfScope {

@@ -177,6 +177,17 @@ class Cache:
         nb = n * torch.empty((), dtype=dtype).element_size()
         return self.base[off:off + nb].view(dtype).view(*shape)
 
+    def sub(self, n0: int, n1: int) -> dla_cache:
+        """dla_cache struct over sequences [n0, n1) of this cache (same memory)."""
+        H, C, d = self.H, self.C, self.d
+        per_u = {"S": C * d * d * 4, "z": C * d * 8, "n": C * 8, "ts": C * 8, "pair_loss": C * 8,
+                 "order": C * 4, "m": 4, "prev_k": d * 4, "prev_r": 8, "t": 8}
+        c = dla_cache()
+        c.N, c.H, c.C, c.d_k, c.d_v = n1 - n0, H, C, d, d
+        for name, sz in per_u.items():
+            setattr(c, name, getattr(self.c, name) + n0 * H * sz)
+        return c
+
     def views(self):
         N, H, C, d = self.N, self.H, self.C, self.d
         return dict(S=self._view("S", torch.float32, (N, H, C, d, d)),
@@ -271,3 +282,26 @@ def prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, cap=None, 
         torch.cuda.synchronize()
         check_device_status(st, "dla_prefill")
     return o, tr
+
+
+class Decoder:
+    """Reusable buffers for dla_decode_step on one cache."""
+
+    def __init__(self, cache: Cache, device="cuda"):
+        self.cache = cache
+        U = cache.N * cache.H
+        nb = dla_decode_workspace_bytes(cache.N, cache.H, cache.C, cache.d, cache.d)
+        if nb == 0:
+            raise DlaError(2, "dla_decode_workspace_bytes")
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=device)
+        self.boundary = torch.zeros(U, dtype=torch.uint8, device=device)
+        self.merge_i = torch.zeros(U, dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(self, q, k, v, tau, o=None, stream=None, profile=None):
+        """One token for every stream: q, k, v [N, H, d] -> o [N, H, d]."""
+        if o is None:
+            o = torch.empty_like(q)
+        dla_decode_step(self.cache.c, tau, _dtype_code(k), q, k, v, o, self.boundary,
+                        self.merge_i, self.ws, self.status, stream, profile)
+        return o
