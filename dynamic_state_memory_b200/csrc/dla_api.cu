@@ -7,6 +7,7 @@
 namespace dla {
 
 int simt_tile_rows();
+int tc_tile_rows();
 
 namespace {
 
@@ -42,14 +43,19 @@ void carve_cache(Carver &cv, dla_cache &c) {
   c.t = cv.take<int64_t>(u);
 }
 
+// The tensor-core path serves bf16 inputs with d = 128; everything else runs
+// the fp32 SIMT readout.
+bool use_tc(const dla_config &cfg) { return cfg.in_dtype == DLA_BF16 && cfg.d_k == 128; }
+
 Dims make_dims(const dla_config &cfg, int policy) {
   Dims dm{};
   dm.heads = cfg.B * cfg.H;
   dm.T = cfg.T;
-  dm.M = simt_tile_rows();
+  const bool tc = use_tc(cfg);
+  dm.M = tc ? tc_tile_rows() : simt_tile_rows();
   dm.D = cfg.d_k;
   dm.C = policy == DLA_POLICY_DYNAMIC ? cfg.C : 64;
-  int W = cfg.window > 0 ? cfg.window : 2048;
+  int W = cfg.window > 0 ? cfg.window : (tc ? 8192 : 2048);
   W = (W + dm.M - 1) / dm.M * dm.M;
   const int Tr = (cfg.T + dm.M - 1) / dm.M * dm.M;
   if (Tr > 0 && W > Tr) W = Tr;
@@ -60,7 +66,7 @@ Dims make_dims(const dla_config &cfg, int policy) {
   const int per_tile = dm.C < 2 * dm.M + 1 ? dm.C : 2 * dm.M + 1;
   dm.vmax = dm.C + dm.tiles * per_tile;
   dm.opsmax = 3 * W + dm.tiles + 1 + dm.vmax + 8;
-  dm.vbytes = dm.D * dm.D * (int)sizeof(float);
+  dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
   return dm;
 }
 
@@ -116,6 +122,7 @@ const char *dla_status_string(dla_status s) {
     case DLA_ERR_TRACE_OVERFLOW: return "more merges than the trace capacity";
     case DLA_ERR_WORKSPACE: return "workspace smaller than dla_workspace_bytes()";
     case DLA_ERR_INVARIANT: return "device invariant violated";
+    case DLA_ERR_TIMEOUT: return "a bounded device wait timed out";
   }
   return "unknown status";
 }
@@ -179,6 +186,9 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
                 trace->cap < 0))
     return DLA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  if (use_tc(*cfg) && (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
+                       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16))
+    return DLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
   Plan pl{};
   Carver cv{static_cast<char *>(ws)};
@@ -214,9 +224,13 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_engine(dm, pl, ca, s); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s); }
+    const bool tc = use_tc(*cfg);
+    { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_READOUT, s); e = launch_readout_simt(dm, pl, ca, s); }
+    {
+      ProfScope ps(pf, DLA_K_READOUT, s);
+      e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
+    }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
   }
   return DLA_OK;

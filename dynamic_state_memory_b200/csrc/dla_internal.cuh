@@ -104,7 +104,8 @@ cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, c
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
-                               cudaStream_t s);
+                               cudaStream_t s, bool bf16_versions);
+cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s);
 cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,

@@ -1,0 +1,501 @@
+// readout_tc.cu -- tcgen05 tensor-core readout of one 128-token tile (bf16
+// inputs, fp32 accumulation, d_k = d_v = 128).
+//
+// Same arithmetic as the SIMT readout (see readout_simt.cu for the atom /
+// piece / epoch formulation of o_t = sum_i lambda_{t,i} S_i phi(q_t) with
+// lambda_{t,i} = softmax_i(phi(q_t) . mu_i / sqrt(d_k)); Dynamic Linear
+// Attention | Chlience Paper Archive, section 5.3), mapped onto Blackwell:
+//
+//   TMA (128B swizzle) loads q, k, v tiles; phi is applied in shared memory.
+//   tcgen05.mma (kind::f16, M = 128 tokens) computes into tensor memory:
+//     A  = phi(Q) phi(K)^T               (128 x 128)   TMEM cols [256, 384)
+//     LA = phi(Q) Mu^T                   (128 x m0)    TMEM cols [384, 512)
+//   Four warps (one TMEM lane = one token row each) turn LA and the row sums
+//   of A into softmax weights per atom / piece, in place in TMEM, and write
+//   P = W o A (causal) as the bf16 A operand of
+//     O_intra = P V                                    TMEM cols [256, 384)
+//   Then, per atom alpha, a bulk copy brings the frozen bf16 state version
+//   (already stored in the UMMA K-major swizzled layout) into one of 3 shared
+//   stages, one thread issues P_alpha = phi(Q) S_alpha^T into one of two TMEM
+//   buffers (cols [0,128) / [128,256)), and 8 epilogue warps accumulate
+//   W_alpha(t) * P_alpha in registers while the next MMA runs.
+// Every wait on an mbarrier is bounded; a timeout sets DLA_ERR_TIMEOUT.
+#include "dla_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace dla {
+namespace {
+using namespace tc;
+
+constexpr int M = 128;
+constexpr int D = 128;
+constexpr int NST = 3;
+constexpr int THREADS = 384;
+constexpr int TILE_BYTES = M * D * 2;
+constexpr uint32_t VER_BYTES = D * D * 2;
+constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
+constexpr uint32_t COL_BUF0 = 0, COL_AI = 256, COL_W = 384;
+constexpr float INV_SQRT_D = 0.08838834764831845f;
+
+struct Smem {
+  uint8_t q[TILE_BYTES];
+  uint8_t kp[TILE_BYTES];
+  uint8_t v[TILE_BYTES];
+  uint8_t st[NST][VER_BYTES];
+  uint64_t bar_load, bar_mma, full[NST], empty[NST], tfull[2], tempty[2];
+  uint32_t tmem_base;
+  int abort;
+  int m0, np, len;
+  float nA[128];
+  int atom[128];
+  int pst[M + 1], pen[M + 1], pidx[M];
+  uint32_t bits[(M + 1) * BW];
+};
+
+__device__ __forceinline__ bool bit_of(const uint32_t *b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
+
+__device__ __forceinline__ void online(float &mx, float &l, float a) {
+  const float nm = fmaxf(mx, a);
+  l = l * expf(mx - nm) + expf(a - nm);
+  mx = nm;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_readout_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                 const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
+  extern __shared__ uint8_t raw[];
+  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                       ~static_cast<uintptr_t>(1023));
+  const int u = blockIdx.y, c = blockIdx.x;
+  const int T0 = c * M;
+  if (T0 >= ca.Tw) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int *abort = &sm.abort;
+  const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
+
+  // ---- setup: TMEM, barriers, tile metadata ------------------------------
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if (tid == 0) {
+    mbar_init(&sm.bar_load, 1);
+    mbar_init(&sm.bar_mma, 1);
+    for (int i = 0; i < NST; i++) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], 8);
+    }
+    fence_mbar_init();
+    sm.abort = 0;
+    const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
+    const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
+    const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
+    const int32_t *evm = pl.tile_ev_mrg + ((size_t)u * dm.tiles + c) * M;
+    const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
+    const int len = min(M, ca.Tw - T0);
+    sm.m0 = m0;
+    sm.len = len;
+    for (int a = 0; a < m0; a++) {
+      sm.atom[a] = atoms[a];
+      sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + atoms[a]];
+    }
+    const bool cont = !(nev > 0 && evo[0] == 0);
+    int np = 0;
+    if (cont) sm.pst[np++] = 0;
+    for (int i = 0; i < nev; i++) sm.pst[np++] = evo[i];
+    for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
+    sm.np = np;
+    uint32_t cur[BW];
+    for (int w = 0; w < BW; w++) cur[w] = 0;
+    for (int a = 0; a < m0; a++) cur[a >> 5] |= 1u << (a & 31);
+    for (int p = 0; p < np; p++) {
+      const int beta = m0 + p;
+      if (p == 0 && cont) {
+        if (m0 > 0) cur[(m0 - 1) >> 5] &= ~(1u << ((m0 - 1) & 31));
+      } else {
+        const int code = evm[p - (cont ? 1 : 0)];
+        int nm = 0, pos = -1;
+        if (code >= 0) {
+          nm = 1;
+          pos = code;
+        } else if (code <= -2) {
+          nm = -code - 1;
+        }
+        for (int r = 0; r < nm; r++) {
+          int total = 0;
+          for (int w = 0; w < BW; w++) total += __popc(cur[w]);
+          const int i = pos >= 0 ? pos : total - 2;
+          int seen = 0;
+          for (int w = 0; w < BW; w++) {
+            const int pc = __popc(cur[w]);
+            if (i < seen + pc) {
+              uint32_t x = cur[w];
+              for (int k2 = 0; k2 < i - seen; k2++) x &= x - 1;
+              cur[w] &= ~(x & (~x + 1));
+              break;
+            }
+            seen += pc;
+          }
+        }
+      }
+      cur[beta >> 5] |= 1u << (beta & 31);
+      for (int w = 0; w < BW; w++) sm.bits[p * BW + w] = cur[w];
+    }
+    for (int p = 0; p < np; p++)
+      for (int t = sm.pst[p]; t < sm.pen[p]; t++) sm.pidx[t] = p;
+    for (int t = len; t < M; t++) sm.pidx[t] = np - 1;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  const int m0 = sm.m0, np = sm.np, len = sm.len;
+
+  // ---- loads --------------------------------------------------------------
+  if (tid == 0) {
+    mbar_expect_tx(&sm.bar_load, 3 * TILE_BYTES);
+    const int row = ca.w0 + T0;
+    for (int h = 0; h < 2; h++) {
+      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, row, u);
+      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, row, u);
+      tma_load_3d(sm.v + h * (TILE_BYTES / 2), &tv, &sm.bar_load, h * 64, row, u);
+    }
+    for (int a = 0; a < m0 && a < NST - 1; a++) {
+      mbar_expect_tx(&sm.full[a], VER_BYTES);
+      bulk_load(sm.st[a], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[a]);
+    }
+  }
+  mbar_wait(&sm.bar_load, 0, abort);
+
+  // ---- phi(q), phi(k) in place; Mu (bf16 means of the atoms) ---------------
+  for (int i = tid; i < 2 * TILE_BYTES / 16; i += THREADS) {
+    uint4 *p = reinterpret_cast<uint4 *>(i < TILE_BYTES / 16 ? sm.q : sm.kp) + (i % (TILE_BYTES / 16));
+    uint4 x = *p;
+    uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi32(bf16_lo(w[j])), phi32(bf16_hi(w[j])));
+    *p = x;
+  }
+  const int n_mu = (m0 + 15) & ~15;
+  uint8_t *mu_buf = sm.st[NST - 1];
+  for (int e = tid; e < n_mu * 16; e += THREADS) {
+    const int a = e >> 4, ch = e & 15;
+    uint4 x = make_uint4(0, 0, 0, 0);
+    if (a < m0) {
+      const float *mu = pl.ver_mu + ((size_t)u * dm.vmax + sm.atom[a]) * D + ch * 8;
+      x.x = pack_bf16(mu[0], mu[1]);
+      x.y = pack_bf16(mu[2], mu[3]);
+      x.z = pack_bf16(mu[4], mu[5]);
+      x.w = pack_bf16(mu[6], mu[7]);
+    }
+    *reinterpret_cast<uint4 *>(mu_buf + sw128_offset(a, ch * 8, 128)) = x;
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+
+  const uint32_t q_s = smem_u32(sm.q), kp_s = smem_u32(sm.kp), v_s = smem_u32(sm.v);
+  auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
+    return sdesc(base + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024);
+  };
+  // ---- A = phi(Q) phi(K)^T and LA = phi(Q) Mu^T ------------------------------
+  if (warp == 1 && lane == 0) {
+    tc_fence_after();
+    for (int k = 0; k < 8; k++)
+      mma_bf16(tbase + COL_AI, kdesc(q_s, k), kdesc(kp_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
+    if (m0 > 0)
+      for (int k = 0; k < 8; k++)
+        mma_bf16(tbase + COL_W, kdesc(q_s, k), kdesc(smem_u32(mu_buf), k),
+                 idesc_bf16(M, n_mu, 0, 0), k > 0);
+    mma_commit(&sm.bar_mma);
+  }
+  mbar_wait(&sm.bar_mma, 0, abort);
+  tc_fence_after();
+  if (tid == 0 && m0 >= NST) {
+    mbar_expect_tx(&sm.full[NST - 1], VER_BYTES);
+    bulk_load(sm.st[NST - 1], verS + (size_t)sm.atom[NST - 1] * VER_BYTES, VER_BYTES,
+              &sm.full[NST - 1]);
+  }
+
+  // ---- softmax weights per row (warps 4..7, row t = TMEM lane) ----------------
+  if (warp >= 4 && warp < 8) {
+    const int qd = warp & 3;
+    const int t = 32 * qd + lane;
+    const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+    const int ep = sm.pidx[t];
+    const uint32_t *bits = sm.bits + ep * BW;
+    // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s] -> TMEM cols [0, np)
+    {
+      float y = 0.f;
+      int p = 0;
+      for (int s0 = 0; s0 < M; s0 += 32) {
+        uint32_t ar[32];
+        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+          const int s = s0 + j;
+          if (s < len) {
+            if (p + 1 < np && s == sm.pst[p + 1]) {
+              tmem_st1(trow + COL_BUF0 + p, __float_as_uint(y));
+              p++;
+              y = 0.f;
+            }
+            if (s <= t) y += __uint_as_float(ar[j]);
+          }
+        }
+      }
+      tmem_st1(trow + COL_BUF0 + p, __float_as_uint(y));
+      tmem_wait_st();
+    }
+    // pass A: state logits at each state's last atom / piece, online softmax
+    float sacc = 0.f, nacc = 0.f, mx = -INFINITY, l = 0.f;
+    for (int a0 = 0; a0 < m0; a0 += 32) {
+      uint32_t r[32];
+      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; j++) {
+        const int beta = a0 + j;
+        if (beta < m0) {
+          const float nn = sm.nA[beta];
+          sacc += nn * __uint_as_float(r[j]);
+          nacc += nn;
+          if (bit_of(bits, beta)) {
+            const float a = sacc / nacc * INV_SQRT_D;
+            r[j] = __float_as_uint(a);
+            online(mx, l, a);
+            sacc = nacc = 0.f;
+          }
+        }
+      }
+      DLA_TMEM_ST32(trow + COL_W + a0, r);
+      tmem_wait_st();
+    }
+    for (int p = 0; p < np; p++) {
+      uint32_t yv = tmem_ld1(trow + COL_BUF0 + p);
+      tmem_wait_ld();
+      if (p <= ep) {
+        const float nn = p < ep ? (float)(sm.pen[p] - sm.pst[p]) : (float)(t - sm.pst[p] + 1);
+        sacc += __uint_as_float(yv);
+        nacc += nn;
+        if (bit_of(bits, m0 + p)) {
+          const float a = sacc / nacc * INV_SQRT_D;
+          yv = __float_as_uint(a);
+          online(mx, l, a);
+          sacc = nacc = 0.f;
+        }
+      }
+      tmem_st1(trow + COL_BUF0 + p, yv);
+    }
+    tmem_wait_st();
+    // pass B (reverse): weight of every atom / piece = lambda of its state
+    float cur = 0.f;
+    for (int p = np - 1; p >= 0; p--) {
+      const uint32_t av = tmem_ld1(trow + COL_BUF0 + p);
+      tmem_wait_ld();
+      float w = 0.f;
+      if (p <= ep) {
+        if (bit_of(bits, m0 + p)) cur = expf(__uint_as_float(av) - mx) / l;
+        w = cur;
+      }
+      tmem_st1(trow + COL_BUF0 + p, __float_as_uint(w));
+    }
+    tmem_wait_st();
+    for (int a0 = ((m0 - 1) >> 5) << 5; m0 > 0 && a0 >= 0; a0 -= 32) {
+      uint32_t r[32];
+      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 31; j >= 0; j--) {
+        const int beta = a0 + j;
+        if (beta < m0) {
+          if (bit_of(bits, beta)) cur = expf(__uint_as_float(r[j]) - mx) / l;
+          r[j] = __float_as_uint(cur);
+        }
+      }
+      DLA_TMEM_ST32(trow + COL_W + a0, r);
+      tmem_wait_st();
+    }
+    // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of P V
+    {
+      int p = 0;
+      float w = __uint_as_float(tmem_ld1(trow + COL_BUF0));
+      tmem_wait_ld();
+      for (int s0 = 0; s0 < M; s0 += 32) {
+        uint32_t ar[32];
+        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float v2[2];
+#pragma unroll
+          for (int h = 0; h < 2; h++) {
+            const int s = s0 + j + h;
+            if (s < len && p + 1 < np && s == sm.pst[p + 1]) {
+              p++;
+              w = __uint_as_float(tmem_ld1(trow + COL_BUF0 + p));
+              tmem_wait_ld();
+            }
+            v2[h] = (s <= t && s < len) ? w * __uint_as_float(ar[j + h]) : 0.f;
+          }
+          pk[j >> 1] = pack_bf16(v2[0], v2[1]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ch++)
+          *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0 + ch * 8, M)) =
+              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      }
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+
+  // ---- P V, then the pipelined readout over atoms --------------------------
+  if (warp == 1 && lane == 0) {
+    tc_fence_after();
+    for (int k = 0; k < 8; k++)
+      mma_bf16(tbase + COL_AI, kdesc(kp_s, k), sdesc(v_s + k * 2048, TILE_BYTES / 2, 1024),
+               idesc_bf16(M, 128, 0, 1), k > 0);
+    mma_commit(&sm.bar_mma);
+    for (int a = 0; a < m0; a++) {
+      const int s = a % NST, b = a & 1;
+      bool ok = mbar_wait(&sm.full[s], (a / NST) & 1, abort);
+      if (a >= 2) ok = mbar_wait(&sm.tempty[b], ((a >> 1) - 1) & 1, abort) && ok;
+      tc_fence_after();
+      if (ok) {
+        const uint32_t st_s = smem_u32(sm.st[s]);
+        for (int k = 0; k < 8; k++)
+          mma_bf16(tbase + b * 128, kdesc(q_s, k), kdesc(st_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
+      }
+      mma_commit(&sm.empty[s]);
+      mma_commit(&sm.tfull[b]);
+    }
+  } else if (warp == 0 && lane == 0) {
+    for (int a = NST; a < m0; a++) {
+      const int s = a % NST;
+      if (!mbar_wait(&sm.empty[s], ((a / NST) - 1) & 1, abort)) break;
+      mbar_expect_tx(&sm.full[s], VER_BYTES);
+      bulk_load(sm.st[s], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
+    }
+  } else if (warp >= 4) {
+    const int qd = warp & 3, hc = (warp - 4) >> 2;
+    const int t = 32 * qd + lane;
+    const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; i++) acc[i] = 0.f;
+    for (int a0 = 0; a0 < m0; a0 += 32) {
+      uint32_t wr[32];
+      DLA_TMEM_LD32(trow + COL_W + a0, wr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; j++) {
+        const int a = a0 + j;
+        if (a < m0) {
+          const int b = a & 1;
+          mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
+          tc_fence_after();
+          const float w = __uint_as_float(wr[j]);
+          uint32_t pr[32];
+          DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i++) acc[i] = fmaf(w, __uint_as_float(pr[i]), acc[i]);
+          DLA_TMEM_LD32(trow + b * 128 + hc * 64 + 32, pr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(w, __uint_as_float(pr[i]), acc[32 + i]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.tempty[b]);
+        }
+      }
+    }
+    mbar_wait(&sm.bar_mma, 1, abort);
+    tc_fence_after();
+    {
+      uint32_t pr[32];
+      DLA_TMEM_LD32(trow + COL_AI + hc * 64, pr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i++) acc[i] += __uint_as_float(pr[i]);
+      DLA_TMEM_LD32(trow + COL_AI + hc * 64 + 32, pr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i++) acc[32 + i] += __uint_as_float(pr[i]);
+    }
+    if (t < len) {
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(ca.o) +
+                                             ((size_t)u * dm.T + ca.w0 + T0 + t) * D + hc * 64);
+#pragma unroll
+      for (int ch = 0; ch < 8; ch++)
+        dst[ch] = make_uint4(pack_bf16(acc[8 * ch], acc[8 * ch + 1]),
+                             pack_bf16(acc[8 * ch + 2], acc[8 * ch + 3]),
+                             pack_bf16(acc[8 * ch + 4], acc[8 * ch + 5]),
+                             pack_bf16(acc[8 * ch + 6], acc[8 * ch + 7]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+  if (tid == 0 && sm.abort) set_status(ca.dev_status, DLA_ERR_TIMEOUT);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, int T, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)M, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int tc_tile_rows() { return M; }
+
+size_t readout_tc_smem() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, ca.q, dm.T, dm.heads) || !make_map(&tk, ca.k, dm.T, dm.heads) ||
+      !make_map(&tv, ca.v, dm.T, dm.heads))
+    return cudaErrorInvalidValue;
+  const size_t sb = readout_tc_smem();
+  cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sb);
+  if (e != cudaSuccess) return e;
+  dim3 g(dm.tiles, dm.heads);
+  k_readout_tc<<<g, THREADS, sb, s>>>(tq, tk, tv, dm, pl, ca);
+  return cudaGetLastError();
+}
+
+}  // namespace dla

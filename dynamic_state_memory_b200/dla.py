@@ -18,7 +18,8 @@ DLA_OK = 0
 DLA_F32, DLA_BF16 = 0, 1
 DLA_POLICY_DYNAMIC, DLA_POLICY_FENWICK = 0, 1
 STATUS_NAMES = {0: "DLA_OK", 1: "DLA_ERR_INVALID_ARG", 2: "DLA_ERR_UNSUPPORTED", 3: "DLA_ERR_CUDA",
-                4: "DLA_ERR_TRACE_OVERFLOW", 5: "DLA_ERR_WORKSPACE", 6: "DLA_ERR_INVARIANT"}
+                4: "DLA_ERR_TRACE_OVERFLOW", 5: "DLA_ERR_WORKSPACE", 6: "DLA_ERR_INVARIANT",
+                7: "DLA_ERR_TIMEOUT"}
 
 c_i32, c_f32, c_vp, c_size = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 

@@ -44,7 +44,8 @@ typedef enum {
   DLA_ERR_CUDA = 3,            /* a CUDA launch failed (see cudaGetLastError) */
   DLA_ERR_TRACE_OVERFLOW = 4,  /* device: more merges than dla_trace.cap */
   DLA_ERR_WORKSPACE = 5,       /* ws_bytes smaller than the size query */
-  DLA_ERR_INVARIANT = 6        /* device: a cache invariant was violated */
+  DLA_ERR_INVARIANT = 6,       /* device: a cache invariant was violated */
+  DLA_ERR_TIMEOUT = 7          /* device: a bounded wait inside a kernel gave up */
 } dla_status;
 
 typedef enum { DLA_F32 = 0, DLA_BF16 = 1 } dla_dtype;

@@ -59,5 +59,5 @@ def test_size_queries_and_argument_errors():
     assert lib.dla_prefill(ctypes.byref(good), None, None, None, None, ctypes.byref(cache), None,
                            None, 0, None, None) == 1
     assert lib.dla_cache_init(ctypes.byref(cache), 1, 1, 4, 32, 32, None, 0, None) == 1
-    for code in range(7):
+    for code in range(8):
         assert dla.status_string(code)
