@@ -535,7 +535,7 @@ def main():
     ap.add_argument("--workload", default="prefill_t8192")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--window", type=int, default=0)
-    ap.add_argument("--path", default="simt")
+    ap.add_argument("--path", default="auto", help="reported path; auto = tc for bf16 d=128")
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--B", type=int, default=0, help="override the batch (profiling runs)")
@@ -545,6 +545,8 @@ def main():
     wl = dict(synth.WORKLOADS[args.workload])
     if args.B:
         wl["B"] = args.B
+    if args.path == "auto":
+        args.path = "tc" if (wl["dtype"] == "bf16" and wl["d"] == 128) else "simt"
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
         if rank == 0:

@@ -26,56 +26,60 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 
-__device__ double score_fp64(const void *k, int32_t dt, size_t a, size_t b, const float *bprev,
-                             int D) {
-  // a: row of k_t; b: row of k_{t-1} in k (ignored when bprev != nullptr)
+// r = 1 - cos(a, b) with the oracle's operation order: three sums in index
+// order, no contraction, cos = dot / (sqrt(|a|^2) sqrt(|b|^2)); a zero norm
+// gives r = 1.  a, b: rows of `stride` floats in shared memory.
+__device__ double score_rows(const float *a, const float *b, int D) {
   double dot = 0.0, na = 0.0, nb = 0.0;
-  for (int c = 0; c < D; c++) {
-    double x = (double)load_in(k, dt, a + c);
-    double y = bprev ? (double)bprev[c] : (double)load_in(k, dt, b + c);
-    dot = __dadd_rn(dot, __dmul_rn(x, y));
-  }
-  for (int c = 0; c < D; c++) {
-    double x = (double)load_in(k, dt, a + c);
-    na = __dadd_rn(na, __dmul_rn(x, x));
-  }
-  for (int c = 0; c < D; c++) {
-    double y = bprev ? (double)bprev[c] : (double)load_in(k, dt, b + c);
-    nb = __dadd_rn(nb, __dmul_rn(y, y));
-  }
+  for (int c = 0; c < D; c++) dot = __dadd_rn(dot, __dmul_rn((double)a[c], (double)b[c]));
+  for (int c = 0; c < D; c++) na = __dadd_rn(na, __dmul_rn((double)a[c], (double)a[c]));
+  for (int c = 0; c < D; c++) nb = __dadd_rn(nb, __dmul_rn((double)b[c], (double)b[c]));
   if (na == 0.0 || nb == 0.0) return 1.0;
   return __dsub_rn(1.0, __ddiv_rn(dot, __dmul_rn(__dsqrt_rn(na), __dsqrt_rn(nb))));
 }
 
-// r for window-local token tl of head u (global index tg = t0 + tl).
-__device__ double score_at(const Dims &dm, const CallArgs &ca, int u, int tl, int64_t t0) {
-  if (t0 + tl == 0) return 0.0;
-  const int D = dm.D;
-  size_t row = ((size_t)u * dm.T + ca.w0 + tl) * D;
-  if (tl == 0) return score_fp64(ca.k, ca.in_dtype, row, 0, ca.cache.prev_k + (size_t)u * D, D);
-  return score_fp64(ca.k, ca.in_dtype, row, row - D, nullptr, D);
-}
+constexpr int SCORE_TOK = 128;  // tokens per block
 
-__global__ void k_score(Dims dm, Plan pl, CallArgs ca, int policy) {
+// Block of SCORE_TOK tokens; rows t-2 .. t+127 are staged (fp32, padded
+// stride D+1 so that thread t reading row t hits distinct banks).
+__global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs ca, int policy) {
+  extern __shared__ float srow[];  // [(SCORE_TOK + 2)][D + 1]
   const int u = blockIdx.y;
-  const int tl = blockIdx.x * blockDim.x + threadIdx.x;
-  __shared__ double rprev[1];
+  const int tb = blockIdx.x * SCORE_TOK;  // first window token of the block
+  const int tl = tb + threadIdx.x;
+  const int D = dm.D, ld = D + 1;
   const int64_t t0 = ca.cache.t[u];
+  __shared__ double rs[SCORE_TOK + 1];
   double r = 0.0;
   if (policy == DLA_POLICY_DYNAMIC) {
-    if (threadIdx.x == 0) {
-      const int tp = blockIdx.x * blockDim.x - 1;  // token before this block
-      rprev[0] = tp < 0 ? ca.cache.prev_r[u] : score_at(dm, ca, u, tp, t0);
+    // rows of window tokens tb-2 .. tb+127 (clipped to the window); row -1 is
+    // the cache's previous key
+    const size_t base = (size_t)u * dm.T + ca.w0;
+    for (int e = threadIdx.x; e < (SCORE_TOK + 2) * D; e += SCORE_TOK) {
+      const int rr = e / D, c = e % D;
+      const int t = tb - 2 + rr;
+      float x = 0.f;
+      if (t >= 0 && t < ca.Tw) x = load_in(ca.k, ca.in_dtype, (base + t) * D + c);
+      else if (t == -1) x = ca.cache.prev_k[(size_t)u * D + c];
+      srow[rr * ld + c] = x;
     }
-    if (tl < ca.Tw) r = score_at(dm, ca, u, tl, t0);
+    __syncthreads();
+    if (tl < ca.Tw)
+      r = (t0 + tl == 0) ? 0.0 : score_rows(srow + (threadIdx.x + 2) * ld, srow + (threadIdx.x + 1) * ld, D);
+    if (threadIdx.x == 0) {
+      const int tp = tb - 1;  // the token before the block
+      double rp;
+      if (tp < 0) rp = ca.cache.prev_r[u];
+      else rp = (t0 + tp == 0) ? 0.0 : score_rows(srow + 1 * ld, srow + 0 * ld, D);
+      rs[0] = rp;
+    }
   }
-  __shared__ double rs[256];
-  rs[threadIdx.x] = r;
+  rs[threadIdx.x + 1] = r;
   __syncthreads();
   if (tl >= ca.Tw) return;
   uint8_t b = 1;
   if (policy == DLA_POLICY_DYNAMIC) {
-    const double rp = threadIdx.x == 0 ? rprev[0] : rs[threadIdx.x - 1];
+    const double rp = rs[threadIdx.x];
     const double tau = (double)ca.tau;
     const bool join = (t0 + tl > 0) && (r < tau) && (rp < tau);
     b = join ? 0 : 1;
@@ -136,42 +140,62 @@ __global__ void k_segsum(Dims dm, Plan pl, CallArgs ca) {
       const int os = ca.cache.order[(size_t)u * dm.C + m - 1];
       z = ca.cache.z[((size_t)u * dm.C + os) * D + c];
     }
-    for (int s = s0; s < s1; s++) {
-      const double x = (double)load_in(ca.k, ca.in_dtype, ((size_t)u * dm.T + ca.w0 + s) * D + c);
-      z = __dadd_rn(z, phi64(x));
-      if ((s + 1) % dm.M == 0 && (s + 1) < ca.Tw)
-        pl.z_tile[((size_t)u * dm.tiles + (s + 1) / dm.M) * D + c] = z;
+    const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
+    for (int sb = s0; sb < s1; sb += 8) {
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; i++) x[i] = sb + i < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)(sb + i) * D) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const int s = sb + i;
+        if (s < s1) {
+          z = __dadd_rn(z, phi64((double)x[i]));
+          if ((s + 1) % dm.M == 0 && (s + 1) < ca.Tw)
+            pl.z_tile[((size_t)u * dm.tiles + (s + 1) / dm.M) * D + c] = z;
+        }
+      }
     }
     pl.z_end[((size_t)u * dm.W + j) * D + c] = z;
   }
 }
 
 // ---------------------------------------------------------------- engine ----
+// One warp per head.  The head's cache summaries (order, n, ts, version of
+// each slot, pair losses and the fp64 z of every slot) live in shared memory
+// for the whole window and are written back at its end.
+
+struct EngSmem {
+  int32_t order[128];
+  int32_t sver[128];
+  long long n[128];
+  long long ts[128];
+  double loss[128];
+  double z[1];  // [C][D], dynamic
+};
 
 struct Eng {
   const Dims *dm;
   const Plan *pl;
   const CallArgs *ca;
+  EngSmem *sm;
   int u, lane, C, D;
-  int32_t *order;
-  int64_t *n, *ts;
-  double *z, *loss;
-  int32_t *slot_ver;
   int4 *ops;
   int nops, nver, m;
   uint32_t used[4];
 
+  __device__ double *zs(int slot) const { return sm->z + (size_t)slot * D; }
+  // lane-local emit at position nops + rank; the caller advances nops
+  __device__ void put(int idx, int op, int a, int b, int c) const {
+    if (idx < dm->opsmax) ops[idx] = make_int4(op, a, b, c);
+    else set_status(ca->dev_status, DLA_ERR_INVARIANT);
+  }
   __device__ void emit(int op, int a, int b, int c) {
-    if (nops < dm->opsmax) {
-      if (lane == 0) ops[nops] = make_int4(op, a, b, c);
-    } else if (lane == 0) {
-      set_status(ca->dev_status, DLA_ERR_INVARIANT);
-    }
+    if (lane == 0) put(nops, op, a, b, c);
     nops++;
   }
   __device__ double ward(int sa, int sb) const {
-    const double na = (double)n[sa], nb = (double)n[sb];
-    const double *za = z + (size_t)sa * D, *zb = z + (size_t)sb * D;
+    const double na = (double)sm->n[sa], nb = (double)sm->n[sb];
+    const double *za = zs(sa), *zb = zs(sb);
     double s = 0.0;
     for (int c = lane; c < D; c += 32) {
       const double diff = __dsub_rn(__ddiv_rn(za[c], na), __ddiv_rn(zb[c], nb));
@@ -186,10 +210,9 @@ struct Eng {
     for (int w = 0; w < 4; w++) {
       const uint32_t freeb = ~used[w];
       if (w * 32 < C && freeb) {
-        const int bit = __ffs(freeb) - 1;
-        const int slot = w * 32 + bit;
+        const int slot = w * 32 + __ffs(freeb) - 1;
         if (slot < C) {
-          used[w] |= 1u << bit;
+          used[w] |= 1u << (slot & 31);
           return slot;
         }
       }
@@ -198,39 +221,39 @@ struct Eng {
     return 0;
   }
   __device__ void free_slot(int s) { used[s >> 5] &= ~(1u << (s & 31)); }
-  // New version of `slot` with mean phi(k) = zsrc / cnt.
-  __device__ int new_version(int slot, const double *zsrc, int64_t cnt) {
-    const int v = nver++;
-    if (v >= dm->vmax) {
-      if (lane == 0) set_status(ca->dev_status, DLA_ERR_INVARIANT);
-      return dm->vmax - 1;
-    }
-    emit(OP_SHADOW, slot, v, 0);
+  // mean phi(k) and count of version v (all lanes)
+  __device__ void write_mu(int v, const double *zsrc, long long cnt) const {
     float *mu = pl->ver_mu + ((size_t)u * dm->vmax + v) * D;
     const double dn = (double)cnt;
     for (int c = lane; c < D; c += 32) mu[c] = (float)__ddiv_rn(zsrc[c], dn);
     if (lane == 0) pl->ver_n[(size_t)u * dm->vmax + v] = (float)cnt;
-    return v;
   }
 };
 
 __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
+  extern __shared__ __align__(16) unsigned char eng_raw[];
+  EngSmem *sm = reinterpret_cast<EngSmem *>(eng_raw);
   Eng e;
   e.dm = &dm;
   e.pl = &pl;
   e.ca = &ca;
+  e.sm = sm;
   e.u = blockIdx.x;
   e.lane = threadIdx.x;
   e.C = dm.C;
   e.D = dm.D;
   const int u = e.u, lane = e.lane, C = dm.C, D = dm.D, M = dm.M;
   const dla_cache &cc = ca.cache;
-  e.order = cc.order + (size_t)u * C;
-  e.n = cc.n + (size_t)u * C;
-  e.ts = cc.ts + (size_t)u * C;
-  e.z = cc.z + (size_t)u * C * D;
-  e.loss = cc.pair_loss + (size_t)u * C;
-  e.slot_ver = pl.slot_ver + (size_t)u * C;
+  // ---- load the head's summaries ------------------------------------------
+  for (int p = lane; p < C; p += 32) {
+    sm->order[p] = cc.order[(size_t)u * C + p];
+    sm->n[p] = cc.n[(size_t)u * C + p];
+    sm->ts[p] = cc.ts[(size_t)u * C + p];
+    sm->loss[p] = cc.pair_loss[(size_t)u * C + p];
+    sm->sver[p] = -1;
+  }
+  for (int i = lane; i < C * D; i += 32) sm->z[i] = cc.z[(size_t)u * C * D + i];
+  __syncwarp();
   e.ops = pl.ops + (size_t)u * dm.opsmax;
   e.nops = 0;
   e.nver = 0;
@@ -238,11 +261,10 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   const int64_t t0 = cc.t[u];
   for (int w = 0; w < 4; w++) e.used[w] = 0;
   for (int p = 0; p < e.m; p++) {
-    const int s = e.order[p];
+    const int s = sm->order[p];
     e.used[s >> 5] |= 1u << (s & 31);
   }
-  for (int s = lane; s < C; s += 32) e.slot_ver[s] = -1;
-  __syncwarp();
+  if (e.m > 0) e.emit(OP_LOAD, sm->order[e.m - 1], 0, 0);
 
   const int nseg = pl.nseg[u];
   const int32_t *ss = pl.seg_start + (size_t)u * (dm.W + 1);
@@ -263,32 +285,47 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     const int Tend = min(T0 + M, ca.Tw);
     // ---- states present just before the tile ----------------------------
     if (e.m > 0) {
-      const int os = e.order[e.m - 1];
+      const int os = sm->order[e.m - 1];
       if (T0 > cur_from) {
         e.emit(OP_ADD, os, cur_from, T0 - cur_from);
-        if (lane == 0) e.n[os] += T0 - cur_from;
+        if (lane == 0) sm->n[os] += T0 - cur_from;
         __syncwarp();
         cur_from = T0;
       }
     }
     const int m0 = e.m;
-    for (int p = 0; p < m0; p++) {
-      const int slot = e.order[p];
-      int v;
-      if (p == m0 - 1) {  // open state: snapshot of its partial sum
-        const double *zs = c == 0 ? e.z + (size_t)slot * D
-                                  : pl.z_tile + ((size_t)u * dm.tiles + c) * D;
-        v = e.new_version(slot, zs, e.n[slot]);
-      } else {
-        v = e.slot_ver[slot];
-        if (v < 0) {
-          v = e.new_version(slot, e.z + (size_t)slot * D, e.n[slot]);
-          if (lane == 0) e.slot_ver[slot] = v;
-        }
+    for (int p0 = 0; p0 < m0; p0 += 32) {
+      const int p = p0 + lane;
+      const int slot = p < m0 ? sm->order[p] : 0;
+      const bool need = p < m0 && (p == m0 - 1 || sm->sver[slot] < 0);
+      const unsigned bal = __ballot_sync(FULL, need);
+      const int rank = __popc(bal & ((1u << lane) - 1u));
+      if (need) {
+        const int v = e.nver + rank;
+        e.put(e.nops + rank, OP_SHADOW, slot, v, 0);
+        if (p != m0 - 1) sm->sver[slot] = v;
+        tat[(size_t)c * dm.amax + p] = v;
+      } else if (p < m0) {
+        tat[(size_t)c * dm.amax + p] = sm->sver[slot];
       }
-      if (lane == 0) tat[(size_t)c * dm.amax + p] = v;
+      // means of the new versions (lanes over dimensions)
+      unsigned todo = bal;
+      while (todo) {
+        const int l = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int pv = p0 + l;
+        const int sl = sm->order[pv];
+        const int v = e.nver + __popc(bal & ((1u << l) - 1u));
+        const double *zsrc = (pv == m0 - 1 && c > 0)
+                                 ? pl.z_tile + ((size_t)u * dm.tiles + c) * D
+                                 : e.zs(sl);
+        e.write_mu(v, zsrc, sm->n[sl]);
+      }
+      e.nver += __popc(bal);
+      e.nops += __popc(bal);
       __syncwarp();
     }
+    if (e.nver > dm.vmax && lane == 0) set_status(ca.dev_status, DLA_ERR_INVARIANT);
     if (lane == 0) tm0[c] = m0;
     // ---- boundaries inside the tile --------------------------------------
     int nev = 0;
@@ -297,18 +334,19 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
       if (!(s == 0 && bflag[0] == 0)) {
         int mrg = EV_NO_MERGE;
         if (e.m > 0) {
-          const int os = e.order[e.m - 1];
+          const int os = sm->order[e.m - 1];
           if (s > cur_from) {
             e.emit(OP_ADD, os, cur_from, s - cur_from);
-            if (lane == 0) e.n[os] += s - cur_from;
+            if (lane == 0) sm->n[os] += s - cur_from;
           }
+          e.emit(OP_STORE, os, 0, 0);
           if (j >= 1)
-            for (int cc2 = lane; cc2 < D; cc2 += 32) e.z[(size_t)os * D + cc2] = zend[(size_t)(j - 1) * D + cc2];
+            for (int d2 = lane; d2 < D; d2 += 32) e.zs(os)[d2] = zend[(size_t)(j - 1) * D + d2];
           __syncwarp();
           // seal: the open state joins the sealed list (all m states sealed)
           if (e.m >= 2) {
-            const double l = e.ward(e.order[e.m - 2], e.order[e.m - 1]);
-            if (lane == 0) e.loss[e.m - 2] = l;
+            const double l = e.ward(sm->order[e.m - 2], sm->order[e.m - 1]);
+            if (lane == 0) sm->loss[e.m - 2] = l;
           }
           __syncwarp();
           if (e.m == C) {
@@ -316,7 +354,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             double best = INFINITY;
             int bi = 0x7fffffff;
             for (int p = lane; p < C - 1; p += 32) {
-              const double l = e.loss[p];
+              const double l = sm->loss[p];
               if (l < best) {
                 best = l;
                 bi = p;
@@ -331,13 +369,12 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
               }
             }
             const int is = __shfl_sync(FULL, bi, 0);
-            const int a = e.order[is], bb = e.order[is + 1];
-            for (int cc2 = lane; cc2 < D; cc2 += 32)
-              e.z[(size_t)a * D + cc2] = __dadd_rn(e.z[(size_t)a * D + cc2], e.z[(size_t)bb * D + cc2]);
+            const int a = sm->order[is], bb = sm->order[is + 1];
+            for (int d2 = lane; d2 < D; d2 += 32) e.zs(a)[d2] = __dadd_rn(e.zs(a)[d2], e.zs(bb)[d2]);
             if (lane == 0) {
-              e.n[a] += e.n[bb];
-              e.slot_ver[a] = -1;
-              e.slot_ver[bb] = -1;
+              sm->n[a] += sm->n[bb];
+              sm->sver[a] = -1;
+              sm->sver[bb] = -1;
             }
             e.emit(OP_MERGE, a, bb, 0);
             e.free_slot(bb);
@@ -346,24 +383,24 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             double lv[4];
             for (int q = 0; q < 4; q++) {
               const int p = lane + 32 * q;
-              ov[q] = (p >= is + 1 && p + 1 < C) ? e.order[p + 1] : 0;
-              lv[q] = (p >= is + 1 && p + 1 < C - 1) ? e.loss[p + 1] : 0.0;
+              ov[q] = (p >= is + 1 && p + 1 < C) ? sm->order[p + 1] : 0;
+              lv[q] = (p >= is + 1 && p + 1 < C - 1) ? sm->loss[p + 1] : 0.0;
             }
             __syncwarp();
             for (int q = 0; q < 4; q++) {
               const int p = lane + 32 * q;
-              if (p >= is + 1 && p + 1 < C) e.order[p] = ov[q];
-              if (p >= is + 1 && p + 1 < C - 1) e.loss[p] = lv[q];
+              if (p >= is + 1 && p + 1 < C) sm->order[p] = ov[q];
+              if (p >= is + 1 && p + 1 < C - 1) sm->loss[p] = lv[q];
             }
             __syncwarp();
             e.m -= 1;  // C - 1 sealed
             if (is >= 1) {
-              const double l = e.ward(e.order[is - 1], e.order[is]);
-              if (lane == 0) e.loss[is - 1] = l;
+              const double l = e.ward(sm->order[is - 1], sm->order[is]);
+              if (lane == 0) sm->loss[is - 1] = l;
             }
             if (is + 1 <= e.m - 1) {
-              const double l = e.ward(e.order[is], e.order[is + 1]);
-              if (lane == 0) e.loss[is] = l;
+              const double l = e.ward(sm->order[is], sm->order[is + 1]);
+              if (lane == 0) sm->loss[is] = l;
             }
             __syncwarp();
             mrg = is;
@@ -383,12 +420,12 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         // open a new state at s
         const int slot = e.alloc_slot();
         e.emit(OP_ZERO, slot, 0, 0);
-        for (int cc2 = lane; cc2 < D; cc2 += 32) e.z[(size_t)slot * D + cc2] = 0.0;
+        for (int d2 = lane; d2 < D; d2 += 32) e.zs(slot)[d2] = 0.0;
         if (lane == 0) {
-          e.n[slot] = 0;
-          e.ts[slot] = t0 + s;
-          e.order[e.m] = slot;
-          e.slot_ver[slot] = -1;
+          sm->n[slot] = 0;
+          sm->ts[slot] = t0 + s;
+          sm->order[e.m] = slot;
+          sm->sver[slot] = -1;
           toff[(size_t)c * M + nev] = s - T0;
           tmrg[(size_t)c * M + nev] = mrg;
         }
@@ -403,13 +440,22 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   }
   // ---- window end -------------------------------------------------------
   if (e.m > 0) {
-    const int os = e.order[e.m - 1];
+    const int os = sm->order[e.m - 1];
     if (ca.Tw > cur_from) {
       e.emit(OP_ADD, os, cur_from, ca.Tw - cur_from);
-      if (lane == 0) e.n[os] += ca.Tw - cur_from;
+      if (lane == 0) sm->n[os] += ca.Tw - cur_from;
     }
-    for (int cc2 = lane; cc2 < D; cc2 += 32) e.z[(size_t)os * D + cc2] = zend[(size_t)(nseg - 1) * D + cc2];
+    e.emit(OP_STORE, os, 0, 0);
+    for (int d2 = lane; d2 < D; d2 += 32) e.zs(os)[d2] = zend[(size_t)(nseg - 1) * D + d2];
   }
+  __syncwarp();
+  for (int p = lane; p < C; p += 32) {
+    cc.order[(size_t)u * C + p] = sm->order[p];
+    cc.n[(size_t)u * C + p] = sm->n[p];
+    cc.ts[(size_t)u * C + p] = sm->ts[p];
+    cc.pair_loss[(size_t)u * C + p] = sm->loss[p];
+  }
+  for (int i = lane; i < C * D; i += 32) cc.z[(size_t)u * C * D + i] = sm->z[i];
   if (lane == 0) {
     cc.m[u] = e.m;
     cc.t[u] = t0 + ca.Tw;
@@ -418,15 +464,18 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     if (tracing) ca.trace.merge_count[u] = mcount;
   }
   const size_t krow = ((size_t)u * dm.T + ca.w0 + ca.Tw - 1) * D;
-  for (int cc2 = lane; cc2 < D; cc2 += 32) cc.prev_k[(size_t)u * D + cc2] = load_in(ca.k, ca.in_dtype, krow + cc2);
+  for (int d2 = lane; d2 < D; d2 += 32) cc.prev_k[(size_t)u * D + d2] = load_in(ca.k, ca.in_dtype, krow + d2);
 }
 
 }  // namespace
 
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
                          cudaStream_t s) {
-  dim3 g((ca.Tw + 255) / 256, dm.heads);
-  k_score<<<g, 256, 0, s>>>(dm, pl, ca, policy);
+  const size_t sb = sizeof(float) * (SCORE_TOK + 2) * (dm.D + 1);
+  cudaError_t e = cudaFuncSetAttribute(k_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+  if (e != cudaSuccess) return e;
+  dim3 g((ca.Tw + SCORE_TOK - 1) / SCORE_TOK, dm.heads);
+  k_score<<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
   return cudaGetLastError();
 }
 
@@ -442,7 +491,10 @@ cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
 }
 
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  k_engine<<<dm.heads, 32, 0, s>>>(dm, pl, ca);
+  const size_t sb = sizeof(EngSmem) + sizeof(double) * ((size_t)dm.C * dm.D - 1);
+  cudaError_t e = cudaFuncSetAttribute(k_engine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+  if (e != cudaSuccess) return e;
+  k_engine<<<dm.heads, 32, sb, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }
 

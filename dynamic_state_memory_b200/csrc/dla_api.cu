@@ -65,7 +65,7 @@ Dims make_dims(const dla_config &cfg, int policy) {
   dm.amax = dm.C;
   const int per_tile = dm.C < 2 * dm.M + 1 ? dm.C : 2 * dm.M + 1;
   dm.vmax = dm.C + dm.tiles * per_tile;
-  dm.opsmax = 3 * W + dm.tiles + 1 + dm.vmax + 8;
+  dm.opsmax = 4 * W + dm.tiles + 2 + dm.vmax + 8;
   dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
   return dm;
 }

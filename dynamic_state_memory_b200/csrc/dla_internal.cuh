@@ -18,7 +18,18 @@
 
 namespace dla {
 
-enum OpCode : int32_t { OP_ZERO = 0, OP_ADD = 1, OP_MERGE = 2, OP_SHADOW = 3 };
+// Ops of the state materializer.  The open state is kept in registers: ZERO
+// or LOAD makes `slot` the register-resident open state, ADD accumulates
+// tokens into it, STORE writes it back to its slot; MERGE and SHADOW of a
+// sealed slot work on memory, SHADOW of the open slot reads the registers.
+enum OpCode : int32_t {
+  OP_ZERO = 0,
+  OP_ADD = 1,
+  OP_MERGE = 2,
+  OP_SHADOW = 3,
+  OP_LOAD = 4,
+  OP_STORE = 5
+};
 
 // Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
 // pair at that time-order position, <= -2 merge the two newest sealed states

@@ -22,24 +22,68 @@ constexpr int TOK = 32;  // tokens staged per ADD step
 template <int D, int R, bool BF16VER>
 __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallArgs ca) {
   constexpr int PER = R * D / THREADS;  // consecutive elements of one row per thread
-  static_assert(R * D % THREADS == 0 && D % PER == 0, "row block must split evenly");
+  static_assert(R * D % THREADS == 0 && D % PER == 0 && PER % 4 == 0, "row block must split evenly");
+  constexpr int KPT = TOK * D / THREADS;  // k values staged per thread per chunk
+  constexpr int VPT = (TOK * R + THREADS - 1) / THREADS;
   const int u = blockIdx.y;
   const int r0 = blockIdx.x * R;
   const int tid = threadIdx.x;
-  const int rr = (tid * PER) / D;       // row inside the block
-  const int c0 = (tid * PER) % D;       // first column
-  __shared__ float s_phik[TOK][D];
-  __shared__ float s_v[TOK][R];
+  const int rr = (tid * PER) / D;  // row inside the block
+  const int c0 = (tid * PER) % D;  // first column
+  __shared__ float s_phik[2][TOK][D];
+  __shared__ float s_v[2][TOK][R];
+  constexpr int OPBUF = 512;
+  __shared__ int4 s_ops[OPBUF];
   const int4 *ops = pl.ops + (size_t)u * dm.opsmax;
   const int nops = pl.nops[u];
   float *Sbase = ca.cache.S + (size_t)u * dm.C * D * D;
   const size_t my = (size_t)(r0 + rr) * D + c0;  // element offset inside a slot
+  float open[PER];
+  int open_slot = -1;
+#pragma unroll
+  for (int i = 0; i < PER; i++) open[i] = 0.f;
+  auto shadow = [&](int v, const float *src) {
+    if constexpr (BF16VER) {
+      uint8_t *Vd = static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D * 2;
+#pragma unroll
+      for (int i = 0; i < PER; i += 8)
+        *reinterpret_cast<uint4 *>(Vd + tc::sw128_offset(r0 + rr, c0 + i, D)) =
+            make_uint4(tc::pack_bf16(src[i], src[i + 1]), tc::pack_bf16(src[i + 2], src[i + 3]),
+                       tc::pack_bf16(src[i + 4], src[i + 5]), tc::pack_bf16(src[i + 6], src[i + 7]));
+    } else {
+      float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D + my;
+#pragma unroll
+      for (int i = 0; i < PER; i += 4)
+        *reinterpret_cast<float4 *>(Vd + i) = make_float4(src[i], src[i + 1], src[i + 2], src[i + 3]);
+    }
+  };
   for (int oi = 0; oi < nops; oi++) {
-    const int4 op = ops[oi];
+    if ((oi % OPBUF) == 0) {  // stage the next ops in shared memory
+      __syncthreads();
+      for (int i = tid; i < OPBUF && oi + i < nops; i += THREADS) s_ops[i] = ops[oi + i];
+      __syncthreads();
+    }
+    const int4 op = s_ops[oi % OPBUF];
     float *Sa = Sbase + (size_t)op.y * D * D + my;
     if (op.x == OP_ZERO) {
+      open_slot = op.y;
 #pragma unroll
-      for (int i = 0; i < PER; i += 4) *reinterpret_cast<float4 *>(Sa + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < PER; i++) open[i] = 0.f;
+    } else if (op.x == OP_LOAD) {
+      open_slot = op.y;
+#pragma unroll
+      for (int i = 0; i < PER; i += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(Sa + i);
+        open[i] = x.x;
+        open[i + 1] = x.y;
+        open[i + 2] = x.z;
+        open[i + 3] = x.w;
+      }
+    } else if (op.x == OP_STORE) {
+#pragma unroll
+      for (int i = 0; i < PER; i += 4)
+        *reinterpret_cast<float4 *>(Sa + i) = make_float4(open[i], open[i + 1], open[i + 2], open[i + 3]);
+      open_slot = -1;
     } else if (op.x == OP_MERGE) {
       const float *Sb = Sbase + (size_t)op.z * D * D + my;
 #pragma unroll
@@ -53,44 +97,60 @@ __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallA
         *reinterpret_cast<float4 *>(Sa + i) = a;
       }
     } else if (op.x == OP_SHADOW) {
-      if constexpr (BF16VER) {
-        // bf16 version in the UMMA K-major 128-byte-swizzle layout (rows d_v)
-        uint8_t *Vd = static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + op.z) * D * D * 2;
-        uint32_t w[PER / 2];
-#pragma unroll
-        for (int i = 0; i < PER; i += 2) w[i / 2] = tc::pack_bf16(Sa[i], Sa[i + 1]);
-        static_assert(!BF16VER || PER == 8, "one 16-byte chunk per thread");
-        *reinterpret_cast<uint4 *>(Vd + tc::sw128_offset(r0 + rr, c0, D)) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (op.y == open_slot) {
+        shadow(op.z, open);
       } else {
-        float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + op.z) * D * D + my;
+        float tmp[PER];
 #pragma unroll
-        for (int i = 0; i < PER; i += 4) *reinterpret_cast<float4 *>(Vd + i) = *reinterpret_cast<const float4 *>(Sa + i);
+        for (int i = 0; i < PER; i += 4) {
+          const float4 x = *reinterpret_cast<const float4 *>(Sa + i);
+          tmp[i] = x.x;
+          tmp[i + 1] = x.y;
+          tmp[i + 2] = x.z;
+          tmp[i + 3] = x.w;
+        }
+        shadow(op.z, tmp);
       }
-    } else {  // OP_ADD
-      float acc[PER];
-#pragma unroll
-      for (int i = 0; i < PER; i++) acc[i] = Sa[i];
+    } else {  // OP_ADD: tokens [op.z, op.z + op.w) of the window into the open state
       const size_t row0 = (size_t)u * dm.T + ca.w0 + op.z;
-      for (int s0 = 0; s0 < op.w; s0 += TOK) {
-        const int nt = min(TOK, op.w - s0);
-        __syncthreads();
-        for (int e = tid; e < nt * D; e += THREADS) {
-          const int s = e / D, c = e % D;
-          s_phik[s][c] = phi32(load_in(ca.k, ca.in_dtype, (row0 + s0 + s) * D + c));
-        }
-        for (int e = tid; e < nt * R; e += THREADS) {
-          const int s = e / R, r = e % R;
-          s_v[s][r] = load_in(ca.v, ca.in_dtype, (row0 + s0 + s) * D + r0 + r);
-        }
-        __syncthreads();
-        for (int s = 0; s < nt; s++) {
-          const float vv = s_v[s][rr];
+      const int nchunk = (op.w + TOK - 1) / TOK;
+      float kr[KPT], vr[VPT];
+      auto fetch = [&](int ch) {
+        const int nt = min(TOK, op.w - ch * TOK);
 #pragma unroll
-          for (int i = 0; i < PER; i++) acc[i] = fmaf(vv, s_phik[s][c0 + i], acc[i]);
+        for (int i = 0; i < KPT; i++) {
+          const int e = tid + THREADS * i, s = e / D, c = e % D;
+          kr[i] = s < nt ? load_in(ca.k, ca.in_dtype, (row0 + ch * TOK + s) * D + c) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; i++) {
+          const int e = tid + THREADS * i, s = e / R, r = e % R;
+          vr[i] = (e < TOK * R && s < nt) ? load_in(ca.v, ca.in_dtype, (row0 + ch * TOK + s) * D + r0 + r) : 0.f;
+        }
+      };
+      fetch(0);
+      for (int ch = 0; ch < nchunk; ch++) {
+        const int buf = ch & 1;
+#pragma unroll
+        for (int i = 0; i < KPT; i++) {
+          const int e = tid + THREADS * i;
+          s_phik[buf][e / D][e % D] = phi32(kr[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; i++) {
+          const int e = tid + THREADS * i;
+          if (e < TOK * R) s_v[buf][e / R][e % R] = vr[i];
+        }
+        __syncthreads();
+        if (ch + 1 < nchunk) fetch(ch + 1);
+        const int nt = min(TOK, op.w - ch * TOK);
+        for (int s = 0; s < nt; s++) {
+          const float vv = s_v[buf][s][rr];
+#pragma unroll
+          for (int i = 0; i < PER; i++) open[i] = fmaf(vv, s_phik[buf][s][c0 + i], open[i]);
         }
       }
-#pragma unroll
-      for (int i = 0; i < PER; i++) Sa[i] = acc[i];
+      __syncthreads();
     }
   }
 }

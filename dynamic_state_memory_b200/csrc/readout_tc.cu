@@ -75,6 +75,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ---- setup: TMEM, barriers, tile metadata ------------------------------
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
+  {
+    const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
+    for (int a = tid; a < m0; a += THREADS) {
+      const int at = atoms[a];
+      sm.atom[a] = at;
+      sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + at];
+    }
+  }
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
     mbar_init(&sm.bar_mma, 1);
@@ -88,18 +97,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     fence_mbar_init();
     sm.abort = 0;
-    const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
+  }
+  if (warp == 2 && lane == 0) {
+    // in-tile pieces and the state partition of each epoch
     const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
     const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
     const int32_t *evm = pl.tile_ev_mrg + ((size_t)u * dm.tiles + c) * M;
-    const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
     const int len = min(M, ca.Tw - T0);
     sm.m0 = m0;
     sm.len = len;
-    for (int a = 0; a < m0; a++) {
-      sm.atom[a] = atoms[a];
-      sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + atoms[a]];
-    }
     const bool cont = !(nev > 0 && evo[0] == 0);
     int np = 0;
     if (cont) sm.pst[np++] = 0;
@@ -149,7 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  const int m0 = sm.m0, np = sm.np, len = sm.len;
+  const int np = sm.np, len = sm.len;
 
   // ---- loads --------------------------------------------------------------
   if (tid == 0) {
