@@ -14,6 +14,8 @@
 //   loads, applies the merge / open-state update in registers, writes back the
 //   changed slots and accumulates o = sum_i lambda_i S_i phi(q).  Each CTA owns
 //   32 rows of d_v of one stream, so o needs no cross-CTA reduction.
+#include <atomic>
+
 #include "dla_internal.cuh"
 
 namespace dla {
@@ -374,5 +376,37 @@ cudaError_t launch_decode_stream(const dla_cache &cc, int32_t dt, const void *q,
   }
   return cudaGetLastError();
 }
+
+// ---- decode step without caller-provided scratch ---------------------------
+// For callers that cannot allocate device memory themselves (see
+// dla_decode_step_static in dla.h).  The scratch is one file-scope device
+// array shared by every call on a device; the host resolves its device
+// address once per device with cudaGetSymbolAddress (the array's name is not
+// a device pointer in host code).
+namespace {
+constexpr size_t STATIC_DECODE_BYTES = (size_t)8 << 20;
+__device__ __align__(256) unsigned char g_decode_scratch[STATIC_DECODE_BYTES];
+constexpr int MAX_DEVICES = 64;
+std::atomic<void *> g_scratch_addr[MAX_DEVICES];
+
+cudaError_t static_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  void *p = g_scratch_addr[dev].load();
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev].store(p);
+  }
+  *out = p;
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t static_decode_max_bytes() { return STATIC_DECODE_BYTES; }
+
+cudaError_t static_decode_scratch(void **out) { return static_scratch(out); }
 
 }  // namespace dla

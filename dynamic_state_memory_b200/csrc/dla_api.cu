@@ -268,6 +268,27 @@ dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype, 
   return DLA_OK;
 }
 
+dla_status dla_decode_step_static(const dla_cache *cache, float tau, int32_t in_dtype,
+                                  const void *q, const void *k, const void *v, void *o,
+                                  uint8_t *boundary, int32_t *merge_i, int32_t *dev_status,
+                                  void *stream) {
+  if (!cache || !q || !k || !v || !o) return DLA_ERR_INVALID_ARG;
+  if (in_dtype != DLA_F32 && in_dtype != DLA_BF16) return DLA_ERR_INVALID_ARG;
+  if (!cache->S || !cache->z || !cache->order || !cache->m) return DLA_ERR_INVALID_ARG;
+  const size_t need = dla_decode_workspace_bytes(cache->N, cache->H, cache->C, cache->d_k,
+                                                 cache->d_v);
+  if (need == 0) return DLA_ERR_UNSUPPORTED;
+  if (need > static_decode_max_bytes()) return DLA_ERR_WORKSPACE;
+  void *ws = nullptr;
+  if (static_decode_scratch(&ws) != cudaSuccess) return DLA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_decode_decide(*cache, tau, in_dtype, q, k, ws, boundary, merge_i, dev_status, s) !=
+      cudaSuccess)
+    return DLA_ERR_CUDA;
+  if (launch_decode_stream(*cache, in_dtype, q, k, v, o, ws, s) != cudaSuccess) return DLA_ERR_CUDA;
+  return DLA_OK;
+}
+
 dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,
                                     const void *v, void *o, void *ws, size_t ws_bytes,
                                     int32_t *dev_status, void *stream) {

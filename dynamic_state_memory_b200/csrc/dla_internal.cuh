@@ -125,6 +125,8 @@ cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, con
 cudaError_t launch_decode_stream(const dla_cache &cc, int32_t dt, const void *q, const void *k,
                                  const void *v, void *o, void *ws, cudaStream_t s);
 size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C);
+size_t static_decode_max_bytes();
+cudaError_t static_decode_scratch(void **out);
 
 // Records a dla_profile event pair around one launch.
 struct ProfScope {

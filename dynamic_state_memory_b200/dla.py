@@ -73,13 +73,16 @@ _lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
 _lib.dla_decode_step.restype = c_i32
 _lib.dla_decode_step.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                  c_vp, c_size, c_vp, c_vp, _P(dla_profile)]
+_lib.dla_decode_step_static.restype = c_i32
+_lib.dla_decode_step_static.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                        c_vp, c_vp, c_vp]
 _lib.dla_fixed_policy_prefill.restype = c_i32
 _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, c_vp, c_size,
                                           c_vp, c_vp]
 
 EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
            "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
-           "dla_fixed_policy_prefill"]
+           "dla_decode_step_static", "dla_fixed_policy_prefill"]
 
 
 def status_string(code: int) -> str:
@@ -145,6 +148,14 @@ def dla_decode_step(cache, tau, in_dtype, q, k, v, o, boundary, merge_i, ws, dev
                                 _stream(stream),
                                 None if profile is None else ctypes.byref(profile)),
            "dla_decode_step")
+
+
+def dla_decode_step_static(cache, tau, in_dtype, q, k, v, o, boundary, merge_i, dev_status,
+                           stream=None):
+    _check(_lib.dla_decode_step_static(ctypes.byref(cache), float(tau), int(in_dtype), _ptr(q),
+                                       _ptr(k), _ptr(v), _ptr(o), _ptr(boundary), _ptr(merge_i),
+                                       _ptr(dev_status), _stream(stream)),
+           "dla_decode_step_static")
 
 
 def dla_fixed_policy_prefill(cfg, q, k, v, o, ws, dev_status, stream=None):

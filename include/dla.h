@@ -161,6 +161,27 @@ dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype,
                            uint8_t *boundary, int32_t *merge_i, void *ws, size_t ws_bytes,
                            int32_t *dev_status, void *stream, dla_profile *profile);
 
+/* dla_decode_step for callers that cannot allocate device memory: runtimes
+ * that own a fixed device-memory budget, plug-ins that run inside another
+ * engine's memory pool, or code paths where an allocation call is not
+ * allowed.  Same arguments and results as dla_decode_step minus the
+ * workspace: its scratch is a library-owned static device array of 8 MiB
+ * (DLA_STATIC_DECODE_MAX_BYTES) that every GPU loading the library keeps until
+ * the process exits.  It accepts caches whose dla_decode_workspace_bytes() is
+ * at most that size (about 30,000 streams at C = 64) and returns
+ * DLA_ERR_WORKSPACE for larger ones.  It allocates nothing.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All
+ * calls share the one array and it keeps the last call's contents (every call
+ * rewrites what it reads, so nothing needs clearing); calls that overlap on
+ * the GPU, from any stream or thread, race on it, so serialise them.  The
+ * pages describing the method have no counterpart of this entry point. */
+#define DLA_STATIC_DECODE_MAX_BYTES ((size_t)8 << 20)
+dla_status dla_decode_step_static(const dla_cache *cache, float tau, int32_t in_dtype,
+                                  const void *q, const void *k, const void *v, void *o,
+                                  uint8_t *boundary, int32_t *merge_i, int32_t *dev_status,
+                                  void *stream);
+
 /* The Log-Linear-style fixed policy through the same engine (Chlience
  * section 2 and section 5.4): token t reads the Fenwick blocks of [0, t-1]
  * (one per set bit of t) plus {t}, with the same softmax over block means.
