@@ -91,6 +91,42 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.slot_ver = cv.take<int32_t>(h * dm.C);
 }
 
+// Fixed Fenwick policy: one pass over the call (no windows); versions are the
+// nodes of a tree over whole tiles.
+Dims make_dims_fenwick(const dla_config &cfg) {
+  Dims dm{};
+  const bool tc = use_tc(cfg);
+  dm.heads = cfg.B * cfg.H;
+  dm.T = cfg.T;
+  dm.M = tc ? tc_tile_rows() : simt_tile_rows();
+  dm.D = cfg.d_k;
+  dm.C = 32;
+  dm.tiles = (cfg.T + dm.M - 1) / dm.M;
+  if (dm.tiles < 1) dm.tiles = 1;
+  dm.W = dm.tiles * dm.M;
+  dm.amax = 32;
+  int nodes = 1, levels = 1;
+  fen_tree_shape(cfg.T > 0 ? cfg.T : 1, dm.M, &nodes, &levels);
+  dm.vmax = nodes;
+  dm.opsmax = 0;
+  dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
+  return dm;
+}
+
+void carve_fenwick(Carver &cv, const Dims &dm, Plan &pl, float **treeS, float **treeZ) {
+  const size_t h = dm.heads;
+  pl.tile_m0 = cv.take<int32_t>(h * dm.tiles);
+  pl.tile_atoms = cv.take<int32_t>(h * dm.tiles * dm.amax);
+  pl.tile_nev = cv.take<int32_t>(h * dm.tiles);
+  pl.tile_ev_off = cv.take<int32_t>(h * dm.tiles * dm.M);
+  pl.tile_ev_mrg = cv.take<int32_t>(h * dm.tiles * dm.M);
+  pl.ver_mu = cv.take<float>(h * dm.vmax * dm.D);
+  pl.ver_n = cv.take<float>(h * dm.vmax);
+  pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
+  *treeS = cv.take<float>(h * dm.vmax * (size_t)dm.D * dm.D);
+  *treeZ = cv.take<float>(h * dm.vmax * (size_t)dm.D);
+}
+
 bool cfg_ok(const dla_config *cfg, int policy) {
   if (!cfg) return false;
   if (cfg->B <= 0 || cfg->H <= 0 || cfg->T < 0) return false;
@@ -164,6 +200,15 @@ dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int
 
 size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
   if (!cfg_ok(cfg, policy) || shape_ok(cfg, policy) != DLA_OK) return 0;
+  if (policy == DLA_POLICY_FENWICK) {
+    const Dims dm = make_dims_fenwick(*cfg);
+    Plan pl{};
+    float *a, *b;
+    Carver cv{nullptr};
+    carve_fenwick(cv, dm, pl, &a, &b);
+    return cv.off;
+  }
+  if (policy != DLA_POLICY_DYNAMIC) return 0;
   const Dims dm = make_dims(*cfg, policy);
   Plan pl{};
   Carver cv{nullptr};
@@ -292,16 +337,44 @@ dla_status dla_decode_step_static(const dla_cache *cache, float tau, int32_t in_
 dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,
                                     const void *v, void *o, void *ws, size_t ws_bytes,
                                     int32_t *dev_status, void *stream) {
-  (void)cfg;
-  (void)q;
-  (void)k;
-  (void)v;
-  (void)o;
-  (void)ws;
-  (void)ws_bytes;
-  (void)dev_status;
-  (void)stream;
-  return DLA_ERR_UNSUPPORTED;
+  if (!cfg_ok(cfg, DLA_POLICY_FENWICK)) return DLA_ERR_INVALID_ARG;
+  const dla_status sh = shape_ok(cfg, DLA_POLICY_FENWICK);
+  if (sh != DLA_OK) return sh;
+  if (cfg->T == 0) return DLA_OK;
+  if (!q || !k || !v || !o || !ws) return DLA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  const bool tc = use_tc(*cfg);
+  if (tc && (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
+             reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16))
+    return DLA_ERR_INVALID_ARG;
+  const Dims dm = make_dims_fenwick(*cfg);
+  Plan pl{};
+  float *treeS = nullptr, *treeZ = nullptr;
+  Carver cv{static_cast<char *>(ws)};
+  carve_fenwick(cv, dm, pl, &treeS, &treeZ);
+  if (cv.off > ws_bytes) return DLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CallArgs ca{};
+  ca.q = q;
+  ca.k = k;
+  ca.v = v;
+  ca.o = o;
+  ca.in_dtype = cfg->in_dtype;
+  ca.tau = cfg->tau;
+  ca.w0 = 0;
+  ca.Tw = cfg->T;
+  ca.dev_status = dev_status;
+  memset(&ca.trace, 0, sizeof ca.trace);
+  dla_profile *pf = cfg->profile;
+  cudaError_t e;
+  { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, s); }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  {
+    ProfScope ps(pf, DLA_K_READOUT, s);
+    e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
+  }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  return DLA_OK;
 }
 
 }  // extern "C"

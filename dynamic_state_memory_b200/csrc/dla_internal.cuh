@@ -117,6 +117,9 @@ cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s, bool bf16_versions);
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+void fen_tree_shape(int T, int M, int *nodes, int *levels);
+cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
+                           float *treeZ, bool bf16, cudaStream_t s);
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s);
 cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,

@@ -1,0 +1,204 @@
+// fenwick.cu -- plan and states of the fixed Fenwick-bucket policy
+// (Dynamic Linear Attention | Chlience Paper Archive, section 2 and section
+// 5.4: Log-Linear Attention keeps O(log T) buckets; token t reads one block of
+// size 2^b of [0, t-1] per set bit b of t, plus {t}).
+//
+// The structure does not depend on the data, so it is planned in parallel:
+//   - a readout tile starts at T0 = c * M (M a power of two), so the blocks of
+//     [0, T0 - 1] are whole-tile dyadic ranges: one tree node per set bit of c;
+//   - k_fen_leaves: per tile, the state sum S = sum v phi(k)^T, z = sum phi(k)
+//     (leaves of the tree);
+//   - k_fen_level: node = left child + right child, level by level;
+//   every node is also written as a frozen version (fp32 or the bf16 UMMA
+//   layout) with its mean phi(k) and count;
+//   - k_fen_plan: per tile, the atoms (tree nodes, oldest first) and the
+//     in-tile events: every token is a boundary, and at offset o >= 1 the
+//     binary-counter carry merges the two newest blocks (trailing ones of
+//     o - 1) times; those blocks are always in-tile pieces.
+// The readout kernels are the same as for the DLA policy.
+#include "dla_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace dla {
+namespace {
+
+constexpr int THREADS = 256;
+
+struct FenTree {
+  float *S;    // [heads][nodes][D][D] fp32
+  float *z;    // [heads][nodes][D]
+  int32_t nodes;
+  int32_t levels;       // leaves are level 0
+  int32_t off[24];      // first node of each level
+};
+
+// node id of (level, index)
+__device__ __forceinline__ int node_id(const FenTree &tr, int level, int index) {
+  return tr.off[level] + index;
+}
+
+template <int D>
+__device__ void write_version(const Dims &dm, const Plan &pl, int u, int v, const float *S,
+                              const float *z, float n, bool bf16) {
+  // S: fp32 [D][D] in global memory; all threads of the block
+  if (bf16) {
+    uint8_t *Vd = static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D * 2;
+    for (int ch = threadIdx.x; ch < D * D / 8; ch += THREADS) {
+      const int r = (ch * 8) / D, c0 = (ch * 8) % D;
+      const float *src = S + (size_t)r * D + c0;
+      *reinterpret_cast<uint4 *>(Vd + tc::sw128_offset(r, c0, D)) =
+          make_uint4(tc::pack_bf16(src[0], src[1]), tc::pack_bf16(src[2], src[3]),
+                     tc::pack_bf16(src[4], src[5]), tc::pack_bf16(src[6], src[7]));
+    }
+  } else {
+    float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D;
+    for (int e = threadIdx.x; e < D * D; e += THREADS) Vd[e] = S[e];
+  }
+  for (int c = threadIdx.x; c < D; c += THREADS) pl.ver_mu[((size_t)u * dm.vmax + v) * D + c] = z[c] / n;
+  if (threadIdx.x == 0) pl.ver_n[(size_t)u * dm.vmax + v] = n;
+}
+
+// Leaves: per (head, tile) the tile's full state sum (only tiles that are
+// blocks of some later tile start are needed, i.e. tiles c < ntiles - 1).
+template <int D>
+__global__ void __launch_bounds__(THREADS) k_fen_leaves(Dims dm, Plan pl, CallArgs ca, FenTree tr,
+                                                        int ntiles, bool bf16) {
+  constexpr int PER = D * D / THREADS;
+  const int u = blockIdx.y, c = blockIdx.x;
+  if (c >= ntiles) return;
+  const int M = dm.M;
+  const int T0 = c * M, len = min(M, dm.T - T0);
+  __shared__ float s_k[32][D];
+  __shared__ float s_v[32][D];
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; i++) acc[i] = 0.f;
+  float zacc = 0.f;
+  const int e0 = threadIdx.x * PER;  // consecutive elements of one row
+  const int r = e0 / D, c0 = e0 % D;
+  const size_t row0 = (size_t)u * dm.T + T0;
+  for (int s0 = 0; s0 < len; s0 += 32) {
+    const int nt = min(32, len - s0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * D; e += THREADS) {
+      const int s = e / D, cc = e % D;
+      const bool ok = s < nt;
+      s_k[s][cc] = ok ? phi32(load_in(ca.k, ca.in_dtype, (row0 + s0 + s) * D + cc)) : 0.f;
+      s_v[s][cc] = ok ? load_in(ca.v, ca.in_dtype, (row0 + s0 + s) * D + cc) : 0.f;
+    }
+    __syncthreads();
+    for (int s = 0; s < nt; s++) {
+      const float vv = s_v[s][r];
+#pragma unroll
+      for (int i = 0; i < PER; i++) acc[i] = fmaf(vv, s_k[s][c0 + i], acc[i]);
+      if (threadIdx.x < D) zacc += s_k[s][threadIdx.x];
+    }
+  }
+  const int nid = node_id(tr, 0, c);
+  float *S = tr.S + ((size_t)u * tr.nodes + nid) * D * D;
+#pragma unroll
+  for (int i = 0; i < PER; i++) S[e0 + i] = acc[i];
+  float *z = tr.z + ((size_t)u * tr.nodes + nid) * D;
+  if (threadIdx.x < D) z[threadIdx.x] = zacc;
+  __syncthreads();
+  write_version<D>(dm, pl, u, nid, S, z, (float)len, bf16);
+}
+
+// One tree level: node (level, i) = (level-1, 2i) + (level-1, 2i+1).
+template <int D>
+__global__ void __launch_bounds__(THREADS) k_fen_level(Dims dm, Plan pl, FenTree tr, int level,
+                                                       int count, bool bf16) {
+  const int u = blockIdx.y, i = blockIdx.x;
+  if (i >= count) return;
+  const int a = node_id(tr, level - 1, 2 * i), b = node_id(tr, level - 1, 2 * i + 1);
+  const int nid = node_id(tr, level, i);
+  const float *Sa = tr.S + ((size_t)u * tr.nodes + a) * D * D;
+  const float *Sb = tr.S + ((size_t)u * tr.nodes + b) * D * D;
+  float *S = tr.S + ((size_t)u * tr.nodes + nid) * D * D;
+  for (int e = threadIdx.x * 4; e < D * D; e += THREADS * 4) {
+    const float4 x = *reinterpret_cast<const float4 *>(Sa + e);
+    const float4 y = *reinterpret_cast<const float4 *>(Sb + e);
+    *reinterpret_cast<float4 *>(S + e) = make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+  }
+  const float *za = tr.z + ((size_t)u * tr.nodes + a) * D;
+  const float *zb = tr.z + ((size_t)u * tr.nodes + b) * D;
+  float *z = tr.z + ((size_t)u * tr.nodes + nid) * D;
+  for (int c = threadIdx.x; c < D; c += THREADS) z[c] = za[c] + zb[c];
+  __syncthreads();
+  write_version<D>(dm, pl, u, nid, S, z, (float)(dm.M << level), bf16);
+}
+
+// Per (head, tile): atoms = tree nodes of the blocks of [0, T0-1], events.
+__global__ void k_fen_plan(Dims dm, Plan pl, FenTree tr, int ntiles) {
+  const int u = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= ntiles) return;
+  const int M = dm.M;
+  const int T0 = c * M, len = min(M, dm.T - T0);
+  int m0 = 0;
+  int start = 0;  // in tiles
+  for (int b = 30; b >= 0; b--) {
+    if ((c >> b) & 1) {
+      pl.tile_atoms[((size_t)u * dm.tiles + c) * dm.amax + m0] = node_id(tr, b, start >> b);
+      m0++;
+      start += 1 << b;
+    }
+  }
+  pl.tile_m0[(size_t)u * dm.tiles + c] = m0;
+  pl.tile_nev[(size_t)u * dm.tiles + c] = len;
+  for (int o = 0; o < len; o++) {
+    pl.tile_ev_off[((size_t)u * dm.tiles + c) * M + o] = o;
+    int code = EV_NO_MERGE;
+    if (o >= 1) {
+      const int ones = __ffs(~(o - 1)) - 1;  // trailing ones of o - 1
+      if (ones > 0) code = -(ones + 1);
+    }
+    pl.tile_ev_mrg[((size_t)u * dm.tiles + c) * M + o] = code;
+  }
+}
+
+template <int D>
+cudaError_t run_d(const Dims &dm, const Plan &pl, const CallArgs &ca, const FenTree &tr,
+                  int ntiles, bool bf16, cudaStream_t s) {
+  k_fen_plan<<<dim3((ntiles + 127) / 128, dm.heads), 128, 0, s>>>(dm, pl, tr, ntiles);
+  k_fen_leaves<D><<<dim3(ntiles, dm.heads), THREADS, 0, s>>>(dm, pl, ca, tr, ntiles, bf16);
+  for (int l = 1; l < tr.levels; l++) {
+    const int count = ntiles >> l;
+    if (count <= 0) break;
+    k_fen_level<D><<<dim3(count, dm.heads), THREADS, 0, s>>>(dm, pl, tr, l, count, bf16);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Tree sizes for T tokens in tiles of M: number of nodes and levels.
+void fen_tree_shape(int T, int M, int *nodes, int *levels) {
+  const int ntiles = (T + M - 1) / M;
+  int n = 0, l = 0;
+  for (int cnt = ntiles; cnt > 0 && l < 24; cnt >>= 1, l++) n += cnt;
+  *nodes = n > 0 ? n : 1;
+  *levels = l > 0 ? l : 1;
+}
+
+cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
+                           float *treeZ, bool bf16, cudaStream_t s) {
+  FenTree tr{};
+  tr.S = treeS;
+  tr.z = treeZ;
+  const int ntiles = (dm.T + dm.M - 1) / dm.M;
+  fen_tree_shape(dm.T, dm.M, &tr.nodes, &tr.levels);
+  int off = 0;
+  for (int l = 0; l < tr.levels; l++) {
+    tr.off[l] = off;
+    off += ntiles >> l;
+  }
+  switch (dm.D) {
+    case 32: return run_d<32>(dm, pl, ca, tr, ntiles, bf16, s);
+    case 64: return run_d<64>(dm, pl, ca, tr, ntiles, bf16, s);
+    case 128: return run_d<128>(dm, pl, ca, tr, ntiles, bf16, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dla

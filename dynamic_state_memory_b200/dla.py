@@ -317,3 +317,18 @@ class Decoder:
         dla_decode_step(self.cache.c, tau, _dtype_code(k), q, k, v, o, self.boundary,
                         self.merge_i, self.ws, self.status, stream, profile)
         return o
+
+
+def fixed_policy_prefill(q, k, v, *, window=0, stream=None, sync=True, profile=None):
+    """o = fixed Fenwick-bucket policy over q, k, v [B, H, T, d] (streams start at t = 0)."""
+    B, H, T, d = k.shape
+    cfg = make_config(B, H, T, d, 2, 0.0, _dtype_code(k), window, profile)
+    ws = torch.empty(max(dla_workspace_bytes(cfg, DLA_POLICY_FENWICK), 1), dtype=torch.uint8,
+                     device=k.device)
+    o = torch.empty_like(q)
+    st = torch.zeros(1, dtype=torch.int32, device=k.device)
+    dla_fixed_policy_prefill(cfg, q, k, v, o, ws, st, stream)
+    if sync:
+        torch.cuda.synchronize()
+        check_device_status(st, "dla_fixed_policy_prefill")
+    return o

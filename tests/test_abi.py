@@ -47,6 +47,8 @@ def test_size_queries_and_argument_errors():
     assert dla.dla_workspace_bytes(bad_c) == 0
     good = dla.make_config(1, 1, 16, 32, 4, 0.5, dla.DLA_F32)
     assert dla.dla_workspace_bytes(good) > 0
+    assert dla.dla_workspace_bytes(good, dla.DLA_POLICY_FENWICK) > 0
+    assert dla.dla_workspace_bytes(good, 7) == 0
     lib = dla._lib
     cache = dla.dla_cache()
     # null config / null cache -> invalid argument, synchronously
