@@ -154,6 +154,21 @@ def prefill_flops(trace_live_sum, heads_tokens, d):
     return readout, build
 
 
+def _time_steps(step, steps, warmup, stream, world, dev):
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return reduce_max(e0.elapsed_time(e1), world, dev) / steps
+
+
 def bench_prefill(args, wl, rank, world, local_rank):
     import torch
     from dynamic_state_memory_b200 import dla
@@ -194,6 +209,21 @@ def bench_prefill(args, wl, rank, world, local_rank):
     def step():
         dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
         dla.dla_prefill(cfg, q, k, v, o, cache.c, None, ws, st, stream)
+
+    fixed = args.workload.startswith("fixed")
+    if fixed:
+        # the fixed Fenwick policy is the timed path; DLA at C is reported beside it
+        dla_ms = _time_steps(step, args.steps, args.warmup, stream, world, dev)
+        dla_live = live_sum
+        fcfg = dla.make_config(B, H, T, d, C, wl["tau"], dcode, 0, prof.p)
+        fws = torch.empty(dla.dla_workspace_bytes(fcfg, dla.DLA_POLICY_FENWICK), dtype=torch.uint8,
+                          device=dev)
+        del ws
+        live_sum = int(sum(bin(t).count("1") + 1 for t in range(T))) * B * H
+        readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
+
+        def step():
+            dla.dla_fixed_policy_prefill(fcfg, q, k, v, o, fws, st, stream)
 
     for _ in range(args.warmup):
         step()
@@ -274,9 +304,16 @@ def bench_prefill(args, wl, rank, world, local_rank):
             "peak_source": peak_note, "launch_ms": round(per_launch_ms, 4),
             "launches": n_launch,
             "kernel_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()}}
-    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(wl, q_h, k_h, v_h)
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(
+        wl, q_h, k_h, v_h, policy="fenwick" if fixed else "dla")
     e2e_val = tokens / (e2e_ms * 1e-3) / 1e6
+    extra = {}
+    if fixed:
+        extra = {"dla_same_inputs": {
+            "C": C, "value": round(tokens / (dla_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
+            "ms_per_step": round(dla_ms, 4), "mean_live_states": round(dla_live / (B * H * T), 2)}}
     return {
+        **({"policy": "fenwick"} if fixed else {}), **extra,
         "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -293,7 +330,7 @@ def bench_prefill(args, wl, rank, world, local_rank):
     }
 
 
-def cpu_baseline_prefill(wl, q, k, v, target_s=15.0):
+def cpu_baseline_prefill(wl, q, k, v, target_s=15.0, policy="dla"):
     """The oracle as it stands on a bounded sample of the same workload."""
     from oracle import oracle as O
     cores = O.cores()
@@ -305,7 +342,7 @@ def cpu_baseline_prefill(wl, q, k, v, target_s=15.0):
         qs = q.reshape(B * H, T, d)[:heads, :Ts]
         ks = k.reshape(B * H, T, d)[:heads, :Ts]
         vs = v.reshape(B * H, T, d)[:heads, :Ts]
-        orc = O.Oracle(heads, d, d, wl["C"])
+        orc = O.Oracle(heads, d, d, wl["C"], policy)
         t0 = time.perf_counter()
         orc.run(ks, qs, vs, tau=wl["tau"], dtype=wl["dtype"], nthreads=cores)
         t_used = time.perf_counter() - t0
@@ -315,7 +352,8 @@ def cpu_baseline_prefill(wl, q, k, v, target_s=15.0):
     head_tokens_s = heads * Ts / t_used
     return {"value": round(head_tokens_s / H / 1e6, 6), "unit": "Mtok/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{heads} heads x first {Ts} tokens of the workload, full per-token work; "
+            "sample": f"{policy} policy, {heads} heads x first {Ts} tokens of the workload, "
+                      f"full per-token work; "
                       f"Mtok/s = head-tokens/s / H ({t_used:.1f} s)"}
 
 

@@ -26,53 +26,111 @@ namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
 
-// r = 1 - cos(a, b) with the oracle's operation order: three sums in index
-// order, no contraction, cos = dot / (sqrt(|a|^2) sqrt(|b|^2)); a zero norm
-// gives r = 1.  a, b: rows of `stride` floats in shared memory.
-__device__ double score_rows(const float *a, const float *b, int D) {
-  double dot = 0.0, na = 0.0, nb = 0.0;
-  for (int c = 0; c < D; c++) dot = __dadd_rn(dot, __dmul_rn((double)a[c], (double)b[c]));
-  for (int c = 0; c < D; c++) na = __dadd_rn(na, __dmul_rn((double)a[c], (double)a[c]));
-  for (int c = 0; c < D; c++) nb = __dadd_rn(nb, __dmul_rn((double)b[c], (double)b[c]));
+constexpr int SCORE_TOK = 128;  // tokens per block
+
+// Element c of a staged key row: rows hold the raw input (bf16 bits or fp32)
+// with a row stride of `ld` 32-bit words (one pad word keeps thread t, which
+// reads row t, on its own bank).
+template <bool BF16>
+__device__ __forceinline__ double key_at(const uint32_t *row, int c) {
+  if (BF16) {
+    const uint32_t w = row[c >> 1];
+    return (double)__uint_as_float((c & 1) ? (w & 0xFFFF0000u) : (w << 16));
+  }
+  return (double)__uint_as_float(row[c]);
+}
+
+// Each token's squared norm is summed once and reused by the next token; dot
+// and norm run as two independent chains, each in index order with explicit
+// round-to-nearest (the oracle's operation sequence):
+// cos = dot / (sqrt(|a|^2) * sqrt(|b|^2)), a zero norm gives r = 1.
+template <bool BF16>
+__device__ __forceinline__ void dot_norm(const uint32_t *a, const uint32_t *b, int D, double &dot,
+                                         double &na) {
+  dot = 0.0;
+  na = 0.0;
+  for (int c = 0; c < D; c++) {
+    const double x = key_at<BF16>(a, c), y = key_at<BF16>(b, c);
+    dot = __dadd_rn(dot, __dmul_rn(x, y));
+    na = __dadd_rn(na, __dmul_rn(x, x));
+  }
+}
+template <bool BF16>
+__device__ __forceinline__ double norm2(const uint32_t *a, int D) {
+  double n = 0.0;
+  for (int c = 0; c < D; c++) {
+    const double x = key_at<BF16>(a, c);
+    n = __dadd_rn(n, __dmul_rn(x, x));
+  }
+  return n;
+}
+__device__ __forceinline__ double score_of(double dot, double na, double nb) {
   if (na == 0.0 || nb == 0.0) return 1.0;
   return __dsub_rn(1.0, __ddiv_rn(dot, __dmul_rn(__dsqrt_rn(na), __dsqrt_rn(nb))));
 }
 
-constexpr int SCORE_TOK = 128;  // tokens per block
-
-// Block of SCORE_TOK tokens; rows t-2 .. t+127 are staged (fp32, padded
-// stride D+1 so that thread t reading row t hits distinct banks).
+// Block of SCORE_TOK tokens; key rows of window tokens tb-2 .. tb+127 are
+// staged with 16-byte loads (row tb-1 < 0 is the cache's previous key).
+template <bool BF16>
 __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs ca, int policy) {
-  extern __shared__ float srow[];  // [(SCORE_TOK + 2)][D + 1]
+  extern __shared__ uint32_t srow[];  // [(SCORE_TOK + 2)][ld]
   const int u = blockIdx.y;
-  const int tb = blockIdx.x * SCORE_TOK;  // first window token of the block
+  const int tb = blockIdx.x * SCORE_TOK;
   const int tl = tb + threadIdx.x;
-  const int D = dm.D, ld = D + 1;
+  const int D = dm.D;
+  const int wpr = BF16 ? D / 2 : D;  // 32-bit words per row
+  const int ld = wpr + 1;
   const int64_t t0 = ca.cache.t[u];
   __shared__ double rs[SCORE_TOK + 1];
+  __shared__ double nsq[SCORE_TOK + 1];  // squared norm of token tb-1+i
   double r = 0.0;
   if (policy == DLA_POLICY_DYNAMIC) {
-    // rows of window tokens tb-2 .. tb+127 (clipped to the window); row -1 is
-    // the cache's previous key
-    const size_t base = (size_t)u * dm.T + ca.w0;
-    for (int e = threadIdx.x; e < (SCORE_TOK + 2) * D; e += SCORE_TOK) {
-      const int rr = e / D, c = e % D;
+    const int vpr = wpr / 4;  // 16-byte vectors per row
+    const uint4 *kv = reinterpret_cast<const uint4 *>(
+        static_cast<const char *>(ca.k) + ((size_t)u * dm.T + ca.w0) * D * (BF16 ? 2 : 4));
+#pragma unroll 4
+    for (int e = threadIdx.x; e < (SCORE_TOK + 2) * vpr; e += SCORE_TOK) {
+      const int rr = e / vpr, cv = e % vpr;
       const int t = tb - 2 + rr;
-      float x = 0.f;
-      if (t >= 0 && t < ca.Tw) x = load_in(ca.k, ca.in_dtype, (base + t) * D + c);
-      else if (t == -1) x = ca.cache.prev_k[(size_t)u * D + c];
-      srow[rr * ld + c] = x;
+      if (t == -1) continue;  // the cache's previous key, written below
+      uint4 x = make_uint4(0, 0, 0, 0);
+      if (t >= 0 && t < ca.Tw) x = kv[(size_t)t * vpr + cv];
+      uint32_t *dst = srow + rr * ld + cv * 4;
+      dst[0] = x.x;
+      dst[1] = x.y;
+      dst[2] = x.z;
+      dst[3] = x.w;
+    }
+    if (tb == 0) {  // row 1 = token -1 = the cache's previous key (fp32 values)
+      for (int c = threadIdx.x; c < D; c += SCORE_TOK) {
+        const float f = ca.cache.prev_k[(size_t)u * D + c];
+        if (BF16) {
+          const uint32_t hb = __float_as_uint(f) >> 16;  // exact: prev_k holds a bf16 value
+          uint16_t *h = reinterpret_cast<uint16_t *>(srow + 1 * ld);
+          h[c] = (uint16_t)hb;
+        } else {
+          srow[1 * ld + c] = __float_as_uint(f);
+        }
+      }
     }
     __syncthreads();
-    if (tl < ca.Tw)
-      r = (t0 + tl == 0) ? 0.0 : score_rows(srow + (threadIdx.x + 2) * ld, srow + (threadIdx.x + 1) * ld, D);
-    if (threadIdx.x == 0) {
-      const int tp = tb - 1;  // the token before the block
-      double rp;
-      if (tp < 0) rp = ca.cache.prev_r[u];
-      else rp = (t0 + tp == 0) ? 0.0 : score_rows(srow + 1 * ld, srow + 0 * ld, D);
-      rs[0] = rp;
+    double dot = 0.0, na = 0.0;
+    if (tl < ca.Tw) dot_norm<BF16>(srow + (threadIdx.x + 2) * ld, srow + (threadIdx.x + 1) * ld, D, dot, na);
+    nsq[threadIdx.x + 1] = na;
+    if (threadIdx.x == 32) {  // a thread of the second warp: token tb-1
+      const int tp = tb - 1;
+      if (tp < 0) {
+        nsq[0] = norm2<BF16>(srow + 1 * ld, D);
+        rs[0] = ca.cache.prev_r[u];
+      } else {
+        double dp, np;
+        dot_norm<BF16>(srow + 1 * ld, srow + 0 * ld, D, dp, np);
+        nsq[0] = np;
+        rs[0] = (t0 + tp == 0) ? 0.0 : score_of(dp, np, norm2<BF16>(srow + 0 * ld, D));
+      }
     }
+    __syncthreads();
+    if (tl < ca.Tw) r = (t0 + tl == 0) ? 0.0 : score_of(dot, na, nsq[threadIdx.x]);
   }
   rs[threadIdx.x + 1] = r;
   __syncthreads();
@@ -87,6 +145,12 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
   pl.r[(size_t)u * dm.W + tl] = r;
   pl.b[(size_t)u * dm.W + tl] = b;
   if (ca.trace.boundary) ca.trace.boundary[(size_t)u * dm.T + ca.w0 + tl] = b;
+}
+
+// phi(x) in fp64 for every bf16 bit pattern (same exp as inline evaluation).
+__global__ void k_phi_table(double *tab) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < 65536) tab[i] = phi64((double)__uint_as_float((uint32_t)i << 16));
 }
 
 // Pieces of the window: seg_start = {0} and every t > 0 with b_t = 1.
@@ -140,20 +204,31 @@ __global__ void k_segsum(Dims dm, Plan pl, CallArgs ca) {
       const int os = ca.cache.order[(size_t)u * dm.C + m - 1];
       z = ca.cache.z[((size_t)u * dm.C + os) * D + c];
     }
+    // software-pipelined: the next 16 keys are in flight while these 16 are
+    // summed, in token order
     const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
-    for (int sb = s0; sb < s1; sb += 8) {
-      float x[8];
+    constexpr int CH = 16;
+    float cur[CH], nxt[CH];
 #pragma unroll
-      for (int i = 0; i < 8; i++) x[i] = sb + i < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)(sb + i) * D) : 0.f;
+    for (int i = 0; i < CH; i++) cur[i] = s0 + i < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)(s0 + i) * D) : 0.f;
+    for (int sb = s0; sb < s1; sb += CH) {
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
+      for (int i = 0; i < CH; i++) {
+        const int sn = sb + CH + i;
+        nxt[i] = sn < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)sn * D) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < CH; i++) {
         const int s = sb + i;
         if (s < s1) {
-          z = __dadd_rn(z, phi64((double)x[i]));
+          const double ph = pl.phi_tab ? pl.phi_tab[__float_as_uint(cur[i]) >> 16] : phi64((double)cur[i]);
+          z = __dadd_rn(z, ph);
           if ((s + 1) % dm.M == 0 && (s + 1) < ca.Tw)
             pl.z_tile[((size_t)u * dm.tiles + (s + 1) / dm.M) * D + c] = z;
         }
       }
+#pragma unroll
+      for (int i = 0; i < CH; i++) cur[i] = nxt[i];
     }
     pl.z_end[((size_t)u * dm.W + j) * D + c] = z;
   }
@@ -180,7 +255,7 @@ struct Eng {
   EngSmem *sm;
   int u, lane, C, D;
   int4 *ops;
-  int nops, nver, m;
+  int nops, nver, m, npieces;
   uint32_t used[4];
 
   __device__ double *zs(int slot) const { return sm->z + (size_t)slot * D; }
@@ -193,12 +268,27 @@ struct Eng {
     if (lane == 0) put(nops, op, a, b, c);
     nops++;
   }
+  // tokens [from, from + cnt) join the open state `slot`: a tensor-core piece
+  // when long enough (and the path has pieces), else SIMT rank-1 adds
+  __device__ void emit_add(int slot, int from, int cnt) {
+    if (dm->pmax > 0 && cnt >= PIECE_MIN) {
+      if (npieces >= dm->pmax && lane == 0) set_status(ca->dev_status, DLA_ERR_INVARIANT);
+      emit(OP_ADDP, slot, npieces, cnt);
+      npieces++;
+    } else {
+      emit(OP_ADD, slot, from, cnt);
+    }
+  }
+  // Ward loss with one reciprocal per state: mu = z * (1 / n) (within an ulp
+  // of z / n; merge choices agree with the oracle whenever the best and
+  // second-best losses differ by more than rounding)
   __device__ double ward(int sa, int sb) const {
     const double na = (double)sm->n[sa], nb = (double)sm->n[sb];
+    const double ia = __drcp_rn(na), ib = __drcp_rn(nb);
     const double *za = zs(sa), *zb = zs(sb);
     double s = 0.0;
     for (int c = lane; c < D; c += 32) {
-      const double diff = __dsub_rn(__ddiv_rn(za[c], na), __ddiv_rn(zb[c], nb));
+      const double diff = __dsub_rn(__dmul_rn(za[c], ia), __dmul_rn(zb[c], ib));
       s = __dadd_rn(s, __dmul_rn(diff, diff));
     }
     for (int off = 16; off; off >>= 1) s = __dadd_rn(s, __shfl_down_sync(FULL, s, off));
@@ -221,11 +311,10 @@ struct Eng {
     return 0;
   }
   __device__ void free_slot(int s) { used[s >> 5] &= ~(1u << (s & 31)); }
-  // mean phi(k) and count of version v (all lanes)
+  // phi(k) sum and count of version v (all lanes); readouts divide
   __device__ void write_mu(int v, const double *zsrc, long long cnt) const {
-    float *mu = pl->ver_mu + ((size_t)u * dm->vmax + v) * D;
-    const double dn = (double)cnt;
-    for (int c = lane; c < D; c += 32) mu[c] = (float)__ddiv_rn(zsrc[c], dn);
+    float *zv = pl->ver_z + ((size_t)u * dm->vmax + v) * D;
+    for (int c = lane; c < D; c += 32) zv[c] = (float)zsrc[c];
     if (lane == 0) pl->ver_n[(size_t)u * dm->vmax + v] = (float)cnt;
   }
 };
@@ -257,6 +346,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   e.ops = pl.ops + (size_t)u * dm.opsmax;
   e.nops = 0;
   e.nver = 0;
+  e.npieces = 0;
   e.m = cc.m[u];
   const int64_t t0 = cc.t[u];
   for (int w = 0; w < 4; w++) e.used[w] = 0;
@@ -287,12 +377,13 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     if (e.m > 0) {
       const int os = sm->order[e.m - 1];
       if (T0 > cur_from) {
-        e.emit(OP_ADD, os, cur_from, T0 - cur_from);
+        e.emit_add(os, cur_from, T0 - cur_from);
         if (lane == 0) sm->n[os] += T0 - cur_from;
         __syncwarp();
         cur_from = T0;
       }
     }
+    if (lane == 0 && dm.pmax > 0) pl.tile_pbase[(size_t)u * dm.tiles + c] = e.npieces;
     const int m0 = e.m;
     for (int p0 = 0; p0 < m0; p0 += 32) {
       const int p = p0 + lane;
@@ -336,7 +427,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         if (e.m > 0) {
           const int os = sm->order[e.m - 1];
           if (s > cur_from) {
-            e.emit(OP_ADD, os, cur_from, s - cur_from);
+            e.emit_add(os, cur_from, s - cur_from);
             if (lane == 0) sm->n[os] += s - cur_from;
           }
           e.emit(OP_STORE, os, 0, 0);
@@ -442,7 +533,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   if (e.m > 0) {
     const int os = sm->order[e.m - 1];
     if (ca.Tw > cur_from) {
-      e.emit(OP_ADD, os, cur_from, ca.Tw - cur_from);
+      e.emit_add(os, cur_from, ca.Tw - cur_from);
       if (lane == 0) sm->n[os] += ca.Tw - cur_from;
     }
     e.emit(OP_STORE, os, 0, 0);
@@ -471,11 +562,23 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
 
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
                          cudaStream_t s) {
-  const size_t sb = sizeof(float) * (SCORE_TOK + 2) * (dm.D + 1);
-  cudaError_t e = cudaFuncSetAttribute(k_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-  if (e != cudaSuccess) return e;
+  const bool bf = ca.in_dtype == DLA_BF16;
+  const size_t sb = sizeof(uint32_t) * (SCORE_TOK + 2) * ((bf ? dm.D / 2 : dm.D) + 1);
   dim3 g((ca.Tw + SCORE_TOK - 1) / SCORE_TOK, dm.heads);
-  k_score<<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
+  if (bf) {
+    cudaError_t e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    if (e != cudaSuccess) return e;
+    k_score<true><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(k_score<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    if (e != cudaSuccess) return e;
+    k_score<false><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_phi_table(double *tab, cudaStream_t s) {
+  k_phi_table<<<256, 256, 0, s>>>(tab);
   return cudaGetLastError();
 }
 

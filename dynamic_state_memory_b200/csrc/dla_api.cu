@@ -67,6 +67,7 @@ Dims make_dims(const dla_config &cfg, int policy) {
   dm.vmax = dm.C + dm.tiles * per_tile;
   dm.opsmax = 4 * W + dm.tiles + 2 + dm.vmax + 8;
   dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
+  dm.pmax = tc ? dm.tiles + W / PIECE_MIN : 0;
   return dm;
 }
 
@@ -85,10 +86,13 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.tile_nev = cv.take<int32_t>(h * dm.tiles);
   pl.tile_ev_off = cv.take<int32_t>(h * dm.tiles * dm.M);
   pl.tile_ev_mrg = cv.take<int32_t>(h * dm.tiles * dm.M);
-  pl.ver_mu = cv.take<float>(h * dm.vmax * dm.D);
+  pl.ver_z = cv.take<float>(h * dm.vmax * dm.D);
   pl.ver_n = cv.take<float>(h * dm.vmax);
   pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
   pl.slot_ver = cv.take<int32_t>(h * dm.C);
+  pl.tile_pbase = cv.take<int32_t>(h * dm.tiles);
+  pl.phi_tab = cv.take<double>(65536);
+  pl.pieces = cv.take<float>(h * (size_t)dm.pmax * dm.D * dm.D);
 }
 
 // Fixed Fenwick policy: one pass over the call (no windows); versions are the
@@ -120,7 +124,7 @@ void carve_fenwick(Carver &cv, const Dims &dm, Plan &pl, float **treeS, float **
   pl.tile_nev = cv.take<int32_t>(h * dm.tiles);
   pl.tile_ev_off = cv.take<int32_t>(h * dm.tiles * dm.M);
   pl.tile_ev_mrg = cv.take<int32_t>(h * dm.tiles * dm.M);
-  pl.ver_mu = cv.take<float>(h * dm.vmax * dm.D);
+  pl.ver_z = cv.take<float>(h * dm.vmax * dm.D);
   pl.ver_n = cv.take<float>(h * dm.vmax);
   pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
   *treeS = cv.take<float>(h * dm.vmax * (size_t)dm.D * dm.D);
@@ -231,8 +235,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
                 trace->cap < 0))
     return DLA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
-  if (use_tc(*cfg) && (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
-                       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16))
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
+      reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16)
     return DLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
   Plan pl{};
@@ -256,6 +260,11 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     memset(&ca.trace, 0, sizeof ca.trace);
   }
   ca.dev_status = dev_status;
+  if (cfg->in_dtype == DLA_BF16) {
+    if (launch_phi_table(pl.phi_tab, s) != cudaSuccess) return DLA_ERR_CUDA;
+  } else {
+    pl.phi_tab = nullptr;
+  }
   for (int w0 = 0; w0 < cfg->T; w0 += dm.W) {
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
@@ -270,6 +279,11 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_engine(dm, pl, ca, s); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     const bool tc = use_tc(*cfg);
+    if (tc) {
+      ProfScope ps(pf, DLA_K_BUILD, s);
+      e = launch_build_tc(dm, pl, ca, s);
+      if (e != cudaSuccess) return DLA_ERR_CUDA;
+    }
     { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     {

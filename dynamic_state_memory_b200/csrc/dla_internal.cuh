@@ -28,8 +28,12 @@ enum OpCode : int32_t {
   OP_MERGE = 2,
   OP_SHADOW = 3,
   OP_LOAD = 4,
-  OP_STORE = 5
+  OP_STORE = 5,
+  OP_ADDP = 6  // add the precomputed piece (tensor-core builder) op.z to the open state
 };
+
+// Pieces shorter than this stay SIMT adds in the materializer.
+constexpr int PIECE_MIN = 16;
 
 // Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
 // pair at that time-order position, <= -2 merge the two newest sealed states
@@ -48,6 +52,7 @@ struct Dims {
   int32_t vmax;    // max versions per head per window
   int32_t opsmax;  // max ops per head per window
   int32_t vbytes;  // bytes of one version's S
+  int32_t pmax;    // max tensor-core pieces per head per window (0 = none)
 };
 
 // Per-window plan, every array strided by head.
@@ -65,10 +70,13 @@ struct Plan {
   int32_t *tile_nev;   // [heads][tiles]
   int32_t *tile_ev_off;// [heads][tiles][M] boundary offset inside the tile
   int32_t *tile_ev_mrg;// [heads][tiles][M] merge code (see EV_NO_MERGE)
-  float *ver_mu;       // [heads][vmax][D] mean phi(k) of each version
+  float *ver_z;        // [heads][vmax][D] sum of phi(k) of each version (mean = z / n)
   float *ver_n;        // [heads][vmax] token count of each version
   void *ver_S;         // [heads][vmax] versions (fp32 [D][D] or bf16 tiled)
   int32_t *slot_ver;   // [heads][C] engine scratch
+  int32_t *tile_pbase; // [heads][tiles] first piece id of each tile
+  float *pieces;       // [heads][pmax][D][D] fp32 piece states
+  double *phi_tab;     // [65536] phi(x) in fp64 for every bf16 bit pattern (or null)
 };
 
 struct CallArgs {
@@ -112,11 +120,13 @@ __device__ __forceinline__ float phi32(float x) { return x > 0.0f ? x + 1.0f : e
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
                          cudaStream_t s);
 cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_phi_table(double *tab, cudaStream_t s);
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s, bool bf16_versions);
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 void fen_tree_shape(int T, int M, int *nodes, int *levels);
 cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
                            float *treeZ, bool bf16, cudaStream_t s);

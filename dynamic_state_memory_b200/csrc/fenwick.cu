@@ -54,7 +54,7 @@ __device__ void write_version(const Dims &dm, const Plan &pl, int u, int v, cons
     float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D;
     for (int e = threadIdx.x; e < D * D; e += THREADS) Vd[e] = S[e];
   }
-  for (int c = threadIdx.x; c < D; c += THREADS) pl.ver_mu[((size_t)u * dm.vmax + v) * D + c] = z[c] / n;
+  for (int c = threadIdx.x; c < D; c += THREADS) pl.ver_z[((size_t)u * dm.vmax + v) * D + c] = z[c];
   if (threadIdx.x == 0) pl.ver_n[(size_t)u * dm.vmax + v] = n;
 }
 

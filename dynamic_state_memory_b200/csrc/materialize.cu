@@ -111,6 +111,16 @@ __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallA
         }
         shadow(op.z, tmp);
       }
+    } else if (op.x == OP_ADDP) {
+      const float *pc = pl.pieces + ((size_t)u * dm.pmax + op.z) * D * D + my;
+#pragma unroll
+      for (int i = 0; i < PER; i += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(pc + i);
+        open[i] += x.x;
+        open[i + 1] += x.y;
+        open[i + 2] += x.z;
+        open[i + 3] += x.w;
+      }
     } else {  // OP_ADD: tokens [op.z, op.z + op.w) of the window into the open state
       const size_t row0 = (size_t)u * dm.T + ca.w0 + op.z;
       const int nchunk = (op.w + TOK - 1) / TOK;

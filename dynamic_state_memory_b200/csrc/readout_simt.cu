@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(THREADS) k_readout(Dims dm, Plan pl, CallArgs 
   const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * dm.M;
   const int32_t *evm = pl.tile_ev_mrg + ((size_t)u * dm.tiles + c) * dm.M;
   const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
-  const float *ver_mu = pl.ver_mu + (size_t)u * dm.vmax * D;
+  const float *ver_z = pl.ver_z + (size_t)u * dm.vmax * D;
   const float *ver_n = pl.ver_n + (size_t)u * dm.vmax;
   const float *ver_S = static_cast<const float *>(pl.ver_S) + (size_t)u * dm.vmax * D * D;
 
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(THREADS) k_readout(Dims dm, Plan pl, CallArgs 
   for (int a0 = 0; a0 < m0; a0 += M) {
     const int na = min(M, m0 - a0);
     for (int e = tid; e < na * D; e += THREADS)
-      sm.Kp[e] = ver_mu[(size_t)atoms[a0 + e / D] * D + e % D];
+      sm.Kp[e] = ver_z[(size_t)atoms[a0 + e / D] * D + e % D] / ver_n[atoms[a0 + e / D]];
     __syncthreads();
     for (int e = tid; e < na * M; e += THREADS) {
       const int al = e / M, t = e % M;

@@ -188,11 +188,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int a = e >> 4, ch = e & 15;
     uint4 x = make_uint4(0, 0, 0, 0);
     if (a < m0) {
-      const float *mu = pl.ver_mu + ((size_t)u * dm.vmax + sm.atom[a]) * D + ch * 8;
-      x.x = pack_bf16(mu[0], mu[1]);
-      x.y = pack_bf16(mu[2], mu[3]);
-      x.z = pack_bf16(mu[4], mu[5]);
-      x.w = pack_bf16(mu[6], mu[7]);
+      const float4 *zz = reinterpret_cast<const float4 *>(pl.ver_z + ((size_t)u * dm.vmax + sm.atom[a]) * D + ch * 8);
+      const float inv = 1.0f / sm.nA[a];
+      const float4 z0 = zz[0], z1 = zz[1];
+      x.x = pack_bf16(z0.x * inv, z0.y * inv);
+      x.y = pack_bf16(z0.z * inv, z0.w * inv);
+      x.z = pack_bf16(z1.x * inv, z1.y * inv);
+      x.w = pack_bf16(z1.z * inv, z1.w * inv);
     }
     *reinterpret_cast<uint4 *>(mu_buf + sw128_offset(a, ch * 8, 128)) = x;
   }
@@ -471,7 +473,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *base, int T, int heads) {
+}  // namespace
+
+// 3D tensor map {d = 128, T, heads} of a bf16 [heads][T][128] tensor, boxes of
+// 64 x 128 x 1 with the 128-byte swizzle (out-of-range rows read as zero).
+bool make_bf16_map(CUtensorMap *m, const void *base, int T, int heads) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)heads};
@@ -483,17 +489,18 @@ bool make_map(CUtensorMap *m, const void *base, int T, int heads) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-int tc_tile_rows() { return M; }
+namespace {
+constexpr int kTileRows = M;
+}
+int tc_tile_rows() { return kTileRows; }
 
 size_t readout_tc_smem() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, ca.q, dm.T, dm.heads) || !make_map(&tk, ca.k, dm.T, dm.heads) ||
-      !make_map(&tv, ca.v, dm.T, dm.heads))
+  if (!make_bf16_map(&tq, ca.q, dm.T, dm.heads) || !make_bf16_map(&tk, ca.k, dm.T, dm.heads) ||
+      !make_bf16_map(&tv, ca.v, dm.T, dm.heads))
     return cudaErrorInvalidValue;
   const size_t sb = readout_tc_smem();
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -26,6 +26,7 @@
  *     workspace or dev_status.
  *   - Layouts are row-major with the last index fastest.  q, k, v are
  *     [B][H][T][d]; o is [B][H][T][d_v] in the input dtype (fp32 accumulation).
+ *     Prefill tensors must start on a 16-byte boundary.
  */
 #ifndef DLA_H_
 #define DLA_H_
@@ -61,7 +62,8 @@ typedef enum {
   DLA_K_MATERIALIZE = 4, /* state build, merges and versions */
   DLA_K_READOUT = 5,     /* multi-state readout */
   DLA_K_DECODE_DECIDE = 6,
-  DLA_K_DECODE_STREAM = 7
+  DLA_K_DECODE_STREAM = 7,
+  DLA_K_BUILD = 8        /* tensor-core state-piece builder */
 } dla_kernel_kind;
 
 /* Optional timing hook (host memory, caller-owned).  When non-NULL, the
