@@ -186,50 +186,81 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
   if (threadIdx.x == 0) pl.nseg[u] = base;
 }
 
-// z per piece (fp64, token order) and the open state's z before each tile.
-__global__ void k_segsum(Dims dm, Plan pl, CallArgs ca) {
+// z = sum of phi(k) of every window piece, in fp64, in two levels:
+//   k_tilesum    per (head, tile): token-order sums of each run of the tile's
+//                tokens between boundaries ("part"), stored at the part's first
+//                token;
+//   k_segcombine per segment: its parts added in time order (the cache's z
+//                of a continued open state first), writing the segment's end
+//                sum and the open state's partial sum before each tile.
+// Each dependent fp64 chain is at most a tile (128 tokens) or the tiles a
+// segment spans; the association differs from a strict token-order sum by
+// rounding only (merge choices are then the same unless two Ward losses tie
+// to within rounding).
+__global__ void k_tilesum(Dims dm, Plan pl, CallArgs ca) {
+  const int u = blockIdx.y, tile = blockIdx.x;
+  const int c = threadIdx.x;  // dimension
+  const int D = dm.D, M = dm.M;
+  const int T0 = tile * M;
+  if (T0 >= ca.Tw) return;
+  const int T1 = min(T0 + M, ca.Tw);
+  const uint8_t *b = pl.b + (size_t)u * dm.W;
+  const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
+  double *zp = pl.z_part + (size_t)u * dm.W * D + c;
+  const double *__restrict__ tab = pl.phi_tab;
+  constexpr int CH = 16;
+  double z = 0.0;
+  int part = T0;
+  for (int s0 = T0; s0 < T1; s0 += CH) {
+    double ph[CH];
+#pragma unroll
+    for (int i = 0; i < CH; i++) {
+      const int s = s0 + i;
+      const float x = s < T1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)s * D) : 0.f;
+      ph[i] = tab ? __ldg(tab + (__float_as_uint(x) >> 16)) : phi64((double)x);
+    }
+#pragma unroll
+    for (int i = 0; i < CH; i++) {
+      const int s = s0 + i;
+      if (s < T1) {
+        if (s > T0 && b[s]) {
+          zp[(size_t)part * D] = z;
+          part = s;
+          z = 0.0;
+        }
+        z = __dadd_rn(z, ph[i]);
+      }
+    }
+  }
+  zp[(size_t)part * D] = z;
+}
+
+__global__ void k_segcombine(Dims dm, Plan pl, CallArgs ca) {
   const int u = blockIdx.y;
   const int c = threadIdx.x;  // dimension
-  const int D = dm.D;
+  const int D = dm.D, M = dm.M;
   const int nseg = pl.nseg[u];
   const int32_t *ss = pl.seg_start + (size_t)u * (dm.W + 1);
   const uint8_t *b = pl.b + (size_t)u * dm.W;
+  const double *zp = pl.z_part + (size_t)u * dm.W * D + c;
   for (int j = blockIdx.x; j < nseg; j += gridDim.x) {
     const int s0 = ss[j];
     const int s1 = j + 1 < nseg ? ss[j + 1] : ca.Tw;
     double z = 0.0;
     if (j == 0 && b[0] == 0) {
-      // continuation of the cache's open state: keep summing its z in order
+      // continuation of the cache's open state
       const int m = ca.cache.m[u];
       const int os = ca.cache.order[(size_t)u * dm.C + m - 1];
       z = ca.cache.z[((size_t)u * dm.C + os) * D + c];
     }
-    // software-pipelined: the next 16 keys are in flight while these 16 are
-    // summed, in token order
-    const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
-    constexpr int CH = 16;
-    float cur[CH], nxt[CH];
-#pragma unroll
-    for (int i = 0; i < CH; i++) cur[i] = s0 + i < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)(s0 + i) * D) : 0.f;
-    for (int sb = s0; sb < s1; sb += CH) {
-#pragma unroll
-      for (int i = 0; i < CH; i++) {
-        const int sn = sb + CH + i;
-        nxt[i] = sn < s1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)sn * D) : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < CH; i++) {
-        const int s = sb + i;
-        if (s < s1) {
-          const double ph = pl.phi_tab ? pl.phi_tab[__float_as_uint(cur[i]) >> 16] : phi64((double)cur[i]);
-          z = __dadd_rn(z, ph);
-          if ((s + 1) % dm.M == 0 && (s + 1) < ca.Tw)
-            pl.z_tile[((size_t)u * dm.tiles + (s + 1) / dm.M) * D + c] = z;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < CH; i++) cur[i] = nxt[i];
+    z = __dadd_rn(z, zp[(size_t)s0 * D]);
+    for (int T0 = (s0 / M + 1) * M; T0 < s1; T0 += M) {
+      pl.z_tile[((size_t)u * dm.tiles + T0 / M) * D + c] = z;
+      z = __dadd_rn(z, zp[(size_t)T0 * D]);
     }
+    // the tile start right after the segment's end (if the segment ends at a
+    // tile boundary the next tile's open state is this one, complete)
+    if (s1 % M == 0 && s1 < ca.Tw) pl.z_tile[((size_t)u * dm.tiles + s1 / M) * D + c] = z;
     pl.z_end[((size_t)u * dm.W + j) * D + c] = z;
   }
 }
@@ -311,6 +342,14 @@ struct Eng {
     return 0;
   }
   __device__ void free_slot(int s) { used[s >> 5] &= ~(1u << (s & 31)); }
+  // the same from per-lane registers (dimension lane + 32 q)
+  __device__ void write_mu_regs(int v, const double *zr, long long cnt) const {
+    float *zv = pl->ver_z + ((size_t)u * dm->vmax + v) * D;
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+      if (lane + 32 * q < D) zv[lane + 32 * q] = (float)zr[q];
+    if (lane == 0) pl->ver_n[(size_t)u * dm->vmax + v] = (float)cnt;
+  }
   // phi(k) sum and count of version v (all lanes); readouts divide
   __device__ void write_mu(int v, const double *zsrc, long long cnt) const {
     float *zv = pl->ver_z + ((size_t)u * dm->vmax + v) * D;
@@ -370,9 +409,23 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
 
   int j = 0;
   int cur_from = 0;  // first window token not yet added to the open state
+  // one step of look-ahead on global reads: the next boundary positions, the
+  // end sum of the segment sealed at the next boundary, the next tile's
+  // open-state partial sum
+  int ss_cur = nseg > 0 ? ss[0] : 0x7fffffff;
+  int ss_nxt = nseg > 1 ? ss[1] : 0x7fffffff;
+  double zprev[4] = {0.0, 0.0, 0.0, 0.0};  // end sum of segment j-1
+  double ztile[4] = {0.0, 0.0, 0.0, 0.0};  // open-state partial sum before tile c
   for (int c = 0; c < dm.tiles && c * M < ca.Tw; c++) {
     const int T0 = c * M;
     const int Tend = min(T0 + M, ca.Tw);
+    double ztile_cur[4];
+#pragma unroll
+    for (int q = 0; q < 4; q++) ztile_cur[q] = ztile[q];
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+      ztile[q] = (c + 1 < dm.tiles && (c + 1) * M < ca.Tw && lane + 32 * q < D)
+                     ? pl.z_tile[((size_t)u * dm.tiles + c + 1) * D + lane + 32 * q] : 0.0;
     // ---- states present just before the tile ----------------------------
     if (e.m > 0) {
       const int os = sm->order[e.m - 1];
@@ -407,10 +460,8 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         const int pv = p0 + l;
         const int sl = sm->order[pv];
         const int v = e.nver + __popc(bal & ((1u << l) - 1u));
-        const double *zsrc = (pv == m0 - 1 && c > 0)
-                                 ? pl.z_tile + ((size_t)u * dm.tiles + c) * D
-                                 : e.zs(sl);
-        e.write_mu(v, zsrc, sm->n[sl]);
+        if (pv == m0 - 1 && c > 0) e.write_mu_regs(v, ztile_cur, sm->n[sl]);
+        else e.write_mu(v, e.zs(sl), sm->n[sl]);
       }
       e.nver += __popc(bal);
       e.nops += __popc(bal);
@@ -420,8 +471,12 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     if (lane == 0) tm0[c] = m0;
     // ---- boundaries inside the tile --------------------------------------
     int nev = 0;
-    while (j < nseg && ss[j] < Tend) {
-      const int s = ss[j];
+    while (j < nseg && ss_cur < Tend) {
+      const int s = ss_cur;
+      const int ss_n2 = j + 2 < nseg ? ss[j + 2] : 0x7fffffff;
+      double znext[4];
+#pragma unroll
+      for (int q = 0; q < 4; q++) znext[q] = lane + 32 * q < D ? zend[(size_t)j * D + lane + 32 * q] : 0.0;
       if (!(s == 0 && bflag[0] == 0)) {
         int mrg = EV_NO_MERGE;
         if (e.m > 0) {
@@ -431,8 +486,11 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             if (lane == 0) sm->n[os] += s - cur_from;
           }
           e.emit(OP_STORE, os, 0, 0);
-          if (j >= 1)
-            for (int d2 = lane; d2 < D; d2 += 32) e.zs(os)[d2] = zend[(size_t)(j - 1) * D + d2];
+          if (j >= 1) {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+              if (lane + 32 * q < D) e.zs(os)[lane + 32 * q] = zprev[q];
+          }
           __syncwarp();
           // seal: the open state joins the sealed list (all m states sealed)
           if (e.m >= 2) {
@@ -525,6 +583,10 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         cur_from = s;
         nev++;
       }
+#pragma unroll
+      for (int q = 0; q < 4; q++) zprev[q] = znext[q];
+      ss_cur = ss_nxt;
+      ss_nxt = ss_n2;
       j++;
     }
     if (lane == 0) tnev[c] = nev;
@@ -588,8 +650,8 @@ cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, c
 }
 
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  dim3 g(64, dm.heads);
-  k_segsum<<<g, dm.D, 0, s>>>(dm, pl, ca);
+  k_tilesum<<<dim3(dm.tiles, dm.heads), dm.D, 0, s>>>(dm, pl, ca);
+  k_segcombine<<<dim3(64, dm.heads), dm.D, 0, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }
 

@@ -79,6 +79,7 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.nseg = cv.take<int32_t>(h);
   pl.z_end = cv.take<double>(h * dm.W * dm.D);
   pl.z_tile = cv.take<double>(h * dm.tiles * dm.D);
+  pl.z_part = cv.take<double>(h * dm.W * dm.D);
   pl.ops = cv.take<int4>(h * dm.opsmax);
   pl.nops = cv.take<int32_t>(h);
   pl.tile_m0 = cv.take<int32_t>(h * dm.tiles);
@@ -114,6 +115,7 @@ Dims make_dims_fenwick(const dla_config &cfg) {
   dm.vmax = nodes;
   dm.opsmax = 0;
   dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
+  dm.fenwick = 1;
   return dm;
 }
 

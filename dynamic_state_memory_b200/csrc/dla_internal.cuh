@@ -53,6 +53,7 @@ struct Dims {
   int32_t opsmax;  // max ops per head per window
   int32_t vbytes;  // bytes of one version's S
   int32_t pmax;    // max tensor-core pieces per head per window (0 = none)
+  int32_t fenwick; // 1: fixed Fenwick policy (every token a piece; closed-form epochs)
 };
 
 // Per-window plan, every array strided by head.
@@ -63,6 +64,7 @@ struct Plan {
   int32_t *nseg;       // [heads]
   double *z_end;       // [heads][W][D] phi(k) sum of each piece's state at its end
   double *z_tile;      // [heads][tiles][D] open state's phi(k) sum before each tile
+  double *z_part;      // [heads][W][D] phi(k) sum of each in-tile run, at its first token
   int4 *ops;           // [heads][opsmax]
   int32_t *nops;       // [heads]
   int32_t *tile_m0;    // [heads][tiles]

@@ -54,12 +54,6 @@ struct Smem {
 
 __device__ __forceinline__ bool bit_of(const uint32_t *b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
 
-__device__ __forceinline__ void online(float &mx, float &l, float a) {
-  const float nm = fmaxf(mx, a);
-  l = l * expf(mx - nm) + expf(a - nm);
-  mx = nm;
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
@@ -98,7 +92,37 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_mbar_init();
     sm.abort = 0;
   }
-  if (warp == 2 && lane == 0) {
+  if (dm.fenwick) {
+    // fixed policy: every token is a piece; at epoch p the in-tile states are
+    // the binary-counter blocks of pieces [0, p) (one per set bit of p, largest
+    // first) and {p}; every atom is its own block
+    const int len = min(M, ca.Tw - T0);
+    if (tid == 0) {
+      sm.m0 = m0;
+      sm.len = len;
+      sm.np = len;
+    }
+    for (int p = tid; p < len; p += THREADS) {
+      sm.pst[p] = p;
+      sm.pen[p] = p + 1;
+      uint32_t cur[BW];
+#pragma unroll
+      for (int w = 0; w < BW; w++)
+        cur[w] = m0 >= 32 * (w + 1) ? ~0u : (m0 > 32 * w ? (1u << (m0 - 32 * w)) - 1u : 0u);
+      int start = 0;
+      for (int b = 6; b >= 0; b--) {
+        if ((p >> b) & 1) {
+          start += 1 << b;
+          const int beta = m0 + start - 1;
+          cur[beta >> 5] |= 1u << (beta & 31);
+        }
+      }
+      const int beta = m0 + p;
+      cur[beta >> 5] |= 1u << (beta & 31);
+#pragma unroll
+      for (int w = 0; w < BW; w++) sm.bits[p * BW + w] = cur[w];
+    }
+  } else if (warp == 2 && lane == 0) {
     // in-tile pieces and the state partition of each epoch
     const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
     const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
@@ -113,8 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
     sm.np = np;
     uint32_t cur[BW];
-    for (int w = 0; w < BW; w++) cur[w] = 0;
-    for (int a = 0; a < m0; a++) cur[a >> 5] |= 1u << (a & 31);
+    for (int w = 0; w < BW; w++)
+      cur[w] = m0 >= 32 * (w + 1) ? ~0u : (m0 > 32 * w ? (1u << (m0 - 32 * w)) - 1u : 0u);
     for (int p = 0; p < np; p++) {
       const int beta = m0 + p;
       if (p == 0 && cont) {
@@ -148,14 +172,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       cur[beta >> 5] |= 1u << (beta & 31);
       for (int w = 0; w < BW; w++) sm.bits[p * BW + w] = cur[w];
     }
-    for (int p = 0; p < np; p++)
-      for (int t = sm.pst[p]; t < sm.pen[p]; t++) sm.pidx[t] = p;
-    for (int t = len; t < M; t++) sm.pidx[t] = np - 1;
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
   const int np = sm.np, len = sm.len;
+  if (tid < M) {  // piece of each row (rows past the tile's end take the last piece)
+    int p = 0;
+    while (p + 1 < np && sm.pst[p + 1] <= tid) p++;
+    sm.pidx[tid] = p;
+  }
 
   // ---- loads --------------------------------------------------------------
   if (tid == 0) {
@@ -226,134 +252,182 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   // ---- softmax weights per row (warps 4..7, row t = TMEM lane) ----------------
+  // Pass A walks the row's atoms (TMEM columns, 32 at a time) and pieces in
+  // time order: segmented sums of x_beta and n_beta give each state's logit at
+  // its last atom / piece (written in place); the softmax max and sum are
+  // merged once per chunk.  Pass B walks backwards and gives every atom /
+  // piece the weight of the state it belongs to.  Piece values live in
+  // registers when there are at most PREG pieces, else in TMEM cols [0, np).
   if (warp >= 4 && warp < 8) {
+    constexpr int PREG = 8;
     const int qd = warp & 3;
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     const int ep = sm.pidx[t];
     const uint32_t *bits = sm.bits + ep * BW;
-    // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s] -> TMEM cols [0, np)
+    float pv[PREG];  // piece sums, then logits, then weights
+#pragma unroll
+    for (int k = 0; k < PREG; k++) pv[k] = 0.f;
+    auto piece_get = [&](int p) -> float {
+      if (p < PREG) {
+        float x = 0.f;
+#pragma unroll
+        for (int k = 0; k < PREG; k++) x = (k == p) ? pv[k] : x;
+        return x;
+      }
+      const float x = __uint_as_float(tmem_ld1(trow + COL_BUF0 + p));
+      tmem_wait_ld();
+      return x;
+    };
+    auto piece_put = [&](int p, float x) {
+      if (p < PREG) {
+#pragma unroll
+        for (int k = 0; k < PREG; k++) pv[k] = (k == p) ? x : pv[k];
+      } else {
+        tmem_st1(trow + COL_BUF0 + p, __float_as_uint(x));
+        tmem_wait_st();
+      }
+    };
+    // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s]   (8 columns per load;
+    // loops are kept rolled so the code stays small)
     {
       float y = 0.f;
       int p = 0;
-      for (int s0 = 0; s0 < M; s0 += 32) {
-        uint32_t ar[32];
-        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+      int nxt = np > 1 ? sm.pst[1] : M + 1;
+#pragma unroll 1
+      for (int s0 = 0; s0 < M; s0 += 8) {
+        uint32_t ar[8];
+        DLA_TMEM_LD8(trow + COL_AI + s0, ar);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j++) {
+        for (int j = 0; j < 8; j++) {
           const int s = s0 + j;
-          if (s < len) {
-            if (p + 1 < np && s == sm.pst[p + 1]) {
-              tmem_st1(trow + COL_BUF0 + p, __float_as_uint(y));
-              p++;
-              y = 0.f;
-            }
-            if (s <= t) y += __uint_as_float(ar[j]);
+          if (s == nxt) {
+            piece_put(p, y);
+            p++;
+            y = 0.f;
+            nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
           }
+          y += (s <= t && s < len) ? __uint_as_float(ar[j]) : 0.f;
         }
       }
-      tmem_st1(trow + COL_BUF0 + p, __float_as_uint(y));
-      tmem_wait_st();
+      piece_put(p, y);
     }
-    // pass A: state logits at each state's last atom / piece, online softmax
-    float sacc = 0.f, nacc = 0.f, mx = -INFINITY, l = 0.f;
-    for (int a0 = 0; a0 < m0; a0 += 32) {
-      uint32_t r[32];
-      DLA_TMEM_LD32(trow + COL_W + a0, r);
+    // pass A
+    float mx = -INFINITY, l = 0.f, sacc = 0.f, nacc = 0.f;
+#pragma unroll 1
+    for (int a0 = 0; a0 < m0; a0 += 8) {
+      uint32_t r[8];
+      DLA_TMEM_LD8(trow + COL_W + a0, r);
       tmem_wait_ld();
+      const uint32_t wb = bits[a0 >> 5] >> (a0 & 31);
+      float cmx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; j++) {
+      for (int j = 0; j < 8; j++) {
         const int beta = a0 + j;
         if (beta < m0) {
           const float nn = sm.nA[beta];
-          sacc += nn * __uint_as_float(r[j]);
+          sacc = fmaf(nn, __uint_as_float(r[j]), sacc);
           nacc += nn;
-          if (bit_of(bits, beta)) {
-            const float a = sacc / nacc * INV_SQRT_D;
+          if ((wb >> j) & 1u) {
+            const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
             r[j] = __float_as_uint(a);
-            online(mx, l, a);
-            sacc = nacc = 0.f;
+            cmx = fmaxf(cmx, a);
+            sacc = 0.f;
+            nacc = 0.f;
           }
         }
       }
-      DLA_TMEM_ST32(trow + COL_W + a0, r);
+      float cl = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+        if (a0 + j < m0 && ((wb >> j) & 1u)) cl += __expf(__uint_as_float(r[j]) - cmx);
+      if (cmx > -INFINITY) {
+        const float nm = fmaxf(mx, cmx);
+        l = l * __expf(mx - nm) + cl * __expf(cmx - nm);
+        mx = nm;
+      }
+      DLA_TMEM_ST8(trow + COL_W + a0, r);
       tmem_wait_st();
     }
+#pragma unroll 1
     for (int p = 0; p < np; p++) {
-      uint32_t yv = tmem_ld1(trow + COL_BUF0 + p);
-      tmem_wait_ld();
+      float y = piece_get(p);
       if (p <= ep) {
         const float nn = p < ep ? (float)(sm.pen[p] - sm.pst[p]) : (float)(t - sm.pst[p] + 1);
-        sacc += __uint_as_float(yv);
+        sacc += y;
         nacc += nn;
         if (bit_of(bits, m0 + p)) {
-          const float a = sacc / nacc * INV_SQRT_D;
-          yv = __float_as_uint(a);
-          online(mx, l, a);
-          sacc = nacc = 0.f;
+          const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
+          y = a;
+          const float nm = fmaxf(mx, a);
+          l = l * __expf(mx - nm) + __expf(a - nm);
+          mx = nm;
+          sacc = 0.f;
+          nacc = 0.f;
         }
       }
-      tmem_st1(trow + COL_BUF0 + p, yv);
+      piece_put(p, y);
     }
-    tmem_wait_st();
-    // pass B (reverse): weight of every atom / piece = lambda of its state
+    // pass B (reverse)
+    const float inv_l = 1.0f / l;
     float cur = 0.f;
+#pragma unroll 1
     for (int p = np - 1; p >= 0; p--) {
-      const uint32_t av = tmem_ld1(trow + COL_BUF0 + p);
-      tmem_wait_ld();
+      const float a = piece_get(p);
       float w = 0.f;
       if (p <= ep) {
-        if (bit_of(bits, m0 + p)) cur = expf(__uint_as_float(av) - mx) / l;
+        if (bit_of(bits, m0 + p)) cur = __expf(a - mx) * inv_l;
         w = cur;
       }
-      tmem_st1(trow + COL_BUF0 + p, __float_as_uint(w));
+      piece_put(p, w);
     }
-    tmem_wait_st();
-    for (int a0 = ((m0 - 1) >> 5) << 5; m0 > 0 && a0 >= 0; a0 -= 32) {
-      uint32_t r[32];
-      DLA_TMEM_LD32(trow + COL_W + a0, r);
+#pragma unroll 1
+    for (int a0 = ((m0 - 1) >> 3) << 3; m0 > 0 && a0 >= 0; a0 -= 8) {
+      uint32_t r[8];
+      DLA_TMEM_LD8(trow + COL_W + a0, r);
       tmem_wait_ld();
+      const uint32_t wb = bits[a0 >> 5] >> (a0 & 31);
 #pragma unroll
-      for (int j = 31; j >= 0; j--) {
-        const int beta = a0 + j;
-        if (beta < m0) {
-          if (bit_of(bits, beta)) cur = expf(__uint_as_float(r[j]) - mx) / l;
+      for (int j = 0; j < 8; j++)
+        if (a0 + j < m0 && ((wb >> j) & 1u)) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
+#pragma unroll
+      for (int j = 7; j >= 0; j--) {
+        if (a0 + j < m0) {
+          if ((wb >> j) & 1u) cur = __uint_as_float(r[j]);
           r[j] = __float_as_uint(cur);
         }
       }
-      DLA_TMEM_ST32(trow + COL_W + a0, r);
+      DLA_TMEM_ST8(trow + COL_W + a0, r);
       tmem_wait_st();
     }
     // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of P V
     {
       int p = 0;
-      float w = __uint_as_float(tmem_ld1(trow + COL_BUF0));
-      tmem_wait_ld();
-      for (int s0 = 0; s0 < M; s0 += 32) {
-        uint32_t ar[32];
-        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+      float w = piece_get(0);
+      int nxt = np > 1 ? sm.pst[1] : M + 1;
+#pragma unroll 1
+      for (int s0 = 0; s0 < M; s0 += 8) {
+        uint32_t ar[8];
+        DLA_TMEM_LD8(trow + COL_AI + s0, ar);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[4];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int j = 0; j < 8; j += 2) {
           float v2[2];
 #pragma unroll
           for (int h = 0; h < 2; h++) {
             const int s = s0 + j + h;
-            if (s < len && p + 1 < np && s == sm.pst[p + 1]) {
+            if (s == nxt) {
               p++;
-              w = __uint_as_float(tmem_ld1(trow + COL_BUF0 + p));
-              tmem_wait_ld();
+              w = piece_get(p);
+              nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
             }
             v2[h] = (s <= t && s < len) ? w * __uint_as_float(ar[j + h]) : 0.f;
           }
           pk[j >> 1] = pack_bf16(v2[0], v2[1]);
         }
-#pragma unroll
-        for (int ch = 0; ch < 4; ch++)
-          *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0 + ch * 8, M)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
   }
@@ -395,32 +469,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     float acc[64];
 #pragma unroll
     for (int i = 0; i < 64; i++) acc[i] = 0.f;
-    for (int a0 = 0; a0 < m0; a0 += 32) {
-      uint32_t wr[32];
-      DLA_TMEM_LD32(trow + COL_W + a0, wr);
+#pragma unroll 1
+    for (int a = 0; a < m0; a++) {
+      const int b = a & 1;
+      const float w = __uint_as_float(tmem_ld1(trow + COL_W + a));
+      mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
+      tc_fence_after();
+      uint32_t pr[32];
+      DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; j++) {
-        const int a = a0 + j;
-        if (a < m0) {
-          const int b = a & 1;
-          mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
-          tc_fence_after();
-          const float w = __uint_as_float(wr[j]);
-          uint32_t pr[32];
-          DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
-          tmem_wait_ld();
+      for (int i = 0; i < 32; i++) acc[i] = fmaf(w, __uint_as_float(pr[i]), acc[i]);
+      DLA_TMEM_LD32(trow + b * 128 + hc * 64 + 32, pr);
+      tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; i++) acc[i] = fmaf(w, __uint_as_float(pr[i]), acc[i]);
-          DLA_TMEM_LD32(trow + b * 128 + hc * 64 + 32, pr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(w, __uint_as_float(pr[i]), acc[32 + i]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.tempty[b]);
-        }
-      }
+      for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(w, __uint_as_float(pr[i]), acc[32 + i]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tempty[b]);
     }
     mbar_wait(&sm.bar_mma, 1, abort);
     tc_fence_after();
