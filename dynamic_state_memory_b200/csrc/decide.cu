@@ -7,8 +7,11 @@
 //              predecessor are low-information; Chlience section 5.1: b_t = 1
 //              opens a new state).
 //   k_segscan  window pieces: {0} and every boundary t > 0 (warp ballots).
-//   k_segsum   z = sum of phi(k) per piece in fp64, token by token, and the open
-//              state's partial z before each readout tile.
+//   k_tilesum  per (tile, head): fp64 sum of phi(k) over each run of a piece
+//              inside the tile, in token order.
+//   k_segcombine  per piece: the runs' sums in time order (after the cached
+//              open state's z for a continuation) give z at the piece's end
+//              and the open state's partial z before each readout tile.
 //   k_engine   one warp per head walks tiles and boundaries in time order:
 //              seals, capacity merges by least Ward loss (Chlience section 5.2
 //              and Corollary 1), slot allocation; emits the materializer op
@@ -266,358 +269,456 @@ __global__ void k_segcombine(Dims dm, Plan pl, CallArgs ca) {
 }
 
 // ---------------------------------------------------------------- engine ----
-// One warp per head.  The head's cache summaries (order, n, ts, version of
-// each slot, pair losses and the fp64 z of every slot) live in shared memory
-// for the whole window and are written back at its end.
+// One warp per head walks the window's tiles and segment starts in time order.
+// Shared memory holds the head's cache summaries for the whole window (time
+// order, counts, first times, versions, sealed-pair losses, 1/n of sealed
+// states and the fp64 z of every slot) and a ring of segment-end sums z_end
+// that asynchronous copies fill ZR segments ahead.  Lane l owns dimensions
+// l, l + 32, ... of every z, so z updates need no warp synchronisation.
+// Kernel parameters are copied to registers (no pointer to them is formed)
+// and segment starts are prefetched 32 at a time into lane registers.
+
+constexpr int ZR = 8;  // z_end ring depth
 
 struct EngSmem {
   int32_t order[128];
   int32_t sver[128];
+  uint32_t used[4];
   long long n[128];
   long long ts[128];
   double loss[128];
-  double z[1];  // [C][D], dynamic
+  double rn[128];          // 1 / n of sealed states (__drcp_rn)
+  double zring[ZR][128];
+  double z[1];             // [C][D], dynamic
 };
 
-struct Eng {
-  const Dims *dm;
-  const Plan *pl;
-  const CallArgs *ca;
-  EngSmem *sm;
-  int u, lane, C, D;
-  int4 *ops;
-  int nops, nver, m, npieces;
-  uint32_t used[4];
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-  __device__ double *zs(int slot) const { return sm->z + (size_t)slot * D; }
-  // lane-local emit at position nops + rank; the caller advances nops
-  __device__ void put(int idx, int op, int a, int b, int c) const {
-    if (idx < dm->opsmax) ops[idx] = make_int4(op, a, b, c);
-    else set_status(ca->dev_status, DLA_ERR_INVARIANT);
+// Sum over the warp of one fp64 value per lane, the same on every lane (xor
+// butterfly: partners add the same two operands, so all lanes agree bit for
+// bit, and lane 0's order is that of a halving tree).
+__device__ __forceinline__ double warp_sum(double s) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) s = __dadd_rn(s, __shfl_xor_sync(FULL, s, off));
+  return s;
+}
+
+// Ward loss n_a n_b / (n_a + n_b) * |z_a / n_a - z_b / n_b|^2 (Chlience
+// section 5.2, Corollary 1), means formed as z * (1 / n): within an ulp of
+// z / n, so merge choices agree with the oracle whenever the best and second
+// best losses differ by more than rounding.
+template <int QD>
+__device__ __forceinline__ double ward_loss(const EngSmem *sm, const double *z, int D, int sa,
+                                            int sb, int lane) {
+  const double na = (double)sm->n[sa], nb = (double)sm->n[sb];
+  const double ia = sm->rn[sa], ib = sm->rn[sb];
+  const double *za = z + (size_t)sa * D + lane, *zb = z + (size_t)sb * D + lane;
+  double s = 0.0;
+#pragma unroll
+  for (int q = 0; q < QD; q++) {
+    const double diff = __dsub_rn(__dmul_rn(za[32 * q], ia), __dmul_rn(zb[32 * q], ib));
+    s = __dadd_rn(s, __dmul_rn(diff, diff));
   }
-  __device__ void emit(int op, int a, int b, int c) {
-    if (lane == 0) put(nops, op, a, b, c);
+  const double f = __ddiv_rn(__dmul_rn(na, nb), __dadd_rn(na, nb));
+  return __dmul_rn(f, warp_sum(s));
+}
+
+// Two independent Ward losses (a, b) and (b, c) in one pass (same arithmetic).
+template <int QD>
+__device__ __forceinline__ void ward_loss2(const EngSmem *sm, const double *z, int D, int sa,
+                                           int sb, int sc, int lane, double &l_ab, double &l_bc) {
+  const double na = (double)sm->n[sa], nb = (double)sm->n[sb], nc = (double)sm->n[sc];
+  const double ia = sm->rn[sa], ib = sm->rn[sb], ic = sm->rn[sc];
+  const double *za = z + (size_t)sa * D + lane, *zb = z + (size_t)sb * D + lane,
+               *zc = z + (size_t)sc * D + lane;
+  double s1 = 0.0, s2 = 0.0;
+#pragma unroll
+  for (int q = 0; q < QD; q++) {
+    const double mb = __dmul_rn(zb[32 * q], ib);
+    const double d1 = __dsub_rn(__dmul_rn(za[32 * q], ia), mb);
+    const double d2 = __dsub_rn(mb, __dmul_rn(zc[32 * q], ic));
+    s1 = __dadd_rn(s1, __dmul_rn(d1, d1));
+    s2 = __dadd_rn(s2, __dmul_rn(d2, d2));
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    s1 = __dadd_rn(s1, __shfl_xor_sync(FULL, s1, off));
+    s2 = __dadd_rn(s2, __shfl_xor_sync(FULL, s2, off));
+  }
+  const double f1 = __ddiv_rn(__dmul_rn(na, nb), __dadd_rn(na, nb));
+  const double f2 = __ddiv_rn(__dmul_rn(nb, nc), __dadd_rn(nb, nc));
+  l_ab = __dmul_rn(f1, s1);
+  l_bc = __dmul_rn(f2, s2);
+}
+
+// Leftmost argmin of loss[0 .. L-1] (L >= 1).  Losses are non-negative and
+// finite, so their bit patterns order like their values: three 32-bit warp
+// reductions (high word, low word, index) replace an fp64 shuffle tree.
+__device__ __forceinline__ int argmin_leftmost(const double *loss, int L, int lane) {
+  unsigned long long best = ~0ull;
+  int bi = 0x7fffffff;
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    const int p = lane + 32 * q;
+    if (p < L) {
+      const unsigned long long key = (unsigned long long)__double_as_longlong(loss[p]);
+      if (key < best) {
+        best = key;
+        bi = p;
+      }
+    }
+  }
+  const unsigned hi = __reduce_min_sync(FULL, (unsigned)(best >> 32));
+  const unsigned lo = __reduce_min_sync(FULL, (unsigned)(best >> 32) == hi ? (unsigned)best : ~0u);
+  const bool cand = best == (((unsigned long long)hi << 32) | lo);
+  return (int)__reduce_min_sync(FULL, cand ? (unsigned)bi : 0x7fffffffu);
+}
+
+template <int D>
+__global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
+  constexpr int QD = D / 32;
+  extern __shared__ __align__(16) unsigned char eng_raw[];
+  EngSmem *sm = reinterpret_cast<EngSmem *>(eng_raw);
+  double *zs = sm->z;
+  const int u = blockIdx.x, lane = threadIdx.x;
+  const int C = dm.C, M = dm.M, W = dm.W, tiles = dm.tiles, amax = dm.amax, vmax = dm.vmax;
+  const int opsmax = dm.opsmax, pmax = dm.pmax;
+  const int Tw = ca.Tw;
+  int32_t *const dev_status = ca.dev_status;
+  // the head's cache
+  int32_t *const c_order = ca.cache.order + (size_t)u * C;
+  int64_t *const c_n = ca.cache.n + (size_t)u * C;
+  int64_t *const c_ts = ca.cache.ts + (size_t)u * C;
+  double *const c_loss = ca.cache.pair_loss + (size_t)u * C;
+  double *const c_z = ca.cache.z + (size_t)u * C * D;
+  // the head's plan
+  const int nseg = pl.nseg[u];
+  const int32_t *const ss = pl.seg_start + (size_t)u * (W + 1);
+  const double *const zend = pl.z_end + (size_t)u * W * D;
+  const double *const ztile_g = pl.z_tile + (size_t)u * tiles * D;
+  int4 *const ops = pl.ops + (size_t)u * opsmax;
+  int32_t *const tm0 = pl.tile_m0 + (size_t)u * tiles;
+  int32_t *const tat = pl.tile_atoms + (size_t)u * tiles * amax;
+  int32_t *const tnev = pl.tile_nev + (size_t)u * tiles;
+  int32_t *const toff = pl.tile_ev_off + (size_t)u * tiles * M;
+  int32_t *const tmrg = pl.tile_ev_mrg + (size_t)u * tiles * M;
+  int32_t *const tpb = pmax > 0 ? pl.tile_pbase + (size_t)u * tiles : nullptr;
+  float *const ver_z = pl.ver_z + (size_t)u * vmax * D;
+  float *const ver_n = pl.ver_n + (size_t)u * vmax;
+  int32_t *const tr_t = ca.trace.merge_t ? ca.trace.merge_t + (size_t)u * ca.trace.cap : nullptr;
+  int32_t *const tr_i = ca.trace.merge_i ? ca.trace.merge_i + (size_t)u * ca.trace.cap : nullptr;
+  const bool tracing = ca.trace.merge_count != nullptr;
+  const int tcap = ca.trace.cap;
+
+  // ---- segment-end sums: prefetch ring ------------------------------------
+  auto zfetch = [&](int g) {
+    if (g < nseg) {
+      double *dst = sm->zring[g % ZR] + lane;
+      const double *src = zend + (size_t)g * D + lane;
+#pragma unroll
+      for (int q = 0; q < QD; q++) cp_async8(dst + 32 * q, src + 32 * q);
+    }
+    cp_async_commit();
+  };
+#pragma unroll 1
+  for (int g = 0; g < ZR; g++) zfetch(g);
+  int zcons = 0;  // next z_end row to take (rows are taken in order)
+  // z_end[zcons] -> dst (lane-owned dims); then refill its ring slot
+  auto ztake = [&](double *dst) {
+    cp_async_wait<ZR - 1>();
+    const double *src = sm->zring[zcons % ZR] + lane;
+#pragma unroll
+    for (int q = 0; q < QD; q++) dst[lane + 32 * q] = src[32 * q];
+    zfetch(zcons + ZR);
+    zcons++;
+  };
+
+  // ---- load the head's summaries ------------------------------------------
+  int m = ca.cache.m[u];
+  const int64_t t0 = ca.cache.t[u];
+  if (lane < 4) sm->used[lane] = 0u;
+  __syncwarp();
+  for (int p = lane; p < C; p += 32) {
+    const int o = c_order[p];
+    sm->order[p] = o;
+    const long long nn = c_n[p];
+    sm->n[p] = nn;
+    sm->rn[p] = __drcp_rn((double)nn);
+    sm->ts[p] = c_ts[p];
+    sm->loss[p] = c_loss[p];
+    sm->sver[p] = -1;
+    if (p < m) atomicOr(&sm->used[o >> 5], 1u << (o & 31));
+  }
+  for (int i = lane; i < C * D; i += 32) zs[i] = c_z[i];
+  __syncwarp();
+  // lane w < 4 keeps the used-slot bits of slots 32w .. 32w + 31
+  uint32_t uw = lane < 4 ? sm->used[lane] : 0u;
+  const uint32_t valid_bits = lane * 32 >= C ? 0u : (C - lane * 32 >= 32 ? ~0u : ((1u << (C - lane * 32)) - 1u));
+  // lowest free slot
+  auto alloc_slot = [&]() -> int {
+    const uint32_t fr = ~uw & valid_bits;
+    const unsigned bal = __ballot_sync(FULL, fr != 0u);
+    if (bal == 0u) {
+      if (lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
+      return 0;
+    }
+    const int w = __ffs(bal) - 1;
+    const int bit = __ffs(__shfl_sync(FULL, fr, w)) - 1;
+    if (lane == w) uw |= 1u << bit;
+    return w * 32 + bit;
+  };
+
+  int nops = 0, nver = 0, npieces = 0;
+  auto emit = [&](int op, int a, int b, int c) {
+    if (lane == 0) {
+      if (nops < opsmax) ops[nops] = make_int4(op, a, b, c);
+      else set_status(dev_status, DLA_ERR_INVARIANT);
+    }
     nops++;
-  }
+  };
   // tokens [from, from + cnt) join the open state `slot`: a tensor-core piece
   // when long enough (and the path has pieces), else SIMT rank-1 adds
-  __device__ void emit_add(int slot, int from, int cnt) {
-    if (dm->pmax > 0 && cnt >= PIECE_MIN) {
-      if (npieces >= dm->pmax && lane == 0) set_status(ca->dev_status, DLA_ERR_INVARIANT);
+  auto emit_add = [&](int slot, int from, int cnt) {
+    if (pmax > 0 && cnt >= PIECE_MIN) {
+      if (npieces >= pmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
       emit(OP_ADDP, slot, npieces, cnt);
       npieces++;
     } else {
       emit(OP_ADD, slot, from, cnt);
     }
-  }
-  // Ward loss with one reciprocal per state: mu = z * (1 / n) (within an ulp
-  // of z / n; merge choices agree with the oracle whenever the best and
-  // second-best losses differ by more than rounding)
-  __device__ double ward(int sa, int sb) const {
-    const double na = (double)sm->n[sa], nb = (double)sm->n[sb];
-    const double ia = __drcp_rn(na), ib = __drcp_rn(nb);
-    const double *za = zs(sa), *zb = zs(sb);
-    double s = 0.0;
-    for (int c = lane; c < D; c += 32) {
-      const double diff = __dsub_rn(__dmul_rn(za[c], ia), __dmul_rn(zb[c], ib));
-      s = __dadd_rn(s, __dmul_rn(diff, diff));
-    }
-    for (int off = 16; off; off >>= 1) s = __dadd_rn(s, __shfl_down_sync(FULL, s, off));
-    s = __shfl_sync(FULL, s, 0);
-    const double f = __ddiv_rn(__dmul_rn(na, nb), __dadd_rn(na, nb));
-    return __dmul_rn(f, s);
-  }
-  __device__ int alloc_slot() {
-    for (int w = 0; w < 4; w++) {
-      const uint32_t freeb = ~used[w];
-      if (w * 32 < C && freeb) {
-        const int slot = w * 32 + __ffs(freeb) - 1;
-        if (slot < C) {
-          used[w] |= 1u << (slot & 31);
-          return slot;
-        }
-      }
-    }
-    if (lane == 0) set_status(ca->dev_status, DLA_ERR_INVARIANT);
-    return 0;
-  }
-  __device__ void free_slot(int s) { used[s >> 5] &= ~(1u << (s & 31)); }
-  // the same from per-lane registers (dimension lane + 32 q)
-  __device__ void write_mu_regs(int v, const double *zr, long long cnt) const {
-    float *zv = pl->ver_z + ((size_t)u * dm->vmax + v) * D;
-#pragma unroll
-    for (int q = 0; q < 4; q++)
-      if (lane + 32 * q < D) zv[lane + 32 * q] = (float)zr[q];
-    if (lane == 0) pl->ver_n[(size_t)u * dm->vmax + v] = (float)cnt;
-  }
-  // phi(k) sum and count of version v (all lanes); readouts divide
-  __device__ void write_mu(int v, const double *zsrc, long long cnt) const {
-    float *zv = pl->ver_z + ((size_t)u * dm->vmax + v) * D;
-    for (int c = lane; c < D; c += 32) zv[c] = (float)zsrc[c];
-    if (lane == 0) pl->ver_n[(size_t)u * dm->vmax + v] = (float)cnt;
-  }
-};
-
-__global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
-  extern __shared__ __align__(16) unsigned char eng_raw[];
-  EngSmem *sm = reinterpret_cast<EngSmem *>(eng_raw);
-  Eng e;
-  e.dm = &dm;
-  e.pl = &pl;
-  e.ca = &ca;
-  e.sm = sm;
-  e.u = blockIdx.x;
-  e.lane = threadIdx.x;
-  e.C = dm.C;
-  e.D = dm.D;
-  const int u = e.u, lane = e.lane, C = dm.C, D = dm.D, M = dm.M;
-  const dla_cache &cc = ca.cache;
-  // ---- load the head's summaries ------------------------------------------
-  for (int p = lane; p < C; p += 32) {
-    sm->order[p] = cc.order[(size_t)u * C + p];
-    sm->n[p] = cc.n[(size_t)u * C + p];
-    sm->ts[p] = cc.ts[(size_t)u * C + p];
-    sm->loss[p] = cc.pair_loss[(size_t)u * C + p];
-    sm->sver[p] = -1;
-  }
-  for (int i = lane; i < C * D; i += 32) sm->z[i] = cc.z[(size_t)u * C * D + i];
-  __syncwarp();
-  e.ops = pl.ops + (size_t)u * dm.opsmax;
-  e.nops = 0;
-  e.nver = 0;
-  e.npieces = 0;
-  e.m = cc.m[u];
-  const int64_t t0 = cc.t[u];
-  for (int w = 0; w < 4; w++) e.used[w] = 0;
-  for (int p = 0; p < e.m; p++) {
-    const int s = sm->order[p];
-    e.used[s >> 5] |= 1u << (s & 31);
-  }
-  if (e.m > 0) e.emit(OP_LOAD, sm->order[e.m - 1], 0, 0);
-
-  const int nseg = pl.nseg[u];
-  const int32_t *ss = pl.seg_start + (size_t)u * (dm.W + 1);
-  const uint8_t *bflag = pl.b + (size_t)u * dm.W;
-  const double *zend = pl.z_end + (size_t)u * dm.W * D;
-  int32_t *tm0 = pl.tile_m0 + (size_t)u * dm.tiles;
-  int32_t *tat = pl.tile_atoms + (size_t)u * dm.tiles * dm.amax;
-  int32_t *tnev = pl.tile_nev + (size_t)u * dm.tiles;
-  int32_t *toff = pl.tile_ev_off + (size_t)u * dm.tiles * M;
-  int32_t *tmrg = pl.tile_ev_mrg + (size_t)u * dm.tiles * M;
-  const bool tracing = ca.trace.merge_count != nullptr;
+  };
+  if (m > 0) emit(OP_LOAD, sm->order[m - 1], 0, 0);
   int mcount = tracing ? ca.trace.merge_count[u] : 0;
+  const bool cont0 = nseg > 0 && pl.b[(size_t)u * W] == 0;  // token 0 continues the open state
+
+  // segment starts, 32 per lane-register chunk, the next chunk in flight
+  int sbase = 0;
+  int ssA = lane < nseg ? ss[lane] : 0x7fffffff;
+  int ssB = 32 + lane < nseg ? ss[32 + lane] : 0x7fffffff;
 
   int j = 0;
   int cur_from = 0;  // first window token not yet added to the open state
-  // one step of look-ahead on global reads: the next boundary positions, the
-  // end sum of the segment sealed at the next boundary, the next tile's
-  // open-state partial sum
-  int ss_cur = nseg > 0 ? ss[0] : 0x7fffffff;
-  int ss_nxt = nseg > 1 ? ss[1] : 0x7fffffff;
-  double zprev[4] = {0.0, 0.0, 0.0, 0.0};  // end sum of segment j-1
-  double ztile[4] = {0.0, 0.0, 0.0, 0.0};  // open-state partial sum before tile c
-  for (int c = 0; c < dm.tiles && c * M < ca.Tw; c++) {
+  double ztile[QD];  // open-state partial sum before the next tile
+#pragma unroll
+  for (int q = 0; q < QD; q++) ztile[q] = 0.0;
+#pragma unroll 1
+  for (int c = 0; c < tiles && c * M < Tw; c++) {
     const int T0 = c * M;
-    const int Tend = min(T0 + M, ca.Tw);
-    double ztile_cur[4];
+    const int Tend = min(T0 + M, Tw);
+    double ztile_cur[QD];
 #pragma unroll
-    for (int q = 0; q < 4; q++) ztile_cur[q] = ztile[q];
-#pragma unroll
-    for (int q = 0; q < 4; q++)
-      ztile[q] = (c + 1 < dm.tiles && (c + 1) * M < ca.Tw && lane + 32 * q < D)
-                     ? pl.z_tile[((size_t)u * dm.tiles + c + 1) * D + lane + 32 * q] : 0.0;
-    // ---- states present just before the tile ----------------------------
-    if (e.m > 0) {
-      const int os = sm->order[e.m - 1];
-      if (T0 > cur_from) {
-        e.emit_add(os, cur_from, T0 - cur_from);
-        if (lane == 0) sm->n[os] += T0 - cur_from;
-        __syncwarp();
-        cur_from = T0;
-      }
+    for (int q = 0; q < QD; q++) {
+      ztile_cur[q] = ztile[q];
+      ztile[q] = (c + 1 < tiles && (c + 1) * M < Tw) ? ztile_g[(size_t)(c + 1) * D + lane + 32 * q] : 0.0;
     }
-    if (lane == 0 && dm.pmax > 0) pl.tile_pbase[(size_t)u * dm.tiles + c] = e.npieces;
-    const int m0 = e.m;
+    // ---- states present just before the tile ----------------------------
+    if (m > 0 && T0 > cur_from) {
+      const int os = sm->order[m - 1];
+      emit_add(os, cur_from, T0 - cur_from);
+      if (lane == 0) sm->n[os] += T0 - cur_from;
+      cur_from = T0;
+    }
+    __syncwarp();
+    if (lane == 0 && tpb) tpb[c] = npieces;
+    const int m0 = m;
+#pragma unroll 1
     for (int p0 = 0; p0 < m0; p0 += 32) {
       const int p = p0 + lane;
       const int slot = p < m0 ? sm->order[p] : 0;
-      const bool need = p < m0 && (p == m0 - 1 || sm->sver[slot] < 0);
+      const int sv = p < m0 ? sm->sver[slot] : 0;
+      const bool need = p < m0 && (p == m0 - 1 || sv < 0);
       const unsigned bal = __ballot_sync(FULL, need);
       const int rank = __popc(bal & ((1u << lane) - 1u));
       if (need) {
-        const int v = e.nver + rank;
-        e.put(e.nops + rank, OP_SHADOW, slot, v, 0);
+        const int v = nver + rank;
+        if (nops + rank < opsmax) ops[nops + rank] = make_int4(OP_SHADOW, slot, v, 0);
+        else set_status(dev_status, DLA_ERR_INVARIANT);
         if (p != m0 - 1) sm->sver[slot] = v;
-        tat[(size_t)c * dm.amax + p] = v;
+        tat[(size_t)c * amax + p] = v;
       } else if (p < m0) {
-        tat[(size_t)c * dm.amax + p] = sm->sver[slot];
+        tat[(size_t)c * amax + p] = sv;
       }
-      // means of the new versions (lanes over dimensions)
+      // sums and counts of the new versions (lanes over dimensions)
       unsigned todo = bal;
       while (todo) {
         const int l = __ffs(todo) - 1;
         todo &= todo - 1;
         const int pv = p0 + l;
-        const int sl = sm->order[pv];
-        const int v = e.nver + __popc(bal & ((1u << l) - 1u));
-        if (pv == m0 - 1 && c > 0) e.write_mu_regs(v, ztile_cur, sm->n[sl]);
-        else e.write_mu(v, e.zs(sl), sm->n[sl]);
+        const int sl = __shfl_sync(FULL, slot, l);
+        const int v = nver + __popc(bal & ((1u << l) - 1u));
+        float *zv = ver_z + (size_t)v * D + lane;
+        if (pv == m0 - 1 && c > 0) {
+#pragma unroll
+          for (int q = 0; q < QD; q++) zv[32 * q] = (float)ztile_cur[q];
+        } else {
+          const double *zsrc = zs + (size_t)sl * D + lane;
+#pragma unroll
+          for (int q = 0; q < QD; q++) zv[32 * q] = (float)zsrc[32 * q];
+        }
+        if (lane == 0) ver_n[v] = (float)sm->n[sl];
       }
-      e.nver += __popc(bal);
-      e.nops += __popc(bal);
+      nver += __popc(bal);
+      nops += __popc(bal);
       __syncwarp();
     }
-    if (e.nver > dm.vmax && lane == 0) set_status(ca.dev_status, DLA_ERR_INVARIANT);
+    if (nver > vmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
     if (lane == 0) tm0[c] = m0;
     // ---- boundaries inside the tile --------------------------------------
     int nev = 0;
-    while (j < nseg && ss_cur < Tend) {
-      const int s = ss_cur;
-      const int ss_n2 = j + 2 < nseg ? ss[j + 2] : 0x7fffffff;
-      double znext[4];
-#pragma unroll
-      for (int q = 0; q < 4; q++) znext[q] = lane + 32 * q < D ? zend[(size_t)j * D + lane + 32 * q] : 0.0;
-      if (!(s == 0 && bflag[0] == 0)) {
+#pragma unroll 1
+    while (j < nseg) {
+      if (j - sbase == 32) {
+        sbase += 32;
+        ssA = ssB;
+        ssB = sbase + 32 + lane < nseg ? ss[sbase + 32 + lane] : 0x7fffffff;
+      }
+      const int s = __shfl_sync(FULL, ssA, j - sbase);
+      if (s >= Tend) break;
+      if (!(s == 0 && cont0)) {
         int mrg = EV_NO_MERGE;
-        if (e.m > 0) {
-          const int os = sm->order[e.m - 1];
+        if (m > 0) {
+          const int os = sm->order[m - 1];
           if (s > cur_from) {
-            e.emit_add(os, cur_from, s - cur_from);
+            emit_add(os, cur_from, s - cur_from);
             if (lane == 0) sm->n[os] += s - cur_from;
           }
-          e.emit(OP_STORE, os, 0, 0);
-          if (j >= 1) {
-#pragma unroll
-            for (int q = 0; q < 4; q++)
-              if (lane + 32 * q < D) e.zs(os)[lane + 32 * q] = zprev[q];
-          }
+          emit(OP_STORE, os, 0, 0);
+          if (j >= 1) ztake(zs + (size_t)os * D);
           __syncwarp();
           // seal: the open state joins the sealed list (all m states sealed)
-          if (e.m >= 2) {
-            const double l = e.ward(sm->order[e.m - 2], sm->order[e.m - 1]);
-            if (lane == 0) sm->loss[e.m - 2] = l;
+          if (lane == 0) sm->rn[os] = __drcp_rn((double)sm->n[os]);
+          __syncwarp();
+          if (m >= 2) {
+            const double l = ward_loss<QD>(sm, zs, D, sm->order[m - 2], os, lane);
+            if (lane == 0) sm->loss[m - 2] = l;
           }
           __syncwarp();
-          if (e.m == C) {
-            // leftmost argmin over the C-1 sealed pairs
-            double best = INFINITY;
-            int bi = 0x7fffffff;
-            for (int p = lane; p < C - 1; p += 32) {
-              const double l = sm->loss[p];
-              if (l < best) {
-                best = l;
-                bi = p;
-              }
-            }
-            for (int off = 16; off; off >>= 1) {
-              const double ob = __shfl_down_sync(FULL, best, off);
-              const int oi = __shfl_down_sync(FULL, bi, off);
-              if (ob < best || (ob == best && oi < bi)) {
-                best = ob;
-                bi = oi;
-              }
-            }
-            const int is = __shfl_sync(FULL, bi, 0);
+          if (m == C) {
+            const int is = argmin_leftmost(sm->loss, C - 1, lane);
             const int a = sm->order[is], bb = sm->order[is + 1];
-            for (int d2 = lane; d2 < D; d2 += 32) e.zs(a)[d2] = __dadd_rn(e.zs(a)[d2], e.zs(bb)[d2]);
-            if (lane == 0) {
-              sm->n[a] += sm->n[bb];
-              sm->sver[a] = -1;
-              sm->sver[bb] = -1;
+            {
+              double *za = zs + (size_t)a * D + lane;
+              const double *zb = zs + (size_t)bb * D + lane;
+#pragma unroll
+              for (int q = 0; q < QD; q++) za[32 * q] = __dadd_rn(za[32 * q], zb[32 * q]);
             }
-            e.emit(OP_MERGE, a, bb, 0);
-            e.free_slot(bb);
-            // drop position is+1 from order and pair (is) from the losses
+            emit(OP_MERGE, a, bb, 0);
+            if (lane == (bb >> 5)) uw &= ~(1u << (bb & 31));
+            // drop position is + 1 from the order and pair is from the losses
             int32_t ov[4];
             double lv[4];
+#pragma unroll
             for (int q = 0; q < 4; q++) {
               const int p = lane + 32 * q;
               ov[q] = (p >= is + 1 && p + 1 < C) ? sm->order[p + 1] : 0;
               lv[q] = (p >= is + 1 && p + 1 < C - 1) ? sm->loss[p + 1] : 0.0;
             }
             __syncwarp();
+#pragma unroll
             for (int q = 0; q < 4; q++) {
               const int p = lane + 32 * q;
               if (p >= is + 1 && p + 1 < C) sm->order[p] = ov[q];
               if (p >= is + 1 && p + 1 < C - 1) sm->loss[p] = lv[q];
             }
-            __syncwarp();
-            e.m -= 1;  // C - 1 sealed
-            if (is >= 1) {
-              const double l = e.ward(sm->order[is - 1], sm->order[is]);
-              if (lane == 0) sm->loss[is - 1] = l;
+            if (lane == 0) {
+              const long long na = sm->n[a] + sm->n[bb];
+              sm->n[a] = na;
+              sm->rn[a] = __drcp_rn((double)na);
+              sm->sver[a] = -1;
+              sm->sver[bb] = -1;
             }
-            if (is + 1 <= e.m - 1) {
-              const double l = e.ward(sm->order[is], sm->order[is + 1]);
-              if (lane == 0) sm->loss[is] = l;
+            __syncwarp();
+            m -= 1;  // C - 1 sealed
+            // the merged state's new neighbour losses
+            const bool left = is >= 1, right = is + 1 <= m - 1;
+            const int sl = sm->order[left ? is - 1 : is];
+            const int sr = sm->order[right ? is + 1 : is];
+            double l_left, l_right;
+            ward_loss2<QD>(sm, zs, D, sl, a, sr, lane, l_left, l_right);
+            if (lane == 0) {
+              if (left) sm->loss[is - 1] = l_left;
+              if (right) sm->loss[is] = l_right;
             }
             __syncwarp();
             mrg = is;
             if (tracing) {
-              if (mcount < ca.trace.cap) {
+              if (mcount < tcap) {
                 if (lane == 0) {
-                  ca.trace.merge_t[(size_t)u * ca.trace.cap + mcount] = (int32_t)(t0 + s);
-                  ca.trace.merge_i[(size_t)u * ca.trace.cap + mcount] = is;
+                  tr_t[mcount] = (int32_t)(t0 + s);
+                  tr_i[mcount] = is;
                 }
               } else if (lane == 0) {
-                set_status(ca.dev_status, DLA_ERR_TRACE_OVERFLOW);
+                set_status(dev_status, DLA_ERR_TRACE_OVERFLOW);
               }
               mcount++;
             }
           }
         }
         // open a new state at s
-        const int slot = e.alloc_slot();
-        e.emit(OP_ZERO, slot, 0, 0);
-        for (int d2 = lane; d2 < D; d2 += 32) e.zs(slot)[d2] = 0.0;
+        const int slot = alloc_slot();
+        emit(OP_ZERO, slot, 0, 0);
+        {
+          double *zn = zs + (size_t)slot * D + lane;
+#pragma unroll
+          for (int q = 0; q < QD; q++) zn[32 * q] = 0.0;
+        }
         if (lane == 0) {
           sm->n[slot] = 0;
           sm->ts[slot] = t0 + s;
-          sm->order[e.m] = slot;
+          sm->order[m] = slot;
           sm->sver[slot] = -1;
           toff[(size_t)c * M + nev] = s - T0;
           tmrg[(size_t)c * M + nev] = mrg;
         }
         __syncwarp();
-        e.m += 1;
+        m += 1;
         cur_from = s;
         nev++;
       }
-#pragma unroll
-      for (int q = 0; q < 4; q++) zprev[q] = znext[q];
-      ss_cur = ss_nxt;
-      ss_nxt = ss_n2;
       j++;
     }
     if (lane == 0) tnev[c] = nev;
   }
   // ---- window end -------------------------------------------------------
-  if (e.m > 0) {
-    const int os = sm->order[e.m - 1];
-    if (ca.Tw > cur_from) {
-      e.emit_add(os, cur_from, ca.Tw - cur_from);
-      if (lane == 0) sm->n[os] += ca.Tw - cur_from;
+  if (m > 0) {
+    const int os = sm->order[m - 1];
+    if (Tw > cur_from) {
+      emit_add(os, cur_from, Tw - cur_from);
+      if (lane == 0) sm->n[os] += Tw - cur_from;
     }
-    e.emit(OP_STORE, os, 0, 0);
-    for (int d2 = lane; d2 < D; d2 += 32) e.zs(os)[d2] = zend[(size_t)(nseg - 1) * D + d2];
+    emit(OP_STORE, os, 0, 0);
+    if (nseg >= 1) ztake(zs + (size_t)os * D);
   }
+  cp_async_wait<0>();
   __syncwarp();
   for (int p = lane; p < C; p += 32) {
-    cc.order[(size_t)u * C + p] = sm->order[p];
-    cc.n[(size_t)u * C + p] = sm->n[p];
-    cc.ts[(size_t)u * C + p] = sm->ts[p];
-    cc.pair_loss[(size_t)u * C + p] = sm->loss[p];
+    c_order[p] = sm->order[p];
+    c_n[p] = sm->n[p];
+    c_ts[p] = sm->ts[p];
+    c_loss[p] = sm->loss[p];
   }
-  for (int i = lane; i < C * D; i += 32) cc.z[(size_t)u * C * D + i] = sm->z[i];
+  for (int i = lane; i < C * D; i += 32) c_z[i] = zs[i];
   if (lane == 0) {
-    cc.m[u] = e.m;
-    cc.t[u] = t0 + ca.Tw;
-    cc.prev_r[u] = pl.r[(size_t)u * dm.W + ca.Tw - 1];
-    pl.nops[u] = min(e.nops, dm.opsmax);
+    ca.cache.m[u] = m;
+    ca.cache.t[u] = t0 + Tw;
+    ca.cache.prev_r[u] = pl.r[(size_t)u * W + Tw - 1];
+    pl.nops[u] = min(nops, opsmax);
     if (tracing) ca.trace.merge_count[u] = mcount;
   }
-  const size_t krow = ((size_t)u * dm.T + ca.w0 + ca.Tw - 1) * D;
-  for (int d2 = lane; d2 < D; d2 += 32) cc.prev_k[(size_t)u * D + d2] = load_in(ca.k, ca.in_dtype, krow + d2);
+  const size_t krow = ((size_t)u * dm.T + ca.w0 + Tw - 1) * D;
+  for (int d2 = lane; d2 < D; d2 += 32) ca.cache.prev_k[(size_t)u * D + d2] = load_in(ca.k, ca.in_dtype, krow + d2);
 }
 
 }  // namespace
@@ -655,12 +756,22 @@ cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
   return cudaGetLastError();
 }
 
-cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  const size_t sb = sizeof(EngSmem) + sizeof(double) * ((size_t)dm.C * dm.D - 1);
-  cudaError_t e = cudaFuncSetAttribute(k_engine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+template <int D>
+static cudaError_t launch_engine_d(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  const size_t sb = sizeof(EngSmem) + sizeof(double) * ((size_t)dm.C * D - 1);
+  cudaError_t e = cudaFuncSetAttribute(k_engine<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
   if (e != cudaSuccess) return e;
-  k_engine<<<dm.heads, 32, sb, s>>>(dm, pl, ca);
+  k_engine<D><<<dm.heads, 32, sb, s>>>(dm, pl, ca);
   return cudaGetLastError();
+}
+
+cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  switch (dm.D) {
+    case 32: return launch_engine_d<32>(dm, pl, ca, s);
+    case 64: return launch_engine_d<64>(dm, pl, ca, s);
+    case 128: return launch_engine_d<128>(dm, pl, ca, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dla
