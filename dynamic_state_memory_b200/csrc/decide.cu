@@ -283,6 +283,7 @@ constexpr int ZR = 8;  // z_end ring depth
 struct EngSmem {
   int32_t order[128];
   int32_t sver[128];
+  int32_t lastmod[128];    // op that produced the slot's sealed value (-1: none)
   uint32_t used[4];
   long long n[128];
   long long ts[128];
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     sm->ts[p] = c_ts[p];
     sm->loss[p] = c_loss[p];
     sm->sver[p] = -1;
+    sm->lastmod[p] = -1;
     if (p < m) atomicOr(&sm->used[o >> 5], 1u << (o & 31));
   }
   for (int i = lane; i < C * D; i += 32) zs[i] = c_z[i];
@@ -539,12 +541,24 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
       const int slot = p < m0 ? sm->order[p] : 0;
       const int sv = p < m0 ? sm->sver[slot] : 0;
       const bool need = p < m0 && (p == m0 - 1 || sv < 0);
+      // a sealed state whose value came from a STORE / MERGE of this window
+      // gets its version id patched into that op; others get a SHADOW op
+      const int lm = (need && p != m0 - 1) ? sm->lastmod[slot] : -1;
+      const bool patch = lm >= 0;
       const unsigned bal = __ballot_sync(FULL, need);
-      const int rank = __popc(bal & ((1u << lane) - 1u));
+      const unsigned bal_emit = __ballot_sync(FULL, need && !patch);
+      const unsigned below = (1u << lane) - 1u;
+      const int rank = __popc(bal & below);
       if (need) {
         const int v = nver + rank;
-        if (nops + rank < opsmax) ops[nops + rank] = make_int4(OP_SHADOW, slot, v, 0);
-        else set_status(dev_status, DLA_ERR_INVARIANT);
+        if (patch) {
+          if (lm < opsmax) ops[lm].w = v + 1;
+          sm->lastmod[slot] = -1;
+        } else {
+          const int erank = __popc(bal_emit & below);
+          if (nops + erank < opsmax) ops[nops + erank] = make_int4(OP_SHADOW, slot, v, 0);
+          else set_status(dev_status, DLA_ERR_INVARIANT);
+        }
         if (p != m0 - 1) sm->sver[slot] = v;
         tat[(size_t)c * amax + p] = v;
       } else if (p < m0) {
@@ -570,7 +584,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         if (lane == 0) ver_n[v] = (float)sm->n[sl];
       }
       nver += __popc(bal);
-      nops += __popc(bal);
+      nops += __popc(bal_emit);
       __syncwarp();
     }
     if (nver > vmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
@@ -594,7 +608,6 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             emit_add(os, cur_from, s - cur_from);
             if (lane == 0) sm->n[os] += s - cur_from;
           }
-          emit(OP_STORE, os, 0, 0);
           if (j >= 1) ztake(zs + (size_t)os * D);
           __syncwarp();
           // seal: the open state joins the sealed list (all m states sealed)
@@ -614,7 +627,19 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
 #pragma unroll
               for (int q = 0; q < QD; q++) za[32 * q] = __dadd_rn(za[32 * q], zb[32 * q]);
             }
-            emit(OP_MERGE, a, bb, 0);
+            if (bb == os) {
+              // the just-sealed state is the right member: its registers go
+              // straight into the left one, it is never stored
+              if (lane == 0) sm->lastmod[a] = nops;
+              emit(OP_MERGEO, a, 0, 0);
+            } else {
+              if (lane == 0) {
+                sm->lastmod[os] = nops;
+                sm->lastmod[a] = nops + 1;
+              }
+              emit(OP_STORE, os, 0, 0);
+              emit(OP_MERGE, a, bb, 0);
+            }
             if (lane == (bb >> 5)) uw &= ~(1u << (bb & 31));
             // drop position is + 1 from the order and pair is from the losses
             int32_t ov[4];
@@ -664,6 +689,9 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
               }
               mcount++;
             }
+          } else {
+            if (lane == 0) sm->lastmod[os] = nops;
+            emit(OP_STORE, os, 0, 0);
           }
         }
         // open a new state at s
@@ -679,6 +707,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
           sm->ts[slot] = t0 + s;
           sm->order[m] = slot;
           sm->sver[slot] = -1;
+          sm->lastmod[slot] = -1;
           toff[(size_t)c * M + nev] = s - T0;
           tmrg[(size_t)c * M + nev] = mrg;
         }

@@ -19,17 +19,22 @@
 namespace dla {
 
 // Ops of the state materializer.  The open state is kept in registers: ZERO
-// or LOAD makes `slot` the register-resident open state, ADD accumulates
-// tokens into it, STORE writes it back to its slot; MERGE and SHADOW of a
-// sealed slot work on memory, SHADOW of the open slot reads the registers.
+// or LOAD makes `slot` the register-resident open state, ADD / ADDP
+// accumulate tokens into it, STORE writes it back to its slot; MERGE works on
+// memory, MERGEO adds the open registers into a sealed slot (the open state
+// is the merge's right member and disappears), SHADOW freezes a version (of
+// the open registers, or of a sealed slot read from memory).  STORE, MERGE
+// and MERGEO carry in .w the version id + 1 of the result (0: none), so a
+// sealed state's version is written from registers without a re-read.
 enum OpCode : int32_t {
-  OP_ZERO = 0,
-  OP_ADD = 1,
-  OP_MERGE = 2,
-  OP_SHADOW = 3,
-  OP_LOAD = 4,
-  OP_STORE = 5,
-  OP_ADDP = 6  // add the precomputed piece (tensor-core builder) op.z to the open state
+  OP_ZERO = 0,    // (ZERO, slot)
+  OP_ADD = 1,     // (ADD, slot, first window token, count)
+  OP_MERGE = 2,   // (MERGE, dst, src, version + 1)
+  OP_SHADOW = 3,  // (SHADOW, slot, version)
+  OP_LOAD = 4,    // (LOAD, slot)
+  OP_STORE = 5,   // (STORE, slot, 0, version + 1)
+  OP_ADDP = 6,    // (ADDP, slot, piece id, count): add the tensor-core builder's piece
+  OP_MERGEO = 7   // (MERGEO, dst, 0, version + 1)
 };
 
 // Pieces shorter than this stay SIMT adds in the materializer.

@@ -2,14 +2,18 @@
 //
 // Each CTA owns R rows (of d_v) of every slot of one head and replays the
 // head's ops in order, so no two CTAs touch the same element and no
-// inter-CTA synchronisation is needed:
-//   ZERO(slot)            S_slot = 0                 (a new open state)
-//   ADD(slot, t, cnt)     S_slot += v_s phi(k_s)^T   for cnt tokens from t
-//                         (Chlience section 5.1: the per-token state joins the
-//                          current state)
-//   MERGE(dst, src)       S_dst += S_src             (Chlience section 5.2)
-//   SHADOW(slot, ver)     version ver = S_slot, frozen for the readout
-//                         (fp32 copy, or bf16 in the tensor-core tile layout)
+// inter-CTA synchronisation is needed.  The open state lives in registers:
+//   ZERO(slot) / LOAD(slot)   the open state starts at 0 / from its slot
+//   ADD(slot, t, cnt)         open += v_s phi(k_s)^T for cnt tokens from t
+//                             (Chlience section 5.1: the per-token state joins
+//                             the current state)
+//   ADDP(slot, piece)         open += the tensor-core builder's piece
+//   STORE(slot, -, ver + 1)   S_slot = open (the state is sealed)
+//   MERGE(dst, src, ver + 1)  S_dst += S_src             (Chlience section 5.2)
+//   MERGEO(dst, -, ver + 1)   S_dst += open (the just-sealed state merges left)
+//   SHADOW(slot, ver)         version ver = S_slot (or the open registers)
+// A non-zero .w of STORE / MERGE / MERGEO also freezes the result as version
+// .w - 1 from registers (fp32 copy, or bf16 in the tensor-core tile layout).
 #include "dla_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -83,19 +87,25 @@ __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallA
 #pragma unroll
       for (int i = 0; i < PER; i += 4)
         *reinterpret_cast<float4 *>(Sa + i) = make_float4(open[i], open[i + 1], open[i + 2], open[i + 3]);
+      if (op.w > 0) shadow(op.w - 1, open);
       open_slot = -1;
-    } else if (op.x == OP_MERGE) {
+    } else if (op.x == OP_MERGE || op.x == OP_MERGEO) {
       const float *Sb = Sbase + (size_t)op.z * D * D + my;
+      float sum[PER];
 #pragma unroll
       for (int i = 0; i < PER; i += 4) {
-        float4 a = *reinterpret_cast<const float4 *>(Sa + i);
-        const float4 b = *reinterpret_cast<const float4 *>(Sb + i);
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-        *reinterpret_cast<float4 *>(Sa + i) = a;
+        const float4 a = *reinterpret_cast<const float4 *>(Sa + i);
+        float4 b;
+        if (op.x == OP_MERGE) b = *reinterpret_cast<const float4 *>(Sb + i);
+        else b = make_float4(open[i], open[i + 1], open[i + 2], open[i + 3]);
+        sum[i] = a.x + b.x;
+        sum[i + 1] = a.y + b.y;
+        sum[i + 2] = a.z + b.z;
+        sum[i + 3] = a.w + b.w;
+        *reinterpret_cast<float4 *>(Sa + i) = make_float4(sum[i], sum[i + 1], sum[i + 2], sum[i + 3]);
       }
+      if (op.w > 0) shadow(op.w - 1, sum);
+      if (op.x == OP_MERGEO) open_slot = -1;
     } else if (op.x == OP_SHADOW) {
       if (op.y == open_slot) {
         shadow(op.z, open);
