@@ -21,27 +21,51 @@ namespace dla {
 namespace {
 
 constexpr int THREADS = 256;
-constexpr int TOK = 32;  // tokens staged per ADD step
+constexpr int TOKC = 16;     // tokens per ADD chunk
+constexpr int OPBUF = 1024;  // ops staged in shared memory at a time
 
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Latency hiding: the op list is known before the replay, so the k / v rows
+// of the next ADD chunk (in op order, across ops) are always in flight into a
+// double-buffered raw staging area, and the next ADDP piece is preloaded into
+// registers.  Both are read-only inputs of this kernel, so reading them early
+// is safe.  The arithmetic per element is the same as a plain replay.
 template <int D, int R, bool BF16VER>
 __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallArgs ca) {
   constexpr int PER = R * D / THREADS;  // consecutive elements of one row per thread
   static_assert(R * D % THREADS == 0 && D % PER == 0 && PER % 4 == 0, "row block must split evenly");
-  constexpr int KPT = TOK * D / THREADS;  // k values staged per thread per chunk
-  constexpr int VPT = (TOK * R + THREADS - 1) / THREADS;
+  constexpr int RAW = TOKC * (D + R) * 4;  // k rows then v rows, fp32-sized
   const int u = blockIdx.y;
   const int r0 = blockIdx.x * R;
   const int tid = threadIdx.x;
   const int rr = (tid * PER) / D;  // row inside the block
   const int c0 = (tid * PER) % D;  // first column
-  __shared__ float s_phik[2][TOK][D];
-  __shared__ float s_v[2][TOK][R];
-  constexpr int OPBUF = 512;
+  __shared__ __align__(16) uint8_t s_raw[2][RAW];
+  __shared__ float s_phik[TOKC][D];
+  __shared__ float s_v[TOKC][R];
   __shared__ int4 s_ops[OPBUF];
   const int4 *ops = pl.ops + (size_t)u * dm.opsmax;
   const int nops = pl.nops[u];
   float *Sbase = ca.cache.S + (size_t)u * dm.C * D * D;
   const size_t my = (size_t)(r0 + rr) * D + c0;  // element offset inside a slot
+  const bool bf_in = ca.in_dtype == DLA_BF16;
+  const int esz = bf_in ? 2 : 4;
+  const uint8_t *kin = static_cast<const uint8_t *>(ca.k);
+  const uint8_t *vin = static_cast<const uint8_t *>(ca.v);
+  const size_t head_row0 = (size_t)u * dm.T + ca.w0;
+  const float *pieces = pl.pieces ? pl.pieces + (size_t)u * dm.pmax * D * D + my : nullptr;
   float open[PER];
   int open_slot = -1;
 #pragma unroll
@@ -61,11 +85,64 @@ __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallA
         *reinterpret_cast<float4 *>(Vd + i) = make_float4(src[i], src[i + 1], src[i + 2], src[i + 3]);
     }
   };
+
+  int staged_end = 0;  // ops [.., staged_end) are in s_ops
+  auto find_op = [&](int code, int from) -> int {
+    for (int i = from; i < staged_end; i++)
+      if (s_ops[i % OPBUF].x == code) return i;
+    return -1;
+  };
+  // ---- ADD chunks: (op, chunk) in flight ----
+  int inf_op = -1, inf_ch = 0, inf_buf = 0, next_buf = 0;
+  auto issue_chunk = [&](int oi, int ch) {
+    const int4 op = s_ops[oi % OPBUF];
+    const int nt = min(TOKC, op.w - ch * TOKC);
+    const size_t row0 = head_row0 + op.z + ch * TOKC;
+    const int kq = D * esz / 16, vq = R * esz / 16, per_tok = kq + vq;
+    uint8_t *dst = s_raw[next_buf];
+    for (int e = tid; e < nt * per_tok; e += THREADS) {
+      const int s = e / per_tok, w = e % per_tok;
+      if (w < kq)
+        cp_async16(dst + (size_t)s * D * esz + w * 16, kin + (row0 + s) * D * esz + w * 16);
+      else
+        cp_async16(dst + (size_t)TOKC * D * esz + (size_t)s * R * esz + (w - kq) * 16,
+                   vin + ((row0 + s) * D + r0) * esz + (w - kq) * 16);
+    }
+    cp_async_commit();
+    inf_op = oi;
+    inf_ch = ch;
+    inf_buf = next_buf;
+    next_buf ^= 1;
+  };
+  // ---- ADDP pieces: the next one preloaded in registers ----
+  float pfv[PER];
+  int pf_op = -1;
+  auto preload_piece = [&](int from) {
+    pf_op = find_op(OP_ADDP, from);
+    if (pf_op >= 0) {
+      const float *pc = pieces + (size_t)s_ops[pf_op % OPBUF].z * D * D;
+#pragma unroll
+      for (int i = 0; i < PER; i += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(pc + i);
+        pfv[i] = x.x;
+        pfv[i + 1] = x.y;
+        pfv[i + 2] = x.z;
+        pfv[i + 3] = x.w;
+      }
+    }
+  };
+
   for (int oi = 0; oi < nops; oi++) {
     if ((oi % OPBUF) == 0) {  // stage the next ops in shared memory
       __syncthreads();
-      for (int i = tid; i < OPBUF && oi + i < nops; i += THREADS) s_ops[i] = ops[oi + i];
+      staged_end = min(nops, oi + OPBUF);
+      for (int i = tid; i < staged_end - oi; i += THREADS) s_ops[i] = ops[oi + i];
       __syncthreads();
+      if (inf_op < 0) {
+        const int f = find_op(OP_ADD, oi);
+        if (f >= 0) issue_chunk(f, 0);
+      }
+      if (pf_op < 0 && pieces) preload_piece(oi);
     }
     const int4 op = s_ops[oi % OPBUF];
     float *Sa = Sbase + (size_t)op.y * D * D + my;
@@ -122,57 +199,46 @@ __global__ void __launch_bounds__(THREADS) k_materialize(Dims dm, Plan pl, CallA
         shadow(op.z, tmp);
       }
     } else if (op.x == OP_ADDP) {
-      const float *pc = pl.pieces + ((size_t)u * dm.pmax + op.z) * D * D + my;
+      if (pf_op != oi) preload_piece(oi);
 #pragma unroll
-      for (int i = 0; i < PER; i += 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(pc + i);
-        open[i] += x.x;
-        open[i + 1] += x.y;
-        open[i + 2] += x.z;
-        open[i + 3] += x.w;
-      }
+      for (int i = 0; i < PER; i++) open[i] += pfv[i];
+      preload_piece(oi + 1);
     } else {  // OP_ADD: tokens [op.z, op.z + op.w) of the window into the open state
-      const size_t row0 = (size_t)u * dm.T + ca.w0 + op.z;
-      const int nchunk = (op.w + TOK - 1) / TOK;
-      float kr[KPT], vr[VPT];
-      auto fetch = [&](int ch) {
-        const int nt = min(TOK, op.w - ch * TOK);
-#pragma unroll
-        for (int i = 0; i < KPT; i++) {
-          const int e = tid + THREADS * i, s = e / D, c = e % D;
-          kr[i] = s < nt ? load_in(ca.k, ca.in_dtype, (row0 + ch * TOK + s) * D + c) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < VPT; i++) {
-          const int e = tid + THREADS * i, s = e / R, r = e % R;
-          vr[i] = (e < TOK * R && s < nt) ? load_in(ca.v, ca.in_dtype, (row0 + ch * TOK + s) * D + r0 + r) : 0.f;
-        }
-      };
-      fetch(0);
+      const int nchunk = (op.w + TOKC - 1) / TOKC;
       for (int ch = 0; ch < nchunk; ch++) {
-        const int buf = ch & 1;
-#pragma unroll
-        for (int i = 0; i < KPT; i++) {
-          const int e = tid + THREADS * i;
-          s_phik[buf][e / D][e % D] = phi32(kr[i]);
+        if (inf_op != oi || inf_ch != ch) issue_chunk(oi, ch);
+        const int b = inf_buf;
+        cp_async_wait_all();
+        __syncthreads();  // chunk visible; the previous chunk's readers are done
+        inf_op = -1;
+        // the following chunk in op order goes in flight now
+        if (ch + 1 < nchunk) {
+          issue_chunk(oi, ch + 1);
+        } else {
+          const int f = find_op(OP_ADD, oi + 1);
+          if (f >= 0) issue_chunk(f, 0);
         }
-#pragma unroll
-        for (int i = 0; i < VPT; i++) {
-          const int e = tid + THREADS * i;
-          if (e < TOK * R) s_v[buf][e / R][e % R] = vr[i];
+        const int nt = min(TOKC, op.w - ch * TOKC);
+        const uint8_t *rk = s_raw[b];
+        const uint8_t *rv = s_raw[b] + (size_t)TOKC * D * esz;
+        for (int e = tid; e < nt * D; e += THREADS) {
+          const float x = bf_in ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(rk)[e] << 16)
+                                : reinterpret_cast<const float *>(rk)[e];
+          s_phik[e / D][e % D] = phi32(x);
         }
+        for (int e = tid; e < nt * R; e += THREADS)
+          s_v[e / R][e % R] = bf_in ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(rv)[e] << 16)
+                                    : reinterpret_cast<const float *>(rv)[e];
         __syncthreads();
-        if (ch + 1 < nchunk) fetch(ch + 1);
-        const int nt = min(TOK, op.w - ch * TOK);
         for (int s = 0; s < nt; s++) {
-          const float vv = s_v[buf][s][rr];
+          const float vv = s_v[s][rr];
 #pragma unroll
-          for (int i = 0; i < PER; i++) open[i] = fmaf(vv, s_phik[buf][s][c0 + i], open[i]);
+          for (int i = 0; i < PER; i++) open[i] = fmaf(vv, s_phik[s][c0 + i], open[i]);
         }
       }
-      __syncthreads();
     }
   }
+  cp_async_wait_all();
 }
 
 template <int D>
