@@ -49,16 +49,65 @@ def dist_env():
 
 
 class ClockSampler:
+    """SM clock and throttle reasons sampled during the timed region.
+
+    A background thread reads NVML (read-only queries) every 10 ms, plus one
+    sample at start and one at stop, so even a short timed region has several
+    samples; without NVML it falls back to ``nvidia-smi -lms 50``.
+    """
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.010
 
     def __init__(self, gpu_index):
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+
+    def _nvml_sample(self):
+        import pynvml as nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:  # older bindings
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.rows.append(dict(sm=float(sm), smax=float(self.smax),
+                              hw=bool(rs & 0x8), hwt=bool(rs & 0x40), swt=bool(rs & 0x20),
+                              pcap=bool(rs & 0x4)))
 
     def start(self):
+        self.rows = []
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            self.h = None
+            try:  # the physical GPU behind cuda:idx (CUDA_VISIBLE_DEVICES may remap)
+                import torch
+                uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+                self.h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = None
+            if self.h is None:
+                self.h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.smax = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.stop_evt = threading.Event()
+            self._nvml_sample()
+
+            def loop():
+                while not self.stop_evt.wait(self.PERIOD_S):
+                    try:
+                        self._nvml_sample()
+                    except Exception:
+                        return
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -66,31 +115,43 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
+        rows = self.rows
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=2)
             try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
+                self._nvml_sample()
+            except Exception:
+                pass
+            rows = self.rows
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     hw=parts[5].lower().startswith("active"),
+                                     hwt=parts[6].lower().startswith("active"),
+                                     swt=parts[7].lower().startswith("active"),
+                                     pcap=parts[8].lower().startswith("active")))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        else:
+            return None
         if not rows:
             return None
         smax = max(r["smax"] for r in rows)
@@ -99,10 +160,10 @@ class ClockSampler:
         for r in rows:
             for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
                               ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower().startswith("active"):
+                if r[key]:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(load), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- inputs ----

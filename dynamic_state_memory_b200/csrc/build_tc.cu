@@ -11,6 +11,10 @@
 // accumulator lives in TMEM; 4 warps (one TMEM lane = one row of d_v) write it
 // to the piece buffer, which the materializer adds to the open state (op
 // ADDP).  Shorter pieces stay SIMT adds in the materializer.
+//
+// Leaf mode (fixed Fenwick policy): the one piece is the whole tile and the
+// result is the tree leaf of that tile: fp32 state and phi(k) sum, plus the
+// frozen bf16 version (UMMA layout), its phi(k) sum and token count.
 #include "dla_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -23,6 +27,12 @@ constexpr int D = 128;
 constexpr int THREADS = 128;
 constexpr int TILE_BYTES = M * D * 2;
 constexpr int BLK = 2048;  // one 16-token block of one 64-column half
+
+struct FenLeaves {
+  float *treeS;  // [heads][nodes][D][D]; null: piece mode
+  float *treeZ;  // [heads][nodes][D]
+  int nodes;
+};
 
 struct Smem {
   uint8_t k[TILE_BYTES];     // phi(k), rows = tokens, MN-major for B
@@ -37,7 +47,7 @@ struct Smem {
 
 __global__ void __launch_bounds__(THREADS, 1)
     k_build_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-               Dims dm, Plan pl, CallArgs ca) {
+               Dims dm, Plan pl, CallArgs ca, FenLeaves fen) {
   extern __shared__ uint8_t raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                        ~static_cast<uintptr_t>(1023));
@@ -53,14 +63,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&sm.bar_mma, 1);
     fence_mbar_init();
     sm.abort = 0;
-    const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
-    const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
-    const bool cont = !(nev > 0 && evo[0] == 0);
-    int np = 0;
-    if (cont) sm.pst[np++] = 0;
-    for (int i = 0; i < nev; i++) sm.pst[np++] = evo[i];
-    for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
-    sm.np = np;
+    if (fen.treeS) {
+      sm.pst[0] = 0;
+      sm.pen[0] = len;
+      sm.np = 1;
+    } else {
+      const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
+      const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
+      const bool cont = !(nev > 0 && evo[0] == 0);
+      int np = 0;
+      if (cont) sm.pst[np++] = 0;
+      for (int i = 0; i < nev; i++) sm.pst[np++] = evo[i];
+      for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
+      sm.np = np;
+    }
     mbar_expect_tx(&sm.bar_load, 2 * TILE_BYTES);
     const int row = ca.w0 + T0;
     for (int h = 0; h < 2; h++) {
@@ -72,6 +88,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
   mbar_wait(&sm.bar_load, 0, abort);
+  if (fen.treeS) {
+    // leaf phi(k) sum in token order, from the raw tile (thread = column)
+    float z = 0.f;
+    for (int r = 0; r < len; r++) {
+      const uint16_t x = *reinterpret_cast<const uint16_t *>(sm.k + sw128_offset(r, tid, M));
+      z += phi32(__uint_as_float((uint32_t)x << 16));
+    }
+    const size_t node = (size_t)u * fen.nodes + c;
+    fen.treeZ[node * D + tid] = z;
+    pl.ver_z[((size_t)u * dm.vmax + c) * D + tid] = z;
+    if (tid == 0) pl.ver_n[(size_t)u * dm.vmax + c] = (float)len;
+    __syncthreads();
+  }
   for (int i = tid; i < TILE_BYTES / 16; i += THREADS) {
     uint4 *p = reinterpret_cast<uint4 *>(sm.k) + i;
     uint4 x = *p;
@@ -84,14 +113,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
 
   const int np = sm.np;
-  const int pbase = pl.tile_pbase[(size_t)u * dm.tiles + c];
-  float *pieces = pl.pieces + (size_t)u * dm.pmax * D * D;
+  const int pbase = fen.treeS ? c : pl.tile_pbase[(size_t)u * dm.tiles + c];
+  float *pieces = fen.treeS ? fen.treeS + (size_t)u * fen.nodes * D * D
+                            : pl.pieces + (size_t)u * dm.pmax * D * D;
   const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);
   int id = pbase;
   int phase = 0;
   for (int p = 0; p < np; p++) {
     const int a = sm.pst[p], b = sm.pen[p];
-    if (b - a < PIECE_MIN) continue;
+    if (b - a < PIECE_MIN && !fen.treeS) continue;
     const int jb0 = a >> 4, jb1 = (b - 1) >> 4;
     // masked copies of the straddling blocks (whole 128-byte rows zeroed)
     const bool edge0 = (a & 15) != 0 || (jb0 == jb1 && (b & 15) != 0);
@@ -133,6 +163,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int r = 32 * warp + (tid & 31);
       const uint32_t trow = tbase + ((uint32_t)(32 * warp) << 16);
       float4 *dst = reinterpret_cast<float4 *>(pieces + ((size_t)id * D + r) * D);
+      uint8_t *ver = fen.treeS ? static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + c) * D * D * 2
+                               : nullptr;
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t x[32];
         DLA_TMEM_LD32(trow + c0, x);
@@ -141,6 +173,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 8; i++)
           dst[c0 / 4 + i] = make_float4(__uint_as_float(x[4 * i]), __uint_as_float(x[4 * i + 1]),
                                         __uint_as_float(x[4 * i + 2]), __uint_as_float(x[4 * i + 3]));
+        if (ver) {
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            *reinterpret_cast<uint4 *>(ver + sw128_offset(r, c0 + 8 * i, D)) =
+                make_uint4(pack_bf16(__uint_as_float(x[8 * i]), __uint_as_float(x[8 * i + 1])),
+                           pack_bf16(__uint_as_float(x[8 * i + 2]), __uint_as_float(x[8 * i + 3])),
+                           pack_bf16(__uint_as_float(x[8 * i + 4]), __uint_as_float(x[8 * i + 5])),
+                           pack_bf16(__uint_as_float(x[8 * i + 6]), __uint_as_float(x[8 * i + 7])));
+        }
       }
     }
     tc_fence_before();
@@ -160,7 +201,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 bool make_bf16_map(CUtensorMap *m, const void *base, int T, int heads);
 
-cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+static cudaError_t launch_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, FenLeaves fen,
+                             int ntiles, cudaStream_t s) {
   if (dm.M != M || dm.D != D || ca.in_dtype != DLA_BF16) return cudaErrorInvalidValue;
   CUtensorMap tk, tv;
   if (!make_bf16_map(&tk, ca.k, dm.T, dm.heads) || !make_bf16_map(&tv, ca.v, dm.T, dm.heads))
@@ -168,8 +210,18 @@ cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, 
   const size_t sb = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_build_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
   if (e != cudaSuccess) return e;
-  k_build_tc<<<dim3(dm.tiles, dm.heads), THREADS, sb, s>>>(tk, tv, dm, pl, ca);
+  k_build_tc<<<dim3(ntiles, dm.heads), THREADS, sb, s>>>(tk, tv, dm, pl, ca, fen);
   return cudaGetLastError();
+}
+
+cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  return launch_tc(dm, pl, ca, FenLeaves{nullptr, nullptr, 0}, dm.tiles, s);
+}
+
+// Fixed-policy tree leaves of tiles [0, ntiles) (version id of a leaf = its tile).
+cudaError_t launch_fen_leaves_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
+                                 float *treeZ, int nodes, int ntiles, cudaStream_t s) {
+  return launch_tc(dm, pl, ca, FenLeaves{treeS, treeZ, nodes}, ntiles, s);
 }
 
 }  // namespace dla

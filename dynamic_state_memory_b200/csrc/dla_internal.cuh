@@ -134,6 +134,8 @@ cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &c
                                cudaStream_t s, bool bf16_versions);
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_fen_leaves_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
+                                 float *treeZ, int nodes, int ntiles, cudaStream_t s);
 void fen_tree_shape(int T, int M, int *nodes, int *levels);
 cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
                            float *treeZ, bool bf16, cudaStream_t s);

@@ -6,8 +6,8 @@
 // The structure does not depend on the data, so it is planned in parallel:
 //   - a readout tile starts at T0 = c * M (M a power of two), so the blocks of
 //     [0, T0 - 1] are whole-tile dyadic ranges: one tree node per set bit of c;
-//   - k_fen_leaves: per tile, the state sum S = sum v phi(k)^T, z = sum phi(k)
-//     (leaves of the tree);
+//   - leaves: per tile, the state sum S = sum v phi(k)^T, z = sum phi(k)
+//     (on the tensor cores for bf16 d = 128, else k_fen_leaves);
 //   - k_fen_level: node = left child + right child, level by level;
 //   every node is also written as a frozen version (fp32 or the bf16 UMMA
 //   layout) with its mean phi(k) and count;
@@ -161,7 +161,13 @@ template <int D>
 cudaError_t run_d(const Dims &dm, const Plan &pl, const CallArgs &ca, const FenTree &tr,
                   int ntiles, bool bf16, cudaStream_t s) {
   k_fen_plan<<<dim3((ntiles + 127) / 128, dm.heads), 128, 0, s>>>(dm, pl, tr, ntiles);
-  k_fen_leaves<D><<<dim3(ntiles, dm.heads), THREADS, 0, s>>>(dm, pl, ca, tr, ntiles, bf16);
+  if (bf16 && D == 128) {
+    // leaves on the tensor cores (tile state sums, phi(k) sums, bf16 versions)
+    const cudaError_t e = launch_fen_leaves_tc(dm, pl, ca, tr.S, tr.z, tr.nodes, ntiles, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    k_fen_leaves<D><<<dim3(ntiles, dm.heads), THREADS, 0, s>>>(dm, pl, ca, tr, ntiles, bf16);
+  }
   for (int l = 1; l < tr.levels; l++) {
     const int count = ntiles >> l;
     if (count <= 0) break;

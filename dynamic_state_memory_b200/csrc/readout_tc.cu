@@ -93,34 +93,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     sm.abort = 0;
   }
   if (dm.fenwick) {
-    // fixed policy: every token is a piece; at epoch p the in-tile states are
-    // the binary-counter blocks of pieces [0, p) (one per set bit of p, largest
-    // first) and {p}; every atom is its own block
-    const int len = min(M, ca.Tw - T0);
+    // fixed policy: the states of row o of the tile are the atoms (tree nodes
+    // of [0, T0)), the binary-counter blocks of [T0, T0 + o) (one per set
+    // bit of o) and {T0 + o}; the weight pass derives them from o directly
     if (tid == 0) {
       sm.m0 = m0;
-      sm.len = len;
-      sm.np = len;
-    }
-    for (int p = tid; p < len; p += THREADS) {
-      sm.pst[p] = p;
-      sm.pen[p] = p + 1;
-      uint32_t cur[BW];
-#pragma unroll
-      for (int w = 0; w < BW; w++)
-        cur[w] = m0 >= 32 * (w + 1) ? ~0u : (m0 > 32 * w ? (1u << (m0 - 32 * w)) - 1u : 0u);
-      int start = 0;
-      for (int b = 6; b >= 0; b--) {
-        if ((p >> b) & 1) {
-          start += 1 << b;
-          const int beta = m0 + start - 1;
-          cur[beta >> 5] |= 1u << (beta & 31);
-        }
-      }
-      const int beta = m0 + p;
-      cur[beta >> 5] |= 1u << (beta & 31);
-#pragma unroll
-      for (int w = 0; w < BW; w++) sm.bits[p * BW + w] = cur[w];
+      sm.len = min(M, ca.Tw - T0);
+      sm.np = 0;
     }
   } else if (warp == 2 && lane == 0) {
     // in-tile pieces and the state partition of each epoch
@@ -177,7 +156,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
   const int np = sm.np, len = sm.len;
-  if (tid < M) {  // piece of each row (rows past the tile's end take the last piece)
+  if (tid < M && !dm.fenwick) {  // piece of each row (rows past the tile's end take the last piece)
     int p = 0;
     while (p + 1 < np && sm.pst[p + 1] <= tid) p++;
     sm.pidx[tid] = p;
@@ -258,7 +237,101 @@ __global__ void __launch_bounds__(THREADS, 1)
   // merged once per chunk.  Pass B walks backwards and gives every atom /
   // piece the weight of the state it belongs to.  Piece values live in
   // registers when there are at most PREG pieces, else in TMEM cols [0, np).
-  if (warp >= 4 && warp < 8) {
+  if (dm.fenwick && warp >= 4 && warp < 8) {
+    // Row o: block sums of A[o][s] over the row's in-tile blocks (s < o lies
+    // in the block of size 2^p, p = the highest bit where s and o differ),
+    // one softmax over atoms, blocks and {o}, then P[o][s] = w(block) A[o][s].
+    const int qd = warp & 3;
+    const int t = 32 * qd + lane;
+    const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+    float bsum[7];
+#pragma unroll
+    for (int q = 0; q < 7; q++) bsum[q] = 0.f;
+    float aself = 0.f;
+#pragma unroll 1
+    for (int s0 = 0; s0 < M; s0 += 8) {
+      uint32_t ar[8];
+      DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int s = s0 + j;
+        const float x = __uint_as_float(ar[j]);
+        const int pb = 31 - __clz(s ^ t);
+#pragma unroll
+        for (int q = 0; q < 7; q++) bsum[q] += (s < t && pb == q) ? x : 0.f;
+        aself = s == t ? x : aself;
+      }
+    }
+    float lg[7];
+    float mx = aself * INV_SQRT_D;
+#pragma unroll
+    for (int q = 0; q < 7; q++) {
+      lg[q] = bsum[q] * (1.0f / (float)(1 << q)) * INV_SQRT_D;
+      if ((t >> q) & 1) mx = fmaxf(mx, lg[q]);
+    }
+#pragma unroll 1
+    for (int a0 = 0; a0 < m0; a0 += 8) {
+      uint32_t r[8];
+      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+        if (a0 + j < m0) mx = fmaxf(mx, __uint_as_float(r[j]) * INV_SQRT_D);
+    }
+    float l = __expf(aself * INV_SQRT_D - mx);
+#pragma unroll
+    for (int q = 0; q < 7; q++)
+      if ((t >> q) & 1) l += __expf(lg[q] - mx);
+#pragma unroll 1
+    for (int a0 = 0; a0 < m0; a0 += 8) {
+      uint32_t r[8];
+      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+        if (a0 + j < m0) l += __expf(__uint_as_float(r[j]) * INV_SQRT_D - mx);
+    }
+    const float inv_l = 1.0f / l;
+#pragma unroll 1
+    for (int a0 = 0; a0 < m0; a0 += 8) {
+      uint32_t r[8];
+      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+        r[j] = __float_as_uint(a0 + j < m0 ? __expf(__uint_as_float(r[j]) * INV_SQRT_D - mx) * inv_l : 0.f);
+      DLA_TMEM_ST8(trow + COL_W + a0, r);
+      tmem_wait_st();
+    }
+    float wb[7];
+#pragma unroll
+    for (int q = 0; q < 7; q++) wb[q] = ((t >> q) & 1) ? __expf(lg[q] - mx) * inv_l : 0.f;
+    const float wself = __expf(aself * INV_SQRT_D - mx) * inv_l;
+#pragma unroll 1
+    for (int s0 = 0; s0 < M; s0 += 8) {
+      uint32_t ar[8];
+      DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+      tmem_wait_ld();
+      uint32_t pk[4];
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        float v2[2];
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+          const int s = s0 + j + h;
+          const int pb = 31 - __clz(s ^ t);
+          float w = 0.f;
+#pragma unroll
+          for (int q = 0; q < 7; q++) w = (pb == q) ? wb[q] : w;
+          w = s < t ? w : (s == t ? wself : 0.f);
+          v2[h] = (s < len) ? w * __uint_as_float(ar[j + h]) : 0.f;
+        }
+        pk[j >> 1] = pack_bf16(v2[0], v2[1]);
+      }
+      *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  } else if (warp >= 4 && warp < 8) {
     constexpr int PREG = 8;
     const int qd = warp & 3;
     const int t = 32 * qd + lane;
