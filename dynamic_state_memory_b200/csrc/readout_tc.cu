@@ -509,13 +509,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
 
   // ---- P V, then the pipelined readout over atoms --------------------------
-  if (warp == 1 && lane == 0) {
-    tc_fence_after();
-    for (int k = 0; k < 8; k++)
-      mma_bf16(tbase + COL_AI, kdesc(kp_s, k), sdesc(v_s + k * 2048, TILE_BYTES / 2, 1024),
-               idesc_bf16(M, 128, 0, 1), k > 0);
-    mma_commit(&sm.bar_mma);
-    for (int a = 0; a < m0; a++) {
+  // Two issuing threads (warp 1: even atoms into TMEM buffer 0, warp 2: odd
+  // atoms into buffer 1).  An issuing thread is held for about the duration
+  // of its MMAs, so with one issuer every barrier wait left the tensor pipe
+  // idle; with two, one waits while the other's MMAs run.
+  auto issue_atoms = [&](int first) {
+    for (int a = first; a < m0; a += 2) {
       const int s = a % NST, b = a & 1;
       bool ok = mbar_wait(&sm.full[s], (a / NST) & 1, abort);
       if (a >= 2) ok = mbar_wait(&sm.tempty[b], ((a >> 1) - 1) & 1, abort) && ok;
@@ -528,6 +527,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_commit(&sm.empty[s]);
       mma_commit(&sm.tfull[b]);
     }
+  };
+  if (warp == 1 && lane == 0) {
+    tc_fence_after();
+    for (int k = 0; k < 8; k++)
+      mma_bf16(tbase + COL_AI, kdesc(kp_s, k), sdesc(v_s + k * 2048, TILE_BYTES / 2, 1024),
+               idesc_bf16(M, 128, 0, 1), k > 0);
+    mma_commit(&sm.bar_mma);
+    issue_atoms(0);
+  } else if (warp == 2 && lane == 0) {
+    tc_fence_after();
+    issue_atoms(1);
   } else if (warp == 0 && lane == 0) {
     for (int a = NST; a < m0; a++) {
       const int s = a % NST;
