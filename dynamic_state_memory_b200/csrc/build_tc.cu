@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint4 x = *p;
     uint32_t *w = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
-    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi32(bf16_lo(w[j])), phi32(bf16_hi(w[j])));
+    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi_bf16op(bf16_lo(w[j])), phi_bf16op(bf16_hi(w[j])));
     *p = x;
   }
   fence_proxy_async();

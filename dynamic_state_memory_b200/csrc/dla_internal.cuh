@@ -122,6 +122,9 @@ __device__ __forceinline__ void store_out(void *p, int32_t dtype, size_t i, floa
 // phi = elu + 1 in fp64 (decision summaries) and fp32 (states, readout).
 __device__ __forceinline__ double phi64(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
 __device__ __forceinline__ float phi32(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
+// phi for a value that is rounded to bf16 right away (tensor-core operands):
+// the fast exponential's error is far below bf16's half-ulp.
+__device__ __forceinline__ float phi_bf16op(float x) { return x > 0.0f ? x + 1.0f : __expf(x); }
 
 // Host launchers (one per kernel file).
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,

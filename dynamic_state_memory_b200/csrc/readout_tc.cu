@@ -15,10 +15,12 @@
 //   P = W o A (causal) as the bf16 A operand of
 //     O_intra = P V                                    TMEM cols [256, 384)
 //   Then, per atom alpha, a bulk copy brings the frozen bf16 state version
-//   (already stored in the UMMA K-major swizzled layout) into one of 3 shared
-//   stages, one thread issues P_alpha = phi(Q) S_alpha^T into one of two TMEM
-//   buffers (cols [0,128) / [128,256)), and 8 epilogue warps accumulate
-//   W_alpha(t) * P_alpha in registers while the next MMA runs.
+//   (already stored in the UMMA K-major swizzled layout) into one of 5 shared
+//   stages (3 of their own, then the k and v tiles once P V has read them),
+//   two threads issue P_alpha = phi(Q) S_alpha^T (even / odd atoms) into three
+//   TMEM buffers (cols [0,128), [128,256), then [256,384) once O_intra has been
+//   read out), and 8 epilogue warps, starting from O_intra, accumulate
+//   W_alpha(t) * P_alpha in registers while the next MMAs run.
 // Every wait on an mbarrier is bounded; a timeout sets DLA_ERR_TIMEOUT.
 #include "dla_internal.cuh"
 #include "tc_ptx.cuh"
@@ -29,12 +31,15 @@ using namespace tc;
 
 constexpr int M = 128;
 constexpr int D = 128;
-constexpr int NST = 3;
+constexpr int NST = 3;   // version stages of their own
+constexpr int NSV = 5;   // + the k and v tiles once P V has read them
 constexpr int THREADS = 384;
 constexpr int TILE_BYTES = M * D * 2;
 constexpr uint32_t VER_BYTES = D * D * 2;
 constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
 constexpr uint32_t COL_BUF0 = 0, COL_AI = 256, COL_W = 384;
+constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and, once its intra-tile
+                        // output has been read, [256,384)
 constexpr float INV_SQRT_D = 0.08838834764831845f;
 
 struct Smem {
@@ -42,7 +47,7 @@ struct Smem {
   uint8_t kp[TILE_BYTES];
   uint8_t v[TILE_BYTES];
   uint8_t st[NST][VER_BYTES];
-  uint64_t bar_load, bar_mma, full[NST], empty[NST], tfull[2], tempty[2];
+  uint64_t bar_load, bar_mma, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
   uint32_t tmem_base;
   int abort;
   int m0, np, len;
@@ -65,6 +70,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (T0 >= ca.Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
+  auto stage = [&](int s) -> uint8_t * { return s < NST ? sm.st[s] : (s == NST ? sm.kp : sm.v); };
   const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
 
   // ---- setup: TMEM, barriers, tile metadata ------------------------------
@@ -81,11 +87,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
     mbar_init(&sm.bar_mma, 1);
-    for (int i = 0; i < NST; i++) {
+    for (int i = 0; i < NSV; i++) {
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
     }
-    for (int i = 0; i < 2; i++) {
+    for (int i = 0; i < NPB; i++) {
       mbar_init(&sm.tfull[i], 1);
       mbar_init(&sm.tempty[i], 8);
     }
@@ -184,7 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint4 x = *p;
     uint32_t *w = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
-    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi32(bf16_lo(w[j])), phi32(bf16_hi(w[j])));
+    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi_bf16op(bf16_lo(w[j])), phi_bf16op(bf16_hi(w[j])));
     *p = x;
   }
   const int n_mu = (m0 + 15) & ~15;
@@ -509,18 +515,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
 
   // ---- P V, then the pipelined readout over atoms --------------------------
-  // Two issuing threads (warp 1: even atoms into TMEM buffer 0, warp 2: odd
-  // atoms into buffer 1).  An issuing thread is held for about the duration
-  // of its MMAs, so with one issuer every barrier wait left the tensor pipe
-  // idle; with two, one waits while the other's MMAs run.
+  // Two issuing threads (warp 1: even atoms, warp 2: odd atoms); an issuing
+  // thread is held for about the duration of its MMAs, so with one issuer
+  // every barrier wait left the tensor pipe idle.  Atom a goes to TMEM buffer
+  // a % 3; the third buffer is the intra-tile output's columns, handed over
+  // once the epilogue has folded that output into its registers.  Three
+  // buffers cover the commit -> drain -> release round trip of a buffer.
   auto issue_atoms = [&](int first) {
     for (int a = first; a < m0; a += 2) {
-      const int s = a % NST, b = a & 1;
-      bool ok = mbar_wait(&sm.full[s], (a / NST) & 1, abort);
-      if (a >= 2) ok = mbar_wait(&sm.tempty[b], ((a >> 1) - 1) & 1, abort) && ok;
+      const int s = a % NSV, b = a % NPB;
+      bool ok = mbar_wait(&sm.full[s], (a / NSV) & 1, abort);
+      if (b == NPB - 1) ok = mbar_wait(&sm.tempty[b], (a / NPB) & 1, abort) && ok;
+      else if (a >= NPB) ok = mbar_wait(&sm.tempty[b], ((a / NPB) - 1) & 1, abort) && ok;
       tc_fence_after();
       if (ok) {
-        const uint32_t st_s = smem_u32(sm.st[s]);
+        const uint32_t st_s = smem_u32(stage(s));
         for (int k = 0; k < 8; k++)
           mma_bf16(tbase + b * 128, kdesc(q_s, k), kdesc(st_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
       }
@@ -539,24 +548,49 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     issue_atoms(1);
   } else if (warp == 0 && lane == 0) {
+    // L2 prefetch PF atoms ahead of the stage loads: versions were just
+    // written by the materializer, so a head's first tiles mostly miss L2
+    constexpr int PF = 6;
+    for (int a = NST; a < m0 && a < NST + PF; a++)
+      bulk_prefetch_l2(verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES);
     for (int a = NST; a < m0; a++) {
-      const int s = a % NST;
-      if (!mbar_wait(&sm.empty[s], ((a / NST) - 1) & 1, abort)) break;
+      if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)sm.atom[a + PF] * VER_BYTES, VER_BYTES);
+      const int s = a % NSV;
+      // stages NST.. are the k / v tiles: free once P V has completed
+      // (bar_mma phase 1; phase 0, the first MMAs, completed before here)
+      const bool ok = a < NSV ? mbar_wait(&sm.bar_mma, 1, abort)
+                              : mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort);
+      if (!ok) break;
       mbar_expect_tx(&sm.full[s], VER_BYTES);
-      bulk_load(sm.st[s], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
+      bulk_load(stage(s), verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
     }
   } else if (warp >= 4) {
     const int qd = warp & 3, hc = (warp - 4) >> 2;
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     float acc[64];
+    // start from the intra-tile output, then release its columns as buffer 2
+    mbar_wait(&sm.bar_mma, 1, abort);
+    tc_fence_after();
+    {
+      uint32_t pr[32];
+      DLA_TMEM_LD32(trow + COL_AI + hc * 64, pr);
+      tmem_wait_ld();
 #pragma unroll
-    for (int i = 0; i < 64; i++) acc[i] = 0.f;
+      for (int i = 0; i < 32; i++) acc[i] = __uint_as_float(pr[i]);
+      DLA_TMEM_LD32(trow + COL_AI + hc * 64 + 32, pr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i++) acc[32 + i] = __uint_as_float(pr[i]);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.tempty[NPB - 1]);
 #pragma unroll 1
     for (int a = 0; a < m0; a++) {
-      const int b = a & 1;
+      const int b = a % NPB;
       const float w = __uint_as_float(tmem_ld1(trow + COL_W + a));
-      mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
+      mbar_wait(&sm.tfull[b], (a / NPB) & 1, abort);
       tc_fence_after();
       uint32_t pr[32];
       DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
@@ -570,19 +604,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tempty[b]);
-    }
-    mbar_wait(&sm.bar_mma, 1, abort);
-    tc_fence_after();
-    {
-      uint32_t pr[32];
-      DLA_TMEM_LD32(trow + COL_AI + hc * 64, pr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i++) acc[i] += __uint_as_float(pr[i]);
-      DLA_TMEM_LD32(trow + COL_AI + hc * 64 + 32, pr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i++) acc[32 + i] += __uint_as_float(pr[i]);
     }
     if (t < len) {
       uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(ca.o) +
