@@ -7,7 +7,7 @@
 //              predecessor are low-information; Chlience section 5.1: b_t = 1
 //              opens a new state).
 //   k_segscan  window pieces: {0} and every boundary t > 0 (warp ballots).
-//   k_tilesum  per (tile, head): fp64 sum of phi(k) over each run of a piece
+//   k_tilesum_*  per (tile, head): fp64 sum of phi(k) over each run of a piece
 //              inside the tile, in token order.
 //   k_segcombine  per piece: the runs' sums in time order (after the cached
 //              open state's z for a continuation) give z at the piece's end
@@ -151,10 +151,6 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
 }
 
 // phi(x) in fp64 for every bf16 bit pattern (same exp as inline evaluation).
-__global__ void k_phi_table(double *tab) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < 65536) tab[i] = phi64((double)__uint_as_float((uint32_t)i << 16));
-}
 
 // Pieces of the window: seg_start = {0} and every t > 0 with b_t = 1.
 __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
@@ -200,7 +196,71 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
 // segment spans; the association differs from a strict token-order sum by
 // rounding only (merge choices are then the same unless two Ward losses tie
 // to within rounding).
-__global__ void k_tilesum(Dims dm, Plan pl, CallArgs ca) {
+// phi of a bf16 input in fp64.  Negative inputs need exp: those with a
+// biased exponent in [PHI_E0, PHI_E0 + PHI_NE) (|x| in [2^-24, 16)) come from
+// a table filled with the same exp() per call; other negatives call exp().
+constexpr int PHI_E0 = 103, PHI_NE = 28, PHI_TAB = PHI_NE * 128;
+
+__global__ void k_phi_table(double *tab) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < PHI_TAB) {
+    const uint32_t bits = 0x8000u | ((uint32_t)(PHI_E0 + i / 128) << 7) | (uint32_t)(i % 128);
+    tab[i] = phi64((double)__uint_as_float(bits << 16));
+  }
+}
+
+__device__ __forceinline__ double phi_bf16_f64(uint32_t bits, const double *s_tab) {
+  const float x = __uint_as_float(bits << 16);
+  if (!(bits & 0x8000u)) return (double)x + 1.0;  // x >= +0 (phi(+0) = 1 either way)
+  const uint32_t e = ((bits >> 7) & 0xFFu) - PHI_E0;
+  return e < (uint32_t)PHI_NE ? s_tab[e * 128 + (bits & 127u)] : phi64((double)x);
+}
+
+__device__ __forceinline__ void cp_async16_cg(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
+// bf16 path: the tile's k rows, the phi table and the boundary flags are
+// staged in shared memory with asynchronous copies (one wait), then thread c
+// runs the fp64 chain of dimension c from shared memory.
+template <int D>
+__global__ void __launch_bounds__(D) k_tilesum_bf16(Dims dm, Plan pl, CallArgs ca) {
+  constexpr int M = 128;
+  extern __shared__ __align__(16) unsigned char ts_raw[];
+  double *s_tab = reinterpret_cast<double *>(ts_raw);                    // PHI_TAB
+  uint16_t *s_k = reinterpret_cast<uint16_t *>(ts_raw + PHI_TAB * 8);    // M x D
+  uint8_t *s_b = ts_raw + PHI_TAB * 8 + M * D * 2;                       // M
+  const int u = blockIdx.y, tile = blockIdx.x;
+  const int c = threadIdx.x;
+  const int T0 = tile * M;
+  if (T0 >= ca.Tw) return;
+  const int T1 = min(T0 + M, ca.Tw), len = T1 - T0;
+  const uint16_t *kg = static_cast<const uint16_t *>(ca.k) + ((size_t)u * dm.T + ca.w0 + T0) * D;
+  for (int i = c; i < len * D / 8; i += D) cp_async16_cg(s_k + 8 * i, kg + 8 * i);
+  for (int i = c; i < PHI_TAB / 2; i += D) cp_async16_cg(s_tab + 2 * i, pl.phi_tab + 2 * i);
+  for (int i = c; i < len; i += D) s_b[i] = pl.b[(size_t)u * dm.W + T0 + i];
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  double *zp = pl.z_part + (size_t)u * dm.W * D + c;
+  double z = 0.0;
+  int part = T0;
+#pragma unroll 4
+  for (int i = 0; i < len; i++) {
+    if (i > 0 && s_b[i]) {
+      zp[(size_t)part * D] = z;
+      part = T0 + i;
+      z = 0.0;
+    }
+    z = __dadd_rn(z, phi_bf16_f64(s_k[i * D + c], s_tab));
+  }
+  zp[(size_t)part * D] = z;
+}
+
+// Other inputs (fp32, or tiles other than 128 rows): direct loads, phi64.
+__global__ void k_tilesum_any(Dims dm, Plan pl, CallArgs ca) {
   const int u = blockIdx.y, tile = blockIdx.x;
   const int c = threadIdx.x;  // dimension
   const int D = dm.D, M = dm.M;
@@ -210,30 +270,15 @@ __global__ void k_tilesum(Dims dm, Plan pl, CallArgs ca) {
   const uint8_t *b = pl.b + (size_t)u * dm.W;
   const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
   double *zp = pl.z_part + (size_t)u * dm.W * D + c;
-  const double *__restrict__ tab = pl.phi_tab;
-  constexpr int CH = 16;
   double z = 0.0;
   int part = T0;
-  for (int s0 = T0; s0 < T1; s0 += CH) {
-    double ph[CH];
-#pragma unroll
-    for (int i = 0; i < CH; i++) {
-      const int s = s0 + i;
-      const float x = s < T1 ? load_in(ca.k, ca.in_dtype, kb + (size_t)s * D) : 0.f;
-      ph[i] = tab ? __ldg(tab + (__float_as_uint(x) >> 16)) : phi64((double)x);
+  for (int s = T0; s < T1; s++) {
+    if (s > T0 && b[s]) {
+      zp[(size_t)part * D] = z;
+      part = s;
+      z = 0.0;
     }
-#pragma unroll
-    for (int i = 0; i < CH; i++) {
-      const int s = s0 + i;
-      if (s < T1) {
-        if (s > T0 && b[s]) {
-          zp[(size_t)part * D] = z;
-          part = s;
-          z = 0.0;
-        }
-        z = __dadd_rn(z, ph[i]);
-      }
-    }
+    z = __dadd_rn(z, phi64((double)load_in(ca.k, ca.in_dtype, kb + (size_t)s * D)));
   }
   zp[(size_t)part * D] = z;
 }
@@ -769,18 +814,35 @@ cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int
   return cudaGetLastError();
 }
 
-cudaError_t launch_phi_table(double *tab, cudaStream_t s) {
-  k_phi_table<<<256, 256, 0, s>>>(tab);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   k_segscan<<<dm.heads, 1024, 0, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }
 
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  k_tilesum<<<dim3(dm.tiles, dm.heads), dm.D, 0, s>>>(dm, pl, ca);
+  const dim3 g(dm.tiles, dm.heads);
+  if (ca.in_dtype == DLA_BF16 && dm.M == 128) {
+    k_phi_table<<<(PHI_TAB + 255) / 256, 256, 0, s>>>(pl.phi_tab);
+    const size_t sb = PHI_TAB * 8 + 128 * (size_t)dm.D * 2 + 128;
+    cudaError_t e = cudaSuccess;
+    switch (dm.D) {
+      case 32:
+        e = cudaFuncSetAttribute(k_tilesum_bf16<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+        if (e == cudaSuccess) k_tilesum_bf16<32><<<g, 32, sb, s>>>(dm, pl, ca);
+        break;
+      case 64:
+        e = cudaFuncSetAttribute(k_tilesum_bf16<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+        if (e == cudaSuccess) k_tilesum_bf16<64><<<g, 64, sb, s>>>(dm, pl, ca);
+        break;
+      default:
+        e = cudaFuncSetAttribute(k_tilesum_bf16<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+        if (e == cudaSuccess) k_tilesum_bf16<128><<<g, 128, sb, s>>>(dm, pl, ca);
+        break;
+    }
+    if (e != cudaSuccess) return e;
+  } else {
+    k_tilesum_any<<<g, dm.D, 0, s>>>(dm, pl, ca);
+  }
   k_segcombine<<<dim3(64, dm.heads), dm.D, 0, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }

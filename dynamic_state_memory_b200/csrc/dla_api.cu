@@ -92,8 +92,8 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
   pl.slot_ver = cv.take<int32_t>(h * dm.C);
   pl.tile_pbase = cv.take<int32_t>(h * dm.tiles);
-  pl.phi_tab = cv.take<double>(65536);
   pl.pieces = cv.take<float>(h * (size_t)dm.pmax * dm.D * dm.D);
+  pl.phi_tab = cv.take<double>(4096);
 }
 
 // Fixed Fenwick policy: one pass over the call (no windows); versions are the
@@ -262,11 +262,6 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     memset(&ca.trace, 0, sizeof ca.trace);
   }
   ca.dev_status = dev_status;
-  if (cfg->in_dtype == DLA_BF16) {
-    if (launch_phi_table(pl.phi_tab, s) != cudaSuccess) return DLA_ERR_CUDA;
-  } else {
-    pl.phi_tab = nullptr;
-  }
   for (int w0 = 0; w0 < cfg->T; w0 += dm.W) {
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;

@@ -82,8 +82,8 @@ struct Plan {
   void *ver_S;         // [heads][vmax] versions (fp32 [D][D] or bf16 tiled)
   int32_t *slot_ver;   // [heads][C] engine scratch
   int32_t *tile_pbase; // [heads][tiles] first piece id of each tile
+  double *phi_tab;     // phi in fp64 of negative bf16 inputs of moderate magnitude
   float *pieces;       // [heads][pmax][D][D] fp32 piece states
-  double *phi_tab;     // [65536] phi(x) in fp64 for every bf16 bit pattern (or null)
 };
 
 struct CallArgs {
@@ -130,7 +130,6 @@ __device__ __forceinline__ float phi_bf16op(float x) { return x > 0.0f ? x + 1.0
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
                          cudaStream_t s);
 cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
-cudaError_t launch_phi_table(double *tab, cudaStream_t s);
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
