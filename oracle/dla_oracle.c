@@ -194,6 +194,7 @@ typedef struct {
   int dtype;
   const void *q, *k, *v; /* [nrun][T][d] */
   double *out;           /* [nrun][T][dv] or NULL */
+  const uint8_t *out_mask; /* [T]: read out only where set (NULL: every token) */
   uint8_t *boundary;     /* [nrun][T] or NULL */
   int32_t *merge_t, *merge_i, *merge_count; /* [nrun][cap], [nrun] */
   int cap;
@@ -310,7 +311,7 @@ static void run_head_dla(job *J, int r) {
     for (int i = 0; i < hd->nsealed; i++) lst[m++] = &hd->sealed[i];
     lst[m++] = &hd->open;
     if (J->live) J->live[(size_t)r * T + tl] = m;
-    if (J->out) {
+    if (J->out && (!J->out_mask || J->out_mask[tl])) {
       for (int c = 0; c < dk; c++) p[c] = phi(widen(J->q, J->dtype, base + c));
       readout(o, lst, m, p, J->out + ((size_t)r * T + tl) * dv);
     }
@@ -359,7 +360,7 @@ static void run_head_fenwick(job *J, int r) {
     for (int i = 0; i < hd->nsealed; i++) lst[m++] = &hd->sealed[i];
     lst[m++] = &hd->open;
     if (J->live) J->live[(size_t)r * T + tl] = m;
-    if (J->out) {
+    if (J->out && (!J->out_mask || J->out_mask[tl])) {
       for (int c = 0; c < dk; c++) p[c] = phi(widen(J->q, J->dtype, base + c));
       readout(o, lst, m, p, J->out + ((size_t)r * T + tl) * dv);
     }
@@ -396,12 +397,14 @@ static void *worker(void *arg) {
 
 /* Run T tokens for heads [head_lo, head_hi).  Inputs are [nrun][T][d] in
  * `dtype`; outputs (all optional) are indexed by the run-local head r.
- * `out` needs the oracle created with want_S = 1.  Returns 0 on success. */
-int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
-                   const void *q, const void *k, const void *v, double *out,
-                   uint8_t *boundary, int32_t *merge_t, int32_t *merge_i,
-                   int32_t *merge_count, int cap, int32_t *live, double *margins,
-                   int nthreads) {
+ * `out` needs the oracle created with want_S = 1; with `out_mask` the readout
+ * runs only at tokens whose mask entry is set (states are updated at every
+ * token either way).  Returns 0 on success. */
+int dla_oracle_run_masked(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+                          const void *q, const void *k, const void *v, double *out,
+                          const uint8_t *out_mask, uint8_t *boundary, int32_t *merge_t,
+                          int32_t *merge_i, int32_t *merge_count, int cap, int32_t *live,
+                          double *margins, int nthreads) {
   if (!o || head_lo < 0 || head_hi > o->nheads || head_lo > head_hi || T < 0) return 1;
   if (out && (!o->want_S || !q || !v)) return 2;
   if (!k) return 3;
@@ -417,6 +420,7 @@ int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int d
   J.k = k;
   J.v = v;
   J.out = out;
+  J.out_mask = out_mask;
   J.boundary = boundary;
   J.merge_t = merge_t;
   J.merge_i = merge_i;
@@ -441,6 +445,16 @@ int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int d
   pthread_mutex_destroy(&J.mu);
   free(mc_local);
   return 0;
+}
+
+/* Same, reading out at every token. */
+int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+                   const void *q, const void *k, const void *v, double *out,
+                   uint8_t *boundary, int32_t *merge_t, int32_t *merge_i,
+                   int32_t *merge_count, int cap, int32_t *live, double *margins,
+                   int nthreads) {
+  return dla_oracle_run_masked(o, head_lo, head_hi, T, tau, dtype, q, k, v, out, NULL, boundary,
+                               merge_t, merge_i, merge_count, cap, live, margins, nthreads);
 }
 
 /* Live states of one head in time order (sealed..., open).  Returns m and

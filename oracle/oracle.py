@@ -44,6 +44,10 @@ def load_library(path: str):
     lib.dla_oracle_run.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
                                    P, ctypes.c_int, P, P, ctypes.c_int]
+    lib.dla_oracle_run_masked.restype = ctypes.c_int
+    lib.dla_oracle_run_masked.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
+                                          P, P, ctypes.c_int, P, P, ctypes.c_int]
     lib.dla_oracle_state.restype = ctypes.c_int
     lib.dla_oracle_state.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
     return lib
@@ -84,10 +88,13 @@ class Oracle:
             self.h = None
 
     def run(self, k, q=None, v=None, *, tau: float, dtype: str, head_lo: int = 0,
-            want_out: bool = True, cap: int | None = None, nthreads: int | None = None):
+            want_out: bool = True, cap: int | None = None, nthreads: int | None = None,
+            out_mask=None):
         """Run T tokens for heads [head_lo, head_lo + k.shape[0]).
 
         k, q, v: arrays [nrun, T, d] (float32, float64 or bf16 uint16 bits).
+        ``out_mask`` ([T] bool) limits the readout to the marked tokens (rows
+        elsewhere stay zero); states are updated at every token regardless.
         Returns dict with out [nrun, T, d_v] (fp64 or None), boundary
         [nrun, T] u8, merges as lists of (t, i) per head, live [nrun, T] and
         margins [nrun, 3] (min |r - tau|, min Ward relative gap, exact ties).
@@ -110,10 +117,14 @@ class Oracle:
         margins[:, 0] = np.inf
         margins[:, 1] = np.inf
         nthreads = cores() if nthreads is None else nthreads
-        rc = self.lib.dla_oracle_run(self.h, head_lo, head_lo + nrun, T, float(tau),
-                                     DTYPES[dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                                     _ptr(boundary), _ptr(mt), _ptr(mi), _ptr(mc), cap,
-                                     _ptr(live), _ptr(margins), nthreads)
+        if out_mask is not None:
+            out_mask = np.ascontiguousarray(out_mask, dtype=np.uint8)
+            if out_mask.shape != (T,):
+                raise ValueError("out_mask must have shape [T]")
+        rc = self.lib.dla_oracle_run_masked(self.h, head_lo, head_lo + nrun, T, float(tau),
+                                            DTYPES[dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                            _ptr(out_mask), _ptr(boundary), _ptr(mt), _ptr(mi),
+                                            _ptr(mc), cap, _ptr(live), _ptr(margins), nthreads)
         if rc != 0:
             raise RuntimeError(f"dla_oracle_run failed with code {rc}")
         merges = [list(zip(mt[r, :min(mc[r], cap)].tolist(), mi[r, :min(mc[r], cap)].tolist()))

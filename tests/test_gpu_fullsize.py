@@ -1,0 +1,155 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times (default windows and tiles, every stream of the workload).
+
+- Decision traces (boundary flags, merge tokens and indices) of every stream
+  are compared bit for bit with the fp64 oracle run in trace-only mode.
+- Outputs of sampled streams are compared at sampled tokens (random ones plus
+  every tile's first and last token and the sequence end) with the oracle's
+  masked readout, which updates states at every token and reads out only at
+  the sampled ones.  The bf16 tolerance is 2e-2 of max|o| over the compared
+  set.
+"""
+import numpy as np
+import pytest
+
+from dynamic_state_memory_b200 import synth
+from oracle import oracle as O
+from tests.gpu_helpers import TOL, from_device, gen_decode_parallel, gen_prefill_parallel, to_device
+
+pytestmark = pytest.mark.gpu
+
+TILE = 128
+
+
+def sample_mask(T, seed, n=384):
+    rng = np.random.default_rng(seed)
+    idx = set(rng.choice(T, size=min(n, T), replace=False).tolist())
+    idx |= {0, T - 1}
+    idx |= set(range(0, T, TILE)) | set(range(TILE - 1, T, TILE))
+    mask = np.zeros(T, dtype=np.uint8)
+    mask[sorted(idx)] = 1
+    return mask
+
+
+def oracle_sampled(q, k, v, C, tau, policy, mask):
+    """Oracle outputs of one stream at the masked tokens."""
+    T, d = k.shape
+    orc = O.Oracle(1, d, d, C, policy)
+    res = orc.run(k[None], q[None], v[None], tau=tau, dtype="bf16", out_mask=mask)
+    return res["out"][0][mask.astype(bool)]
+
+
+def check_outputs(o, q, k, v, C, tau, policy, heads, seed):
+    T = k.shape[2]
+    mask = sample_mask(T, seed)
+    for (b, h) in heads:
+        ref = oracle_sampled(q[b, h], k[b, h], v[b, h], C, tau, policy, mask)
+        got = o[b, h][mask.astype(bool)]
+        err = float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+        assert err <= TOL["bf16"], (policy, b, h, err)
+
+
+def check_trace(tr, k, C, tau):
+    B, H, T, d = k.shape
+    orc = O.Oracle(B * H, d, d, C, want_S=False)
+    res = orc.run(k.reshape(B * H, T, d), tau=tau, dtype="bf16", want_out=False)
+    gap = float(res["margins"][:, 1].min())
+    assert np.array_equal(tr.boundary.cpu().numpy().reshape(B * H, T), res["boundary"]), gap
+    assert tr.merges() == res["merges"], gap
+
+
+def gpu_prefill(q, k, v, C, tau):
+    import torch
+    from dynamic_state_memory_b200 import dla
+    B, H, T, d = k.shape
+    cache = dla.Cache(B, H, C, d)
+    o, tr = dla.prefill(to_device(q, "bf16"), to_device(k, "bf16"), to_device(v, "bf16"), cache, tau)
+    torch.cuda.synchronize()
+    return from_device(o), tr
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("prefill_t8192", [(0, 0), (3, 15)]),
+    ("prefill_t131072", [(0, 0), (0, 11)]),
+])
+def test_prefill_full_size(gpu, name, heads):
+    wl = synth.WORKLOADS[name]
+    q, k, v = gen_prefill_parallel(wl)
+    o, tr = gpu_prefill(q, k, v, wl["C"], wl["tau"])
+    check_trace(tr, k, wl["C"], wl["tau"])
+    check_outputs(o, q, k, v, wl["C"], wl["tau"], "dla", heads, wl["seed"])
+
+
+def test_fixed_policy_full_size(gpu):
+    """Fixed Fenwick policy and, on the same inputs, DLA at C = 16."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    wl = synth.WORKLOADS["fixed_t32768"]
+    q, k, v = gen_prefill_parallel(wl)
+    o = dla.fixed_policy_prefill(to_device(q, "bf16"), to_device(k, "bf16"), to_device(v, "bf16"))
+    torch.cuda.synchronize()
+    check_outputs(from_device(o), q, k, v, 64, 0.0, "fenwick", [(0, 0), (1, 15)], wl["seed"])
+    od, tr = gpu_prefill(q, k, v, wl["C"], wl["tau"])
+    check_trace(tr, k, wl["C"], wl["tau"])
+    check_outputs(od, q, k, v, wl["C"], wl["tau"], "dla", [(1, 3)], wl["seed"] + 1)
+
+
+def test_decode_full_size(gpu):
+    """All 256 x 16 streams pre-filled with 4096 tokens (as the benchmark does),
+    then decode steps; every stream's decisions checked in the prefill and at
+    every step, sampled streams' outputs at every step."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    wl = synth.WORKLOADS["decode_n256"]
+    steps = 8
+    (pq, pk, pv), (sq, sk, sv) = gen_decode_parallel(wl, steps)
+    N, H, T, d = pk.shape
+    C, tau = wl["C"], wl["tau"]
+    cache = dla.Cache(N, H, C, d)
+    # pre-fill the cache as the benchmark does: 8 sequences per call, 1024-token windows
+    chunk = 8
+    cfg = dla.make_config(chunk, H, T, d, C, tau, dla.DLA_BF16, 1024)
+    ws = torch.empty(dla.dla_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pre_bnd, pre_mrg = [], []
+    for n0 in range(0, N, chunk):
+        qq, kk, vv = (to_device(np.ascontiguousarray(x[n0:n0 + chunk]), "bf16") for x in (pq, pk, pv))
+        o = torch.empty_like(qq)
+        tr = dla.Trace(chunk * H, T, T + 1)
+        dla.dla_prefill(cfg, qq, kk, vv, o, cache.sub(n0, n0 + chunk), tr.c, ws, st)
+        torch.cuda.synchronize()
+        dla.check_device_status(st, "prefill of the decode cache")
+        pre_bnd.append(tr.boundary.cpu().numpy().reshape(chunk * H, T))
+        pre_mrg += tr.merges()
+    del ws
+    dec = dla.Decoder(cache)
+    outs, bnd, mrg = [], [], []
+    for s in range(steps):
+        o = dec.step(to_device(sq[s], "bf16"), to_device(sk[s], "bf16"), to_device(sv[s], "bf16"), tau)
+        torch.cuda.synchronize()
+        dla.check_device_status(dec.status, "decode")
+        outs.append(from_device(o))
+        bnd.append(dec.boundary.cpu().numpy().copy())
+        mrg.append(dec.merge_i.cpu().numpy().copy())
+    # decisions of every stream: prefill trace, then one token per step
+    orc = O.Oracle(N * H, d, d, C, want_S=False)
+    res = orc.run(pk.reshape(N * H, T, d), tau=tau, dtype="bf16", want_out=False)
+    assert np.array_equal(np.concatenate(pre_bnd), res["boundary"])
+    assert pre_mrg == res["merges"]
+    for s in range(steps):
+        r1 = orc.run(np.ascontiguousarray(sk[s].reshape(N * H, 1, d)), tau=tau, dtype="bf16",
+                     want_out=False)
+        assert np.array_equal(bnd[s], r1["boundary"][:, 0]), s
+        want = np.array([m[0][1] if m else -1 for m in r1["merges"]], dtype=np.int32)
+        assert np.array_equal(mrg[s], want), s
+    # outputs of sampled streams at every step
+    for (n, h) in [(0, 0), (255, 15), (97, 6)]:
+        ref_o = O.Oracle(1, d, d, C)
+        ref_o.run(pk[n, h][None], pq[n, h][None], pv[n, h][None], tau=tau, dtype="bf16",
+                  out_mask=np.zeros(T, dtype=np.uint8))
+        ref = np.stack([ref_o.run(sk[s, n, h][None, None], sq[s, n, h][None, None],
+                                  sv[s, n, h][None, None], tau=tau, dtype="bf16")["out"][0, 0]
+                        for s in range(steps)])
+        got = np.stack([outs[s][n, h] for s in range(steps)])
+        err = float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
+        assert err <= TOL["bf16"], (n, h, err)

@@ -219,3 +219,22 @@ def test_synth_recipe():
     assert abs(lens.mean() - 48.0) < 1.5 and lens.min() >= 1
     ln = synth._draw_lengths(np.random.default_rng(0), ("lognormal", 64.0, 1.5), 2_000_000)
     assert abs(np.median(ln) - 64) <= 4
+
+
+@pytest.mark.parametrize("policy", ["dla", "fenwick"])
+def test_masked_readout_equals_full_readout(policy):
+    """The masked readout (used for sampled outputs at full workload sizes)
+    updates states at every token: its rows equal the full run's at the marked
+    tokens and are zero elsewhere."""
+    T, d = 200, 6
+    q, k, v = small_case(3, T, d)
+    full = O.Oracle(1, d, d, 4, policy).run(k[None], q[None], v[None], tau=0.5, dtype="f64")
+    mask = np.zeros(T, dtype=np.uint8)
+    mask[[0, 1, 63, 64, 127, 150, 199]] = 1
+    part = O.Oracle(1, d, d, 4, policy).run(k[None], q[None], v[None], tau=0.5, dtype="f64",
+                                            out_mask=mask)
+    sel = mask.astype(bool)
+    assert np.array_equal(part["out"][0, sel], full["out"][0, sel])
+    assert not part["out"][0, ~sel].any()
+    assert np.array_equal(part["boundary"], full["boundary"])
+    assert part["merges"] == full["merges"]
