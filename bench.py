@@ -166,6 +166,50 @@ class ClockSampler:
                 "samples": len(rows), "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
+# ------------------------------------------------------------ ncu traffic ----
+
+# kernel slot -> (ncu summary under profiles/, source files the kernel is built from)
+TRAFFIC_SOURCES = {
+    ("readout", "tc"): ("readout_tc", ["readout_tc.cu", "tc_ptx.cuh", "dla_internal.cuh"]),
+    ("decode_stream", "-"): ("decode_stream", ["decode.cu", "dla_internal.cuh"]),
+}
+
+
+def source_sha256(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "dynamic_state_memory_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel, path, workload):
+    """DRAM bytes per launch (read + write) from the committed ncu summary of
+    this kernel and workload, or None when there is none or the kernel's
+    source has changed since it was captured."""
+    key = TRAFFIC_SOURCES.get((kernel, path))
+    if key is None:
+        return None
+    name, files = key
+    fn = os.path.join(ROOT, "profiles", f"{name}_{workload}.md")
+    if not os.path.exists(fn):
+        return None
+    fields = {}
+    for line in open(fn):
+        line = line.strip()
+        if ":" in line and line.split(":", 1)[0] in ("source_sha256", "dram_bytes_per_launch",
+                                                    "units_per_launch_scale"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    if fields.get("source_sha256") != source_sha256(files):
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"]) * float(fields.get("units_per_launch_scale", 1))
+    except (KeyError, ValueError):
+        return None
+
+
 # ---------------------------------------------------------------- inputs ----
 
 def _gen_head(args):
@@ -342,7 +386,10 @@ def bench_prefill(args, wl, rank, world, local_rank):
     value = tokens / (ms_step * 1e-3) / 1e6
     # dominant kernel
     tot = {kname: sum(v_) for kname, v_ in kt.items()}
-    dom = max(tot, key=tot.get)
+    dominant = max(tot, key=tot.get)
+    # the roofline is the readout's (the contraction); it is the dominant
+    # kernel on every prefill workload here, and `dominant` says so if not
+    dom = "readout" if "readout" in kt else dominant
     per_launch_ms = statistics.mean(kt[dom])
     n_launch = len(kt[dom])
     steps_recorded = args.steps
@@ -360,8 +407,10 @@ def bench_prefill(args, wl, rank, world, local_rank):
     else:
         bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
         achieved = float("nan")
-    roof = {"kernel": dom, "bound": bound, "achieved": round(achieved, 3), "peak": peak,
-            "unit": unit, "frac": round(achieved / peak, 4), "traffic": None,
+    traffic = ncu_traffic(dom, "simt" if args.path == "simt" else "tc", args.workload)
+    roof = {"kernel": dom, "dominant_kernel": dominant, "bound": bound,
+            "achieved": round(achieved, 3), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
             "peak_source": peak_note, "launch_ms": round(per_launch_ms, 4),
             "launches": n_launch,
             "kernel_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()}}
@@ -525,7 +574,8 @@ def bench_decode(args, wl, rank, world, local_rank):
     achieved = state_bytes / (stream_ms * 1e-3) / 1e9
     peak = peaks.get("hbm_gbs", 6540.8)
     roof = {"kernel": "decode_stream", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": ncu_traffic("decode_stream", "-", args.workload),
             "peak_source": f"{peaks_kind} copy bandwidth",
             "algorithmic_bytes_per_launch": state_bytes, "launch_ms": round(stream_ms, 4),
             "launches": len(kt["decode_stream"]),
