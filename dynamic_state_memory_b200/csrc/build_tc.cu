@@ -68,12 +68,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       sm.pen[0] = len;
       sm.np = 1;
     } else {
-      const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
-      const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
-      const bool cont = !(nev > 0 && evo[0] == 0);
+      // runs of the tile: it starts one, and every boundary flag after its
+      // first token starts the next (the first token either continues the
+      // open state or opens a new one; the run starts there either way)
+      const uint8_t *bf = pl.b + (size_t)u * dm.W + T0;
       int np = 0;
-      if (cont) sm.pst[np++] = 0;
-      for (int i = 0; i < nev; i++) sm.pst[np++] = evo[i];
+      sm.pst[np++] = 0;
+      for (int i = 1; i < len; i++)
+        if (bf[i]) sm.pst[np++] = i;
       for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
       sm.np = np;
     }
@@ -113,7 +115,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
 
   const int np = sm.np;
-  const int pbase = fen.treeS ? c : pl.tile_pbase[(size_t)u * dm.tiles + c];
+  const int pbase = fen.treeS ? c : c * PIECES_PER_TILE;
   float *pieces = fen.treeS ? fen.treeS + (size_t)u * fen.nodes * D * D
                             : pl.pieces + (size_t)u * dm.pmax * D * D;
   const uint32_t k_s = smem_u32(sm.k), v_s = smem_u32(sm.v);

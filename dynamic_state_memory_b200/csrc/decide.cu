@@ -460,7 +460,6 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   int32_t *const tnev = pl.tile_nev + (size_t)u * tiles;
   int32_t *const toff = pl.tile_ev_off + (size_t)u * tiles * M;
   int32_t *const tmrg = pl.tile_ev_mrg + (size_t)u * tiles * M;
-  int32_t *const tpb = pmax > 0 ? pl.tile_pbase + (size_t)u * tiles : nullptr;
   float *const ver_z = pl.ver_z + (size_t)u * vmax * D;
   float *const ver_n = pl.ver_n + (size_t)u * vmax;
   int32_t *const tr_t = ca.trace.merge_t ? ca.trace.merge_t + (size_t)u * ca.trace.cap : nullptr;
@@ -527,7 +526,8 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     return w * 32 + bit;
   };
 
-  int nops = 0, nver = 0, npieces = 0;
+  int nops = 0, nver = 0;
+  int ptile = -1, pk = 0;  // tile of the last piece and pieces emitted in it
   auto emit = [&](int op, int a, int b, int c) {
     if (lane == 0) {
       if (nops < opsmax) ops[nops] = make_int4(op, a, b, c);
@@ -539,9 +539,14 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   // when long enough (and the path has pieces), else SIMT rank-1 adds
   auto emit_add = [&](int slot, int from, int cnt) {
     if (pmax > 0 && cnt >= PIECE_MIN) {
-      if (npieces >= pmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
-      emit(OP_ADDP, slot, npieces, cnt);
-      npieces++;
+      const int tl = from / M;  // a run never crosses a tile boundary
+      if (tl != ptile) {
+        ptile = tl;
+        pk = 0;
+      }
+      const int id = tl * PIECES_PER_TILE + pk++;
+      if (id >= pmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
+      emit(OP_ADDP, slot, id, cnt);
     } else {
       emit(OP_ADD, slot, from, cnt);
     }
@@ -578,7 +583,6 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
       cur_from = T0;
     }
     __syncwarp();
-    if (lane == 0 && tpb) tpb[c] = npieces;
     const int m0 = m;
 #pragma unroll 1
     for (int p0 = 0; p0 < m0; p0 += 32) {

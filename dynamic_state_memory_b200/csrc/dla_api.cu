@@ -67,7 +67,7 @@ Dims make_dims(const dla_config &cfg, int policy) {
   dm.vmax = dm.C + dm.tiles * per_tile;
   dm.opsmax = 4 * W + dm.tiles + 2 + dm.vmax + 8;
   dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
-  dm.pmax = tc ? dm.tiles + W / PIECE_MIN : 0;
+  dm.pmax = tc ? dm.tiles * PIECES_PER_TILE : 0;
   return dm;
 }
 
@@ -91,7 +91,6 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.ver_n = cv.take<float>(h * dm.vmax);
   pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
   pl.slot_ver = cv.take<int32_t>(h * dm.C);
-  pl.tile_pbase = cv.take<int32_t>(h * dm.tiles);
   pl.pieces = cv.take<float>(h * (size_t)dm.pmax * dm.D * dm.D);
   pl.phi_tab = cv.take<double>(4096);
 }
@@ -146,6 +145,31 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
   if (cfg->d_k != cfg->d_v || !d_ok(cfg->d_k)) return DLA_ERR_UNSUPPORTED;
   if (policy == DLA_POLICY_DYNAMIC && (cfg->C < 2 || cfg->C > 128)) return DLA_ERR_UNSUPPORTED;
   return DLA_OK;
+}
+
+// The second stream of a prefill call and its fork / join events, one set
+// per host thread and device, created on first use and kept for the thread's
+// lifetime (non-blocking, so it never synchronises with the legacy stream).
+enum { EV_START = 0, EV_SCAN, EV_ENGINE, EV_DONE0, EV_DONE1, EV_COUNT };
+struct Aux {
+  cudaStream_t s = nullptr;
+  cudaEvent_t ev[EV_COUNT] = {};
+  bool ok = false;
+};
+constexpr int MAX_DEVICES = 64;
+
+Aux *aux_streams() {
+  thread_local Aux aux[MAX_DEVICES];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return nullptr;
+  Aux &a = aux[dev];
+  if (!a.ok) {
+    if (!a.s && cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (cudaEvent_t &e : a.ev)
+      if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    a.ok = true;
+  }
+  return &a;
 }
 
 }  // namespace
@@ -219,6 +243,7 @@ size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
   Plan pl{};
   Carver cv{nullptr};
   carve_plan(cv, dm, pl);
+  if (cfg->T > dm.W) carve_plan(cv, dm, pl);  // windows alternate between two plans
   return cv.off;
 }
 
@@ -241,11 +266,16 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16)
     return DLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
-  Plan pl{};
+  Plan plans[2];
   Carver cv{static_cast<char *>(ws)};
-  carve_plan(cv, dm, pl);
+  carve_plan(cv, dm, plans[0]);
+  if (cfg->T > dm.W) carve_plan(cv, dm, plans[1]);
+  else plans[1] = plans[0];
   if (cv.off > ws_bytes) return DLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Aux *ax = aux_streams();
+  if (!ax) return DLA_ERR_CUDA;
+  cudaStream_t sd = ax->s;  // decisions: score, pieces, sums, engine
   CallArgs ca{};
   ca.q = q;
   ca.k = k;
@@ -262,32 +292,49 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     memset(&ca.trace, 0, sizeof ca.trace);
   }
   ca.dev_status = dev_status;
-  for (int w0 = 0; w0 < cfg->T; w0 += dm.W) {
+  // Fork: the decision kernels and the engine run on the auxiliary stream,
+  // the state build, materializer and readout on the caller's stream.  The
+  // builder needs only the boundary flags, so it overlaps the sums and the
+  // engine; window w + 1's decisions overlap window w's heavy kernels.  Every
+  // auxiliary launch is ordered before a later wait of the caller's stream,
+  // so the call ends (joins) on the caller's stream.
+  if (cudaEventRecord(ax->ev[EV_START], s) != cudaSuccess ||
+      cudaStreamWaitEvent(sd, ax->ev[EV_START], 0) != cudaSuccess)
+    return DLA_ERR_CUDA;
+  const bool tc = use_tc(*cfg);
+  dla_profile *pf = cfg->profile;
+  int wi = 0;
+  for (int w0 = 0; w0 < cfg->T; w0 += dm.W, wi++) {
+    const Plan &pl = plans[wi & 1];
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
-    dla_profile *pf = cfg->profile;
-    cudaError_t e;
-    { ProfScope ps(pf, DLA_K_SCORE, s); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, s); }
+    cudaError_t e = cudaSuccess;
+    // this plan was last read by window wi - 2's readout
+    if (wi >= 2 && cudaStreamWaitEvent(sd, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_SCORE, sd); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, sd); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_SEGSCAN, s); e = launch_segscan(dm, pl, ca, s); }
+    { ProfScope ps(pf, DLA_K_SEGSCAN, sd); e = launch_segscan(dm, pl, ca, sd); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SCAN], sd) != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_SEGSUM, sd); e = launch_segsum(dm, pl, ca, sd); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_SEGSUM, s); e = launch_segsum(dm, pl, ca, s); }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_engine(dm, pl, ca, s); }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
-    const bool tc = use_tc(*cfg);
+    { ProfScope ps(pf, DLA_K_ENGINE, sd); e = launch_engine(dm, pl, ca, sd); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], sd) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc) {
+      if (cudaStreamWaitEvent(s, ax->ev[EV_SCAN], 0) != cudaSuccess) return DLA_ERR_CUDA;
       ProfScope ps(pf, DLA_K_BUILD, s);
       e = launch_build_tc(dm, pl, ca, s);
       if (e != cudaSuccess) return DLA_ERR_CUDA;
     }
+    if (cudaStreamWaitEvent(s, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     {
       ProfScope ps(pf, DLA_K_READOUT, s);
       e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
     }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_DONE0 + (wi & 1)], s) != cudaSuccess)
+      return DLA_ERR_CUDA;
   }
   return DLA_OK;
 }

@@ -39,6 +39,10 @@ enum OpCode : int32_t {
 
 // Pieces shorter than this stay SIMT adds in the materializer.
 constexpr int PIECE_MIN = 16;
+// Piece ids are tile-based: run k (in token order) of the pieces of tile c
+// is piece c * PIECES_PER_TILE + k, so the builder needs only the boundary
+// flags and runs concurrently with the capacity-merge engine.
+constexpr int PIECES_PER_TILE = 128 / PIECE_MIN;
 
 // Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
 // pair at that time-order position, <= -2 merge the two newest sealed states
@@ -81,7 +85,6 @@ struct Plan {
   float *ver_n;        // [heads][vmax] token count of each version
   void *ver_S;         // [heads][vmax] versions (fp32 [D][D] or bf16 tiled)
   int32_t *slot_ver;   // [heads][C] engine scratch
-  int32_t *tile_pbase; // [heads][tiles] first piece id of each tile
   double *phi_tab;     // phi in fp64 of negative bf16 inputs of moderate magnitude
   float *pieces;       // [heads][pmax][D][D] fp32 piece states
 };
