@@ -147,12 +147,15 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
   return DLA_OK;
 }
 
-// The second stream of a prefill call and its fork / join events, one set
-// per host thread and device, created on first use and kept for the thread's
-// lifetime (non-blocking, so it never synchronises with the legacy stream).
-enum { EV_START = 0, EV_SCAN, EV_ENGINE, EV_DONE0, EV_DONE1, EV_COUNT };
+// The auxiliary streams of a prefill call and their fork / join events, one
+// set per host thread and device, created on first use and kept for the
+// thread's lifetime (non-blocking, so they never synchronise with the legacy
+// stream).  `s` runs the score and sums at normal priority; `se` runs the
+// engine at the highest priority: it is latency-bound and on the critical
+// path of a single window, so its few CTAs should get SMs first.
+enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_DONE0, EV_DONE1, EV_COUNT };
 struct Aux {
-  cudaStream_t s = nullptr;
+  cudaStream_t s = nullptr, se = nullptr;
   cudaEvent_t ev[EV_COUNT] = {};
   bool ok = false;
 };
@@ -164,7 +167,11 @@ Aux *aux_streams() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return nullptr;
   Aux &a = aux[dev];
   if (!a.ok) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
     if (!a.s && cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (!a.se && cudaStreamCreateWithPriority(&a.se, cudaStreamNonBlocking, hi) != cudaSuccess)
+      return nullptr;
     for (cudaEvent_t &e : a.ev)
       if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
     a.ok = true;
@@ -275,7 +282,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Aux *ax = aux_streams();
   if (!ax) return DLA_ERR_CUDA;
-  cudaStream_t sd = ax->s;  // decisions: score, pieces, sums, engine
+  cudaStream_t sd = ax->s;   // decisions: score, pieces, sums
+  cudaStream_t se = ax->se;  // the engine
   CallArgs ca{};
   ca.q = q;
   ca.k = k;
@@ -294,8 +302,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   ca.dev_status = dev_status;
   // Fork: the decision kernels and the engine run on the auxiliary stream,
   // the state build, materializer and readout on the caller's stream.  The
-  // builder needs only the boundary flags, so it overlaps the sums and the
-  // engine; window w + 1's decisions overlap window w's heavy kernels.  Every
+  // builder needs only the boundary flags, so it overlaps the engine; window
+  // w + 1's decisions overlap window w's heavy kernels.  Every
   // auxiliary launch is ordered before a later wait of the caller's stream,
   // so the call ends (joins) on the caller's stream.
   if (cudaEventRecord(ax->ev[EV_START], s) != cudaSuccess ||
@@ -309,19 +317,26 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
     cudaError_t e = cudaSuccess;
-    // this plan was last read by window wi - 2's readout
+    // this plan was last read by window wi - 2's readout; the score reads the
+    // cache's last key and score, written by window wi - 1's engine
     if (wi >= 2 && cudaStreamWaitEvent(sd, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
+    if (wi >= 1 && cudaStreamWaitEvent(sd, ax->ev[EV_ENGINE], 0) != cudaSuccess)
       return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SCORE, sd); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, sd); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SEGSCAN, sd); e = launch_segscan(dm, pl, ca, sd); }
-    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SCAN], sd) != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_SEGSUM, sd); e = launch_segsum(dm, pl, ca, sd); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_ENGINE, sd); e = launch_engine(dm, pl, ca, sd); }
-    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], sd) != cudaSuccess) return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_SEGSUM, sd); e = launch_segsum(dm, pl, ca, sd); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SUMS], sd) != cudaSuccess ||
+        cudaStreamWaitEvent(se, ax->ev[EV_SUMS], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_ENGINE, se); e = launch_engine(dm, pl, ca, se); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], se) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc) {
-      if (cudaStreamWaitEvent(s, ax->ev[EV_SCAN], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      // after the sums (not just the boundary flags it reads), so it overlaps
+      // the engine without slowing the sums ahead of it
+      if (cudaStreamWaitEvent(s, ax->ev[EV_SUMS], 0) != cudaSuccess) return DLA_ERR_CUDA;
       ProfScope ps(pf, DLA_K_BUILD, s);
       e = launch_build_tc(dm, pl, ca, s);
       if (e != cudaSuccess) return DLA_ERR_CUDA;
