@@ -229,7 +229,10 @@ dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int
   c.d_v = d_v;
   Carver cv{static_cast<char *>(dev_base)};
   carve_cache(cv, c);
-  if (cudaMemsetAsync(dev_base, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // S is carved first; everything after it is reset
+  const size_t s_end = reinterpret_cast<char *>(c.z) - static_cast<char *>(dev_base);
+  if (cudaMemsetAsync(static_cast<char *>(dev_base) + s_end, 0, need - s_end,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DLA_ERR_CUDA;
   *cache = c;
   return DLA_OK;

@@ -133,7 +133,9 @@ typedef struct {
 size_t dla_cache_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v);
 
 /* Lay out a cache in [dev_base, dev_base + bytes) and reset it to the empty
- * state (m = 0, t = 0, prev_r = 0, S = 0) with kernels on `stream`.
+ * state (m = 0, t = 0, prev_r = 0; every array but S zeroed) with an
+ * asynchronous memset on `stream`.  S is left as it is: a slot's state is
+ * always written (new open state, store, merge) before it is read.
  * dev_base must be 256-byte aligned. */
 dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int32_t d_k,
                           int32_t d_v, void *dev_base, size_t bytes, void *stream);
