@@ -15,12 +15,14 @@
 //   P = W o A (causal) as the bf16 A operand of
 //     O_intra = P V                                    TMEM cols [256, 384)
 //   Then, per atom alpha, a bulk copy brings the frozen bf16 state version
-//   (already stored in the UMMA K-major swizzled layout) into one of 5 shared
-//   stages (3 of their own, then the k and v tiles once P V has read them),
-//   two threads issue P_alpha = phi(Q) S_alpha^T (even / odd atoms) into three
-//   TMEM buffers (cols [0,128), [128,256), then [256,384) once O_intra has been
-//   read out), and 8 epilogue warps, starting from O_intra, accumulate
-//   W_alpha(t) * P_alpha in registers while the next MMAs run.
+//   (already stored in the UMMA K-major swizzled layout) into one of 6 shared
+//   stages (3 of their own, then the k and v tiles once P V has read them and
+//   the q tile once phi(Q) is in tensor memory),
+//   two threads issue P_alpha = phi(Q) S_alpha^T (even / odd atoms) into two
+//   TMEM buffers (cols [0,128) / [128,256)), with phi(Q) read from tensor
+//   memory (written into O_intra's columns once it has been read out), and 8
+//   epilogue warps, starting from O_intra, accumulate W_alpha(t) * P_alpha in
+//   registers while the next MMAs run.
 // Every wait on an mbarrier is bounded; a timeout sets DLA_ERR_TIMEOUT.
 #include "dla_internal.cuh"
 #include "tc_ptx.cuh"
@@ -32,14 +34,20 @@ using namespace tc;
 constexpr int M = 128;
 constexpr int D = 128;
 constexpr int NST = 3;   // version stages of their own
-constexpr int NSV = 5;   // + the k and v tiles once P V has read them
+constexpr int NSV = 6;   // + the k and v tiles once P V has read them, and the q tile
+                         // once phi(Q) is in tensor memory
 constexpr int THREADS = 384;
 constexpr int TILE_BYTES = M * D * 2;
 constexpr uint32_t VER_BYTES = D * D * 2;
 constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
 constexpr uint32_t COL_BUF0 = 0, COL_AI = 256, COL_W = 384;
-constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and, once its intra-tile
-                        // output has been read, [256,384)
+constexpr int NPB = 2;  // TMEM P buffers: cols [0,128), [128,256)
+// phi(Q) as the A operand of the atom MMAs, in tensor memory once the
+// intra-tile output has been read out of the same columns: elements
+// [64h, 64h + 64) of a row in cols COL_AI + 64h + [0, 32), two per column
+__device__ __forceinline__ uint32_t qa_col(int kstep) {
+  return COL_AI + (kstep < 4 ? 8 * kstep : 64 + 8 * (kstep - 4));
+}
 constexpr float INV_SQRT_D = 0.08838834764831845f;
 
 struct Smem {
@@ -47,7 +55,7 @@ struct Smem {
   uint8_t kp[TILE_BYTES];
   uint8_t v[TILE_BYTES];
   uint8_t st[NST][VER_BYTES];
-  uint64_t bar_load, bar_mma, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
+  uint64_t bar_load, bar_mma, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
   uint32_t tmem_base;
   int abort;
   int m0, np, len;
@@ -70,11 +78,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (T0 >= ca.Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
-  auto stage = [&](int s) -> uint8_t * { return s < NST ? sm.st[s] : (s == NST ? sm.kp : sm.v); };
+  auto stage = [&](int s) -> uint8_t * {
+    return s < NST ? sm.st[s] : (s == NST ? sm.kp : (s == NST + 1 ? sm.v : sm.q));
+  };
   const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
 
-  // ---- setup: TMEM, barriers, tile metadata ------------------------------
+  // ---- setup: TMEM, barriers, tile loads first, then tile metadata --------
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if (tid == 0) {
+    mbar_init(&sm.bar_load, 1);
+    fence_mbar_init();
+    mbar_expect_tx(&sm.bar_load, 3 * TILE_BYTES);
+    const int row = ca.w0 + T0;
+    for (int h = 0; h < 2; h++) {
+      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, row, u);
+      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, row, u);
+      tma_load_3d(sm.v + h * (TILE_BYTES / 2), &tv, &sm.bar_load, h * 64, row, u);
+    }
+  }
   const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
   {
     const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
@@ -85,12 +106,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
   if (tid == 0) {
-    mbar_init(&sm.bar_load, 1);
     mbar_init(&sm.bar_mma, 1);
     for (int i = 0; i < NSV; i++) {
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
     }
+    mbar_init(&sm.bar_qa, 8);
     for (int i = 0; i < NPB; i++) {
       mbar_init(&sm.tfull[i], 1);
       mbar_init(&sm.tempty[i], 8);
@@ -170,13 +191,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // ---- loads --------------------------------------------------------------
   if (tid == 0) {
-    mbar_expect_tx(&sm.bar_load, 3 * TILE_BYTES);
-    const int row = ca.w0 + T0;
-    for (int h = 0; h < 2; h++) {
-      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, row, u);
-      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, row, u);
-      tma_load_3d(sm.v + h * (TILE_BYTES / 2), &tv, &sm.bar_load, h * 64, row, u);
-    }
     for (int a = 0; a < m0 && a < NST - 1; a++) {
       mbar_expect_tx(&sm.full[a], VER_BYTES);
       bulk_load(sm.st[a], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[a]);
@@ -515,23 +529,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
 
   // ---- P V, then the pipelined readout over atoms --------------------------
-  // Two issuing threads (warp 1: even atoms, warp 2: odd atoms); an issuing
-  // thread is held for about the duration of its MMAs, so with one issuer
-  // every barrier wait left the tensor pipe idle.  Atom a goes to TMEM buffer
-  // a % 3; the third buffer is the intra-tile output's columns, handed over
-  // once the epilogue has folded that output into its registers.  Three
-  // buffers cover the commit -> drain -> release round trip of a buffer.
+  // Two issuing threads (warp 1: even atoms into TMEM buffer 0, warp 2: odd
+  // atoms into buffer 1); an issuing thread is held for about the duration of
+  // its MMAs, so with one issuer every barrier wait left the tensor pipe idle.
+  // The atom MMAs read phi(Q) from tensor memory: with both operands in shared
+  // memory, their reads plus the version copies exceeded its bandwidth.
   auto issue_atoms = [&](int first) {
+    bool ok_qa = first < m0 ? mbar_wait(&sm.bar_qa, 0, abort) : true;
     for (int a = first; a < m0; a += 2) {
-      const int s = a % NSV, b = a % NPB;
-      bool ok = mbar_wait(&sm.full[s], (a / NSV) & 1, abort);
-      if (b == NPB - 1) ok = mbar_wait(&sm.tempty[b], (a / NPB) & 1, abort) && ok;
-      else if (a >= NPB) ok = mbar_wait(&sm.tempty[b], ((a / NPB) - 1) & 1, abort) && ok;
+      const int s = a % NSV, b = a & 1;
+      bool ok = mbar_wait(&sm.full[s], (a / NSV) & 1, abort) && ok_qa;
+      if (a >= 2) ok = mbar_wait(&sm.tempty[b], ((a >> 1) - 1) & 1, abort) && ok;
       tc_fence_after();
       if (ok) {
         const uint32_t st_s = smem_u32(stage(s));
         for (int k = 0; k < 8; k++)
-          mma_bf16(tbase + b * 128, kdesc(q_s, k), kdesc(st_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
+          mma_bf16_ta(tbase + b * 128, tbase + qa_col(k), kdesc(st_s, k), idesc_bf16(M, 128, 0, 0),
+                      k > 0);
       }
       mma_commit(&sm.empty[s]);
       mma_commit(&sm.tfull[b]);
@@ -556,10 +570,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int a = NST; a < m0; a++) {
       if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)sm.atom[a + PF] * VER_BYTES, VER_BYTES);
       const int s = a % NSV;
-      // stages NST.. are the k / v tiles: free once P V has completed
-      // (bar_mma phase 1; phase 0, the first MMAs, completed before here)
-      const bool ok = a < NSV ? mbar_wait(&sm.bar_mma, 1, abort)
-                              : mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort);
+      // stages NST, NST + 1 are the k / v tiles: free once P V has completed
+      // (bar_mma phase 1; phase 0, the first MMAs, completed before here);
+      // stage NST + 2 is the q tile, free once phi(Q) is in tensor memory
+      const bool ok = a >= NSV        ? mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort)
+                      : s == NST + 2 ? mbar_wait(&sm.bar_qa, 0, abort)
+                                     : mbar_wait(&sm.bar_mma, 1, abort);
       if (!ok) break;
       mbar_expect_tx(&sm.full[s], VER_BYTES);
       bulk_load(stage(s), verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
@@ -569,7 +585,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     float acc[64];
-    // start from the intra-tile output, then release its columns as buffer 2
+    // start from the intra-tile output, then put phi(Q) in its columns
     mbar_wait(&sm.bar_mma, 1, abort);
     tc_fence_after();
     {
@@ -583,14 +599,28 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 32; i++) acc[32 + i] = __uint_as_float(pr[i]);
     }
+    {
+      // row t, elements [64 hc, 64 hc + 64) of phi(q_t), from the swizzled tile
+      uint32_t qw[32];
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(sm.q + sw128_offset(t, 64 * hc + 8 * i, M));
+        qw[4 * i] = x.x;
+        qw[4 * i + 1] = x.y;
+        qw[4 * i + 2] = x.z;
+        qw[4 * i + 3] = x.w;
+      }
+      DLA_TMEM_ST32(trow + COL_AI + 64 * hc, qw);
+      tmem_wait_st();
+    }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.tempty[NPB - 1]);
+    if (lane == 0) mbar_arrive(&sm.bar_qa);
 #pragma unroll 1
     for (int a = 0; a < m0; a++) {
-      const int b = a % NPB;
+      const int b = a & 1;
       const float w = __uint_as_float(tmem_ld1(trow + COL_W + a));
-      mbar_wait(&sm.tfull[b], (a / NPB) & 1, abort);
+      mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
       tc_fence_after();
       uint32_t pr[32];
       DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
