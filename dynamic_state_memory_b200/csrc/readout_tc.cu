@@ -34,14 +34,15 @@ using namespace tc;
 constexpr int M = 128;
 constexpr int D = 128;
 constexpr int NST = 3;   // version stages of their own
-constexpr int NSV = 6;   // + the k and v tiles once P V has read them, and the q tile
-                         // once phi(Q) is in tensor memory
+constexpr int NSV = 4;   // + the k tile once P V has read it
 constexpr int THREADS = 384;
 constexpr int TILE_BYTES = M * D * 2;
 constexpr uint32_t VER_BYTES = D * D * 2;
 constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
 constexpr uint32_t COL_BUF0 = 0, COL_AI = 256, COL_W = 384;
-constexpr int NPB = 2;  // TMEM P buffers: cols [0,128), [128,256)
+constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and, once the weights have
+                        // been moved to shared memory, [384,512)
+__device__ __forceinline__ uint32_t pbuf_col(int b) { return b == 2 ? 384u : (uint32_t)b * 128u; }
 // phi(Q) as the A operand of the atom MMAs, in tensor memory once the
 // intra-tile output has been read out of the same columns: elements
 // [64h, 64h + 64) of a row in cols COL_AI + 64h + [0, 32), two per column
@@ -51,9 +52,9 @@ __device__ __forceinline__ uint32_t qa_col(int kstep) {
 constexpr float INV_SQRT_D = 0.08838834764831845f;
 
 struct Smem {
-  uint8_t q[TILE_BYTES];
-  uint8_t kp[TILE_BYTES];
+  uint8_t q[TILE_BYTES];   // then (with v) the atom weights during the atom loop
   uint8_t v[TILE_BYTES];
+  uint8_t kp[TILE_BYTES];
   uint8_t st[NST][VER_BYTES];
   uint64_t bar_load, bar_mma, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
   uint32_t tmem_base;
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
   auto stage = [&](int s) -> uint8_t * {
-    return s < NST ? sm.st[s] : (s == NST ? sm.kp : (s == NST + 1 ? sm.v : sm.q));
+    return s < NST ? sm.st[s] : sm.kp;
   };
   const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
 
@@ -533,19 +534,21 @@ __global__ void __launch_bounds__(THREADS, 1)
   // atoms into buffer 1); an issuing thread is held for about the duration of
   // its MMAs, so with one issuer every barrier wait left the tensor pipe idle.
   // The atom MMAs read phi(Q) from tensor memory: with both operands in shared
-  // memory, their reads plus the version copies exceeded its bandwidth.
+  // memory, their reads plus the version copies exceeded its bandwidth.  Atom
+  // a goes to product buffer a % 3: three buffers cover a buffer's round trip
+  // (MMAs, commit, epilogue drain, release) at the MMA rate.
   auto issue_atoms = [&](int first) {
     bool ok_qa = first < m0 ? mbar_wait(&sm.bar_qa, 0, abort) : true;
     for (int a = first; a < m0; a += 2) {
-      const int s = a % NSV, b = a & 1;
+      const int s = a % NSV, b = a % NPB;
       bool ok = mbar_wait(&sm.full[s], (a / NSV) & 1, abort) && ok_qa;
-      if (a >= 2) ok = mbar_wait(&sm.tempty[b], ((a >> 1) - 1) & 1, abort) && ok;
+      if (a >= NPB) ok = mbar_wait(&sm.tempty[b], ((a / NPB) - 1) & 1, abort) && ok;
       tc_fence_after();
       if (ok) {
         const uint32_t st_s = smem_u32(stage(s));
         for (int k = 0; k < 8; k++)
-          mma_bf16_ta(tbase + b * 128, tbase + qa_col(k), kdesc(st_s, k), idesc_bf16(M, 128, 0, 0),
-                      k > 0);
+          mma_bf16_ta(tbase + pbuf_col(b), tbase + qa_col(k), kdesc(st_s, k),
+                      idesc_bf16(M, 128, 0, 0), k > 0);
       }
       mma_commit(&sm.empty[s]);
       mma_commit(&sm.tfull[b]);
@@ -570,12 +573,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int a = NST; a < m0; a++) {
       if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)sm.atom[a + PF] * VER_BYTES, VER_BYTES);
       const int s = a % NSV;
-      // stages NST, NST + 1 are the k / v tiles: free once P V has completed
-      // (bar_mma phase 1; phase 0, the first MMAs, completed before here);
-      // stage NST + 2 is the q tile, free once phi(Q) is in tensor memory
-      const bool ok = a >= NSV        ? mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort)
-                      : s == NST + 2 ? mbar_wait(&sm.bar_qa, 0, abort)
-                                     : mbar_wait(&sm.bar_mma, 1, abort);
+      // stage NST is the k tile: free once P V has completed (bar_mma phase
+      // 1; phase 0, the first MMAs, completed before here)
+      const bool ok = a >= NSV ? mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort)
+                               : mbar_wait(&sm.bar_mma, 1, abort);
       if (!ok) break;
       mbar_expect_tx(&sm.full[s], VER_BYTES);
       bulk_load(stage(s), verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
@@ -613,21 +614,38 @@ __global__ void __launch_bounds__(THREADS, 1)
       DLA_TMEM_ST32(trow + COL_AI + 64 * hc, qw);
       tmem_wait_st();
     }
+    // every epilogue warp has read its phi(Q) rows: the q and v tiles now take
+    // the weights, W[atom][row] in fp32, and their TMEM columns become buffer 2
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    float *sW = reinterpret_cast<float *>(sm.q);
+    {
+      const int half = (m0 + 15) / 16 * 8;  // atoms per warp half, in chunks of 8
+      const int a_lo = hc * half, a_hi = min(m0, a_lo + half);
+#pragma unroll 1
+      for (int a0 = a_lo; a0 < a_hi; a0 += 8) {
+        uint32_t r[8];
+        DLA_TMEM_LD8(trow + COL_W + a0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+          if (a0 + j < a_hi) sW[(a0 + j) * M + t] = __uint_as_float(r[j]);
+      }
+    }
     tc_fence_before();
-    __syncwarp();
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (lane == 0) mbar_arrive(&sm.bar_qa);
 #pragma unroll 1
     for (int a = 0; a < m0; a++) {
-      const int b = a & 1;
-      const float w = __uint_as_float(tmem_ld1(trow + COL_W + a));
-      mbar_wait(&sm.tfull[b], (a >> 1) & 1, abort);
+      const int b = a % NPB;
+      const float w = sW[a * M + t];
+      mbar_wait(&sm.tfull[b], (a / NPB) & 1, abort);
       tc_fence_after();
       uint32_t pr[32];
-      DLA_TMEM_LD32(trow + b * 128 + hc * 64, pr);
+      DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64, pr);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; i++) acc[i] = fmaf(w, __uint_as_float(pr[i]), acc[i]);
-      DLA_TMEM_LD32(trow + b * 128 + hc * 64 + 32, pr);
+      DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64 + 32, pr);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(w, __uint_as_float(pr[i]), acc[32 + i]);
