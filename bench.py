@@ -407,7 +407,8 @@ def bench_prefill(args, wl, rank, world, local_rank):
     else:
         bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
         achieved = float("nan")
-    traffic = ncu_traffic(dom, "simt" if args.path == "simt" else "tc", args.workload)
+    traffic = None if args.B else ncu_traffic(dom, "simt" if args.path == "simt" else "tc",
+                                              args.workload)
     roof = {"kernel": dom, "dominant_kernel": dominant, "bound": bound,
             "achieved": round(achieved, 3), "peak": peak,
             "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -575,7 +576,7 @@ def bench_decode(args, wl, rank, world, local_rank):
     peak = peaks.get("hbm_gbs", 6540.8)
     roof = {"kernel": "decode_stream", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": ncu_traffic("decode_stream", "-", args.workload),
+            "traffic": None if args.B else ncu_traffic("decode_stream", "-", args.workload),
             "peak_source": f"{peaks_kind} copy bandwidth",
             "algorithmic_bytes_per_launch": state_bytes, "launch_ms": round(stream_ms, 4),
             "launches": len(kt["decode_stream"]),
