@@ -353,12 +353,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   } else if (warp >= 4 && warp < 8) {
+    // One thread per row.  Chunks of 8 columns / entries take a branch-free
+    // fast path when no piece boundary (resp. no multi-entry state) falls
+    // inside them; boundaries are the same for every row, so the test is
+    // warp-uniform and only the few chunks holding one take the per-element
+    // path.
     constexpr int PREG = 8;
     const int qd = warp & 3;
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     const int ep = sm.pidx[t];
     const uint32_t *bits = sm.bits + ep * BW;
+    const int smax = min(32 * qd + 31, len - 1);  // last column a row of this warp reads
     float pv[PREG];  // piece sums, then logits, then weights
 #pragma unroll
     for (int k = 0; k < PREG; k++) pv[k] = 0.f;
@@ -382,60 +388,86 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_wait_st();
       }
     };
-    // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s]   (8 columns per load;
-    // loops are kept rolled so the code stays small)
+    // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s]; pieces that start
+    // past the warp's last row are never read (p > ep for all its rows)
     {
       float y = 0.f;
       int p = 0;
       int nxt = np > 1 ? sm.pst[1] : M + 1;
 #pragma unroll 1
-      for (int s0 = 0; s0 < M; s0 += 8) {
+      for (int s0 = 0; s0 <= smax; s0 += 8) {
         uint32_t ar[8];
         DLA_TMEM_LD8(trow + COL_AI + s0, ar);
         tmem_wait_ld();
+        float x[8];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-          const int s = s0 + j;
-          if (s == nxt) {
-            piece_put(p, y);
-            p++;
-            y = 0.f;
-            nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
+        for (int j = 0; j < 8; j++) x[j] = (s0 + j <= t && s0 + j < len) ? __uint_as_float(ar[j]) : 0.f;
+        if (nxt >= s0 + 8) {
+          y += ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
+        } else {
+#pragma unroll 1
+          for (int j = 0; j < 8; j++) {
+            if (s0 + j == nxt) {
+              piece_put(p, y);
+              p++;
+              y = 0.f;
+              nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
+            }
+            float xj = x[0];
+#pragma unroll
+            for (int i = 1; i < 8; i++) xj = (i == j) ? x[i] : xj;
+            y += xj;
           }
-          y += (s <= t && s < len) ? __uint_as_float(ar[j]) : 0.f;
         }
       }
       piece_put(p, y);
     }
-    // pass A
+    // pass A: each state's logit at its last atom / piece (in place), online
+    // softmax max and sum.  A chunk whose atoms are all states of their own
+    // (the common case) needs no segmented sums: its logits are LA / sqrt(d).
     float mx = -INFINITY, l = 0.f, sacc = 0.f, nacc = 0.f;
 #pragma unroll 1
     for (int a0 = 0; a0 < m0; a0 += 8) {
       uint32_t r[8];
       DLA_TMEM_LD8(trow + COL_W + a0, r);
-      tmem_wait_ld();
-      const uint32_t wb = bits[a0 >> 5] >> (a0 & 31);
-      float cmx = -INFINITY;
+      const int nval = min(8, m0 - a0);
+      const uint32_t vmask = (1u << nval) - 1u;
+      const uint32_t wb = (bits[a0 >> 5] >> (a0 & 31)) & vmask;
+      const bool fast = wb == vmask && (a0 == 0 || bit_of(bits, a0 - 1));
+      float nn[8];
 #pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const int beta = a0 + j;
-        if (beta < m0) {
-          const float nn = sm.nA[beta];
-          sacc = fmaf(nn, __uint_as_float(r[j]), sacc);
-          nacc += nn;
-          if ((wb >> j) & 1u) {
-            const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
-            r[j] = __float_as_uint(a);
-            cmx = fmaxf(cmx, a);
-            sacc = 0.f;
-            nacc = 0.f;
+      for (int j = 0; j < 8; j++) nn[j] = sm.nA[a0 + j];
+      tmem_wait_ld();
+      float cmx = -INFINITY, cl = 0.f;
+      if (__all_sync(0xffffffffu, fast)) {
+        float a[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) a[j] = j < nval ? __uint_as_float(r[j]) * INV_SQRT_D : -INFINITY;
+        cmx = fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])), fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          cl += __expf(a[j] - cmx);
+          if (j < nval) r[j] = __float_as_uint(a[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          if (j < nval) {
+            sacc = fmaf(nn[j], __uint_as_float(r[j]), sacc);
+            nacc += nn[j];
+            if ((wb >> j) & 1u) {
+              const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
+              r[j] = __float_as_uint(a);
+              cmx = fmaxf(cmx, a);
+              sacc = 0.f;
+              nacc = 0.f;
+            }
           }
         }
-      }
-      float cl = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; j++)
-        if (a0 + j < m0 && ((wb >> j) & 1u)) cl += __expf(__uint_as_float(r[j]) - cmx);
+        for (int j = 0; j < 8; j++)
+          if (j < nval && ((wb >> j) & 1u)) cl += __expf(__uint_as_float(r[j]) - cmx);
+      }
       if (cmx > -INFINITY) {
         const float nm = fmaxf(mx, cmx);
         l = l * __expf(mx - nm) + cl * __expf(cmx - nm);
@@ -463,7 +495,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       piece_put(p, y);
     }
-    // pass B (reverse)
+    // pass B (reverse): every atom / piece gets the weight of its state
     const float inv_l = 1.0f / l;
     float cur = 0.f;
 #pragma unroll 1
@@ -480,46 +512,67 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int a0 = ((m0 - 1) >> 3) << 3; m0 > 0 && a0 >= 0; a0 -= 8) {
       uint32_t r[8];
       DLA_TMEM_LD8(trow + COL_W + a0, r);
+      const int nval = min(8, m0 - a0);
+      const uint32_t vmask = (1u << nval) - 1u;
+      const uint32_t wb = (bits[a0 >> 5] >> (a0 & 31)) & vmask;
+      const bool fast = wb == vmask && (a0 == 0 || bit_of(bits, a0 - 1));
       tmem_wait_ld();
-      const uint32_t wb = bits[a0 >> 5] >> (a0 & 31);
+      if (__all_sync(0xffffffffu, fast)) {
+        // every entry ends its own state; the entry before the chunk ends one
+        // too, so the carried weight restarts there
 #pragma unroll
-      for (int j = 0; j < 8; j++)
-        if (a0 + j < m0 && ((wb >> j) & 1u)) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
+        for (int j = 0; j < 8; j++)
+          if (j < nval) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
+      } else {
 #pragma unroll
-      for (int j = 7; j >= 0; j--) {
-        if (a0 + j < m0) {
-          if ((wb >> j) & 1u) cur = __uint_as_float(r[j]);
-          r[j] = __float_as_uint(cur);
+        for (int j = 0; j < 8; j++)
+          if (j < nval && ((wb >> j) & 1u)) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
+#pragma unroll
+        for (int j = 7; j >= 0; j--) {
+          if (j < nval) {
+            if ((wb >> j) & 1u) cur = __uint_as_float(r[j]);
+            r[j] = __float_as_uint(cur);
+          }
         }
       }
       DLA_TMEM_ST8(trow + COL_W + a0, r);
       tmem_wait_st();
     }
-    // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of P V
+    // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of
+    // P V; columns past the warp's last row are zero
     {
       int p = 0;
       float w = piece_get(0);
       int nxt = np > 1 ? sm.pst[1] : M + 1;
 #pragma unroll 1
       for (int s0 = 0; s0 < M; s0 += 8) {
-        uint32_t ar[8];
-        DLA_TMEM_LD8(trow + COL_AI + s0, ar);
-        tmem_wait_ld();
-        uint32_t pk[4];
+        uint32_t pk[4] = {0u, 0u, 0u, 0u};
+        if (s0 <= smax) {
+          uint32_t ar[8];
+          DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+          tmem_wait_ld();
+          float v[8];
+          if (nxt >= s0 + 8) {
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          float v2[2];
+            for (int j = 0; j < 8; j++) v[j] = (s0 + j <= t && s0 + j < len) ? w * __uint_as_float(ar[j]) : 0.f;
+          } else {
+#pragma unroll 1
+            for (int j = 0; j < 8; j++) {
+              if (s0 + j == nxt) {
+                p++;
+                w = piece_get(p);
+                nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
+              }
+              float xj = __uint_as_float(ar[0]);
 #pragma unroll
-          for (int h = 0; h < 2; h++) {
-            const int s = s0 + j + h;
-            if (s == nxt) {
-              p++;
-              w = piece_get(p);
-              nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
+              for (int i = 1; i < 8; i++) xj = (i == j) ? __uint_as_float(ar[i]) : xj;
+              const float vj = (s0 + j <= t && s0 + j < len) ? w * xj : 0.f;
+#pragma unroll
+              for (int i = 0; i < 8; i++) v[i] = (i == j) ? vj : v[i];
             }
-            v2[h] = (s <= t && s < len) ? w * __uint_as_float(ar[j + h]) : 0.f;
           }
-          pk[j >> 1] = pack_bf16(v2[0], v2[1]);
+#pragma unroll
+          for (int j = 0; j < 4; j++) pk[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
         }
         *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
