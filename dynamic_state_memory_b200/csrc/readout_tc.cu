@@ -68,6 +68,28 @@ struct Smem {
 
 __device__ __forceinline__ bool bit_of(const uint32_t *b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
 
+// pairwise sum / max of 32 values (depth 5: the terms are independent)
+__device__ __forceinline__ float sum32(const float (&x)[32]) {
+  float y[16];
+#pragma unroll
+  for (int j = 0; j < 16; j++) y[j] = x[j] + x[j + 16];
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; j++) y[j] += y[j + w];
+  return y[0];
+}
+__device__ __forceinline__ float max32(const float (&x)[32]) {
+  float y[16];
+#pragma unroll
+  for (int j = 0; j < 16; j++) y[j] = fmaxf(x[j], x[j + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; j++) y[j] = fmaxf(y[j], y[j + w]);
+  return y[0];
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
@@ -353,11 +375,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   } else if (warp >= 4 && warp < 8) {
-    // One thread per row.  Chunks of 8 columns / entries take a branch-free
-    // fast path when no piece boundary (resp. no multi-entry state) falls
-    // inside them; boundaries are the same for every row, so the test is
-    // warp-uniform and only the few chunks holding one take the per-element
-    // path.
+    // One thread per row, blocks of 32 columns / atoms: one TMEM load per
+    // block and 32 independent operations per step (a single warp per
+    // scheduler cannot hide dependent latencies).  Piece boundaries are the
+    // same for every row, so the loops over them are warp-uniform; a block
+    // whose atoms are all states of their own (the common case) needs no
+    // segmented sums: its logits are LA / sqrt(d).
     constexpr int PREG = 8;
     const int qd = warp & 3;
     const int t = 32 * qd + lane;
@@ -395,85 +418,82 @@ __global__ void __launch_bounds__(THREADS, 1)
       int p = 0;
       int nxt = np > 1 ? sm.pst[1] : M + 1;
 #pragma unroll 1
-      for (int s0 = 0; s0 <= smax; s0 += 8) {
-        uint32_t ar[8];
-        DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+      for (int s0 = 0; s0 <= smax; s0 += 32) {
+        uint32_t ar[32];
+        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
         tmem_wait_ld();
-        float x[8];
+        float x[32];
 #pragma unroll
-        for (int j = 0; j < 8; j++) x[j] = (s0 + j <= t && s0 + j < len) ? __uint_as_float(ar[j]) : 0.f;
-        if (nxt >= s0 + 8) {
-          y += ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
-        } else {
+        for (int j = 0; j < 32; j++) x[j] = (s0 + j <= t && s0 + j < len) ? __uint_as_float(ar[j]) : 0.f;
+        int lo = s0;
 #pragma unroll 1
-          for (int j = 0; j < 8; j++) {
-            if (s0 + j == nxt) {
-              piece_put(p, y);
-              p++;
-              y = 0.f;
-              nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
-            }
-            float xj = x[0];
+        while (true) {
+          const int hi = min(nxt, s0 + 32);
+          float xs[32];
 #pragma unroll
-            for (int i = 1; i < 8; i++) xj = (i == j) ? x[i] : xj;
-            y += xj;
-          }
+          for (int j = 0; j < 32; j++) xs[j] = (s0 + j >= lo && s0 + j < hi) ? x[j] : 0.f;
+          y += sum32(xs);
+          if (nxt >= s0 + 32) break;
+          piece_put(p, y);
+          p++;
+          y = 0.f;
+          lo = nxt;
+          nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
         }
       }
       piece_put(p, y);
     }
-    // pass A: each state's logit at its last atom / piece (in place), online
-    // softmax max and sum.  A chunk whose atoms are all states of their own
-    // (the common case) needs no segmented sums: its logits are LA / sqrt(d).
+    // pass A: each state's logit at its last atom / piece, online softmax max
+    // and sum; atom columns keep exp(logit - block max) (0 for atoms that do
+    // not end a state), pieces keep their logits
     float mx = -INFINITY, l = 0.f, sacc = 0.f, nacc = 0.f;
+    float bmx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // block maxima
 #pragma unroll 1
-    for (int a0 = 0; a0 < m0; a0 += 8) {
-      uint32_t r[8];
-      DLA_TMEM_LD8(trow + COL_W + a0, r);
-      const int nval = min(8, m0 - a0);
-      const uint32_t vmask = (1u << nval) - 1u;
-      const uint32_t wb = (bits[a0 >> 5] >> (a0 & 31)) & vmask;
-      const bool fast = wb == vmask && (a0 == 0 || bit_of(bits, a0 - 1));
-      float nn[8];
-#pragma unroll
-      for (int j = 0; j < 8; j++) nn[j] = sm.nA[a0 + j];
+    for (int b = 0; b * 32 < m0; b++) {
+      const int a0 = b * 32;
+      uint32_t r[32];
+      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      const int nval = min(32, m0 - a0);
+      const uint32_t vmask = nval == 32 ? ~0u : (1u << nval) - 1u;
+      const uint32_t wb = bits[b] & vmask;
+      const bool fast = wb == vmask && (b == 0 || (bits[b - 1] >> 31));
       tmem_wait_ld();
-      float cmx = -INFINITY, cl = 0.f;
+      float a[32];
       if (__all_sync(0xffffffffu, fast)) {
-        float a[8];
 #pragma unroll
-        for (int j = 0; j < 8; j++) a[j] = j < nval ? __uint_as_float(r[j]) * INV_SQRT_D : -INFINITY;
-        cmx = fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])), fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
-#pragma unroll
-        for (int j = 0; j < 8; j++) {
-          cl += __expf(a[j] - cmx);
-          if (j < nval) r[j] = __float_as_uint(a[j]);
-        }
+        for (int j = 0; j < 32; j++) a[j] = j < nval ? __uint_as_float(r[j]) * INV_SQRT_D : -INFINITY;
       } else {
+        float s = sacc, n = nacc;
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-          if (j < nval) {
-            sacc = fmaf(nn[j], __uint_as_float(r[j]), sacc);
-            nacc += nn[j];
-            if ((wb >> j) & 1u) {
-              const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
-              r[j] = __float_as_uint(a);
-              cmx = fmaxf(cmx, a);
-              sacc = 0.f;
-              nacc = 0.f;
-            }
-          }
+        for (int j = 0; j < 32; j++) {
+          const bool valid = j < nval, end = (wb >> j) & 1u;
+          const float nn = sm.nA[a0 + j];
+          s = valid ? fmaf(nn, __uint_as_float(r[j]), s) : s;
+          n = valid ? n + nn : n;
+          a[j] = end ? __fdividef(s, n) * INV_SQRT_D : -INFINITY;
+          s = end ? 0.f : s;
+          n = end ? 0.f : n;
         }
-#pragma unroll
-        for (int j = 0; j < 8; j++)
-          if (j < nval && ((wb >> j) & 1u)) cl += __expf(__uint_as_float(r[j]) - cmx);
+        sacc = s;
+        nacc = n;
       }
+      const float cmx = max32(a);
       if (cmx > -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) a[j] = __expf(a[j] - cmx);
+        const float cl = sum32(a);
         const float nm = fmaxf(mx, cmx);
         l = l * __expf(mx - nm) + cl * __expf(cmx - nm);
         mx = nm;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j++) a[j] = 0.f;
       }
-      DLA_TMEM_ST8(trow + COL_W + a0, r);
+#pragma unroll
+      for (int k = 0; k < 4; k++) bmx[k] = (k == b) ? cmx : bmx[k];
+#pragma unroll
+      for (int j = 0; j < 32; j++) r[j] = __float_as_uint(a[j]);
+      DLA_TMEM_ST32(trow + COL_W + a0, r);
       tmem_wait_st();
     }
 #pragma unroll 1
@@ -509,33 +529,33 @@ __global__ void __launch_bounds__(THREADS, 1)
       piece_put(p, w);
     }
 #pragma unroll 1
-    for (int a0 = ((m0 - 1) >> 3) << 3; m0 > 0 && a0 >= 0; a0 -= 8) {
-      uint32_t r[8];
-      DLA_TMEM_LD8(trow + COL_W + a0, r);
-      const int nval = min(8, m0 - a0);
-      const uint32_t vmask = (1u << nval) - 1u;
-      const uint32_t wb = (bits[a0 >> 5] >> (a0 & 31)) & vmask;
-      const bool fast = wb == vmask && (a0 == 0 || bit_of(bits, a0 - 1));
+    for (int b = (m0 - 1) >> 5; m0 > 0 && b >= 0; b--) {
+      const int a0 = b * 32;
+      uint32_t r[32];
+      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      const int nval = min(32, m0 - a0);
+      const uint32_t vmask = nval == 32 ? ~0u : (1u << nval) - 1u;
+      const uint32_t wb = bits[b] & vmask;
+      const bool fast = wb == vmask && (b == 0 || (bits[b - 1] >> 31));
+      float cb = bmx[0];
+#pragma unroll
+      for (int k = 1; k < 4; k++) cb = (k == b) ? bmx[k] : cb;
+      const float f = cb > -INFINITY ? __expf(cb - mx) * inv_l : 0.f;
       tmem_wait_ld();
       if (__all_sync(0xffffffffu, fast)) {
-        // every entry ends its own state; the entry before the chunk ends one
-        // too, so the carried weight restarts there
+        // the atom before the block ends a state, so no weight carries over
 #pragma unroll
-        for (int j = 0; j < 8; j++)
-          if (j < nval) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
+        for (int j = 0; j < 32; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * f);
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; j++)
-          if (j < nval && ((wb >> j) & 1u)) r[j] = __float_as_uint(__expf(__uint_as_float(r[j]) - mx) * inv_l);
-#pragma unroll
-        for (int j = 7; j >= 0; j--) {
+        for (int j = 31; j >= 0; j--) {
           if (j < nval) {
-            if ((wb >> j) & 1u) cur = __uint_as_float(r[j]);
+            if ((wb >> j) & 1u) cur = __uint_as_float(r[j]) * f;
             r[j] = __float_as_uint(cur);
           }
         }
       }
-      DLA_TMEM_ST8(trow + COL_W + a0, r);
+      DLA_TMEM_ST32(trow + COL_W + a0, r);
       tmem_wait_st();
     }
     // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of
@@ -545,36 +565,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       float w = piece_get(0);
       int nxt = np > 1 ? sm.pst[1] : M + 1;
 #pragma unroll 1
-      for (int s0 = 0; s0 < M; s0 += 8) {
-        uint32_t pk[4] = {0u, 0u, 0u, 0u};
+      for (int s0 = 0; s0 < M; s0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; j++) pk[j] = 0u;
         if (s0 <= smax) {
-          uint32_t ar[8];
-          DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+          uint32_t ar[32];
+          DLA_TMEM_LD32(trow + COL_AI + s0, ar);
           tmem_wait_ld();
-          float v[8];
-          if (nxt >= s0 + 8) {
+          float v[32];
 #pragma unroll
-            for (int j = 0; j < 8; j++) v[j] = (s0 + j <= t && s0 + j < len) ? w * __uint_as_float(ar[j]) : 0.f;
-          } else {
+          for (int j = 0; j < 32; j++) v[j] = 0.f;
+          int lo = s0;
 #pragma unroll 1
-            for (int j = 0; j < 8; j++) {
-              if (s0 + j == nxt) {
-                p++;
-                w = piece_get(p);
-                nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
-              }
-              float xj = __uint_as_float(ar[0]);
+          while (true) {
+            const int hi = min(nxt, s0 + 32);
 #pragma unroll
-              for (int i = 1; i < 8; i++) xj = (i == j) ? __uint_as_float(ar[i]) : xj;
-              const float vj = (s0 + j <= t && s0 + j < len) ? w * xj : 0.f;
-#pragma unroll
-              for (int i = 0; i < 8; i++) v[i] = (i == j) ? vj : v[i];
-            }
+            for (int j = 0; j < 32; j++)
+              v[j] = (s0 + j >= lo && s0 + j < hi) ? w * __uint_as_float(ar[j]) : v[j];
+            if (nxt >= s0 + 32) break;
+            p++;
+            w = piece_get(p);
+            lo = nxt;
+            nxt = p + 1 < np ? sm.pst[p + 1] : M + 1;
           }
 #pragma unroll
-          for (int j = 0; j < 4; j++) pk[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
+          for (int j = 0; j < 16; j++) {
+            const int s = s0 + 2 * j;
+            pk[j] = pack_bf16((s <= t && s < len) ? v[2 * j] : 0.f, (s + 1 <= t && s + 1 < len) ? v[2 * j + 1] : 0.f);
+          }
         }
-        *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+          *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0 + 8 * i, M)) =
+              make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
     }
   }
