@@ -259,6 +259,21 @@ def prefill_flops(trace_live_sum, heads_tokens, d):
     return readout, build
 
 
+def atom_flops(m0_rows_sum, d):
+    """FLOPs of the tensor-core readout's atom loop: each row of a 128-token
+    tile takes one d x d product per state present before the tile (atom)."""
+    return 2.0 * m0_rows_sum * d * d
+
+
+def tile_atoms_rows(m, T, M=128):
+    """sum over tiles of (rows in the tile) x (states live just before it), for
+    one head with m[t] = states live after token t."""
+    tot = 0
+    for c in range(1, (T + M - 1) // M):
+        tot += min(M, T - c * M) * int(m[c * M - 1])
+    return tot
+
+
 def _time_steps(step, steps, warmup, stream, world, dev):
     import torch
     for _ in range(warmup):
@@ -303,13 +318,16 @@ def bench_prefill(args, wl, rank, world, local_rank):
     mt = tr.merge_t.cpu().numpy()
     mc = tr.merge_count.cpu().numpy()
     live_sum = 0
+    m0_rows = 0
     for h in range(B * H):
         m = np.cumsum(bnd[h].astype(np.int64))
         merges_at = np.zeros(T, dtype=np.int64)
         np.add.at(merges_at, mt[h, :mc[h]], 1)
         m = m - np.cumsum(merges_at)
         live_sum += int(m.sum())
+        m0_rows += tile_atoms_rows(m, T)
     readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
+    loop_flops = atom_flops(m0_rows, d)
 
     def step():
         dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
@@ -326,6 +344,9 @@ def bench_prefill(args, wl, rank, world, local_rank):
         del ws
         live_sum = int(sum(bin(t).count("1") + 1 for t in range(T))) * B * H
         readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
+        # Fenwick atoms of tile c: the tree blocks of [0, 128 c), one per set bit of c
+        loop_flops = atom_flops(sum(min(128, T - c * 128) * bin(c).count("1")
+                                    for c in range((T + 127) // 128)) * B * H, d)
 
         def step():
             dla.dla_fixed_policy_prefill(fcfg, q, k, v, o, fws, st, stream)
@@ -394,7 +415,11 @@ def bench_prefill(args, wl, rank, world, local_rank):
     n_launch = len(kt[dom])
     steps_recorded = args.steps
     if dom == "readout":
-        flops_per_launch = readout_flops / (n_launch / steps_recorded)
+        # the tensor-core readout's timed kernel is its atom loop (the prologue,
+        # "readout_pre", runs beside the materializer); the SIMT readout is one
+        # kernel doing all of the readout's work
+        work = readout_flops if args.path == "simt" else loop_flops
+        flops_per_launch = work / (n_launch / steps_recorded)
         if args.path == "simt":
             bound, unit = "alu", "TFLOP/s"
             peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12

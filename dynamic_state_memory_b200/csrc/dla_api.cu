@@ -71,6 +71,15 @@ Dims make_dims(const dla_config &cfg, int policy) {
   return dm;
 }
 
+// Per-tile outputs of the tensor-core readout's prologue kernel.
+void carve_pre(Carver &cv, const Dims &dm, Plan &pl) {
+  if (dm.vbytes != dm.D * dm.D * 2) return;  // SIMT path: none
+  const size_t g = (size_t)dm.heads * dm.tiles;
+  pl.pre_q = cv.take<char>(g * dm.M * dm.D * 2);
+  pl.pre_w = cv.take<float>(g * dm.amax * dm.M);
+  pl.pre_o = cv.take<float>(g * dm.M * dm.D);
+}
+
 void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   const size_t h = dm.heads;
   pl.r = cv.take<double>(h * dm.W);
@@ -93,6 +102,7 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.slot_ver = cv.take<int32_t>(h * dm.C);
   pl.pieces = cv.take<float>(h * (size_t)dm.pmax * dm.D * dm.D);
   pl.phi_tab = cv.take<double>(4096);
+  carve_pre(cv, dm, pl);
 }
 
 // Fixed Fenwick policy: one pass over the call (no windows); versions are the
@@ -130,6 +140,7 @@ void carve_fenwick(Carver &cv, const Dims &dm, Plan &pl, float **treeS, float **
   pl.ver_S = cv.take<char>(h * dm.vmax * (size_t)dm.vbytes);
   *treeS = cv.take<float>(h * dm.vmax * (size_t)dm.D * dm.D);
   *treeZ = cv.take<float>(h * dm.vmax * (size_t)dm.D);
+  carve_pre(cv, dm, pl);
 }
 
 bool cfg_ok(const dla_config *cfg, int policy) {
@@ -152,10 +163,12 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
 // thread's lifetime (non-blocking, so they never synchronise with the legacy
 // stream).  `s` runs the score and sums at normal priority; `se` runs the
 // engine at the highest priority: it is latency-bound and on the critical
-// path of a single window, so its few CTAs should get SMs first.
-enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_DONE0, EV_DONE1, EV_COUNT };
+// path of a single window, so its few CTAs should get SMs first; `sp` runs the
+// tensor-core readout's prologue beside the materializer at the lowest
+// priority, so that the materializer's CTAs are placed first.
+enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_PRE, EV_DONE0, EV_DONE1, EV_COUNT };
 struct Aux {
-  cudaStream_t s = nullptr, se = nullptr;
+  cudaStream_t s = nullptr, se = nullptr, sp = nullptr;
   cudaEvent_t ev[EV_COUNT] = {};
   bool ok = false;
 };
@@ -171,6 +184,8 @@ Aux *aux_streams() {
     if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
     if (!a.s && cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     if (!a.se && cudaStreamCreateWithPriority(&a.se, cudaStreamNonBlocking, hi) != cudaSuccess)
+      return nullptr;
+    if (!a.sp && cudaStreamCreateWithPriority(&a.sp, cudaStreamNonBlocking, lo) != cudaSuccess)
       return nullptr;
     for (cudaEvent_t &e : a.ev)
       if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
@@ -276,7 +291,7 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16)
     return DLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
-  Plan plans[2];
+  Plan plans[2] = {};
   Carver cv{static_cast<char *>(ws)};
   carve_plan(cv, dm, plans[0]);
   if (cfg->T > dm.W) carve_plan(cv, dm, plans[1]);
@@ -287,6 +302,7 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   if (!ax) return DLA_ERR_CUDA;
   cudaStream_t sd = ax->s;   // decisions: score, pieces, sums
   cudaStream_t se = ax->se;  // the engine
+  cudaStream_t sp = ax->sp;  // the tensor-core readout's prologue
   CallArgs ca{};
   ca.q = q;
   ca.k = k;
@@ -344,9 +360,17 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       e = launch_build_tc(dm, pl, ca, s);
       if (e != cudaSuccess) return DLA_ERR_CUDA;
     }
+    if (tc) {
+      // the readout's prologue needs the engine's atom lists and means, not
+      // the versions: it runs beside the materializer
+      if (cudaStreamWaitEvent(sp, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      { ProfScope ps(pf, DLA_K_READOUT_PRE, sp); e = launch_readout_pre_tc(dm, pl, ca, sp); }
+      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
+    }
     if (cudaStreamWaitEvent(s, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
+    if (tc && cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess) return DLA_ERR_CUDA;
     {
       ProfScope ps(pf, DLA_K_READOUT, s);
       e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
@@ -445,6 +469,10 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
   cudaError_t e;
   { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, s); }
   if (e != cudaSuccess) return DLA_ERR_CUDA;
+  if (tc) {
+    { ProfScope ps(pf, DLA_K_READOUT_PRE, s); e = launch_readout_pre_tc(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
+  }
   {
     ProfScope ps(pf, DLA_K_READOUT, s);
     e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);

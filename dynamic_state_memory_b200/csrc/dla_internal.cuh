@@ -87,6 +87,11 @@ struct Plan {
   int32_t *slot_ver;   // [heads][C] engine scratch
   double *phi_tab;     // phi in fp64 of negative bf16 inputs of moderate magnitude
   float *pieces;       // [heads][pmax][D][D] fp32 piece states
+  // tensor-core readout: per-tile outputs of the prologue kernel (null on
+  // the SIMT path)
+  void *pre_q;         // [heads][tiles] phi(Q) tiles, bf16 in the UMMA layout
+  float *pre_w;        // [heads][tiles][amax][M] atom weights
+  float *pre_o;        // [heads][tiles][M * D] intra-tile outputs
 };
 
 struct CallArgs {
@@ -137,6 +142,8 @@ cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s, bool bf16_versions);
+cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs &ca,
+                                  cudaStream_t s);
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_fen_leaves_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,

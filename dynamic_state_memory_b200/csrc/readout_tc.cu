@@ -1,28 +1,31 @@
-// readout_tc.cu -- tcgen05 tensor-core readout of one 128-token tile (bf16
-// inputs, fp32 accumulation, d_k = d_v = 128).
+// readout_tc.cu -- tcgen05 tensor-core readout of 128-token tiles (bf16
+// inputs, fp32 accumulation, d_k = d_v = 128), in two kernels.
 //
 // Same arithmetic as the SIMT readout (see readout_simt.cu for the atom /
 // piece / epoch formulation of o_t = sum_i lambda_{t,i} S_i phi(q_t) with
 // lambda_{t,i} = softmax_i(phi(q_t) . mu_i / sqrt(d_k)); Dynamic Linear
-// Attention | Chlience Paper Archive, section 5.3), mapped onto Blackwell:
+// Attention | Chlience Paper Archive, section 5.3), mapped onto Blackwell.
 //
+// k_readout_pre needs only the plan's atom lists and means, not the frozen
+// state versions, so it runs beside the materializer:
 //   TMA (128B swizzle) loads q, k, v tiles; phi is applied in shared memory.
 //   tcgen05.mma (kind::f16, M = 128 tokens) computes into tensor memory:
 //     A  = phi(Q) phi(K)^T               (128 x 128)   TMEM cols [256, 384)
 //     LA = phi(Q) Mu^T                   (128 x m0)    TMEM cols [384, 512)
 //   Four warps (one TMEM lane = one token row each) turn LA and the row sums
-//   of A into softmax weights per atom / piece, in place in TMEM, and write
+//   of A into softmax weights per atom / piece and write
 //   P = W o A (causal) as the bf16 A operand of
 //     O_intra = P V                                    TMEM cols [256, 384)
-//   Then, per atom alpha, a bulk copy brings the frozen bf16 state version
-//   (already stored in the UMMA K-major swizzled layout) into one of 6 shared
-//   stages (3 of their own, then the k and v tiles once P V has read them and
-//   the q tile once phi(Q) is in tensor memory),
-//   two threads issue P_alpha = phi(Q) S_alpha^T (even / odd atoms) into two
-//   TMEM buffers (cols [0,128) / [128,256)), with phi(Q) read from tensor
-//   memory (written into O_intra's columns once it has been read out), and 8
-//   epilogue warps, starting from O_intra, accumulate W_alpha(t) * P_alpha in
-//   registers while the next MMAs run.
+//   It stores phi(Q) (bf16, in the UMMA layout), the atom weights W[atom][row]
+//   and O_intra (fp32) to the plan.
+// k_readout_tc then runs the pipelined loop over atoms: the epilogue warps
+// start from O_intra and put phi(Q) into tensor memory; per atom alpha, a
+// bulk copy brings the frozen bf16 state version (already in the UMMA K-major
+// swizzled layout) into one of 4 shared stages (3 of their own, then the
+// phi(Q) tile), two threads issue P_alpha = phi(Q) S_alpha^T (even / odd
+// atoms) into three TMEM buffers with phi(Q) read from tensor memory, and 8
+// epilogue warps accumulate W_alpha(t) * P_alpha in registers while the next
+// MMAs run.
 // Every wait on an mbarrier is bounded; a timeout sets DLA_ERR_TIMEOUT.
 #include "dla_internal.cuh"
 #include "tc_ptx.cuh"
@@ -34,29 +37,44 @@ using namespace tc;
 constexpr int M = 128;
 constexpr int D = 128;
 constexpr int NST = 3;   // version stages of their own
-constexpr int NSV = 4;   // + the k tile once P V has read it
-constexpr int THREADS = 384;
+constexpr int NSV = 4;   // + the phi(Q) tile once it is in tensor memory
+constexpr int THREADS = 384;      // atom loop
+constexpr int PRE_THREADS = 256;  // per-tile prologue
 constexpr int TILE_BYTES = M * D * 2;
 constexpr uint32_t VER_BYTES = D * D * 2;
 constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
-constexpr uint32_t COL_BUF0 = 0, COL_AI = 256, COL_W = 384;
-constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and, once the weights have
-                        // been moved to shared memory, [384,512)
+constexpr uint32_t COL_AI = 256;  // phi(Q) of the atom loop
+constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and [384,512)
 __device__ __forceinline__ uint32_t pbuf_col(int b) { return b == 2 ? 384u : (uint32_t)b * 128u; }
-// phi(Q) as the A operand of the atom MMAs, in tensor memory once the
-// intra-tile output has been read out of the same columns: elements
+// phi(Q) as the A operand of the atom MMAs, in tensor memory: elements
 // [64h, 64h + 64) of a row in cols COL_AI + 64h + [0, 32), two per column
 __device__ __forceinline__ uint32_t qa_col(int kstep) {
   return COL_AI + (kstep < 4 ? 8 * kstep : 64 + 8 * (kstep - 4));
 }
 constexpr float INV_SQRT_D = 0.08838834764831845f;
+// Tensor memory of the prologue (256 columns, two CTAs per SM): A, then P in
+// place (the bf16 A operand of P V, laid out like phi(Q) above), in cols
+// [0, 128); LA, then O_intra, in cols [128, 256).
+constexpr uint32_t PRE_A = 0, PRE_LA = 128, PRE_COLS = 256;
+__device__ __forceinline__ uint32_t pa_col(int kstep) {
+  return PRE_A + (kstep < 4 ? 8 * kstep : 64 + 8 * (kstep - 4));
+}
+// column of P's elements [s0, s0 + 2n) (s0 even, within one half of 64)
+__device__ __forceinline__ uint32_t p_col(int s0) { return PRE_A + 64 * (s0 >> 6) + ((s0 & 63) >> 1); }
 
-struct Smem {
-  uint8_t q[TILE_BYTES];   // then (with v) the atom weights during the atom loop
-  uint8_t v[TILE_BYTES];
-  uint8_t kp[TILE_BYTES];
-  uint8_t st[NST][VER_BYTES];
-  uint64_t bar_load, bar_mma, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
+// ---- per-tile outputs of the prologue in the plan ----------------------------
+// phi(Q) of tile g: bf16 bytes [g * TILE_BYTES, +TILE_BYTES), the shared
+// layout (K-major, 128-byte swizzle).  W: fp32 [g][amax][M].  O_intra: fp32
+// [g][2][16][M][4] -- column 64 h + 4 i + e of row t at ((h * 16 + i) * M + t)
+// * 4 + e, so that a warp's 32 rows read or write 512 contiguous bytes.
+__device__ __forceinline__ size_t pre_o_index(int t, int h, int i) { return ((size_t)(h * 16 + i) * M + t) * 4; }
+
+struct PreSmem {
+  uint8_t q[TILE_BYTES];   // phi(Q)
+  uint8_t kp[TILE_BYTES];  // phi(K), then the v tile
+  uint8_t mu[TILE_BYTES];  // bf16 atom means in the 128-row UMMA layout (its second
+                           // K-half is 16 KB after the first, whatever the atom count)
+  uint64_t bar_load, bar_mma, bar_v;
   uint32_t tmem_base;
   int abort;
   int m0, np, len;
@@ -64,6 +82,17 @@ struct Smem {
   int atom[128];
   int pst[M + 1], pen[M + 1], pidx[M];
   uint32_t bits[(M + 1) * BW];
+};
+
+
+struct Smem {
+  uint8_t q[TILE_BYTES];  // phi(Q) on its way to tensor memory, then version stage NST
+  uint8_t st[NST][VER_BYTES];
+  float w[128 * M];       // W[atom][row]
+  uint64_t bar_load, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
+  uint32_t tmem_base;
+  int abort;
+  int atom[128];
 };
 
 __device__ __forceinline__ bool bit_of(const uint32_t *b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
@@ -90,39 +119,37 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return y[0];
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    k_readout_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                 const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
+__global__ void __launch_bounds__(PRE_THREADS, 2)
+    k_readout_pre(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
   extern __shared__ uint8_t raw[];
-  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
-                                       ~static_cast<uintptr_t>(1023));
+  PreSmem &sm = *reinterpret_cast<PreSmem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
   const int u = blockIdx.y, c = blockIdx.x;
   const int T0 = c * M;
   if (T0 >= ca.Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
-  auto stage = [&](int s) -> uint8_t * {
-    return s < NST ? sm.st[s] : sm.kp;
-  };
-  const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
+  const size_t g = (size_t)u * dm.tiles + c;  // tile index in the plan
+  float *const preW = pl.pre_w + g * dm.amax * M;
+  uint8_t *const mu_buf = sm.mu;
 
   // ---- setup: TMEM, barriers, tile loads first, then tile metadata --------
-  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if (warp == 1) tmem_alloc(&sm.tmem_base, PRE_COLS);
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
     fence_mbar_init();
-    mbar_expect_tx(&sm.bar_load, 3 * TILE_BYTES);
+    mbar_expect_tx(&sm.bar_load, 2 * TILE_BYTES);
     const int row = ca.w0 + T0;
     for (int h = 0; h < 2; h++) {
       tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, row, u);
       tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, row, u);
-      tma_load_3d(sm.v + h * (TILE_BYTES / 2), &tv, &sm.bar_load, h * 64, row, u);
     }
   }
   const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
   {
     const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
-    for (int a = tid; a < m0; a += THREADS) {
+    for (int a = tid; a < m0; a += PRE_THREADS) {
       const int at = atoms[a];
       sm.atom[a] = at;
       sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + at];
@@ -130,15 +157,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (tid == 0) {
     mbar_init(&sm.bar_mma, 1);
-    for (int i = 0; i < NSV; i++) {
-      mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], 1);
-    }
-    mbar_init(&sm.bar_qa, 8);
-    for (int i = 0; i < NPB; i++) {
-      mbar_init(&sm.tfull[i], 1);
-      mbar_init(&sm.tempty[i], 8);
-    }
+    mbar_init(&sm.bar_v, 1);
     fence_mbar_init();
     sm.abort = 0;
   }
@@ -212,17 +231,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     sm.pidx[tid] = p;
   }
 
-  // ---- loads --------------------------------------------------------------
-  if (tid == 0) {
-    for (int a = 0; a < m0 && a < NST - 1; a++) {
-      mbar_expect_tx(&sm.full[a], VER_BYTES);
-      bulk_load(sm.st[a], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[a]);
-    }
-  }
   mbar_wait(&sm.bar_load, 0, abort);
 
   // ---- phi(q), phi(k) in place; Mu (bf16 means of the atoms) ---------------
-  for (int i = tid; i < 2 * TILE_BYTES / 16; i += THREADS) {
+  for (int i = tid; i < 2 * TILE_BYTES / 16; i += PRE_THREADS) {
     uint4 *p = reinterpret_cast<uint4 *>(i < TILE_BYTES / 16 ? sm.q : sm.kp) + (i % (TILE_BYTES / 16));
     uint4 x = *p;
     uint32_t *w = reinterpret_cast<uint32_t *>(&x);
@@ -231,8 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     *p = x;
   }
   const int n_mu = (m0 + 15) & ~15;
-  uint8_t *mu_buf = sm.st[NST - 1];
-  for (int e = tid; e < n_mu * 16; e += THREADS) {
+  for (int e = tid; e < n_mu * 16; e += PRE_THREADS) {
     const int a = e >> 4, ch = e & 15;
     uint4 x = make_uint4(0, 0, 0, 0);
     if (a < m0) {
@@ -249,8 +260,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
+  if (tid == 0) {  // phi(Q) is final: store it for the atom loop
+    bulk_store(static_cast<uint8_t *>(pl.pre_q) + g * TILE_BYTES, sm.q, TILE_BYTES);
+    bulk_commit();
+  }
 
-  const uint32_t q_s = smem_u32(sm.q), kp_s = smem_u32(sm.kp), v_s = smem_u32(sm.v);
+  const uint32_t q_s = smem_u32(sm.q), kp_s = smem_u32(sm.kp);
   auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
     return sdesc(base + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024);
   };
@@ -258,19 +273,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1 && lane == 0) {
     tc_fence_after();
     for (int k = 0; k < 8; k++)
-      mma_bf16(tbase + COL_AI, kdesc(q_s, k), kdesc(kp_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
+      mma_bf16(tbase + PRE_A, kdesc(q_s, k), kdesc(kp_s, k), idesc_bf16(M, 128, 0, 0), k > 0);
     if (m0 > 0)
       for (int k = 0; k < 8; k++)
-        mma_bf16(tbase + COL_W, kdesc(q_s, k), kdesc(smem_u32(mu_buf), k),
+        mma_bf16(tbase + PRE_LA, kdesc(q_s, k), kdesc(smem_u32(mu_buf), k),
                  idesc_bf16(M, n_mu, 0, 0), k > 0);
     mma_commit(&sm.bar_mma);
   }
   mbar_wait(&sm.bar_mma, 0, abort);
   tc_fence_after();
-  if (tid == 0 && m0 >= NST) {
-    mbar_expect_tx(&sm.full[NST - 1], VER_BYTES);
-    bulk_load(sm.st[NST - 1], verS + (size_t)sm.atom[NST - 1] * VER_BYTES, VER_BYTES,
-              &sm.full[NST - 1]);
+  if (tid == 0) {  // phi(K) has been read: the v tile takes its place
+    mbar_expect_tx(&sm.bar_v, TILE_BYTES);
+    for (int h = 0; h < 2; h++)
+      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tv, &sm.bar_v, h * 64, ca.w0 + T0, u);
   }
 
   // ---- softmax weights per row (warps 4..7, row t = TMEM lane) ----------------
@@ -279,7 +294,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   // its last atom / piece (written in place); the softmax max and sum are
   // merged once per chunk.  Pass B walks backwards and gives every atom /
   // piece the weight of the state it belongs to.  Piece values live in
-  // registers when there are at most PREG pieces, else in TMEM cols [0, np).
+  // registers when there are at most PREG pieces, else in the tile's O_intra
+  // slot of the plan (written only at the end).  P replaces A in place.
   if (dm.fenwick && warp >= 4 && warp < 8) {
     // Row o: block sums of A[o][s] over the row's in-tile blocks (s < o lies
     // in the block of size 2^p, p = the highest bit where s and o differ),
@@ -294,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int s0 = 0; s0 < M; s0 += 8) {
       uint32_t ar[8];
-      DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+      DLA_TMEM_LD8(trow + PRE_A + s0, ar);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 8; j++) {
@@ -316,7 +332,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int a0 = 0; a0 < m0; a0 += 8) {
       uint32_t r[8];
-      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      DLA_TMEM_LD8(trow + PRE_LA + a0, r);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 8; j++)
@@ -329,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int a0 = 0; a0 < m0; a0 += 8) {
       uint32_t r[8];
-      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      DLA_TMEM_LD8(trow + PRE_LA + a0, r);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 8; j++)
@@ -339,13 +355,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int a0 = 0; a0 < m0; a0 += 8) {
       uint32_t r[8];
-      DLA_TMEM_LD8(trow + COL_W + a0, r);
+      DLA_TMEM_LD8(trow + PRE_LA + a0, r);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 8; j++)
-        r[j] = __float_as_uint(a0 + j < m0 ? __expf(__uint_as_float(r[j]) * INV_SQRT_D - mx) * inv_l : 0.f);
-      DLA_TMEM_ST8(trow + COL_W + a0, r);
-      tmem_wait_st();
+        if (a0 + j < m0) preW[(a0 + j) * M + t] = __expf(__uint_as_float(r[j]) * INV_SQRT_D - mx) * inv_l;
     }
     float wb[7];
 #pragma unroll
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int s0 = 0; s0 < M; s0 += 8) {
       uint32_t ar[8];
-      DLA_TMEM_LD8(trow + COL_AI + s0, ar);
+      DLA_TMEM_LD8(trow + PRE_A + s0, ar);
       tmem_wait_ld();
       uint32_t pk[4];
 #pragma unroll
@@ -372,8 +386,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         pk[j >> 1] = pack_bf16(v2[0], v2[1]);
       }
-      *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0, M)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      DLA_TMEM_ST4(trow + p_col(s0), pk);
     }
+    tmem_wait_st();
   } else if (warp >= 4 && warp < 8) {
     // One thread per row, blocks of 32 columns / atoms: one TMEM load per
     // block and 32 independent operations per step (a single warp per
@@ -389,6 +404,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t *bits = sm.bits + ep * BW;
     const int smax = min(32 * qd + 31, len - 1);  // last column a row of this warp reads
     float pv[PREG];  // piece sums, then logits, then weights
+    float *const ovf = pl.pre_o + g * M * D;  // pieces PREG.. (rows in columns)
 #pragma unroll
     for (int k = 0; k < PREG; k++) pv[k] = 0.f;
     auto piece_get = [&](int p) -> float {
@@ -398,17 +414,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int k = 0; k < PREG; k++) x = (k == p) ? pv[k] : x;
         return x;
       }
-      const float x = __uint_as_float(tmem_ld1(trow + COL_BUF0 + p));
-      tmem_wait_ld();
-      return x;
+      return ovf[(size_t)p * M + t];
     };
     auto piece_put = [&](int p, float x) {
       if (p < PREG) {
 #pragma unroll
         for (int k = 0; k < PREG; k++) pv[k] = (k == p) ? x : pv[k];
       } else {
-        tmem_st1(trow + COL_BUF0 + p, __float_as_uint(x));
-        tmem_wait_st();
+        ovf[(size_t)p * M + t] = x;
       }
     };
     // piece sums y_p(t) = sum_{s in p, s <= t} A[t][s]; pieces that start
@@ -420,7 +433,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
       for (int s0 = 0; s0 <= smax; s0 += 32) {
         uint32_t ar[32];
-        DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+        DLA_TMEM_LD32(trow + PRE_A + s0, ar);
         tmem_wait_ld();
         float x[32];
 #pragma unroll
@@ -452,7 +465,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int b = 0; b * 32 < m0; b++) {
       const int a0 = b * 32;
       uint32_t r[32];
-      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      DLA_TMEM_LD32(trow + PRE_LA + a0, r);
       const int nval = min(32, m0 - a0);
       const uint32_t vmask = nval == 32 ? ~0u : (1u << nval) - 1u;
       const uint32_t wb = bits[b] & vmask;
@@ -493,7 +506,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int k = 0; k < 4; k++) bmx[k] = (k == b) ? cmx : bmx[k];
 #pragma unroll
       for (int j = 0; j < 32; j++) r[j] = __float_as_uint(a[j]);
-      DLA_TMEM_ST32(trow + COL_W + a0, r);
+      DLA_TMEM_ST32(trow + PRE_LA + a0, r);
       tmem_wait_st();
     }
 #pragma unroll 1
@@ -532,7 +545,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int b = (m0 - 1) >> 5; m0 > 0 && b >= 0; b--) {
       const int a0 = b * 32;
       uint32_t r[32];
-      DLA_TMEM_LD32(trow + COL_W + a0, r);
+      DLA_TMEM_LD32(trow + PRE_LA + a0, r);
       const int nval = min(32, m0 - a0);
       const uint32_t vmask = nval == 32 ? ~0u : (1u << nval) - 1u;
       const uint32_t wb = bits[b] & vmask;
@@ -555,8 +568,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      DLA_TMEM_ST32(trow + COL_W + a0, r);
-      tmem_wait_st();
+#pragma unroll
+      for (int j = 0; j < 32; j++)
+        if (j < nval) preW[(a0 + j) * M + t] = __uint_as_float(r[j]);
     }
     // P[t][s] = W_{piece(s)}(t) A[t][s] for s <= t, as the bf16 A operand of
     // P V; columns past the warp's last row are zero
@@ -571,7 +585,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < 16; j++) pk[j] = 0u;
         if (s0 <= smax) {
           uint32_t ar[32];
-          DLA_TMEM_LD32(trow + COL_AI + s0, ar);
+          DLA_TMEM_LD32(trow + PRE_A + s0, ar);
           tmem_wait_ld();
           float v[32];
 #pragma unroll
@@ -595,25 +609,116 @@ __global__ void __launch_bounds__(THREADS, 1)
             pk[j] = pack_bf16((s <= t && s < len) ? v[2 * j] : 0.f, (s + 1 <= t && s + 1 < len) ? v[2 * j + 1] : 0.f);
           }
         }
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-          *reinterpret_cast<uint4 *>(sm.kp + sw128_offset(t, s0 + 8 * i, M)) =
-              make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        DLA_TMEM_ST16(trow + p_col(s0), pk);
       }
+      tmem_wait_st();
     }
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
 
-  // ---- P V, then the pipelined readout over atoms --------------------------
-  // Two issuing threads (warp 1: even atoms into TMEM buffer 0, warp 2: odd
-  // atoms into buffer 1); an issuing thread is held for about the duration of
-  // its MMAs, so with one issuer every barrier wait left the tensor pipe idle.
-  // The atom MMAs read phi(Q) from tensor memory: with both operands in shared
-  // memory, their reads plus the version copies exceeded its bandwidth.  Atom
-  // a goes to product buffer a % 3: three buffers cover a buffer's round trip
-  // (MMAs, commit, epilogue drain, release) at the MMA rate.
+  // ---- O_intra = P V, stored for the atom loop -------------------------------
+  if (warp == 1 && lane == 0) {
+    const bool ok = mbar_wait(&sm.bar_v, 0, abort);
+    tc_fence_after();
+    if (ok)
+      for (int k = 0; k < 8; k++)
+        mma_bf16_ta(tbase + PRE_LA, tbase + pa_col(k), sdesc(kp_s + k * 2048, TILE_BYTES / 2, 1024),
+                    idesc_bf16(M, 128, 0, 1), k > 0);
+    mma_commit(&sm.bar_mma);
+  }
+  mbar_wait(&sm.bar_mma, 1, abort);
+  tc_fence_after();
+  {
+    const int qd = warp & 3, hc = warp >> 2;
+    const int t = 32 * qd + lane;
+    const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+    float4 *dst = reinterpret_cast<float4 *>(pl.pre_o + g * M * D);
+#pragma unroll
+    for (int half = 0; half < 2; half++) {
+      uint32_t pr[32];
+      DLA_TMEM_LD32(trow + PRE_LA + hc * 64 + 32 * half, pr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 8; i++)
+        dst[pre_o_index(t, hc, 8 * half + i) / 4] =
+            make_float4(__uint_as_float(pr[4 * i]), __uint_as_float(pr[4 * i + 1]),
+                        __uint_as_float(pr[4 * i + 2]), __uint_as_float(pr[4 * i + 3]));
+    }
+  }
+  if (tid == 0) bulk_wait_read();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, PRE_COLS);
+  }
+  if (tid == 0 && sm.abort) set_status(ca.dev_status, DLA_ERR_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) k_readout_tc(Dims dm, Plan pl, CallArgs ca) {
+  extern __shared__ uint8_t raw[];
+  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                       ~static_cast<uintptr_t>(1023));
+  const int u = blockIdx.y, c = blockIdx.x;
+  const int T0 = c * M;
+  if (T0 >= ca.Tw) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int *abort = &sm.abort;
+  auto stage = [&](int s) -> uint8_t * {
+    return s < NST ? sm.st[s] : sm.q;
+  };
+  const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
+  const size_t g = (size_t)u * dm.tiles + c;
+  const int m0 = pl.tile_m0[g];
+  const int len = min(M, ca.Tw - T0);
+
+  // ---- setup: TMEM, barriers, the prologue's phi(Q) and weights -------------
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if (tid == 0) {
+    mbar_init(&sm.bar_load, 1);
+    mbar_init(&sm.bar_qa, 8);
+    for (int i = 0; i < NSV; i++) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < NPB; i++) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], 8);
+    }
+    fence_mbar_init();
+    sm.abort = 0;
+    const uint32_t wbytes = (uint32_t)m0 * M * 4;
+    mbar_expect_tx(&sm.bar_load, TILE_BYTES + wbytes);
+    bulk_load(sm.q, static_cast<const uint8_t *>(pl.pre_q) + g * TILE_BYTES, TILE_BYTES, &sm.bar_load);
+    if (m0 > 0) bulk_load(sm.w, pl.pre_w + g * dm.amax * M, wbytes, &sm.bar_load);
+  }
+  {
+    const int32_t *atoms = pl.tile_atoms + g * dm.amax;
+    for (int a = tid; a < m0; a += THREADS) sm.atom[a] = atoms[a];
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  if (tid == 0) {
+    for (int a = 0; a < m0 && a < NST; a++) {
+      mbar_expect_tx(&sm.full[a], VER_BYTES);
+      bulk_load(sm.st[a], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[a]);
+    }
+  }
+  auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
+    return sdesc(base + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024);
+  };
+
+  // ---- the pipelined readout over atoms --------------------------------------
+  // Two issuing threads (warp 1: even atoms, warp 2: odd atoms); an issuing
+  // thread is held for about the duration of its MMAs, so with one issuer
+  // every barrier wait left the tensor pipe idle.  The atom MMAs read phi(Q)
+  // from tensor memory: with both operands in shared memory, their reads plus
+  // the version copies exceeded its bandwidth.  Atom a goes to product buffer
+  // a % 3: three buffers cover a buffer's round trip (MMAs, commit, epilogue
+  // drain, release) at the MMA rate.
   auto issue_atoms = [&](int first) {
     bool ok_qa = first < m0 ? mbar_wait(&sm.bar_qa, 0, abort) : true;
     for (int a = first; a < m0; a += 2) {
@@ -633,10 +738,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   };
   if (warp == 1 && lane == 0) {
     tc_fence_after();
-    for (int k = 0; k < 8; k++)
-      mma_bf16(tbase + COL_AI, kdesc(kp_s, k), sdesc(v_s + k * 2048, TILE_BYTES / 2, 1024),
-               idesc_bf16(M, 128, 0, 1), k > 0);
-    mma_commit(&sm.bar_mma);
     issue_atoms(0);
   } else if (warp == 2 && lane == 0) {
     tc_fence_after();
@@ -650,10 +751,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int a = NST; a < m0; a++) {
       if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)sm.atom[a + PF] * VER_BYTES, VER_BYTES);
       const int s = a % NSV;
-      // stage NST is the k tile: free once P V has completed (bar_mma phase
-      // 1; phase 0, the first MMAs, completed before here)
+      // stage NST is the phi(Q) tile: free once every epilogue warp has put
+      // its rows into tensor memory (bar_qa)
       const bool ok = a >= NSV ? mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort)
-                               : mbar_wait(&sm.bar_mma, 1, abort);
+                               : mbar_wait(&sm.bar_qa, 0, abort);
       if (!ok) break;
       mbar_expect_tx(&sm.full[s], VER_BYTES);
       bulk_load(stage(s), verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
@@ -663,20 +764,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     float acc[64];
-    // start from the intra-tile output, then put phi(Q) in its columns
-    mbar_wait(&sm.bar_mma, 1, abort);
-    tc_fence_after();
-    {
-      uint32_t pr[32];
-      DLA_TMEM_LD32(trow + COL_AI + hc * 64, pr);
-      tmem_wait_ld();
+    {  // start from the intra-tile output
+      const float4 *src = reinterpret_cast<const float4 *>(pl.pre_o + g * M * D);
 #pragma unroll
-      for (int i = 0; i < 32; i++) acc[i] = __uint_as_float(pr[i]);
-      DLA_TMEM_LD32(trow + COL_AI + hc * 64 + 32, pr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i++) acc[32 + i] = __uint_as_float(pr[i]);
+      for (int i = 0; i < 16; i++) {
+        const float4 x = src[pre_o_index(t, hc, i) / 4];
+        acc[4 * i] = x.x;
+        acc[4 * i + 1] = x.y;
+        acc[4 * i + 2] = x.z;
+        acc[4 * i + 3] = x.w;
+      }
     }
+    mbar_wait(&sm.bar_load, 0, abort);
     {
       // row t, elements [64 hc, 64 hc + 64) of phi(q_t), from the swizzled tile
       uint32_t qw[32];
@@ -691,26 +790,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       DLA_TMEM_ST32(trow + COL_AI + 64 * hc, qw);
       tmem_wait_st();
     }
-    // every epilogue warp has read its phi(Q) rows: the q and v tiles now take
-    // the weights, W[atom][row] in fp32, and their TMEM columns become buffer 2
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    float *sW = reinterpret_cast<float *>(sm.q);
-    {
-      const int half = (m0 + 15) / 16 * 8;  // atoms per warp half, in chunks of 8
-      const int a_lo = hc * half, a_hi = min(m0, a_lo + half);
-#pragma unroll 1
-      for (int a0 = a_lo; a0 < a_hi; a0 += 8) {
-        uint32_t r[8];
-        DLA_TMEM_LD8(trow + COL_W + a0, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 8; j++)
-          if (a0 + j < a_hi) sW[(a0 + j) * M + t] = __uint_as_float(r[j]);
-      }
-    }
+    // the tile's shared copy is read (it becomes a version stage)
+    fence_proxy_async();
     tc_fence_before();
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    __syncwarp();
     if (lane == 0) mbar_arrive(&sm.bar_qa);
+    const float *sW = sm.w;
 #pragma unroll 1
     for (int a = 0; a < m0; a++) {
       const int b = a % NPB;
@@ -789,20 +874,32 @@ constexpr int kTileRows = M;
 }
 int tc_tile_rows() { return kTileRows; }
 
-size_t readout_tc_smem() { return sizeof(Smem) + 1024; }
-
-cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16) return cudaErrorInvalidValue;
+cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs &ca,
+                                  cudaStream_t s) {
+  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.pre_q)
+    return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   if (!make_bf16_map(&tq, ca.q, dm.T, dm.heads) || !make_bf16_map(&tk, ca.k, dm.T, dm.heads) ||
       !make_bf16_map(&tv, ca.v, dm.T, dm.heads))
     return cudaErrorInvalidValue;
-  const size_t sb = readout_tc_smem();
+  const size_t sb = sizeof(PreSmem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_readout_pre, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sb);
+  if (e != cudaSuccess) return e;
+  dim3 g(dm.tiles, dm.heads);
+  k_readout_pre<<<g, PRE_THREADS, sb, s>>>(tq, tk, tv, dm, pl, ca);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.pre_q)
+    return cudaErrorInvalidValue;
+  const size_t sb = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sb);
   if (e != cudaSuccess) return e;
   dim3 g(dm.tiles, dm.heads);
-  k_readout_tc<<<g, THREADS, sb, s>>>(tq, tk, tv, dm, pl, ca);
+  k_readout_tc<<<g, THREADS, sb, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }
 
