@@ -75,9 +75,10 @@ Dims make_dims(const dla_config &cfg, int policy) {
 void carve_pre(Carver &cv, const Dims &dm, Plan &pl) {
   if (dm.vbytes != dm.D * dm.D * 2) return;  // SIMT path: none
   const size_t g = (size_t)dm.heads * dm.tiles;
-  pl.pre_q = cv.take<char>(g * dm.M * dm.D * 2);
+  pl.phi_q = cv.take<char>((size_t)dm.heads * dm.W * dm.D * 2);
+  pl.phi_k = cv.take<char>((size_t)dm.heads * dm.W * dm.D * 2);
   pl.pre_w = cv.take<float>(g * dm.amax * dm.M);
-  pl.pre_o = cv.take<float>(g * dm.M * dm.D);
+  pl.pre_o = cv.take<char>(g * dm.M * dm.D * 2);
 }
 
 void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
@@ -163,12 +164,13 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
 // thread's lifetime (non-blocking, so they never synchronise with the legacy
 // stream).  `s` runs the score and sums at normal priority; `se` runs the
 // engine at the highest priority: it is latency-bound and on the critical
-// path of a single window, so its few CTAs should get SMs first; `sp` runs the
-// tensor-core readout's prologue beside the materializer at the lowest
-// priority, so that the materializer's CTAs are placed first.
-enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_PRE, EV_DONE0, EV_DONE1, EV_COUNT };
+// path of a single window, so its few CTAs should get SMs first.  With the
+// tensor-core readout, `sx` runs the materializer at the highest priority and
+// `sp` the readout's prologue beside it at the lowest, so that the
+// materializer's CTAs are placed first.
+enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_BUILD, EV_MAT, EV_PRE, EV_DONE0, EV_DONE1, EV_COUNT };
 struct Aux {
-  cudaStream_t s = nullptr, se = nullptr, sp = nullptr;
+  cudaStream_t s = nullptr, se = nullptr, sp = nullptr, sx = nullptr;
   cudaEvent_t ev[EV_COUNT] = {};
   bool ok = false;
 };
@@ -186,6 +188,8 @@ Aux *aux_streams() {
     if (!a.se && cudaStreamCreateWithPriority(&a.se, cudaStreamNonBlocking, hi) != cudaSuccess)
       return nullptr;
     if (!a.sp && cudaStreamCreateWithPriority(&a.sp, cudaStreamNonBlocking, lo) != cudaSuccess)
+      return nullptr;
+    if (!a.sx && cudaStreamCreateWithPriority(&a.sx, cudaStreamNonBlocking, hi) != cudaSuccess)
       return nullptr;
     for (cudaEvent_t &e : a.ev)
       if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
@@ -303,6 +307,7 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   cudaStream_t sd = ax->s;   // decisions: score, pieces, sums
   cudaStream_t se = ax->se;  // the engine
   cudaStream_t sp = ax->sp;  // the tensor-core readout's prologue
+  cudaStream_t sx = ax->sx;  // the materializer, with the tensor-core readout
   CallArgs ca{};
   ca.q = q;
   ca.k = k;
@@ -326,7 +331,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   // auxiliary launch is ordered before a later wait of the caller's stream,
   // so the call ends (joins) on the caller's stream.
   if (cudaEventRecord(ax->ev[EV_START], s) != cudaSuccess ||
-      cudaStreamWaitEvent(sd, ax->ev[EV_START], 0) != cudaSuccess)
+      cudaStreamWaitEvent(sd, ax->ev[EV_START], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(sp, ax->ev[EV_START], 0) != cudaSuccess)
     return DLA_ERR_CUDA;
   const bool tc = use_tc(*cfg);
   dla_profile *pf = cfg->profile;
@@ -353,12 +359,21 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     { ProfScope ps(pf, DLA_K_ENGINE, se); e = launch_engine(dm, pl, ca, se); }
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], se) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc) {
+      // phi(q), phi(k) of the window beside the latency-bound engine (after
+      // the sums, whose memory traffic it would slow); the plan's phi buffers
+      // were last read by window wi - 2's readout
+      if (cudaStreamWaitEvent(sp, ax->ev[EV_SUMS], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      if (wi >= 2 && cudaStreamWaitEvent(sp, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)
+        return DLA_ERR_CUDA;
+      { ProfScope ps(pf, DLA_K_PHI, sp); e = launch_phi_tc(dm, pl, ca, sp); }
+      if (e != cudaSuccess) return DLA_ERR_CUDA;
+    }
+    if (tc) {
       // after the sums (not just the boundary flags it reads), so it overlaps
       // the engine without slowing the sums ahead of it
       if (cudaStreamWaitEvent(s, ax->ev[EV_SUMS], 0) != cudaSuccess) return DLA_ERR_CUDA;
-      ProfScope ps(pf, DLA_K_BUILD, s);
-      e = launch_build_tc(dm, pl, ca, s);
-      if (e != cudaSuccess) return DLA_ERR_CUDA;
+      { ProfScope ps(pf, DLA_K_BUILD, s); e = launch_build_tc(dm, pl, ca, s); }
+      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_BUILD], s) != cudaSuccess) return DLA_ERR_CUDA;
     }
     if (tc) {
       // the readout's prologue needs the engine's atom lists and means, not
@@ -367,10 +382,20 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       { ProfScope ps(pf, DLA_K_READOUT_PRE, sp); e = launch_readout_pre_tc(dm, pl, ca, sp); }
       if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
     }
-    if (cudaStreamWaitEvent(s, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_materialize(dm, pl, ca, s, tc); }
+    // the materializer: after the engine (ops) and the builder (pieces); on
+    // sx it also waits for window wi - 2's readout, the last reader of this
+    // plan's versions, and for the previous materializer through stream order
+    cudaStream_t sm_ = tc ? sx : s;
+    if (cudaStreamWaitEvent(sm_, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
+    if (tc && (cudaStreamWaitEvent(sx, ax->ev[EV_BUILD], 0) != cudaSuccess ||
+               (wi >= 2 && cudaStreamWaitEvent(sx, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)))
+      return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_MATERIALIZE, sm_); e = launch_materialize(dm, pl, ca, sm_, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
-    if (tc && cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess) return DLA_ERR_CUDA;
+    if (tc && (cudaEventRecord(ax->ev[EV_MAT], sx) != cudaSuccess ||
+               cudaStreamWaitEvent(s, ax->ev[EV_MAT], 0) != cudaSuccess ||
+               cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess))
+      return DLA_ERR_CUDA;
     {
       ProfScope ps(pf, DLA_K_READOUT, s);
       e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
@@ -470,6 +495,8 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
   { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, s); }
   if (e != cudaSuccess) return DLA_ERR_CUDA;
   if (tc) {
+    { ProfScope ps(pf, DLA_K_PHI, s); e = launch_phi_tc(dm, pl, ca, s); }
+    if (e != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_READOUT_PRE, s); e = launch_readout_pre_tc(dm, pl, ca, s); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
   }

@@ -89,9 +89,9 @@ struct Plan {
   float *pieces;       // [heads][pmax][D][D] fp32 piece states
   // tensor-core readout: per-tile outputs of the prologue kernel (null on
   // the SIMT path)
-  void *pre_q;         // [heads][tiles] phi(Q) tiles, bf16 in the UMMA layout
+  void *phi_q, *phi_k; // [heads][W][D] bf16 phi(q), phi(k) of the window's rows
   float *pre_w;        // [heads][tiles][amax][M] atom weights
-  float *pre_o;        // [heads][tiles][M * D] intra-tile outputs
+  void *pre_o;         // [heads][tiles][M * D] intra-tile outputs (bf16)
 };
 
 struct CallArgs {
@@ -142,6 +142,7 @@ cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s, bool bf16_versions);
+cudaError_t launch_phi_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                   cudaStream_t s);
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);

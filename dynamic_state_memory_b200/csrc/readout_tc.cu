@@ -6,9 +6,11 @@
 // lambda_{t,i} = softmax_i(phi(q_t) . mu_i / sqrt(d_k)); Dynamic Linear
 // Attention | Chlience Paper Archive, section 5.3), mapped onto Blackwell.
 //
+// k_phi_tc writes phi(q) and phi(k) of the window as bf16 operands (it needs
+// only the inputs, so it runs beside the decision kernels).
 // k_readout_pre needs only the plan's atom lists and means, not the frozen
 // state versions, so it runs beside the materializer:
-//   TMA (128B swizzle) loads q, k, v tiles; phi is applied in shared memory.
+//   TMA (128B swizzle) loads the phi(q), phi(k) and v tiles.
 //   tcgen05.mma (kind::f16, M = 128 tokens) computes into tensor memory:
 //     A  = phi(Q) phi(K)^T               (128 x 128)   TMEM cols [256, 384)
 //     LA = phi(Q) Mu^T                   (128 x m0)    TMEM cols [384, 512)
@@ -16,8 +18,7 @@
 //   of A into softmax weights per atom / piece and write
 //   P = W o A (causal) as the bf16 A operand of
 //     O_intra = P V                                    TMEM cols [256, 384)
-//   It stores phi(Q) (bf16, in the UMMA layout), the atom weights W[atom][row]
-//   and O_intra (fp32) to the plan.
+//   It stores the atom weights W[atom][row] and O_intra (fp32) to the plan.
 // k_readout_tc then runs the pipelined loop over atoms: the epilogue warps
 // start from O_intra and put phi(Q) into tensor memory; per atom alpha, a
 // bulk copy brings the frozen bf16 state version (already in the UMMA K-major
@@ -63,17 +64,19 @@ __device__ __forceinline__ uint32_t pa_col(int kstep) {
 __device__ __forceinline__ uint32_t p_col(int s0) { return PRE_A + 64 * (s0 >> 6) + ((s0 & 63) >> 1); }
 
 // ---- per-tile outputs of the prologue in the plan ----------------------------
-// phi(Q) of tile g: bf16 bytes [g * TILE_BYTES, +TILE_BYTES), the shared
-// layout (K-major, 128-byte swizzle).  W: fp32 [g][amax][M].  O_intra: fp32
-// [g][2][16][M][4] -- column 64 h + 4 i + e of row t at ((h * 16 + i) * M + t)
-// * 4 + e, so that a warp's 32 rows read or write 512 contiguous bytes.
-__device__ __forceinline__ size_t pre_o_index(int t, int h, int i) { return ((size_t)(h * 16 + i) * M + t) * 4; }
+// W: fp32 [g][amax][M].  O_intra: bf16 [g][2][8][M][8] -- column 64 h + 8 i + e
+// of row t at ((h * 8 + i) * M + t) * 8 + e, so that a warp's 32 rows read or
+// write 512 contiguous bytes (its rounding is far inside the bf16 output's
+// tolerance; the atom loop accumulates in fp32).
+__device__ __forceinline__ size_t pre_o_chunk(int t, int h, int i) { return (size_t)(h * 8 + i) * M + t; }
 
 struct PreSmem {
-  uint8_t q[TILE_BYTES];   // phi(Q)
   uint8_t kp[TILE_BYTES];  // phi(K), then the v tile
+  uint8_t q[TILE_BYTES];   // phi(Q)
   uint8_t mu[TILE_BYTES];  // bf16 atom means in the 128-row UMMA layout (its second
                            // K-half is 16 KB after the first, whatever the atom count)
+                           // q and mu, once the first MMAs have read them, hold the
+                           // values of pieces PREG.. (fp32 [piece][row], 128 pieces)
   uint64_t bar_load, bar_mma, bar_v;
   uint32_t tmem_base;
   int abort;
@@ -84,6 +87,8 @@ struct PreSmem {
   uint32_t bits[(M + 1) * BW];
 };
 
+
+static_assert(offsetof(PreSmem, mu) == offsetof(PreSmem, q) + TILE_BYTES, "q, mu adjacent");
 
 struct Smem {
   uint8_t q[TILE_BYTES];  // phi(Q) on its way to tensor memory, then version stage NST
@@ -119,6 +124,25 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return y[0];
 }
 
+// phi(q), phi(k) of the window's rows as the bf16 operands of the readout:
+// phi_q / phi_k [heads][W][D], rows [0, Tw) (16 bytes per thread and step).
+__global__ void __launch_bounds__(256) k_phi_tc(Dims dm, Plan pl, CallArgs ca) {
+  const size_t per_head = (size_t)ca.Tw * (D / 8);
+  const size_t half = per_head * dm.heads;
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < 2 * half; i += (size_t)gridDim.x * 256) {
+    const bool is_k = i >= half;
+    const size_t j = is_k ? i - half : i;
+    const size_t u = j / per_head, r = j - u * per_head;
+    const uint4 *src = static_cast<const uint4 *>(is_k ? ca.k : ca.q) + (u * dm.T + ca.w0) * (D / 8) + r;
+    uint4 *dst = static_cast<uint4 *>(is_k ? pl.phi_k : pl.phi_q) + u * dm.W * (D / 8) + r;
+    uint4 x = *src;
+    uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+    for (int e = 0; e < 4; e++) w[e] = pack_bf16(phi_bf16op(bf16_lo(w[e])), phi_bf16op(bf16_hi(w[e])));
+    *dst = x;
+  }
+}
+
 __global__ void __launch_bounds__(PRE_THREADS, 2)
     k_readout_pre(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
@@ -140,10 +164,9 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     mbar_init(&sm.bar_load, 1);
     fence_mbar_init();
     mbar_expect_tx(&sm.bar_load, 2 * TILE_BYTES);
-    const int row = ca.w0 + T0;
     for (int h = 0; h < 2; h++) {
-      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, row, u);
-      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, row, u);
+      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, T0, u);
+      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, T0, u);
     }
   }
   const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
@@ -233,15 +256,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
 
   mbar_wait(&sm.bar_load, 0, abort);
 
-  // ---- phi(q), phi(k) in place; Mu (bf16 means of the atoms) ---------------
-  for (int i = tid; i < 2 * TILE_BYTES / 16; i += PRE_THREADS) {
-    uint4 *p = reinterpret_cast<uint4 *>(i < TILE_BYTES / 16 ? sm.q : sm.kp) + (i % (TILE_BYTES / 16));
-    uint4 x = *p;
-    uint32_t *w = reinterpret_cast<uint32_t *>(&x);
-#pragma unroll
-    for (int j = 0; j < 4; j++) w[j] = pack_bf16(phi_bf16op(bf16_lo(w[j])), phi_bf16op(bf16_hi(w[j])));
-    *p = x;
-  }
+  // ---- Mu (bf16 means of the atoms) -------------------------------------------
   const int n_mu = (m0 + 15) & ~15;
   for (int e = tid; e < n_mu * 16; e += PRE_THREADS) {
     const int a = e >> 4, ch = e & 15;
@@ -260,10 +275,6 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
-  if (tid == 0) {  // phi(Q) is final: store it for the atom loop
-    bulk_store(static_cast<uint8_t *>(pl.pre_q) + g * TILE_BYTES, sm.q, TILE_BYTES);
-    bulk_commit();
-  }
 
   const uint32_t q_s = smem_u32(sm.q), kp_s = smem_u32(sm.kp);
   auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     const uint32_t *bits = sm.bits + ep * BW;
     const int smax = min(32 * qd + 31, len - 1);  // last column a row of this warp reads
     float pv[PREG];  // piece sums, then logits, then weights
-    float *const ovf = pl.pre_o + g * M * D;  // pieces PREG.. (rows in columns)
+    float *const ovf = reinterpret_cast<float *>(sm.q);  // pieces PREG.. (rows in columns)
 #pragma unroll
     for (int k = 0; k < PREG; k++) pv[k] = 0.f;
     auto piece_get = [&](int p) -> float {
@@ -634,20 +645,21 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     const int qd = warp & 3, hc = warp >> 2;
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
-    float4 *dst = reinterpret_cast<float4 *>(pl.pre_o + g * M * D);
+    uint4 *dst = reinterpret_cast<uint4 *>(pl.pre_o) + g * (M * D / 8);
 #pragma unroll
     for (int half = 0; half < 2; half++) {
       uint32_t pr[32];
       DLA_TMEM_LD32(trow + PRE_LA + hc * 64 + 32 * half, pr);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 8; i++)
-        dst[pre_o_index(t, hc, 8 * half + i) / 4] =
-            make_float4(__uint_as_float(pr[4 * i]), __uint_as_float(pr[4 * i + 1]),
-                        __uint_as_float(pr[4 * i + 2]), __uint_as_float(pr[4 * i + 3]));
+      for (int i = 0; i < 4; i++)
+        dst[pre_o_chunk(t, hc, 4 * half + i)] =
+            make_uint4(pack_bf16(__uint_as_float(pr[8 * i]), __uint_as_float(pr[8 * i + 1])),
+                       pack_bf16(__uint_as_float(pr[8 * i + 2]), __uint_as_float(pr[8 * i + 3])),
+                       pack_bf16(__uint_as_float(pr[8 * i + 4]), __uint_as_float(pr[8 * i + 5])),
+                       pack_bf16(__uint_as_float(pr[8 * i + 6]), __uint_as_float(pr[8 * i + 7])));
     }
   }
-  if (tid == 0) bulk_wait_read();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -657,7 +669,8 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
   if (tid == 0 && sm.abort) set_status(ca.dev_status, DLA_ERR_TIMEOUT);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) k_readout_tc(Dims dm, Plan pl, CallArgs ca) {
+__global__ void __launch_bounds__(THREADS, 1)
+    k_readout_tc(const __grid_constant__ CUtensorMap tq, Dims dm, Plan pl, CallArgs ca) {
   extern __shared__ uint8_t raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                        ~static_cast<uintptr_t>(1023));
@@ -674,7 +687,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_readout_tc(Dims dm, Plan pl, Cal
   const int m0 = pl.tile_m0[g];
   const int len = min(M, ca.Tw - T0);
 
-  // ---- setup: TMEM, barriers, the prologue's phi(Q) and weights -------------
+  // ---- setup: TMEM, barriers, the phi(Q) tile and the prologue's weights ----
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
@@ -691,7 +704,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_readout_tc(Dims dm, Plan pl, Cal
     sm.abort = 0;
     const uint32_t wbytes = (uint32_t)m0 * M * 4;
     mbar_expect_tx(&sm.bar_load, TILE_BYTES + wbytes);
-    bulk_load(sm.q, static_cast<const uint8_t *>(pl.pre_q) + g * TILE_BYTES, TILE_BYTES, &sm.bar_load);
+    for (int h = 0; h < 2; h++)
+      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, T0, u);
     if (m0 > 0) bulk_load(sm.w, pl.pre_w + g * dm.amax * M, wbytes, &sm.bar_load);
   }
   {
@@ -765,14 +779,18 @@ __global__ void __launch_bounds__(THREADS, 1) k_readout_tc(Dims dm, Plan pl, Cal
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
     float acc[64];
     {  // start from the intra-tile output
-      const float4 *src = reinterpret_cast<const float4 *>(pl.pre_o + g * M * D);
+      const uint4 *src = reinterpret_cast<const uint4 *>(pl.pre_o) + g * (M * D / 8);
 #pragma unroll
-      for (int i = 0; i < 16; i++) {
-        const float4 x = src[pre_o_index(t, hc, i) / 4];
-        acc[4 * i] = x.x;
-        acc[4 * i + 1] = x.y;
-        acc[4 * i + 2] = x.z;
-        acc[4 * i + 3] = x.w;
+      for (int i = 0; i < 8; i++) {
+        const uint4 x = src[pre_o_chunk(t, hc, i)];
+        acc[8 * i] = bf16_lo(x.x);
+        acc[8 * i + 1] = bf16_hi(x.x);
+        acc[8 * i + 2] = bf16_lo(x.y);
+        acc[8 * i + 3] = bf16_hi(x.y);
+        acc[8 * i + 4] = bf16_lo(x.z);
+        acc[8 * i + 5] = bf16_hi(x.z);
+        acc[8 * i + 6] = bf16_lo(x.w);
+        acc[8 * i + 7] = bf16_hi(x.w);
       }
     }
     mbar_wait(&sm.bar_load, 0, abort);
@@ -855,13 +873,19 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+bool make_bf16_map_rows(CUtensorMap *m, const void *base, int rows, int stride_rows, int heads);
+
 // 3D tensor map {d = 128, T, heads} of a bf16 [heads][T][128] tensor, boxes of
 // 64 x 128 x 1 with the 128-byte swizzle (out-of-range rows read as zero).
 bool make_bf16_map(CUtensorMap *m, const void *base, int T, int heads) {
+  return make_bf16_map_rows(m, base, T, T, heads);
+}
+// The same over the first `rows` of every head's `stride_rows` rows.
+bool make_bf16_map_rows(CUtensorMap *m, const void *base, int rows, int stride_rows, int heads) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)stride_rows * D * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)M, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
@@ -874,12 +898,19 @@ constexpr int kTileRows = M;
 }
 int tc_tile_rows() { return kTileRows; }
 
+cudaError_t launch_phi_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  if (dm.D != D || ca.in_dtype != DLA_BF16 || !pl.phi_q) return cudaErrorInvalidValue;
+  k_phi_tc<<<148 * 8, 256, 0, s>>>(dm, pl, ca);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                   cudaStream_t s) {
-  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.pre_q)
+  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.phi_q)
     return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!make_bf16_map(&tq, ca.q, dm.T, dm.heads) || !make_bf16_map(&tk, ca.k, dm.T, dm.heads) ||
+  if (!make_bf16_map_rows(&tq, pl.phi_q, ca.Tw, dm.W, dm.heads) ||
+      !make_bf16_map_rows(&tk, pl.phi_k, ca.Tw, dm.W, dm.heads) ||
       !make_bf16_map(&tv, ca.v, dm.T, dm.heads))
     return cudaErrorInvalidValue;
   const size_t sb = sizeof(PreSmem) + 1024;
@@ -892,14 +923,16 @@ cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs
 }
 
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.pre_q)
+  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.phi_q)
     return cudaErrorInvalidValue;
+  CUtensorMap tq;
+  if (!make_bf16_map_rows(&tq, pl.phi_q, ca.Tw, dm.W, dm.heads)) return cudaErrorInvalidValue;
   const size_t sb = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sb);
   if (e != cudaSuccess) return e;
   dim3 g(dm.tiles, dm.heads);
-  k_readout_tc<<<g, THREADS, sb, s>>>(dm, pl, ca);
+  k_readout_tc<<<g, THREADS, sb, s>>>(tq, dm, pl, ca);
   return cudaGetLastError();
 }
 

@@ -225,7 +225,7 @@ class Profiler:
     """Caller-owned CUDA events the library records around each launch."""
 
     KINDS = ["score", "segscan", "segsum", "engine", "materialize", "readout",
-             "decode_decide", "decode_stream", "build", "readout_pre"]
+             "decode_decide", "decode_stream", "build", "readout_pre", "phi"]
 
     def __init__(self, cap=4096):
         self.events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -64,7 +64,8 @@ typedef enum {
   DLA_K_DECODE_DECIDE = 6,
   DLA_K_DECODE_STREAM = 7,
   DLA_K_BUILD = 8,       /* tensor-core state-piece builder */
-  DLA_K_READOUT_PRE = 9  /* tensor-core readout prologue (weights, intra-tile output) */
+  DLA_K_READOUT_PRE = 9, /* tensor-core readout prologue (weights, intra-tile output) */
+  DLA_K_PHI = 10         /* phi(q), phi(k) as bf16 tensor-core operands */
 } dla_kernel_kind;
 
 /* Optional timing hook (host memory, caller-owned).  When non-NULL, the
