@@ -7,8 +7,10 @@
 //              predecessor are low-information; Chlience section 5.1: b_t = 1
 //              opens a new state).
 //   k_segscan  window pieces: {0} and every boundary t > 0 (warp ballots).
-//   k_tilesum_*  per (tile, head): fp64 sum of phi(k) over each run of a piece
-//              inside the tile, in token order.
+//   k_score    also writes the tile sums below for bf16 keys (its block of
+//              128 tokens is then one readout tile);
+//   k_tilesum_any  otherwise, per (tile, head): fp64 sum of phi(k) over each
+//              run of a piece inside the tile, in token order.
 //   k_segcombine  per piece: the runs' sums in time order (after the cached
 //              open state's z for a continuation) give z at the piece's end
 //              and the open state's partial z before each readout tile.
@@ -47,6 +49,9 @@ __device__ __forceinline__ double key_at(const uint32_t *row, int c) {
 // and norm run as two independent chains, each in index order with explicit
 // round-to-nearest (the oracle's operation sequence):
 // cos = dot / (sqrt(|a|^2) * sqrt(|b|^2)), a zero norm gives r = 1.
+// The product of two bf16 (or fp32) values is exact in fp64, so
+// fma(x, y, acc) rounds exactly like acc + x * y with the product rounded
+// first: one fp64 operation per term instead of two.
 template <bool BF16>
 __device__ __forceinline__ void dot_norm(const uint32_t *a, const uint32_t *b, int D, double &dot,
                                          double &na) {
@@ -54,8 +59,8 @@ __device__ __forceinline__ void dot_norm(const uint32_t *a, const uint32_t *b, i
   na = 0.0;
   for (int c = 0; c < D; c++) {
     const double x = key_at<BF16>(a, c), y = key_at<BF16>(b, c);
-    dot = __dadd_rn(dot, __dmul_rn(x, y));
-    na = __dadd_rn(na, __dmul_rn(x, x));
+    dot = __fma_rn(x, y, dot);
+    na = __fma_rn(x, x, na);
   }
 }
 template <bool BF16>
@@ -63,7 +68,7 @@ __device__ __forceinline__ double norm2(const uint32_t *a, int D) {
   double n = 0.0;
   for (int c = 0; c < D; c++) {
     const double x = key_at<BF16>(a, c);
-    n = __dadd_rn(n, __dmul_rn(x, x));
+    n = __fma_rn(x, x, n);
   }
   return n;
 }
@@ -72,10 +77,34 @@ __device__ __forceinline__ double score_of(double dot, double na, double nb) {
   return __dsub_rn(1.0, __ddiv_rn(dot, __dmul_rn(__dsqrt_rn(na), __dsqrt_rn(nb))));
 }
 
+// phi of a bf16 input in fp64.  Negative inputs need exp: those with a
+// biased exponent in [PHI_E0, PHI_E0 + PHI_NE) (|x| in [2^-24, 16)) come from
+// a table filled with the same exp() per call; other negatives call exp().
+constexpr int PHI_E0 = 103, PHI_NE = 28, PHI_TAB = PHI_NE * 128;
+
+__global__ void k_phi_table(double *tab) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < PHI_TAB) {
+    const uint32_t bits = 0x8000u | ((uint32_t)(PHI_E0 + i / 128) << 7) | (uint32_t)(i % 128);
+    tab[i] = phi64((double)__uint_as_float(bits << 16));
+  }
+}
+
+__device__ __forceinline__ double phi_bf16_f64(uint32_t bits, const double *s_tab) {
+  const float x = __uint_as_float(bits << 16);
+  if (!(bits & 0x8000u)) return (double)x + 1.0;  // x >= +0 (phi(+0) = 1 either way)
+  const uint32_t e = ((bits >> 7) & 0xFFu) - PHI_E0;
+  return e < (uint32_t)PHI_NE ? s_tab[e * 128 + (bits & 127u)] : phi64((double)x);
+}
+
 // Block of SCORE_TOK tokens; key rows of window tokens tb-2 .. tb+127 are
 // staged with 16-byte loads (row tb-1 < 0 is the cache's previous key).
+// With `sums` (bf16 keys, readout tiles of SCORE_TOK rows) the block, which is
+// then one tile, also writes the tile's per-run sums of phi(k) from the
+// staged rows.
 template <bool BF16>
-__global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs ca, int policy) {
+__global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs ca, int policy,
+                                                     int sums) {
   extern __shared__ uint32_t srow[];  // [(SCORE_TOK + 2)][ld]
   const int u = blockIdx.y;
   const int tb = blockIdx.x * SCORE_TOK;
@@ -86,6 +115,7 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
   const int64_t t0 = ca.cache.t[u];
   __shared__ double rs[SCORE_TOK + 1];
   __shared__ double nsq[SCORE_TOK + 1];  // squared norm of token tb-1+i
+  __shared__ uint8_t s_b[SCORE_TOK];
   double r = 0.0;
   if (policy == DLA_POLICY_DYNAMIC) {
     const int vpr = wpr / 4;  // 16-byte vectors per row
@@ -137,17 +167,40 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
   }
   rs[threadIdx.x + 1] = r;
   __syncthreads();
-  if (tl >= ca.Tw) return;
   uint8_t b = 1;
-  if (policy == DLA_POLICY_DYNAMIC) {
-    const double rp = rs[threadIdx.x];
-    const double tau = (double)ca.tau;
-    const bool join = (t0 + tl > 0) && (r < tau) && (rp < tau);
-    b = join ? 0 : 1;
+  if (tl < ca.Tw) {
+    if (policy == DLA_POLICY_DYNAMIC) {
+      const double rp = rs[threadIdx.x];
+      const double tau = (double)ca.tau;
+      const bool join = (t0 + tl > 0) && (r < tau) && (rp < tau);
+      b = join ? 0 : 1;
+    }
+    pl.r[(size_t)u * dm.W + tl] = r;
+    pl.b[(size_t)u * dm.W + tl] = b;
+    if (ca.trace.boundary) ca.trace.boundary[(size_t)u * dm.T + ca.w0 + tl] = b;
   }
-  pl.r[(size_t)u * dm.W + tl] = r;
-  pl.b[(size_t)u * dm.W + tl] = b;
-  if (ca.trace.boundary) ca.trace.boundary[(size_t)u * dm.T + ca.w0 + tl] = b;
+  if (!BF16 || !sums) return;
+  // thread c: token-order fp64 sum of phi(k[.][c]) over each run of the tile
+  // between boundaries, stored at the run's first token
+  s_b[threadIdx.x] = b;
+  __syncthreads();
+  const int len = min(SCORE_TOK, ca.Tw - tb);
+  for (int c = threadIdx.x; c < D; c += SCORE_TOK) {
+    double *zp = pl.z_part + (size_t)u * dm.W * D + c;
+    double z = 0.0;
+    int part = tb;
+#pragma unroll 4
+    for (int i = 0; i < len; i++) {
+      if (i > 0 && s_b[i]) {
+        zp[(size_t)part * D] = z;
+        part = tb + i;
+        z = 0.0;
+      }
+      const uint32_t w = srow[(i + 2) * ld + (c >> 1)];
+      z = __dadd_rn(z, phi_bf16_f64((c & 1) ? (w >> 16) : (w & 0xFFFFu), pl.phi_tab));
+    }
+    zp[(size_t)part * D] = z;
+  }
 }
 
 // phi(x) in fp64 for every bf16 bit pattern (same exp as inline evaluation).
@@ -186,9 +239,9 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
 }
 
 // z = sum of phi(k) of every window piece, in fp64, in two levels:
-//   k_tilesum    per (head, tile): token-order sums of each run of the tile's
+//   tile sums    per (head, tile): token-order sums of each run of the tile's
 //                tokens between boundaries ("part"), stored at the part's first
-//                token;
+//                token (k_score for bf16 keys, else k_tilesum_any);
 //   k_segcombine per segment: its parts added in time order (the cache's z
 //                of a continued open state first), writing the segment's end
 //                sum and the open state's partial sum before each tile.
@@ -196,70 +249,8 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
 // segment spans; the association differs from a strict token-order sum by
 // rounding only (merge choices are then the same unless two Ward losses tie
 // to within rounding).
-// phi of a bf16 input in fp64.  Negative inputs need exp: those with a
-// biased exponent in [PHI_E0, PHI_E0 + PHI_NE) (|x| in [2^-24, 16)) come from
-// a table filled with the same exp() per call; other negatives call exp().
-constexpr int PHI_E0 = 103, PHI_NE = 28, PHI_TAB = PHI_NE * 128;
-
-__global__ void k_phi_table(double *tab) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < PHI_TAB) {
-    const uint32_t bits = 0x8000u | ((uint32_t)(PHI_E0 + i / 128) << 7) | (uint32_t)(i % 128);
-    tab[i] = phi64((double)__uint_as_float(bits << 16));
-  }
-}
-
-__device__ __forceinline__ double phi_bf16_f64(uint32_t bits, const double *s_tab) {
-  const float x = __uint_as_float(bits << 16);
-  if (!(bits & 0x8000u)) return (double)x + 1.0;  // x >= +0 (phi(+0) = 1 either way)
-  const uint32_t e = ((bits >> 7) & 0xFFu) - PHI_E0;
-  return e < (uint32_t)PHI_NE ? s_tab[e * 128 + (bits & 127u)] : phi64((double)x);
-}
-
-__device__ __forceinline__ void cp_async16_cg(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src)
-               : "memory");
-}
-
-// bf16 path: the tile's k rows, the phi table and the boundary flags are
-// staged in shared memory with asynchronous copies (one wait), then thread c
-// runs the fp64 chain of dimension c from shared memory.
-template <int D>
-__global__ void __launch_bounds__(D) k_tilesum_bf16(Dims dm, Plan pl, CallArgs ca) {
-  constexpr int M = 128;
-  extern __shared__ __align__(16) unsigned char ts_raw[];
-  double *s_tab = reinterpret_cast<double *>(ts_raw);                    // PHI_TAB
-  uint16_t *s_k = reinterpret_cast<uint16_t *>(ts_raw + PHI_TAB * 8);    // M x D
-  uint8_t *s_b = ts_raw + PHI_TAB * 8 + M * D * 2;                       // M
-  const int u = blockIdx.y, tile = blockIdx.x;
-  const int c = threadIdx.x;
-  const int T0 = tile * M;
-  if (T0 >= ca.Tw) return;
-  const int T1 = min(T0 + M, ca.Tw), len = T1 - T0;
-  const uint16_t *kg = static_cast<const uint16_t *>(ca.k) + ((size_t)u * dm.T + ca.w0 + T0) * D;
-  for (int i = c; i < len * D / 8; i += D) cp_async16_cg(s_k + 8 * i, kg + 8 * i);
-  for (int i = c; i < PHI_TAB / 2; i += D) cp_async16_cg(s_tab + 2 * i, pl.phi_tab + 2 * i);
-  for (int i = c; i < len; i += D) s_b[i] = pl.b[(size_t)u * dm.W + T0 + i];
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-  double *zp = pl.z_part + (size_t)u * dm.W * D + c;
-  double z = 0.0;
-  int part = T0;
-#pragma unroll 4
-  for (int i = 0; i < len; i++) {
-    if (i > 0 && s_b[i]) {
-      zp[(size_t)part * D] = z;
-      part = T0 + i;
-      z = 0.0;
-    }
-    z = __dadd_rn(z, phi_bf16_f64(s_k[i * D + c], s_tab));
-  }
-  zp[(size_t)part * D] = z;
-}
-
-// Other inputs (fp32, or tiles other than 128 rows): direct loads, phi64.
+// Tile sums of other inputs (fp32 keys, or tiles other than the score's
+// blocks): direct loads, phi64.
 __global__ void k_tilesum_any(Dims dm, Plan pl, CallArgs ca) {
   const int u = blockIdx.y, tile = blockIdx.x;
   const int c = threadIdx.x;  // dimension
@@ -801,19 +792,27 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
 
 }  // namespace
 
+// The score kernel also forms the tile sums for bf16 keys with tiles of
+// SCORE_TOK rows; k_segsum then only combines them.
+bool sums_in_score(const Dims &dm, const CallArgs &ca, int policy) {
+  return ca.in_dtype == DLA_BF16 && dm.M == SCORE_TOK && policy == DLA_POLICY_DYNAMIC;
+}
+
 cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int policy,
                          cudaStream_t s) {
   const bool bf = ca.in_dtype == DLA_BF16;
+  const int sums = sums_in_score(dm, ca, policy) ? 1 : 0;
+  if (sums) k_phi_table<<<(PHI_TAB + 255) / 256, 256, 0, s>>>(pl.phi_tab);
   const size_t sb = sizeof(uint32_t) * (SCORE_TOK + 2) * ((bf ? dm.D / 2 : dm.D) + 1);
   dim3 g((ca.Tw + SCORE_TOK - 1) / SCORE_TOK, dm.heads);
   if (bf) {
     cudaError_t e = cudaFuncSetAttribute(k_score<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
     if (e != cudaSuccess) return e;
-    k_score<true><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
+    k_score<true><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy, sums);
   } else {
     cudaError_t e = cudaFuncSetAttribute(k_score<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
     if (e != cudaSuccess) return e;
-    k_score<false><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy);
+    k_score<false><<<g, SCORE_TOK, sb, s>>>(dm, pl, ca, policy, 0);
   }
   return cudaGetLastError();
 }
@@ -825,25 +824,8 @@ cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, c
 
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   const dim3 g(dm.tiles, dm.heads);
-  if (ca.in_dtype == DLA_BF16 && dm.M == 128) {
-    k_phi_table<<<(PHI_TAB + 255) / 256, 256, 0, s>>>(pl.phi_tab);
-    const size_t sb = PHI_TAB * 8 + 128 * (size_t)dm.D * 2 + 128;
-    cudaError_t e = cudaSuccess;
-    switch (dm.D) {
-      case 32:
-        e = cudaFuncSetAttribute(k_tilesum_bf16<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-        if (e == cudaSuccess) k_tilesum_bf16<32><<<g, 32, sb, s>>>(dm, pl, ca);
-        break;
-      case 64:
-        e = cudaFuncSetAttribute(k_tilesum_bf16<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-        if (e == cudaSuccess) k_tilesum_bf16<64><<<g, 64, sb, s>>>(dm, pl, ca);
-        break;
-      default:
-        e = cudaFuncSetAttribute(k_tilesum_bf16<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-        if (e == cudaSuccess) k_tilesum_bf16<128><<<g, 128, sb, s>>>(dm, pl, ca);
-        break;
-    }
-    if (e != cudaSuccess) return e;
+  if (sums_in_score(dm, ca, DLA_POLICY_DYNAMIC)) {
+    // the tile sums came with the score
   } else {
     k_tilesum_any<<<g, dm.D, 0, s>>>(dm, pl, ca);
   }
