@@ -369,11 +369,11 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       if (e != cudaSuccess) return DLA_ERR_CUDA;
     }
     if (tc) {
-      // after the sums (not just the boundary flags it reads), so it overlaps
-      // the engine without slowing the sums ahead of it
-      if (cudaStreamWaitEvent(s, ax->ev[EV_SUMS], 0) != cudaSuccess) return DLA_ERR_CUDA;
-      { ProfScope ps(pf, DLA_K_BUILD, s); e = launch_build_tc(dm, pl, ca, s); }
-      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_BUILD], s) != cudaSuccess) return DLA_ERR_CUDA;
+      // the builder reads only the boundary flags; after the sums (so it does
+      // not slow them) on the decision stream it overlaps the engine, and the
+      // previous window's readout
+      { ProfScope ps(pf, DLA_K_BUILD, sd); e = launch_build_tc(dm, pl, ca, sd); }
+      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_BUILD], sd) != cudaSuccess) return DLA_ERR_CUDA;
     }
     if (tc) {
       // the readout's prologue needs the engine's atom lists and means, not
