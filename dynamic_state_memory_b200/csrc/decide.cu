@@ -98,7 +98,10 @@ __device__ __forceinline__ double phi_bf16_f64(uint32_t bits, const double *s_ta
 }
 
 // Block of SCORE_TOK tokens; key rows of window tokens tb-2 .. tb+127 are
-// staged with 16-byte loads (row tb-1 < 0 is the cache's previous key).
+// staged with 16-byte loads.  In a call's first window, row tb-1 < 0 is the
+// cache's previous key and r of token -1 the cache's; later windows take both
+// from the call's own input (the same fp64 sequence as the window before), so
+// they need nothing the previous window's engine writes.
 // With `sums` (bf16 keys, readout tiles of SCORE_TOK rows) the block, which is
 // then one tile, also writes the tile's per-run sums of phi(k) from the
 // staged rows.
@@ -112,7 +115,9 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
   const int D = dm.D;
   const int wpr = BF16 ? D / 2 : D;  // 32-bit words per row
   const int ld = wpr + 1;
-  const int64_t t0 = ca.cache.t[u];
+  // the stream's token count before the window (read only in a call's first
+  // window: later ones never hold the stream's first token)
+  const int64_t t0 = ca.w0 == 0 ? ca.cache.t[u] : 1;
   __shared__ double rs[SCORE_TOK + 1];
   __shared__ double nsq[SCORE_TOK + 1];  // squared norm of token tb-1+i
   __shared__ uint8_t s_b[SCORE_TOK];
@@ -125,16 +130,16 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
     for (int e = threadIdx.x; e < (SCORE_TOK + 2) * vpr; e += SCORE_TOK) {
       const int rr = e / vpr, cv = e % vpr;
       const int t = tb - 2 + rr;
-      if (t == -1) continue;  // the cache's previous key, written below
+      if (t == -1 && ca.w0 == 0) continue;  // the cache's previous key, written below
       uint4 x = make_uint4(0, 0, 0, 0);
-      if (t >= 0 && t < ca.Tw) x = kv[(size_t)t * vpr + cv];
+      if (ca.w0 + t >= 0 && t < ca.Tw) x = kv[(ptrdiff_t)t * vpr + cv];
       uint32_t *dst = srow + rr * ld + cv * 4;
       dst[0] = x.x;
       dst[1] = x.y;
       dst[2] = x.z;
       dst[3] = x.w;
     }
-    if (tb == 0) {  // row 1 = token -1 = the cache's previous key (fp32 values)
+    if (tb == 0 && ca.w0 == 0) {  // row 1 = token -1 = the cache's previous key (fp32 values)
       for (int c = threadIdx.x; c < D; c += SCORE_TOK) {
         const float f = ca.cache.prev_k[(size_t)u * D + c];
         if (BF16) {
@@ -152,18 +157,18 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
     nsq[threadIdx.x + 1] = na;
     if (threadIdx.x == 32) {  // a thread of the second warp: token tb-1
       const int tp = tb - 1;
-      if (tp < 0) {
+      if (tp < 0 && ca.w0 == 0) {
         nsq[0] = norm2<BF16>(srow + 1 * ld, D);
         rs[0] = ca.cache.prev_r[u];
       } else {
         double dp, np;
         dot_norm<BF16>(srow + 1 * ld, srow + 0 * ld, D, dp, np);
         nsq[0] = np;
-        rs[0] = (t0 + tp == 0) ? 0.0 : score_of(dp, np, norm2<BF16>(srow + 0 * ld, D));
+        rs[0] = (ca.w0 == 0 && t0 + tp == 0) ? 0.0 : score_of(dp, np, norm2<BF16>(srow + 0 * ld, D));
       }
     }
     __syncthreads();
-    if (tl < ca.Tw) r = (t0 + tl == 0) ? 0.0 : score_of(dot, na, nsq[threadIdx.x]);
+    if (tl < ca.Tw) r = (ca.w0 == 0 && t0 + tl == 0) ? 0.0 : score_of(dot, na, nsq[threadIdx.x]);
   }
   rs[threadIdx.x + 1] = r;
   __syncthreads();
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
     if (policy == DLA_POLICY_DYNAMIC) {
       const double rp = rs[threadIdx.x];
       const double tau = (double)ca.tau;
-      const bool join = (t0 + tl > 0) && (r < tau) && (rp < tau);
+      const bool join = (ca.w0 > 0 || t0 + tl > 0) && (r < tau) && (rp < tau);
       b = join ? 0 : 1;
     }
     pl.r[(size_t)u * dm.W + tl] = r;

@@ -165,12 +165,21 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
 // stream).  `s` runs the score and sums at normal priority; `se` runs the
 // engine at the highest priority: it is latency-bound and on the critical
 // path of a single window, so its few CTAs should get SMs first.  With the
-// tensor-core readout, `sx` runs the materializer at the highest priority and
-// `sp` the readout's prologue beside it at the lowest, so that the
-// materializer's CTAs are placed first.
-enum { EV_START = 0, EV_SUMS, EV_ENGINE, EV_BUILD, EV_MAT, EV_PRE, EV_DONE0, EV_DONE1, EV_COUNT };
+// tensor-core readout, `sb` runs the state builder, `sx` the materializer at
+// the highest priority and `sp` the phi operands and the readout's prologue
+// beside it at the lowest, so that the materializer's CTAs are placed first.
+// Windows cycle through NPLAN plans: a plan is reused three windows later, so
+// window w + 1's decisions and window w + 2's never wait for window w's
+// readout.
+constexpr int NPLAN = 3;
+enum { EV_START = 0, EV_SCAN, EV_SUMS, EV_ENGINE, EV_BUILD, EV_MAT, EV_PRE, EV_DONE0,
+       EV_COUNT = EV_DONE0 + NPLAN };
+int plan_count(const dla_config &cfg, const Dims &dm) {
+  const int windows = (cfg.T + dm.W - 1) / dm.W;
+  return windows < 1 ? 1 : (windows < NPLAN ? windows : NPLAN);
+}
 struct Aux {
-  cudaStream_t s = nullptr, se = nullptr, sp = nullptr, sx = nullptr;
+  cudaStream_t s = nullptr, se = nullptr, sp = nullptr, sx = nullptr, sb = nullptr;
   cudaEvent_t ev[EV_COUNT] = {};
   bool ok = false;
 };
@@ -191,6 +200,7 @@ Aux *aux_streams() {
       return nullptr;
     if (!a.sx && cudaStreamCreateWithPriority(&a.sx, cudaStreamNonBlocking, hi) != cudaSuccess)
       return nullptr;
+    if (!a.sb && cudaStreamCreateWithFlags(&a.sb, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
     for (cudaEvent_t &e : a.ev)
       if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
     a.ok = true;
@@ -271,8 +281,7 @@ size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
   const Dims dm = make_dims(*cfg, policy);
   Plan pl{};
   Carver cv{nullptr};
-  carve_plan(cv, dm, pl);
-  if (cfg->T > dm.W) carve_plan(cv, dm, pl);  // windows alternate between two plans
+  for (int i = 0, n = plan_count(*cfg, dm); i < n; i++) carve_plan(cv, dm, pl);
   return cv.off;
 }
 
@@ -295,11 +304,10 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16)
     return DLA_ERR_INVALID_ARG;
   const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
-  Plan plans[2] = {};
+  Plan plans[NPLAN] = {};
   Carver cv{static_cast<char *>(ws)};
-  carve_plan(cv, dm, plans[0]);
-  if (cfg->T > dm.W) carve_plan(cv, dm, plans[1]);
-  else plans[1] = plans[0];
+  const int nplan = plan_count(*cfg, dm);
+  for (int i = 0; i < nplan; i++) carve_plan(cv, dm, plans[i]);
   if (cv.off > ws_bytes) return DLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Aux *ax = aux_streams();
@@ -308,6 +316,7 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   cudaStream_t se = ax->se;  // the engine
   cudaStream_t sp = ax->sp;  // the tensor-core readout's prologue
   cudaStream_t sx = ax->sx;  // the materializer, with the tensor-core readout
+  cudaStream_t sb = ax->sb;  // the tensor-core state builder
   CallArgs ca{};
   ca.q = q;
   ca.k = k;
@@ -338,20 +347,23 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   dla_profile *pf = cfg->profile;
   int wi = 0;
   for (int w0 = 0; w0 < cfg->T; w0 += dm.W, wi++) {
-    const Plan &pl = plans[wi & 1];
+    const int pi = wi % nplan;  // this window's plan, last used by window wi - nplan
+    const Plan &pl = plans[pi];
+    const bool reuse = wi >= nplan;
     ca.w0 = w0;
     ca.Tw = cfg->T - w0 < dm.W ? cfg->T - w0 : dm.W;
     cudaError_t e = cudaSuccess;
-    // this plan was last read by window wi - 2's readout; the score reads the
-    // cache's last key and score, written by window wi - 1's engine
-    if (wi >= 2 && cudaStreamWaitEvent(sd, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)
-      return DLA_ERR_CUDA;
-    if (wi >= 1 && cudaStreamWaitEvent(sd, ax->ev[EV_ENGINE], 0) != cudaSuccess)
+    // this plan was last read by window wi - nplan's readout.  The score and scan
+    // of a later window read only the call's input; the piece sums read the
+    // cache's open state, written by window wi - 1's engine
+    if (reuse && cudaStreamWaitEvent(sd, ax->ev[EV_DONE0 + pi], 0) != cudaSuccess)
       return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SCORE, sd); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, sd); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SEGSCAN, sd); e = launch_segscan(dm, pl, ca, sd); }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SCAN], sd) != cudaSuccess) return DLA_ERR_CUDA;
+    if (wi >= 1 && cudaStreamWaitEvent(sd, ax->ev[EV_ENGINE], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SEGSUM, sd); e = launch_segsum(dm, pl, ca, sd); }
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SUMS], sd) != cudaSuccess ||
         cudaStreamWaitEvent(se, ax->ev[EV_SUMS], 0) != cudaSuccess)
@@ -360,20 +372,22 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], se) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc) {
       // phi(q), phi(k) of the window beside the latency-bound engine (after
-      // the sums, whose memory traffic it would slow); the plan's phi buffers
-      // were last read by window wi - 2's readout
-      if (cudaStreamWaitEvent(sp, ax->ev[EV_SUMS], 0) != cudaSuccess) return DLA_ERR_CUDA;
-      if (wi >= 2 && cudaStreamWaitEvent(sp, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)
+      // the score, whose memory traffic it would slow); the plan's phi buffers
+      // were last read by window wi - nplan's readout
+      if (cudaStreamWaitEvent(sp, ax->ev[EV_SCAN], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      if (reuse && cudaStreamWaitEvent(sp, ax->ev[EV_DONE0 + pi], 0) != cudaSuccess)
         return DLA_ERR_CUDA;
       { ProfScope ps(pf, DLA_K_PHI, sp); e = launch_phi_tc(dm, pl, ca, sp); }
       if (e != cudaSuccess) return DLA_ERR_CUDA;
     }
     if (tc) {
-      // the builder reads only the boundary flags; after the sums (so it does
-      // not slow them) on the decision stream it overlaps the engine, and the
-      // previous window's readout
-      { ProfScope ps(pf, DLA_K_BUILD, sd); e = launch_build_tc(dm, pl, ca, sd); }
-      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_BUILD], sd) != cudaSuccess) return DLA_ERR_CUDA;
+      // the builder reads only the boundary flags (after the score, so it does
+      // not slow it); it overlaps the engine and the previous window's
+      // readout.  Its pieces were last read by window wi - nplan's materializer,
+      // before the decision stream's wait above
+      if (cudaStreamWaitEvent(sb, ax->ev[EV_SCAN], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      { ProfScope ps(pf, DLA_K_BUILD, sb); e = launch_build_tc(dm, pl, ca, sb); }
+      if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_BUILD], sb) != cudaSuccess) return DLA_ERR_CUDA;
     }
     if (tc) {
       // the readout's prologue needs the engine's atom lists and means, not
@@ -383,12 +397,12 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
     }
     // the materializer: after the engine (ops) and the builder (pieces); on
-    // sx it also waits for window wi - 2's readout, the last reader of this
+    // sx it also waits for window wi - nplan's readout, the last reader of this
     // plan's versions, and for the previous materializer through stream order
     cudaStream_t sm_ = tc ? sx : s;
     if (cudaStreamWaitEvent(sm_, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc && (cudaStreamWaitEvent(sx, ax->ev[EV_BUILD], 0) != cudaSuccess ||
-               (wi >= 2 && cudaStreamWaitEvent(sx, ax->ev[EV_DONE0 + (wi & 1)], 0) != cudaSuccess)))
+               (reuse && cudaStreamWaitEvent(sx, ax->ev[EV_DONE0 + pi], 0) != cudaSuccess)))
       return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_MATERIALIZE, sm_); e = launch_materialize(dm, pl, ca, sm_, tc); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
@@ -400,7 +414,7 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       ProfScope ps(pf, DLA_K_READOUT, s);
       e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);
     }
-    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_DONE0 + (wi & 1)], s) != cudaSuccess)
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_DONE0 + pi], s) != cudaSuccess)
       return DLA_ERR_CUDA;
   }
   return DLA_OK;
