@@ -506,11 +506,21 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
   memset(&ca.trace, 0, sizeof ca.trace);
   dla_profile *pf = cfg->profile;
   cudaError_t e;
+  Aux *ax = tc ? aux_streams() : nullptr;
+  if (tc && !ax) return DLA_ERR_CUDA;
+  if (tc) {
+    // phi(q), phi(k) need only the inputs: beside the tree build
+    cudaStream_t sp = ax->sp;
+    if (cudaEventRecord(ax->ev[EV_START], s) != cudaSuccess ||
+        cudaStreamWaitEvent(sp, ax->ev[EV_START], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_PHI, sp); e = launch_phi_tc(dm, pl, ca, sp); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
+  }
   { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, s); }
   if (e != cudaSuccess) return DLA_ERR_CUDA;
   if (tc) {
-    { ProfScope ps(pf, DLA_K_PHI, s); e = launch_phi_tc(dm, pl, ca, s); }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    if (cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_READOUT_PRE, s); e = launch_readout_pre_tc(dm, pl, ca, s); }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
   }
