@@ -517,13 +517,21 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
     { ProfScope ps(pf, DLA_K_PHI, sp); e = launch_phi_tc(dm, pl, ca, sp); }
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
   }
-  { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, s); }
+  { ProfScope ps(pf, DLA_K_ENGINE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, false, s); }
   if (e != cudaSuccess) return DLA_ERR_CUDA;
   if (tc) {
-    if (cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess) return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_READOUT_PRE, s); e = launch_readout_pre_tc(dm, pl, ca, s); }
-    if (e != cudaSuccess) return DLA_ERR_CUDA;
+    // the prologue needs the plan and the nodes' means, not their states: it
+    // runs beside the tree levels
+    cudaStream_t sp = ax->sp;
+    if (cudaEventRecord(ax->ev[EV_SUMS], s) != cudaSuccess ||
+        cudaStreamWaitEvent(sp, ax->ev[EV_SUMS], 0) != cudaSuccess)
+      return DLA_ERR_CUDA;
+    { ProfScope ps(pf, DLA_K_READOUT_PRE, sp); e = launch_readout_pre_tc(dm, pl, ca, sp); }
+    if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
   }
+  { ProfScope ps(pf, DLA_K_MATERIALIZE, s); e = launch_fenwick(dm, pl, ca, treeS, treeZ, tc, true, s); }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  if (tc && cudaStreamWaitEvent(s, ax->ev[EV_PRE], 0) != cudaSuccess) return DLA_ERR_CUDA;
   {
     ProfScope ps(pf, DLA_K_READOUT, s);
     e = tc ? launch_readout_tc(dm, pl, ca, s) : launch_readout_simt(dm, pl, ca, s);

@@ -150,8 +150,10 @@ cudaError_t launch_build_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, 
 cudaError_t launch_fen_leaves_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
                                  float *treeZ, int nodes, int ntiles, cudaStream_t s);
 void fen_tree_shape(int T, int M, int *nodes, int *levels);
+// Fixed policy: levels == false launches the plan, the leaves and every tree
+// node's means; levels == true then the node states and versions.
 cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
-                           float *treeZ, bool bf16, cudaStream_t s);
+                           float *treeZ, bool bf16, bool levels, cudaStream_t s);
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s);
 cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,

@@ -8,9 +8,14 @@
 //     [0, T0 - 1] are whole-tile dyadic ranges: one tree node per set bit of c;
 //   - leaves: per tile, the state sum S = sum v phi(k)^T, z = sum phi(k)
 //     (on the tensor cores for bf16 d = 128, else k_fen_leaves);
-//   - k_fen_level: node = left child + right child, level by level;
-//   every node is also written as a frozen version (fp32 or the bf16 UMMA
-//   layout) with its mean phi(k) and count;
+//   - k_fen_means: every node's phi(k) sum and count (children added level by
+//   level, one block per head), so the readout's prologue can start while the
+//   states are still being summed;
+//   - k_fen_level: node state = left child + right child, level by level;
+//   even-indexed nodes are also written as frozen versions (fp32 or the bf16
+//   UMMA layout).  A block of size 2^b in a prefix [0, T0) starts at a
+//   multiple of 2^(b+1), so only even-indexed nodes are ever atoms; odd ones
+//   only build their parents;
 //   - k_fen_plan: per tile, the atoms (tree nodes, oldest first) and the
 //     in-tile events: every token is a boundary, and at offset o >= 1 the
 //     binary-counter carry merges the two newest blocks (trailing ones of
@@ -37,10 +42,12 @@ __device__ __forceinline__ int node_id(const FenTree &tr, int level, int index) 
   return tr.off[level] + index;
 }
 
+// The frozen version of node v (all threads of the block): the state, and
+// with `means` its phi(k) sum and count.
 template <int D>
 __device__ void write_version(const Dims &dm, const Plan &pl, int u, int v, const float *S,
-                              const float *z, float n, bool bf16) {
-  // S: fp32 [D][D] in global memory; all threads of the block
+                              const float *z, float n, bool bf16, bool means = true) {
+  // S: fp32 [D][D] in global memory
   if (bf16) {
     uint8_t *Vd = static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D * 2;
     for (int ch = threadIdx.x; ch < D * D / 8; ch += THREADS) {
@@ -54,6 +61,7 @@ __device__ void write_version(const Dims &dm, const Plan &pl, int u, int v, cons
     float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + v) * D * D;
     for (int e = threadIdx.x; e < D * D; e += THREADS) Vd[e] = S[e];
   }
+  if (!means) return;
   for (int c = threadIdx.x; c < D; c += THREADS) pl.ver_z[((size_t)u * dm.vmax + v) * D + c] = z[c];
   if (threadIdx.x == 0) pl.ver_n[(size_t)u * dm.vmax + v] = n;
 }
@@ -104,6 +112,26 @@ __global__ void __launch_bounds__(THREADS) k_fen_leaves(Dims dm, Plan pl, CallAr
   write_version<D>(dm, pl, u, nid, S, z, (float)len, bf16);
 }
 
+// phi(k) sums and counts of every node above the leaves (one block per head,
+// level by level): z(l, i) = z(l-1, 2i) + z(l-1, 2i+1), also as version means.
+template <int D>
+__global__ void __launch_bounds__(THREADS) k_fen_means(Dims dm, Plan pl, FenTree tr, int ntiles) {
+  const int u = blockIdx.x;
+  for (int l = 1; l < tr.levels; l++) {
+    const int count = ntiles >> l;
+    __syncthreads();  // level l - 1 is complete
+    for (int e = threadIdx.x; e < count * D; e += THREADS) {
+      const int i = e / D, c = e % D;
+      const int a = node_id(tr, l - 1, 2 * i), b = node_id(tr, l - 1, 2 * i + 1);
+      const int nid = node_id(tr, l, i);
+      const float z = tr.z[((size_t)u * tr.nodes + a) * D + c] + tr.z[((size_t)u * tr.nodes + b) * D + c];
+      tr.z[((size_t)u * tr.nodes + nid) * D + c] = z;
+      pl.ver_z[((size_t)u * dm.vmax + nid) * D + c] = z;
+      if (c == 0) pl.ver_n[(size_t)u * dm.vmax + nid] = (float)(dm.M << l);
+    }
+  }
+}
+
 // One tree level: node (level, i) = (level-1, 2i) + (level-1, 2i+1).
 template <int D>
 __global__ void __launch_bounds__(THREADS) k_fen_level(Dims dm, Plan pl, FenTree tr, int level,
@@ -120,12 +148,9 @@ __global__ void __launch_bounds__(THREADS) k_fen_level(Dims dm, Plan pl, FenTree
     const float4 y = *reinterpret_cast<const float4 *>(Sb + e);
     *reinterpret_cast<float4 *>(S + e) = make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
   }
-  const float *za = tr.z + ((size_t)u * tr.nodes + a) * D;
-  const float *zb = tr.z + ((size_t)u * tr.nodes + b) * D;
-  float *z = tr.z + ((size_t)u * tr.nodes + nid) * D;
-  for (int c = threadIdx.x; c < D; c += THREADS) z[c] = za[c] + zb[c];
+  if (i & 1) return;  // never an atom
   __syncthreads();
-  write_version<D>(dm, pl, u, nid, S, z, (float)(dm.M << level), bf16);
+  write_version<D>(dm, pl, u, nid, S, nullptr, 0.f, bf16, false);
 }
 
 // Per (head, tile): atoms = tree nodes of the blocks of [0, T0-1], events.
@@ -157,9 +182,19 @@ __global__ void k_fen_plan(Dims dm, Plan pl, FenTree tr, int ntiles) {
   }
 }
 
+// Plan, leaves and every node's means (what the readout's prologue needs),
+// then (levels == true) the node states and versions.
 template <int D>
 cudaError_t run_d(const Dims &dm, const Plan &pl, const CallArgs &ca, const FenTree &tr,
-                  int ntiles, bool bf16, cudaStream_t s) {
+                  int ntiles, bool bf16, bool levels, cudaStream_t s) {
+  if (levels) {
+    for (int l = 1; l < tr.levels; l++) {
+      const int count = ntiles >> l;
+      if (count <= 0) break;
+      k_fen_level<D><<<dim3(count, dm.heads), THREADS, 0, s>>>(dm, pl, tr, l, count, bf16);
+    }
+    return cudaGetLastError();
+  }
   k_fen_plan<<<dim3((ntiles + 127) / 128, dm.heads), 128, 0, s>>>(dm, pl, tr, ntiles);
   if (bf16 && D == 128) {
     // leaves on the tensor cores (tile state sums, phi(k) sums, bf16 versions)
@@ -168,11 +203,7 @@ cudaError_t run_d(const Dims &dm, const Plan &pl, const CallArgs &ca, const FenT
   } else {
     k_fen_leaves<D><<<dim3(ntiles, dm.heads), THREADS, 0, s>>>(dm, pl, ca, tr, ntiles, bf16);
   }
-  for (int l = 1; l < tr.levels; l++) {
-    const int count = ntiles >> l;
-    if (count <= 0) break;
-    k_fen_level<D><<<dim3(count, dm.heads), THREADS, 0, s>>>(dm, pl, tr, l, count, bf16);
-  }
+  if (tr.levels > 1) k_fen_means<D><<<dm.heads, THREADS, 0, s>>>(dm, pl, tr, ntiles);
   return cudaGetLastError();
 }
 
@@ -188,7 +219,7 @@ void fen_tree_shape(int T, int M, int *nodes, int *levels) {
 }
 
 cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, float *treeS,
-                           float *treeZ, bool bf16, cudaStream_t s) {
+                           float *treeZ, bool bf16, bool levels, cudaStream_t s) {
   FenTree tr{};
   tr.S = treeS;
   tr.z = treeZ;
@@ -200,9 +231,9 @@ cudaError_t launch_fenwick(const Dims &dm, const Plan &pl, const CallArgs &ca, f
     off += ntiles >> l;
   }
   switch (dm.D) {
-    case 32: return run_d<32>(dm, pl, ca, tr, ntiles, bf16, s);
-    case 64: return run_d<64>(dm, pl, ca, tr, ntiles, bf16, s);
-    case 128: return run_d<128>(dm, pl, ca, tr, ntiles, bf16, s);
+    case 32: return run_d<32>(dm, pl, ca, tr, ntiles, bf16, levels, s);
+    case 64: return run_d<64>(dm, pl, ca, tr, ntiles, bf16, levels, s);
+    case 128: return run_d<128>(dm, pl, ca, tr, ntiles, bf16, levels, s);
   }
   return cudaErrorInvalidValue;
 }
