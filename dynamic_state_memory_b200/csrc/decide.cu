@@ -106,7 +106,7 @@ __device__ __forceinline__ double phi_bf16_f64(uint32_t bits, const double *s_ta
 // then one tile, also writes the tile's per-run sums of phi(k) from the
 // staged rows.
 template <bool BF16>
-__global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs ca, int policy,
+__global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallArgs ca, int policy,
                                                      int sums) {
   extern __shared__ uint32_t srow[];  // [(SCORE_TOK + 2)][ld]
   const int u = blockIdx.y;
@@ -126,18 +126,50 @@ __global__ void __launch_bounds__(SCORE_TOK) k_score(Dims dm, Plan pl, CallArgs 
     const int vpr = wpr / 4;  // 16-byte vectors per row
     const uint4 *kv = reinterpret_cast<const uint4 *>(
         static_cast<const char *>(ca.k) + ((size_t)u * dm.T + ca.w0) * D * (BF16 ? 2 : 4));
+    if (BF16) {
+      // the block's rows in two batches of 16-byte loads, each batch in flight
+      // at once (at most 17 loads per thread for d = 128), then its stores
+      // into the padded rows
+      constexpr int MAXIT = ((SCORE_TOK + 2) * 16 + SCORE_TOK - 1) / SCORE_TOK;
+      constexpr int BATCH = (MAXIT + 1) / 2;
+#pragma unroll
+      for (int b0 = 0; b0 < MAXIT; b0 += BATCH) {
+        uint4 xs[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; i++) {
+          const int e = threadIdx.x + (b0 + i) * SCORE_TOK;
+          const int rr = e / vpr, cv = e % vpr;
+          const int t = tb - 2 + rr;
+          xs[i] = make_uint4(0, 0, 0, 0);
+          if (b0 + i < MAXIT && e < (SCORE_TOK + 2) * vpr && ca.w0 + t >= 0 && t < ca.Tw)
+            xs[i] = kv[(ptrdiff_t)t * vpr + cv];
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; i++) {
+          const int e = threadIdx.x + (b0 + i) * SCORE_TOK;
+          const int rr = e / vpr, cv = e % vpr;
+          if (b0 + i >= MAXIT || e >= (SCORE_TOK + 2) * vpr || (tb - 2 + rr == -1 && ca.w0 == 0)) continue;
+          uint32_t *dst = srow + rr * ld + cv * 4;
+          dst[0] = xs[i].x;
+          dst[1] = xs[i].y;
+          dst[2] = xs[i].z;
+          dst[3] = xs[i].w;
+        }
+      }
+    } else {
 #pragma unroll 4
-    for (int e = threadIdx.x; e < (SCORE_TOK + 2) * vpr; e += SCORE_TOK) {
-      const int rr = e / vpr, cv = e % vpr;
-      const int t = tb - 2 + rr;
-      if (t == -1 && ca.w0 == 0) continue;  // the cache's previous key, written below
-      uint4 x = make_uint4(0, 0, 0, 0);
-      if (ca.w0 + t >= 0 && t < ca.Tw) x = kv[(ptrdiff_t)t * vpr + cv];
-      uint32_t *dst = srow + rr * ld + cv * 4;
-      dst[0] = x.x;
-      dst[1] = x.y;
-      dst[2] = x.z;
-      dst[3] = x.w;
+      for (int e = threadIdx.x; e < (SCORE_TOK + 2) * vpr; e += SCORE_TOK) {
+        const int rr = e / vpr, cv = e % vpr;
+        const int t = tb - 2 + rr;
+        if (t == -1 && ca.w0 == 0) continue;  // the cache's previous key, written below
+        uint4 x = make_uint4(0, 0, 0, 0);
+        if (ca.w0 + t >= 0 && t < ca.Tw) x = kv[(ptrdiff_t)t * vpr + cv];
+        uint32_t *dst = srow + rr * ld + cv * 4;
+        dst[0] = x.x;
+        dst[1] = x.y;
+        dst[2] = x.z;
+        dst[3] = x.w;
+      }
     }
     if (tb == 0 && ca.w0 == 0) {  // row 1 = token -1 = the cache's previous key (fp32 values)
       for (int c = threadIdx.x; c < D; c += SCORE_TOK) {
