@@ -12,6 +12,10 @@
 // to the piece buffer, which the materializer adds to the open state (op
 // ADDP).  Shorter pieces stay SIMT adds in the materializer.
 //
+// The phi(k) tile, as it sits in shared memory (two 64-column halves of 128
+// rows, 128-byte swizzle), is also stored to the plan: it is the readout
+// prologue's phi(K) operand.
+//
 // Leaf mode (fixed Fenwick policy): the one piece is the whole tile and the
 // result is the tree leaf of that tile: fp32 state and phi(k) sum, plus the
 // frozen bf16 version (UMMA layout), its phi(k) sum and token count.
@@ -113,6 +117,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   fence_proxy_async();
   __syncthreads();
+  if (tid == 0 && pl.phi_k) {  // sm.k is not written again
+    bulk_store(static_cast<uint8_t *>(pl.phi_k) + ((size_t)u * dm.tiles + c) * TILE_BYTES, sm.k,
+               TILE_BYTES);
+    bulk_commit();
+  }
 
   const int np = sm.np;
   const int pbase = fen.treeS ? c : c * PIECES_PER_TILE;
@@ -190,6 +199,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     id++;
   }
+  if (tid == 0 && pl.phi_k) bulk_wait_read();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

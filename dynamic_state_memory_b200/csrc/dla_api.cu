@@ -371,8 +371,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     { ProfScope ps(pf, DLA_K_ENGINE, se); e = launch_engine(dm, pl, ca, se); }
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_ENGINE], se) != cudaSuccess) return DLA_ERR_CUDA;
     if (tc) {
-      // phi(q), phi(k) of the window beside the latency-bound engine (after
-      // the score, whose memory traffic it would slow); the plan's phi buffers
+      // phi(q) of the window beside the latency-bound engine (after the
+      // score, whose memory traffic it would slow); the plan's phi buffers
       // were last read by window wi - nplan's readout
       if (cudaStreamWaitEvent(sp, ax->ev[EV_SCAN], 0) != cudaSuccess) return DLA_ERR_CUDA;
       if (reuse && cudaStreamWaitEvent(sp, ax->ev[EV_DONE0 + pi], 0) != cudaSuccess)
@@ -392,7 +392,9 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     if (tc) {
       // the readout's prologue needs the engine's atom lists and means, not
       // the versions: it runs beside the materializer
-      if (cudaStreamWaitEvent(sp, ax->ev[EV_ENGINE], 0) != cudaSuccess) return DLA_ERR_CUDA;
+      if (cudaStreamWaitEvent(sp, ax->ev[EV_ENGINE], 0) != cudaSuccess ||
+          cudaStreamWaitEvent(sp, ax->ev[EV_BUILD], 0) != cudaSuccess)  // phi(k) tiles
+        return DLA_ERR_CUDA;
       { ProfScope ps(pf, DLA_K_READOUT_PRE, sp); e = launch_readout_pre_tc(dm, pl, ca, sp); }
       if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_PRE], sp) != cudaSuccess) return DLA_ERR_CUDA;
     }
@@ -509,7 +511,8 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
   Aux *ax = tc ? aux_streams() : nullptr;
   if (tc && !ax) return DLA_ERR_CUDA;
   if (tc) {
-    // phi(q), phi(k) need only the inputs: beside the tree build
+    // phi(q) needs only the input: beside the tree build (the leaves store
+    // the phi(k) tiles)
     cudaStream_t sp = ax->sp;
     if (cudaEventRecord(ax->ev[EV_START], s) != cudaSuccess ||
         cudaStreamWaitEvent(sp, ax->ev[EV_START], 0) != cudaSuccess)

@@ -89,7 +89,8 @@ struct Plan {
   float *pieces;       // [heads][pmax][D][D] fp32 piece states
   // tensor-core readout: per-tile outputs of the prologue kernel (null on
   // the SIMT path)
-  void *phi_q, *phi_k; // [heads][W][D] bf16 phi(q), phi(k) of the window's rows
+  void *phi_q;         // [heads][W][D] bf16 phi(q) of the window's rows
+  void *phi_k;         // [heads][tiles][2][128][64] bf16 phi(k) tiles, as in shared memory
   float *pre_w;        // [heads][tiles][amax][M] atom weights
   void *pre_o;         // [heads][tiles][M * D] intra-tile outputs (bf16)
 };

@@ -6,11 +6,13 @@
 // lambda_{t,i} = softmax_i(phi(q_t) . mu_i / sqrt(d_k)); Dynamic Linear
 // Attention | Chlience Paper Archive, section 5.3), mapped onto Blackwell.
 //
-// k_phi_tc writes phi(q) and phi(k) of the window as bf16 operands (it needs
-// only the inputs, so it runs beside the decision kernels).
+// k_phi_tc writes phi(q) of the window as the bf16 operand (it needs only the
+// input, so it runs beside the engine); the state builder stores the phi(k)
+// tiles it forms for its own products.
 // k_readout_pre needs only the plan's atom lists and means, not the frozen
 // state versions, so it runs beside the materializer:
-//   TMA (128B swizzle) loads the phi(q), phi(k) and v tiles.
+//   TMA (128B swizzle) loads the phi(q) and v tiles, a bulk copy the builder's
+//   phi(k) tile.
 //   tcgen05.mma (kind::f16, M = 128 tokens) computes into tensor memory:
 //     A  = phi(Q) phi(K)^T               (128 x 128)   TMEM cols [256, 384)
 //     LA = phi(Q) Mu^T                   (128 x m0)    TMEM cols [384, 512)
@@ -124,17 +126,15 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
   return y[0];
 }
 
-// phi(q), phi(k) of the window's rows as the bf16 operands of the readout:
-// phi_q / phi_k [heads][W][D], rows [0, Tw) (16 bytes per thread and step).
+// phi(q) of the window's rows as the bf16 operand of the readout: phi_q
+// [heads][W][D], rows [0, Tw) (16 bytes per thread and step).
 __global__ void __launch_bounds__(256) k_phi_tc(Dims dm, Plan pl, CallArgs ca) {
   const size_t per_head = (size_t)ca.Tw * (D / 8);
-  const size_t half = per_head * dm.heads;
-  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < 2 * half; i += (size_t)gridDim.x * 256) {
-    const bool is_k = i >= half;
-    const size_t j = is_k ? i - half : i;
-    const size_t u = j / per_head, r = j - u * per_head;
-    const uint4 *src = static_cast<const uint4 *>(is_k ? ca.k : ca.q) + (u * dm.T + ca.w0) * (D / 8) + r;
-    uint4 *dst = static_cast<uint4 *>(is_k ? pl.phi_k : pl.phi_q) + u * dm.W * (D / 8) + r;
+  const size_t total = per_head * dm.heads;
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < total; i += (size_t)gridDim.x * 256) {
+    const size_t u = i / per_head, r = i - u * per_head;
+    const uint4 *src = static_cast<const uint4 *>(ca.q) + (u * dm.T + ca.w0) * (D / 8) + r;
+    uint4 *dst = static_cast<uint4 *>(pl.phi_q) + u * dm.W * (D / 8) + r;
     uint4 x = *src;
     uint32_t *w = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(256) k_phi_tc(Dims dm, Plan pl, CallArgs ca) {
 }
 
 __global__ void __launch_bounds__(PRE_THREADS, 2)
-    k_readout_pre(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, Dims dm, Plan pl, CallArgs ca) {
+    k_readout_pre(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tv,
+                  Dims dm, Plan pl, CallArgs ca) {
   extern __shared__ uint8_t raw[];
   PreSmem &sm = *reinterpret_cast<PreSmem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -164,10 +164,9 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     mbar_init(&sm.bar_load, 1);
     fence_mbar_init();
     mbar_expect_tx(&sm.bar_load, 2 * TILE_BYTES);
-    for (int h = 0; h < 2; h++) {
+    for (int h = 0; h < 2; h++)
       tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, T0, u);
-      tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tk, &sm.bar_load, h * 64, T0, u);
-    }
+    bulk_load(sm.kp, static_cast<const uint8_t *>(pl.phi_k) + g * TILE_BYTES, TILE_BYTES, &sm.bar_load);
   }
   const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
   {
@@ -900,7 +899,9 @@ int tc_tile_rows() { return kTileRows; }
 
 cudaError_t launch_phi_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   if (dm.D != D || ca.in_dtype != DLA_BF16 || !pl.phi_q) return cudaErrorInvalidValue;
-  k_phi_tc<<<148 * 8, 256, 0, s>>>(dm, pl, ca);
+  // 32 KB of (unused) shared memory keeps its CTAs off the SMs that hold
+  // the engine, which reserves most of their shared memory
+  k_phi_tc<<<148 * 8, 256, 32 * 1024, s>>>(dm, pl, ca);
   return cudaGetLastError();
 }
 
@@ -908,9 +909,8 @@ cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs
                                   cudaStream_t s) {
   if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.phi_q)
     return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tv;
   if (!make_bf16_map_rows(&tq, pl.phi_q, ca.Tw, dm.W, dm.heads) ||
-      !make_bf16_map_rows(&tk, pl.phi_k, ca.Tw, dm.W, dm.heads) ||
       !make_bf16_map(&tv, ca.v, dm.T, dm.heads))
     return cudaErrorInvalidValue;
   const size_t sb = sizeof(PreSmem) + 1024;
@@ -918,7 +918,7 @@ cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs
                                        (int)sb);
   if (e != cudaSuccess) return e;
   dim3 g(dm.tiles, dm.heads);
-  k_readout_pre<<<g, PRE_THREADS, sb, s>>>(tq, tk, tv, dm, pl, ca);
+  k_readout_pre<<<g, PRE_THREADS, sb, s>>>(tq, tv, dm, pl, ca);
   return cudaGetLastError();
 }
 
