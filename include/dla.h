@@ -15,9 +15,14 @@
  *
  * Conventions for every entry point:
  *   - All tensor arguments are DEVICE pointers to caller-owned memory; the
- *     library allocates no device memory and keeps no global state.
+ *     library allocates no device memory and keeps no state between calls
+ *     (apart from the scratch of dla_decode_step_static, below).
  *   - Every call is enqueued on `stream` (a cudaStream_t passed as void*;
- *     NULL = legacy default stream) and returns without synchronising.
+ *     NULL = legacy default stream) and returns without synchronising.  A
+ *     prefill forks its kernels onto auxiliary non-blocking streams (created
+ *     on first use, once per host thread and device) with events recorded on
+ *     `stream`, and joins back on `stream`: later work on `stream` sees all
+ *     of its results, as if every kernel had run there.
  *   - Argument errors are returned synchronously (nothing is enqueued).
  *   - Errors found on the device (trace overflow, broken invariant) are
  *     written to *dev_status (a device int32 the caller zeroes beforehand and
@@ -65,7 +70,7 @@ typedef enum {
   DLA_K_DECODE_STREAM = 7,
   DLA_K_BUILD = 8,       /* tensor-core state-piece builder */
   DLA_K_READOUT_PRE = 9, /* tensor-core readout prologue (weights, intra-tile output) */
-  DLA_K_PHI = 10         /* phi(q), phi(k) as bf16 tensor-core operands */
+  DLA_K_PHI = 10         /* phi(q) as the bf16 tensor-core operand */
 } dla_kernel_kind;
 
 /* Optional timing hook (host memory, caller-owned).  When non-NULL, the
