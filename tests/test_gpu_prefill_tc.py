@@ -67,3 +67,51 @@ def test_single_state(gpu):
 def test_many_heads_regime_switching(gpu):
     q, k, v = case(3, 5, 1100, 128, "bf16", seed=13, n_centres=16, mean_len=40.0)
     check(q, k, v, 16, 0.5)
+
+
+@pytest.mark.parametrize("window", [0, 256])
+def test_cuda_graph_capture_and_replay(gpu, window):
+    """A prefill (cache reset + call) captured in a CUDA graph and replayed
+    gives the eager call's outputs and trace bit for bit: the library's fork
+    onto its auxiliary streams and the join go through events on the caller's
+    stream, which stream capture follows."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    q, k, v = case(2, 2, 700, 128, "bf16", seed=77, mean_len=14.0)
+    B, H, T, d = k.shape
+    C, tau = 8, 0.5
+    tq, tk, tv = (to_device(x, "bf16") for x in (q, k, v))
+    cache = dla.Cache(B, H, C, d)
+    cfg = dla.make_config(B, H, T, d, C, tau, dla.DLA_BF16, window, None)
+    ws = torch.empty(dla.dla_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    tr = dla.Trace(B * H, T, T + 1, "cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.empty_like(tq)
+
+    def call(stream):
+        dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
+        dla.dla_prefill(cfg, tq, tk, tv, o, cache.c, tr.c, ws, st, stream)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        call(s)
+    torch.cuda.synchronize()
+    o_eager = o.clone()
+    b_eager = tr.boundary.clone()
+    m_eager = tr.merges()
+    o.zero_()
+    tr.boundary.zero_()
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call(s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    dla.check_device_status(st, "graph replay")
+    assert torch.equal(o, o_eager)
+    assert torch.equal(tr.boundary, b_eager)
+    assert tr.merges() == m_eager
+    ref = oracle_run(q, k, v, C, tau, "bf16")
+    assert tr.merges() == ref["merges"]
+    assert rel_err(from_device(o), ref["out"]) <= TOL["bf16"]
