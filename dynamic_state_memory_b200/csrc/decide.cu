@@ -870,15 +870,28 @@ cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
   return cudaGetLastError();
 }
 
-// The engine is one latency-bound warp per head.  Its CTA reserves most of an
-// SM's shared memory, so the builder and phi kernels that run beside it take
-// other SMs instead of competing for its issue slots.
+// The engine is one latency-bound warp per head.  When every head gets an SM
+// of its own, its CTA reserves most of that SM's shared memory, so the
+// builder and phi kernels that run beside it take other SMs instead of
+// competing for its issue slots (with more heads than SMs it keeps its own
+// size, so that several engines share an SM rather than queue).
 constexpr size_t ENGINE_SM_RESERVE = 200 * 1024;
+
+static int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 1;
+  }
+  return n;
+}
 
 template <int D>
 static cudaError_t launch_engine_d(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   size_t sb = sizeof(EngSmem) + sizeof(double) * ((size_t)dm.C * D - 1);
-  if (sb < ENGINE_SM_RESERVE) sb = ENGINE_SM_RESERVE;
+  if (dm.heads <= sm_count() && sb < ENGINE_SM_RESERVE) sb = ENGINE_SM_RESERVE;
   cudaError_t e = cudaFuncSetAttribute(k_engine<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
   if (e != cudaSuccess) return e;
   k_engine<D><<<dm.heads, 32, sb, s>>>(dm, pl, ca);
