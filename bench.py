@@ -329,9 +329,9 @@ def bench_prefill(args, wl, rank, world, local_rank):
     readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
     loop_flops = atom_flops(m0_rows, d)
 
-    def step():
+    def step(qq=q, kk=k, vv=v, oo=o):
         dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
-        dla.dla_prefill(cfg, q, k, v, o, cache.c, None, ws, st, stream)
+        dla.dla_prefill(cfg, qq, kk, vv, oo, cache.c, None, ws, st, stream)
 
     fixed = args.workload.startswith("fixed")
     if fixed:
@@ -348,8 +348,8 @@ def bench_prefill(args, wl, rank, world, local_rank):
         loop_flops = atom_flops(sum(min(128, T - c * 128) * bin(c).count("1")
                                     for c in range((T + 127) // 128)) * B * H, d)
 
-        def step():
-            dla.dla_fixed_policy_prefill(fcfg, q, k, v, o, fws, st, stream)
+        def step(qq=q, kk=k, vv=v, oo=o):
+            dla.dla_fixed_policy_prefill(fcfg, qq, kk, vv, oo, fws, st, stream)
 
     for _ in range(args.warmup):
         step()
@@ -374,29 +374,54 @@ def bench_prefill(args, wl, rank, world, local_rank):
     launches = prof.p.count
     kt = prof.times_ms()
 
-    # end to end through the public API with host buffers
+    # End to end through the public API with host buffers: every step copies
+    # its q, k, v in from pinned host memory and its o back out. Two device
+    # buffer sets and two copy streams let step i+1's upload and step i's
+    # download run while step i computes, as a stream of requests would.
     pin = [torch.from_numpy(x.view(np.int16) if dt == "bf16" else x).pin_memory()
            for x in (q_h, k_h, v_h)]
     o_host = torch.empty(o.shape, dtype=torch.int16 if dt == "bf16" else torch.float32).pin_memory()
+    sets = [(q, k, v, o), tuple(torch.empty_like(x) for x in (q, k, v, o))]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in sets]    # inputs of the set uploaded
+    ev_used = [torch.cuda.Event() for _ in sets]  # its step has read the inputs, written o
+    ev_out = [torch.cuda.Event() for _ in sets]   # its o downloaded
 
-    def e2e_step():
-        for hsrc, ddst in zip(pin, (q, k, v)):
-            ddst.view(hsrc.dtype).copy_(hsrc, non_blocking=True)
-        step()
-        o_host.copy_(o.view(o_host.dtype), non_blocking=True)
+    def e2e_run(n):
+        up.wait_stream(stream)
+        for i in range(n):
+            j = i % 2
+            qq, kk, vv, oo = sets[j]
+            up.wait_event(ev_used[j])
+            with torch.cuda.stream(up):
+                for hsrc, ddst in zip(pin, (qq, kk, vv)):
+                    ddst.view(hsrc.dtype).copy_(hsrc, non_blocking=True)
+                ev_in[j].record(up)
+            stream.wait_event(ev_in[j])
+            stream.wait_event(ev_out[j])
+            step(qq, kk, vv, oo)
+            ev_used[j].record(stream)
+            down.wait_event(ev_used[j])
+            with torch.cuda.stream(down):
+                o_host.copy_(oo.view(o_host.dtype), non_blocking=True)
+                ev_out[j].record(down)
+        stream.wait_stream(down)
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    e2e_run(max(2, args.warmup // 2))
     torch.cuda.synchronize(dev)
     barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    e2e_steps = max(1, args.steps // 2)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_steps = max(2, args.steps)
+    e2e_run(e2e_steps)
     f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, world, dev)
+    dla.check_device_status(st, "dla_prefill")
+    # the pipelined output is the device-timed step's output, bit for bit
+    if not torch.equal(o_host, o.view(o_host.dtype).cpu()):
+        raise RuntimeError("end-to-end output differs from the device-timed output")
+    del sets
     in_bytes = sum(x.nbytes for x in (q_h, k_h, v_h))
     out_bytes = o_host.numel() * o_host.element_size()
 
@@ -573,25 +598,46 @@ def bench_decode(args, wl, rank, world, local_rank):
     ms = reduce_max(e0.elapsed_time(e1), world, dev)
     kt = prof.times_ms()
     launches = prof.p.count
-    # end to end: host q, k, v per step, o back to the host
+    # End to end: each step's q, k, v come in from pinned host memory and its o
+    # goes back. Steps depend on one another through the cache, so only the
+    # copies overlap: step i+1's upload and step i's download run on copy
+    # streams while step i computes (two device buffer sets).
     hq, hk, hv = (torch.from_numpy(x.view(np.int16)).pin_memory() for x in stp_h)
-    dq, dk_, dv = (torch.empty(N, H, d, dtype=torch.int16, device=dev) for _ in range(3))
+    dsets = [tuple(torch.empty(N, H, d, dtype=torch.int16, device=dev) for _ in range(4))
+             for _ in range(2)]
     ho = torch.empty(N, H, d, dtype=torch.int16).pin_memory()
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in dsets]
+    ev_used = [torch.cuda.Event() for _ in dsets]
+    ev_out = [torch.cuda.Event() for _ in dsets]
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     f0.record(stream)
+    up.wait_stream(stream)
     e2e_steps = min(args.steps, 8)
     for i in range(e2e_steps):
-        j = args.warmup + i
-        dq.copy_(hq[j], non_blocking=True)
-        dk_.copy_(hk[j], non_blocking=True)
-        dv.copy_(hv[j], non_blocking=True)
+        j, b = args.warmup + i, i % 2
+        dq, dk_, dv, do = dsets[b]
+        up.wait_event(ev_used[b])
+        with torch.cuda.stream(up):
+            dq.copy_(hq[j], non_blocking=True)
+            dk_.copy_(hk[j], non_blocking=True)
+            dv.copy_(hv[j], non_blocking=True)
+            ev_in[b].record(up)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])
         dec.step(dq.view(torch.bfloat16), dk_.view(torch.bfloat16), dv.view(torch.bfloat16), tau,
-                 o, stream)
-        ho.copy_(o.view(torch.int16), non_blocking=True)
+                 do.view(torch.bfloat16), stream)
+        ev_used[b].record(stream)
+        down.wait_event(ev_used[b])
+        with torch.cuda.stream(down):
+            ho.copy_(do, non_blocking=True)
+            ev_out[b].record(down)
+    stream.wait_stream(down)
     f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, world, dev)
+    dla.check_device_status(dec.status, "dla_decode_step")
     if rank != 0:
         return None
     ms_step = ms / args.steps
