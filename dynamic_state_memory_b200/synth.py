@@ -14,6 +14,12 @@ draws in float32, in this order):
    draws its centre uniformly from the centres other than the current one.
 4. Keys: ``k_t = centre(t) + sigma * N(0, I_d)`` (no re-normalisation).
 5. Queries ``q ~ N(0, I)``, then values ``v ~ N(0, I)``.
+6. Only with ``value_regimes`` (inputs for the information-score policy, whose
+   score compares the token's rank-1 state v phi(k)^T with the open state, so
+   values must follow the regimes too): ``n_centres`` value centres ~ N(0, I_d),
+   unit-normalised, then ``v_t = value_centre(t) + sigma * N(0, I_d)``,
+   replacing the draw of step 5.  These draws come after all others, so the
+   other inputs are the same with or without the option.
 
 Decode continuation (the decode-step workload): after the prefill tokens, each
 step switches to another centre with probability ``switch_p`` and draws fresh
@@ -97,7 +103,8 @@ def _centre_sequence(rng, n_regimes, n_centres, first=None):
 class HeadStream:
     """One (batch, head) stream: prefill tokens, then optional decode steps."""
 
-    def __init__(self, stream_seed, b, h, *, T, d, n_centres, lengths, sigma, **_):
+    def __init__(self, stream_seed, b, h, *, T, d, n_centres, lengths, sigma,
+                 value_regimes=False, **_):
         self.rng = np.random.default_rng([int(stream_seed), int(b), int(h)])
         self.d = d
         self.sigma = np.float32(sigma)
@@ -112,6 +119,13 @@ class HeadStream:
         self.k = self.centres[tok_centre] + self.sigma * noise
         self.q = self.rng.standard_normal((T, d), dtype=np.float32)
         self.v = self.rng.standard_normal((T, d), dtype=np.float32)
+        self.vcentres = None
+        if value_regimes:
+            vc = self.rng.standard_normal((n_centres, d), dtype=np.float32)
+            vc /= np.linalg.norm(vc, axis=1, keepdims=True).astype(np.float32)
+            self.vcentres = vc.astype(np.float32)
+            vnoise = self.rng.standard_normal((T, d), dtype=np.float32)
+            self.v = self.vcentres[tok_centre] + self.sigma * vnoise
 
     def decode_steps(self, steps, switch_p):
         """Keys continue the last regime and switch w.p. switch_p per step."""
@@ -130,6 +144,9 @@ class HeadStream:
         k = self.centres[idx] + self.sigma * noise
         q = self.rng.standard_normal((steps, self.d), dtype=np.float32)
         v = self.rng.standard_normal((steps, self.d), dtype=np.float32)
+        if self.vcentres is not None:
+            vnoise = self.rng.standard_normal((steps, self.d), dtype=np.float32)
+            v = self.vcentres[idx] + self.sigma * vnoise
         return q, k, v
 
 

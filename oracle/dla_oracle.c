@@ -34,6 +34,19 @@
  *     lambda_{t,i} = softmax_i( phi(q_t) . mu_i / sqrt(d_k) )
  *       (Chlience section 5.3, reading from bounded states).
  *
+ * The information policy (the pages' own criteria, Chlience section 5.1 and
+ * section 5.2) decides and merges on the states themselves:
+ *   - I_t = || N(s_t) - N(S) ||_F / ( || N(S) ||_F + eps ), with s_t the
+ *     per-token state v_t phi(k_t)^T, S the open state before token t and
+ *     N(X) = X / sqrt(mean of the entries of X^2 + eps) (RMSNorm over the
+ *     whole d_v x d_k state, no gain), eps = 1e-6 in both places;
+ *   - b_t = [I_t >= tau]; the first token of a stream has no open state to
+ *     compare with, so it opens one, with I_0 = 0;
+ *   - each state keeps the sum of the scores of its tokens (I-bar); at
+ *     capacity the adjacent sealed pair with the least information density
+ *     (I-bar_i + I-bar_{i+1}) / (n_i + n_{i+1}) is merged (leftmost on ties)
+ *     and the sums add.
+ *
  * The fixed-bucket policy (Chlience section 2 and section 5.4, Log-Linear
  * Attention's Fenwick buckets) keeps a binary-counter list of blocks over
  * [0, t-1]; token t reads the blocks plus {t} with the same softmax, then {t}
@@ -62,12 +75,17 @@
 
 #define OR_POLICY_DLA 0
 #define OR_POLICY_FENWICK 1
+#define OR_POLICY_INFO 2
+
+/* RMSNorm epsilon and the information score's denominator epsilon. */
+#define OR_INFO_EPS 1e-6
 
 typedef struct {
   double *S; /* [dv][dk] sum of v phi(k)^T */
   double *z; /* [dk] sum of phi(k) */
   int64_t n;
   int64_t ts;
+  double info; /* sum of the information scores of its tokens (information policy) */
 } ostate;
 
 typedef struct {
@@ -103,6 +121,7 @@ static void st_alloc(ostate *s, int dk, int dv, int want_S) {
   s->z = (double *)calloc((size_t)dk, sizeof(double));
   s->n = 0;
   s->ts = 0;
+  s->info = 0.0;
 }
 
 static void st_zero(ostate *s, int dk, int dv) {
@@ -110,6 +129,7 @@ static void st_zero(ostate *s, int dk, int dv) {
   memset(s->z, 0, sizeof(double) * (size_t)dk);
   s->n = 0;
   s->ts = 0;
+  s->info = 0.0;
 }
 
 static void st_copy(ostate *dst, const ostate *src, int dk, int dv) {
@@ -117,14 +137,16 @@ static void st_copy(ostate *dst, const ostate *src, int dk, int dv) {
   memcpy(dst->z, src->z, sizeof(double) * (size_t)dk);
   dst->n = src->n;
   dst->ts = src->ts;
+  dst->info = src->info;
 }
 
-/* left <- left + right (S, z, n); left keeps its timestamp. */
+/* left <- left + right (S, z, n, info); left keeps its timestamp. */
 static void st_absorb(ostate *left, const ostate *right, int dk, int dv) {
   if (left->S && right->S)
     for (size_t i = 0; i < (size_t)dv * dk; i++) left->S[i] = left->S[i] + right->S[i];
   for (int i = 0; i < dk; i++) left->z[i] = left->z[i] + right->z[i];
   left->n = left->n + right->n;
+  left->info = left->info + right->info;
 }
 
 /* Ward loss n_a n_b / (n_a + n_b) * sum_i (z_a[i]/n_a - z_b[i]/n_b)^2. */
@@ -149,6 +171,33 @@ static double score(const double *a, const double *b, int dk) {
   return 1.0 - dot / (sqrt(na) * sqrt(nb));
 }
 
+/* Information score of a token against the open state S ([dv][dk]):
+ * || N(v u^T) - N(S) ||_F / (|| N(S) ||_F + eps), N = RMSNorm over all entries. */
+static double info_score(const double *vv, const double *u, const double *S, int dk, int dv) {
+  double cnt = (double)dk * (double)dv;
+  double ss = 0.0, sS = 0.0;
+  for (int a = 0; a < dv; a++)
+    for (int c = 0; c < dk; c++) {
+      double x = vv[a] * u[c];
+      ss = ss + x * x;
+    }
+  for (size_t i = 0; i < (size_t)dv * dk; i++) sS = sS + S[i] * S[i];
+  double rs = sqrt(ss / cnt + OR_INFO_EPS), rS = sqrt(sS / cnt + OR_INFO_EPS);
+  double diff = 0.0, norm = 0.0;
+  for (int a = 0; a < dv; a++)
+    for (int c = 0; c < dk; c++) {
+      double ns = (vv[a] * u[c]) / rs, nS = S[(size_t)a * dk + c] / rS;
+      diff = diff + (ns - nS) * (ns - nS);
+      norm = norm + nS * nS;
+    }
+  return sqrt(diff) / (sqrt(norm) + OR_INFO_EPS);
+}
+
+/* Information density of the union of two adjacent states. */
+static double density(const ostate *a, const ostate *b) {
+  return (a->info + b->info) / ((double)a->n + (double)b->n);
+}
+
 oracle *dla_oracle_new(int nheads, int dk, int dv, int C, int policy, int want_S) {
   oracle *o = (oracle *)calloc(1, sizeof(oracle));
   o->nheads = nheads;
@@ -156,9 +205,11 @@ oracle *dla_oracle_new(int nheads, int dk, int dv, int C, int policy, int want_S
   o->dv = dv;
   o->C = C;
   o->policy = policy;
-  o->want_S = want_S;
+  /* the information policy decides on the states themselves */
+  o->want_S = policy == OR_POLICY_INFO ? 1 : want_S;
+  want_S = o->want_S;
   o->heads = (ohead *)calloc((size_t)nheads, sizeof(ohead));
-  int cap = policy == OR_POLICY_DLA ? C : 64;
+  int cap = policy == OR_POLICY_FENWICK ? 64 : C;
   for (int h = 0; h < nheads; h++) {
     ohead *hd = &o->heads[h];
     hd->cap_sealed = cap;
@@ -199,7 +250,9 @@ typedef struct {
   int32_t *merge_t, *merge_i, *merge_count; /* [nrun][cap], [nrun] */
   int cap;
   int32_t *live; /* [nrun][T] live states read by token t, or NULL */
-  double *margins; /* [nrun][3]: min |r - tau|, min Ward relative gap, #exact ties */
+  double *margins; /* [nrun][3]: min |score - tau|, min relative gap of the merge
+                      criterion (Ward loss or density), #exact ties */
+  double *score;   /* [nrun][T] decision score of each token (r_t or I_t), or NULL */
   int next;        /* work counter */
   pthread_mutex_t mu;
 } job;
@@ -259,6 +312,7 @@ static void run_head_dla(job *J, int r) {
     for (int c = 0; c < dk; c++) kk[c] = widen(J->k, J->dtype, base + c);
     for (int c = 0; c < dk; c++) u[c] = phi(kk[c]);
     double rt = hd->t == 0 ? 0.0 : score(kk, hd->prev_k, dk);
+    if (J->score) J->score[(size_t)r * T + tl] = rt;
     if (hd->t > 0) {
       double mrg = fabs(rt - J->tau);
       if (mrg < min_rm) min_rm = mrg;
@@ -332,6 +386,91 @@ static void run_head_dla(job *J, int r) {
   free(lst);
 }
 
+static void run_head_info(job *J, int r) {
+  oracle *o = J->o;
+  int dk = o->dk, dv = o->dv, C = o->C, T = J->T;
+  ohead *hd = &o->heads[J->head_lo + r];
+  double *u = (double *)malloc(sizeof(double) * dk);
+  double *p = (double *)malloc(sizeof(double) * dk);
+  double *vv = (double *)malloc(sizeof(double) * dv);
+  ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(C + 1));
+  double min_im = INFINITY, min_gap = INFINITY, ties = 0.0;
+  for (int tl = 0; tl < T; tl++) {
+    size_t base = ((size_t)r * T + tl) * dk;
+    size_t vb = ((size_t)r * T + tl) * dv;
+    for (int c = 0; c < dk; c++) u[c] = phi(widen(J->k, J->dtype, base + c));
+    for (int c = 0; c < dv; c++) vv[c] = widen(J->v, J->dtype, vb + c);
+    double it = 0.0;
+    int join = 0;
+    if (hd->has_open) {
+      it = info_score(vv, u, hd->open.S, dk, dv);
+      double mrg = fabs(it - J->tau);
+      if (mrg < min_im) min_im = mrg;
+      join = it < J->tau;
+    }
+    if (J->score) J->score[(size_t)r * T + tl] = it;
+    if (J->boundary) J->boundary[(size_t)r * T + tl] = (uint8_t)(!join);
+    if (!join) {
+      if (hd->has_open) {
+        st_copy(&hd->sealed[hd->nsealed], &hd->open, dk, dv);
+        hd->nsealed++;
+      }
+      if (hd->nsealed == C) {
+        int best = 0;
+        double bl = density(&hd->sealed[0], &hd->sealed[1]);
+        double second = INFINITY;
+        for (int i = 1; i < C - 1; i++) {
+          double l = density(&hd->sealed[i], &hd->sealed[i + 1]);
+          if (l < bl) {
+            second = bl;
+            bl = l;
+            best = i;
+          } else if (l < second) {
+            second = l;
+          }
+        }
+        if (second == bl) ties += 1.0;
+        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;
+        st_absorb(&hd->sealed[best], &hd->sealed[best + 1], dk, dv);
+        ostate tmp = hd->sealed[best + 1];
+        for (int i = best + 1; i < hd->nsealed - 1; i++) hd->sealed[i] = hd->sealed[i + 1];
+        hd->sealed[hd->nsealed - 1] = tmp;
+        hd->nsealed--;
+        record_merge(J, r, hd->t, best);
+      }
+      st_zero(&hd->open, dk, dv);
+      hd->open.ts = hd->t;
+      hd->has_open = 1;
+    }
+    for (int a = 0; a < dv; a++)
+      for (int c = 0; c < dk; c++)
+        hd->open.S[(size_t)a * dk + c] = hd->open.S[(size_t)a * dk + c] + vv[a] * u[c];
+    for (int c = 0; c < dk; c++) hd->open.z[c] = hd->open.z[c] + u[c];
+    hd->open.n = hd->open.n + 1;
+    hd->open.info = hd->open.info + it;
+    int m = 0;
+    for (int i = 0; i < hd->nsealed; i++) lst[m++] = &hd->sealed[i];
+    lst[m++] = &hd->open;
+    if (J->live) J->live[(size_t)r * T + tl] = m;
+    if (J->out && (!J->out_mask || J->out_mask[tl])) {
+      for (int c = 0; c < dk; c++) p[c] = phi(widen(J->q, J->dtype, base + c));
+      readout(o, lst, m, p, J->out + ((size_t)r * T + tl) * dv);
+    }
+    hd->prev_r = it;
+    hd->t = hd->t + 1;
+  }
+  if (J->margins) {
+    double *mg = J->margins + (size_t)r * 3;
+    if (min_im < mg[0]) mg[0] = min_im;
+    if (min_gap < mg[1]) mg[1] = min_gap;
+    mg[2] += ties;
+  }
+  free(u);
+  free(p);
+  free(vv);
+  free(lst);
+}
+
 static void run_head_fenwick(job *J, int r) {
   oracle *o = J->o;
   int dk = o->dk, dv = o->dv, T = J->T;
@@ -390,6 +529,7 @@ static void *worker(void *arg) {
     pthread_mutex_unlock(&J->mu);
     if (r >= J->head_hi - J->head_lo) break;
     if (J->o->policy == OR_POLICY_DLA) run_head_dla(J, r);
+    else if (J->o->policy == OR_POLICY_INFO) run_head_info(J, r);
     else run_head_fenwick(J, r);
   }
   return NULL;
@@ -399,14 +539,16 @@ static void *worker(void *arg) {
  * `dtype`; outputs (all optional) are indexed by the run-local head r.
  * `out` needs the oracle created with want_S = 1; with `out_mask` the readout
  * runs only at tokens whose mask entry is set (states are updated at every
- * token either way).  Returns 0 on success. */
-int dla_oracle_run_masked(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+ * token either way); `score` receives each token's decision score.  The
+ * information policy needs v even without outputs.  Returns 0 on success. */
+int dla_oracle_run_scored(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
                           const void *q, const void *k, const void *v, double *out,
                           const uint8_t *out_mask, uint8_t *boundary, int32_t *merge_t,
                           int32_t *merge_i, int32_t *merge_count, int cap, int32_t *live,
-                          double *margins, int nthreads) {
+                          double *margins, double *score, int nthreads) {
   if (!o || head_lo < 0 || head_hi > o->nheads || head_lo > head_hi || T < 0) return 1;
   if (out && (!o->want_S || !q || !v)) return 2;
+  if (o->policy == OR_POLICY_INFO && !v) return 2;
   if (!k) return 3;
   job J;
   memset(&J, 0, sizeof J);
@@ -428,6 +570,7 @@ int dla_oracle_run_masked(oracle *o, int head_lo, int head_hi, int T, double tau
   J.cap = cap;
   J.live = live;
   J.margins = margins;
+  J.score = score;
   int nrun = head_hi - head_lo;
   int32_t *mc_local = NULL;
   if (!merge_count) {
@@ -447,6 +590,17 @@ int dla_oracle_run_masked(oracle *o, int head_lo, int head_hi, int T, double tau
   return 0;
 }
 
+/* Same, without the per-token scores. */
+int dla_oracle_run_masked(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+                          const void *q, const void *k, const void *v, double *out,
+                          const uint8_t *out_mask, uint8_t *boundary, int32_t *merge_t,
+                          int32_t *merge_i, int32_t *merge_count, int cap, int32_t *live,
+                          double *margins, int nthreads) {
+  return dla_oracle_run_scored(o, head_lo, head_hi, T, tau, dtype, q, k, v, out, out_mask,
+                               boundary, merge_t, merge_i, merge_count, cap, live, margins, NULL,
+                               nthreads);
+}
+
 /* Same, reading out at every token. */
 int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
                    const void *q, const void *k, const void *v, double *out,
@@ -459,9 +613,9 @@ int dla_oracle_run(oracle *o, int head_lo, int head_hi, int T, double tau, int d
 
 /* Live states of one head in time order (sealed..., open).  Returns m and
  * fills up to `maxm` entries: S [m][dv][dk] (if non-NULL and kept), z
- * [m][dk], n [m], ts [m]; plus prev_r and t. */
-int dla_oracle_state(const oracle *o, int head, int maxm, double *S, double *z, int64_t *n,
-                     int64_t *ts, double *prev_r, int64_t *t) {
+ * [m][dk], n [m], ts [m], info [m] (score sums); plus prev_r and t. */
+int dla_oracle_state_info(const oracle *o, int head, int maxm, double *S, double *z, int64_t *n,
+                          int64_t *ts, double *info, double *prev_r, int64_t *t) {
   if (!o || head < 0 || head >= o->nheads) return -1;
   const ohead *hd = &o->heads[head];
   int m = hd->nsealed + (hd->has_open ? 1 : 0);
@@ -472,8 +626,15 @@ int dla_oracle_state(const oracle *o, int head, int maxm, double *S, double *z, 
     if (z) memcpy(z + (size_t)i * dk, s->z, sizeof(double) * (size_t)dk);
     if (n) n[i] = s->n;
     if (ts) ts[i] = s->ts;
+    if (info) info[i] = s->info;
   }
   if (prev_r) *prev_r = hd->prev_r;
   if (t) *t = hd->t;
   return m;
+}
+
+/* Same, without the score sums. */
+int dla_oracle_state(const oracle *o, int head, int maxm, double *S, double *z, int64_t *n,
+                     int64_t *ts, double *prev_r, int64_t *t) {
+  return dla_oracle_state_info(o, head, maxm, S, z, n, ts, NULL, prev_r, t);
 }

@@ -17,7 +17,7 @@ _SRC = os.path.join(_HERE, "dla_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPES = {"f32": 0, "bf16": 1, "f64": 2}
-POLICIES = {"dla": 0, "fenwick": 1}
+POLICIES = {"dla": 0, "fenwick": 1, "info": 2}
 
 
 def build(force: bool = False) -> str:
@@ -48,8 +48,14 @@ def load_library(path: str):
     lib.dla_oracle_run_masked.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
                                           P, P, ctypes.c_int, P, P, ctypes.c_int]
+    lib.dla_oracle_run_scored.restype = ctypes.c_int
+    lib.dla_oracle_run_scored.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
+                                          P, P, ctypes.c_int, P, P, P, ctypes.c_int]
     lib.dla_oracle_state.restype = ctypes.c_int
     lib.dla_oracle_state.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
+    lib.dla_oracle_state_info.restype = ctypes.c_int
+    lib.dla_oracle_state_info.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P]
     return lib
 
 
@@ -78,9 +84,9 @@ class Oracle:
                  want_S: bool = True, lib=None):
         self.lib = _load() if lib is None else lib
         self.nheads, self.d_k, self.d_v, self.C = nheads, d_k, d_v, C
-        self.want_S = want_S
+        self.want_S = want_S or policy == "info"
         self.policy = policy
-        self.h = self.lib.dla_oracle_new(nheads, d_k, d_v, C, POLICIES[policy], int(want_S))
+        self.h = self.lib.dla_oracle_new(nheads, d_k, d_v, C, POLICIES[policy], int(self.want_S))
 
     def __del__(self):
         if getattr(self, "h", None):
@@ -96,8 +102,11 @@ class Oracle:
         ``out_mask`` ([T] bool) limits the readout to the marked tokens (rows
         elsewhere stay zero); states are updated at every token regardless.
         Returns dict with out [nrun, T, d_v] (fp64 or None), boundary
-        [nrun, T] u8, merges as lists of (t, i) per head, live [nrun, T] and
-        margins [nrun, 3] (min |r - tau|, min Ward relative gap, exact ties).
+        [nrun, T] u8, merges as lists of (t, i) per head, live [nrun, T],
+        score [nrun, T] (each token's decision score: r_t, or I_t for the
+        information policy) and margins [nrun, 3] (min |score - tau|, min
+        relative gap of the merge criterion, exact ties).  The information
+        policy needs v even without outputs.
         """
         k = np.ascontiguousarray(k)
         nrun, T = k.shape[0], k.shape[1]
@@ -105,7 +114,8 @@ class Oracle:
             q = np.ascontiguousarray(q)
             v = np.ascontiguousarray(v)
         else:
-            q = v = None
+            q = None
+            v = np.ascontiguousarray(v) if self.policy == "info" else None
         out = np.zeros((nrun, T, self.d_v), dtype=np.float64) if want_out else None
         boundary = np.zeros((nrun, T), dtype=np.uint8)
         cap = (T + 1) if cap is None else cap
@@ -116,34 +126,38 @@ class Oracle:
         margins = np.zeros((nrun, 3), dtype=np.float64)
         margins[:, 0] = np.inf
         margins[:, 1] = np.inf
+        score = np.zeros((nrun, T), dtype=np.float64)
         nthreads = cores() if nthreads is None else nthreads
         if out_mask is not None:
             out_mask = np.ascontiguousarray(out_mask, dtype=np.uint8)
             if out_mask.shape != (T,):
                 raise ValueError("out_mask must have shape [T]")
-        rc = self.lib.dla_oracle_run_masked(self.h, head_lo, head_lo + nrun, T, float(tau),
+        rc = self.lib.dla_oracle_run_scored(self.h, head_lo, head_lo + nrun, T, float(tau),
                                             DTYPES[dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                             _ptr(out_mask), _ptr(boundary), _ptr(mt), _ptr(mi),
-                                            _ptr(mc), cap, _ptr(live), _ptr(margins), nthreads)
+                                            _ptr(mc), cap, _ptr(live), _ptr(margins),
+                                            _ptr(score), nthreads)
         if rc != 0:
             raise RuntimeError(f"dla_oracle_run failed with code {rc}")
         merges = [list(zip(mt[r, :min(mc[r], cap)].tolist(), mi[r, :min(mc[r], cap)].tolist()))
                   for r in range(nrun)]
         return dict(out=out, boundary=boundary, merges=merges, merge_count=mc, live=live,
-                    margins=margins)
+                    margins=margins, score=score)
 
     def state(self, head: int):
-        """Live states of a head in time order: S, z, n, ts, prev_r, t."""
-        maxm = self.C if self.policy == "dla" else 64
+        """Live states of a head in time order: S, z, n, ts, info (score sums),
+        prev_r, t."""
+        maxm = 64 if self.policy == "fenwick" else self.C
         S = np.zeros((maxm, self.d_v, self.d_k)) if self.want_S else None
         z = np.zeros((maxm, self.d_k))
         n = np.zeros(maxm, dtype=np.int64)
         ts = np.zeros(maxm, dtype=np.int64)
+        info = np.zeros(maxm)
         pr = np.zeros(1)
         t = np.zeros(1, dtype=np.int64)
-        m = self.lib.dla_oracle_state(self.h, head, maxm, _ptr(S), _ptr(z), _ptr(n), _ptr(ts),
-                                      _ptr(pr), _ptr(t))
-        return dict(S=None if S is None else S[:m], z=z[:m], n=n[:m], ts=ts[:m],
+        m = self.lib.dla_oracle_state_info(self.h, head, maxm, _ptr(S), _ptr(z), _ptr(n),
+                                           _ptr(ts), _ptr(info), _ptr(pr), _ptr(t))
+        return dict(S=None if S is None else S[:m], z=z[:m], n=n[:m], ts=ts[:m], info=info[:m],
                     prev_r=float(pr[0]), t=int(t[0]), m=m)
 
 
@@ -154,12 +168,13 @@ def prefill(q, k, v, *, C: int, tau: float, dtype: str, policy: str = "dla",
     d_v = v.shape[-1] if v is not None else d
     orc = Oracle(B * H, d, d_v, C, policy, want_S=want_out)
     res = orc.run(k.reshape(B * H, T, d),
-                  None if q is None else q.reshape(B * H, T, d),
+                  None if q is None or not want_out else q.reshape(B * H, T, d),
                   None if v is None else v.reshape(B * H, T, d_v),
                   tau=tau, dtype=dtype, want_out=want_out, nthreads=nthreads)
     if res["out"] is not None:
         res["out"] = res["out"].reshape(B, H, T, d_v)
     res["boundary"] = res["boundary"].reshape(B, H, T)
     res["live"] = res["live"].reshape(B, H, T)
+    res["score"] = res["score"].reshape(B, H, T)
     res["oracle"] = orc
     return res

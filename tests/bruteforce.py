@@ -114,3 +114,69 @@ def fenwick_ranges(t):
             start += 1 << b
     out.append((t, t))
     return out
+
+
+# ---- information policy (the pages' own decision and merge criteria) --------
+
+INFO_EPS = 1e-6
+
+
+def info_score_gram(U, V, t, a):
+    """Information score of token t against the open state over tokens [a, t-1].
+
+    Written from Gram sums instead of the d_v x d_k matrices: with
+    s_t = v_t u_t^T and S = sum_s v_s u_s^T,
+    <s_t, S> = sum_s (v_t.v_s)(u_t.u_s), |S|^2 = sum_{s,s'} (v_s.v_s')(u_s.u_s'),
+    |s_t|^2 = |v_t|^2 |u_t|^2; N(X) = X / sqrt(|X|^2 / (d_k d_v) + eps), and
+    |N(s) - N(S)|^2 = |s|^2/a + |S|^2/b - 2 <s,S>/sqrt(ab) with a, b the two
+    RMS denominators squared.
+    """
+    D2 = U.shape[1] * V.shape[1]
+    Ur, Vr = U[a:t], V[a:t]
+    x = float(((Vr @ V[t]) * (Ur @ U[t])).sum())
+    SS = float(((Vr @ Vr.T) * (Ur @ Ur.T)).sum())
+    ss = float(V[t] @ V[t]) * float(U[t] @ U[t])
+    ra = ss / D2 + INFO_EPS
+    rb = SS / D2 + INFO_EPS
+    num2 = ss / ra + SS / rb - 2.0 * x / np.sqrt(ra * rb)
+    return float(np.sqrt(max(num2, 0.0)) / (np.sqrt(SS / rb) + INFO_EPS))
+
+
+def info_simulate(k, v, C, tau):
+    """The information policy's decisions from scratch, on token ranges.
+
+    A token with no open state opens one (score 0); otherwise it joins the
+    open state when its score is below tau.  Each state is a range with the sum
+    of its tokens' scores; at capacity the adjacent sealed pair of least
+    (sum_i + sum_{i+1}) / (tokens in both ranges) merges, first minimum on ties.
+    Returns (boundary [T], merges [(t, i)], score [T]).
+    """
+    T = k.shape[0]
+    U = phi(k)
+    V = np.asarray(v, dtype=np.float64)
+    score = np.zeros(T)
+    boundary = np.zeros(T, dtype=np.uint8)
+    merges = []
+    sealed = []  # [first, last, score sum]
+    open_ = None
+    for t in range(T):
+        if open_ is None:
+            it, join = 0.0, False
+        else:
+            it = info_score_gram(U, V, t, open_[0])
+            join = it < tau
+        score[t] = it
+        if not join:
+            boundary[t] = 1
+            if open_ is not None:
+                sealed.append(open_)
+            if len(sealed) == C:
+                dens = [(sealed[i][2] + sealed[i + 1][2]) / (sealed[i + 1][1] - sealed[i][0] + 1)
+                        for i in range(C - 1)]
+                i = int(np.argmin(dens))
+                sealed[i:i + 2] = [[sealed[i][0], sealed[i + 1][1], sealed[i][2] + sealed[i + 1][2]]]
+                merges.append((t, i))
+            open_ = [t, t, 0.0]
+        open_[1] = t
+        open_[2] += it
+    return boundary, merges, score

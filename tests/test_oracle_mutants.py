@@ -10,6 +10,7 @@ import tempfile
 import pytest
 
 from oracle import oracle as O
+from tests import test_oracle_info as info_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(O.__file__), "dla_oracle.c")
@@ -39,8 +40,27 @@ MUTANTS = {
 }
 
 
+# Plausible mistakes in the information policy, caught by its own pins.
+INFO_MUTANTS = {
+    "info_no_rmsnorm": ("double rs = sqrt(ss / cnt + OR_INFO_EPS), rS = sqrt(sS / cnt + OR_INFO_EPS);",
+                        "double rs = 1.0, rS = 1.0;"),
+    "info_denominator_not_normalised": ("return sqrt(diff) / (sqrt(norm) + OR_INFO_EPS);",
+                                        "return sqrt(diff) / (sqrt(sS) + OR_INFO_EPS);"),
+    "info_transposed_token_state": ("double ns = (vv[a] * u[c]) / rs,",
+                                    "double ns = (vv[c] * u[a]) / rs,"),
+    "info_non_strict_join": ("join = it < J->tau;", "join = it <= J->tau;"),
+    "info_density_left_only": ("return (a->info + b->info) / ((double)a->n + (double)b->n);",
+                               "return a->info / ((double)a->n + (double)b->n);"),
+    "info_density_mean_of_means": ("return (a->info + b->info) / ((double)a->n + (double)b->n);",
+                                   "return a->info / (double)a->n + b->info / (double)b->n;"),
+    "info_rightmost_tie": ("double l = density(&hd->sealed[i], &hd->sealed[i + 1]);\n          if (l < bl) {",
+                           "double l = density(&hd->sealed[i], &hd->sealed[i + 1]);\n          if (l <= bl) {"),
+    "info_sum_not_carried": ("  left->info = left->info + right->info;\n", ""),
+}
+
+
 def build_mutant(name):
-    old, new = MUTANTS[name]
+    old, new = {**MUTANTS, **INFO_MUTANTS}[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     src = src.replace(old, new, 1)
@@ -73,3 +93,14 @@ def test_mutant_is_caught(name):
     lib = build_mutant(name)
     with pytest.raises(AssertionError):
         all_pins(lib)
+
+
+def test_real_oracle_passes_info_pins():
+    info_pins.all_info_pins(None)
+
+
+@pytest.mark.parametrize("name", sorted(INFO_MUTANTS))
+def test_info_mutant_is_caught(name):
+    lib = build_mutant(name)
+    with pytest.raises(AssertionError):
+        info_pins.all_info_pins(lib)
