@@ -17,7 +17,10 @@
 //   k_engine   one warp per head walks tiles and boundaries in time order:
 //              seals, capacity merges by least Ward loss (Chlience section 5.2
 //              and Corollary 1), slot allocation; emits the materializer op
-//              list, the per-tile atoms/events and the merge trace.
+//              list, the per-tile atoms/events and the merge trace.  Under the
+//              information policy the pair criterion is the information
+//              density (I_a + I_b) / (n_a + n_b) of the pair's score sums
+//              (Chlience section 5.2) and the boundaries come from info.cu.
 //
 // Arithmetic that decides an integer is fp64 with explicit round-to-nearest
 // intrinsics (no contraction): r_t is summed in index order exactly like the
@@ -362,6 +365,7 @@ struct EngSmem {
   long long ts[128];
   double loss[128];
   double rn[128];          // 1 / n of sealed states (__drcp_rn)
+  double info[128];        // score sum of each slot's state (information policy)
   double zring[ZR][128];
   double z[1];             // [C][D], dynamic
 };
@@ -437,6 +441,13 @@ __device__ __forceinline__ void ward_loss2(const EngSmem *sm, const double *z, i
   l_bc = __dmul_rn(f2, s2);
 }
 
+// Information density of the union of slots a and b (Chlience section 5.2):
+// (I_a + I_b) / (n_a + n_b), the oracle's operation order.
+__device__ __forceinline__ double info_density(const EngSmem *sm, int sa, int sb) {
+  return __ddiv_rn(__dadd_rn(sm->info[sa], sm->info[sb]),
+                   __dadd_rn((double)sm->n[sa], (double)sm->n[sb]));
+}
+
 // Leftmost argmin of loss[0 .. L-1] (L >= 1).  Losses are non-negative and
 // finite, so their bit patterns order like their values: three 32-bit warp
 // reductions (high word, low word, index) replace an fp64 shuffle tree.
@@ -494,6 +505,9 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   int32_t *const tr_i = ca.trace.merge_i ? ca.trace.merge_i + (size_t)u * ca.trace.cap : nullptr;
   const bool tracing = ca.trace.merge_count != nullptr;
   const int tcap = ca.trace.cap;
+  const bool info = dm.info != 0;
+  double *const c_info = info ? ca.info_slot + (size_t)u * C : nullptr;
+  const double *const seg_info = info ? pl.seg_info + (size_t)u * W : nullptr;
 
   // ---- segment-end sums: prefetch ring ------------------------------------
   auto zfetch = [&](int g) {
@@ -533,6 +547,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     sm->loss[p] = c_loss[p];
     sm->sver[p] = -1;
     sm->lastmod[p] = -1;
+    sm->info[p] = info ? c_info[p] : 0.0;
     if (p < m) atomicOr(&sm->used[o >> 5], 1u << (o & 31));
   }
   for (int i = lane; i < C * D; i += 32) zs[i] = c_z[i];
@@ -686,12 +701,14 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             if (lane == 0) sm->n[os] += s - cur_from;
           }
           if (j >= 1) ztake(zs + (size_t)os * D);
+          if (info && j >= 1 && lane == 0) sm->info[os] = seg_info[j - 1];
           __syncwarp();
           // seal: the open state joins the sealed list (all m states sealed)
           if (lane == 0) sm->rn[os] = __drcp_rn((double)sm->n[os]);
           __syncwarp();
           if (m >= 2) {
-            const double l = ward_loss<QD>(sm, zs, D, sm->order[m - 2], os, lane);
+            const double l = info ? info_density(sm, sm->order[m - 2], os)
+                                  : ward_loss<QD>(sm, zs, D, sm->order[m - 2], os, lane);
             if (lane == 0) sm->loss[m - 2] = l;
           }
           __syncwarp();
@@ -738,6 +755,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
               const long long na = sm->n[a] + sm->n[bb];
               sm->n[a] = na;
               sm->rn[a] = __drcp_rn((double)na);
+              if (info) sm->info[a] = __dadd_rn(sm->info[a], sm->info[bb]);
               sm->sver[a] = -1;
               sm->sver[bb] = -1;
             }
@@ -748,7 +766,12 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
             const int sl = sm->order[left ? is - 1 : is];
             const int sr = sm->order[right ? is + 1 : is];
             double l_left, l_right;
-            ward_loss2<QD>(sm, zs, D, sl, a, sr, lane, l_left, l_right);
+            if (info) {
+              l_left = info_density(sm, sl, a);
+              l_right = info_density(sm, a, sr);
+            } else {
+              ward_loss2<QD>(sm, zs, D, sl, a, sr, lane, l_left, l_right);
+            }
             if (lane == 0) {
               if (left) sm->loss[is - 1] = l_left;
               if (right) sm->loss[is] = l_right;
@@ -782,6 +805,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
         if (lane == 0) {
           sm->n[slot] = 0;
           sm->ts[slot] = t0 + s;
+          sm->info[slot] = 0.0;
           sm->order[m] = slot;
           sm->sver[slot] = -1;
           sm->lastmod[slot] = -1;
@@ -806,6 +830,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     }
     emit(OP_STORE, os, 0, 0);
     if (nseg >= 1) ztake(zs + (size_t)os * D);
+    if (info && nseg >= 1 && lane == 0) sm->info[os] = seg_info[nseg - 1];
   }
   cp_async_wait<0>();
   __syncwarp();
@@ -814,6 +839,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     c_n[p] = sm->n[p];
     c_ts[p] = sm->ts[p];
     c_loss[p] = sm->loss[p];
+    if (info) c_info[p] = sm->info[p];
   }
   for (int i = lane; i < C * D; i += 32) c_z[i] = zs[i];
   if (lane == 0) {
@@ -861,7 +887,7 @@ cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, c
 
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
   const dim3 g(dm.tiles, dm.heads);
-  if (sums_in_score(dm, ca, DLA_POLICY_DYNAMIC)) {
+  if (!dm.info && sums_in_score(dm, ca, DLA_POLICY_DYNAMIC)) {
     // the tile sums came with the score
   } else {
     k_tilesum_any<<<g, dm.D, 0, s>>>(dm, pl, ca);

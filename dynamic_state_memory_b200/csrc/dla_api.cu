@@ -54,7 +54,8 @@ Dims make_dims(const dla_config &cfg, int policy) {
   const bool tc = use_tc(cfg);
   dm.M = tc ? tc_tile_rows() : simt_tile_rows();
   dm.D = cfg.d_k;
-  dm.C = policy == DLA_POLICY_DYNAMIC ? cfg.C : 64;
+  dm.C = cfg.C;
+  dm.info = policy == DLA_POLICY_INFO ? 1 : 0;
   int W = cfg.window > 0 ? cfg.window : (tc ? 8192 : 2048);
   W = (W + dm.M - 1) / dm.M * dm.M;
   const int Tr = (cfg.T + dm.M - 1) / dm.M * dm.M;
@@ -104,6 +105,15 @@ void carve_plan(Carver &cv, const Dims &dm, Plan &pl) {
   pl.pieces = cv.take<float>(h * (size_t)dm.pmax * dm.D * dm.D);
   pl.phi_tab = cv.take<double>(4096);
   carve_pre(cv, dm, pl);
+  pl.seg_info = dm.info ? cv.take<double>(h * dm.W) : nullptr;
+}
+
+// The information policy's state carried across a call's windows.
+void carve_info(Carver &cv, const Dims &dm, CallArgs &ca) {
+  const size_t h = dm.heads;
+  ca.info_S = cv.take<double>(h * dm.D * dm.D);
+  ca.info_aux = cv.take<double>(h * 4);
+  ca.info_slot = cv.take<double>(h * dm.C);
 }
 
 // Fixed Fenwick policy: one pass over the call (no windows); versions are the
@@ -155,7 +165,8 @@ bool cfg_ok(const dla_config *cfg, int policy) {
 
 dla_status shape_ok(const dla_config *cfg, int policy) {
   if (cfg->d_k != cfg->d_v || !d_ok(cfg->d_k)) return DLA_ERR_UNSUPPORTED;
-  if (policy == DLA_POLICY_DYNAMIC && (cfg->C < 2 || cfg->C > 128)) return DLA_ERR_UNSUPPORTED;
+  if ((policy == DLA_POLICY_DYNAMIC || policy == DLA_POLICY_INFO) && (cfg->C < 2 || cfg->C > 128))
+    return DLA_ERR_UNSUPPORTED;
   return DLA_OK;
 }
 
@@ -277,19 +288,30 @@ size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
     carve_fenwick(cv, dm, pl, &a, &b);
     return cv.off;
   }
-  if (policy != DLA_POLICY_DYNAMIC) return 0;
+  if (policy != DLA_POLICY_DYNAMIC && policy != DLA_POLICY_INFO) return 0;
   const Dims dm = make_dims(*cfg, policy);
   Plan pl{};
   Carver cv{nullptr};
   for (int i = 0, n = plan_count(*cfg, dm); i < n; i++) carve_plan(cv, dm, pl);
+  if (policy == DLA_POLICY_INFO) {
+    CallArgs ca{};
+    carve_info(cv, dm, ca);
+  }
   return cv.off;
 }
 
-dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, const void *v,
-                       void *o, const dla_cache *cache, const dla_trace *trace, void *ws,
-                       size_t ws_bytes, int32_t *dev_status, void *stream) {
-  if (!cfg_ok(cfg, DLA_POLICY_DYNAMIC) || !cache) return DLA_ERR_INVALID_ARG;
-  const dla_status sh = shape_ok(cfg, DLA_POLICY_DYNAMIC);
+}  // extern "C"
+
+namespace {
+
+// A prefill call of the dynamic policy (cosine score, Ward merges) or the
+// information policy (state score, density merges): the same windows,
+// streams and kernels but the score and the engine's pair criterion.
+dla_status prefill_impl(int policy, const dla_config *cfg, const void *q, const void *k,
+                        const void *v, void *o, const dla_cache *cache, const dla_trace *trace,
+                        void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!cfg_ok(cfg, policy) || !cache) return DLA_ERR_INVALID_ARG;
+  const dla_status sh = shape_ok(cfg, policy);
   if (sh != DLA_OK) return sh;
   if (cache->N != cfg->B || cache->H != cfg->H || cache->C != cfg->C || cache->d_k != cfg->d_k ||
       cache->d_v != cfg->d_v)
@@ -303,11 +325,14 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16 ||
       reinterpret_cast<uintptr_t>(v) % 16 || reinterpret_cast<uintptr_t>(o) % 16)
     return DLA_ERR_INVALID_ARG;
-  const Dims dm = make_dims(*cfg, DLA_POLICY_DYNAMIC);
+  const bool info = policy == DLA_POLICY_INFO;
+  const Dims dm = make_dims(*cfg, policy);
   Plan plans[NPLAN] = {};
   Carver cv{static_cast<char *>(ws)};
   const int nplan = plan_count(*cfg, dm);
   for (int i = 0; i < nplan; i++) carve_plan(cv, dm, plans[i]);
+  CallArgs ca{};
+  if (info) carve_info(cv, dm, ca);
   if (cv.off > ws_bytes) return DLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Aux *ax = aux_streams();
@@ -317,7 +342,6 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   cudaStream_t sp = ax->sp;  // the tensor-core readout's prologue
   cudaStream_t sx = ax->sx;  // the materializer, with the tensor-core readout
   cudaStream_t sb = ax->sb;  // the tensor-core state builder
-  CallArgs ca{};
   ca.q = q;
   ca.k = k;
   ca.v = v;
@@ -332,6 +356,8 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
   } else {
     memset(&ca.trace, 0, sizeof ca.trace);
   }
+  if (info && cudaMemsetAsync(ca.info_slot, 0, sizeof(double) * dm.heads * dm.C, s) != cudaSuccess)
+    return DLA_ERR_CUDA;
   ca.dev_status = dev_status;
   // Fork: the decision kernels and the engine run on the auxiliary stream,
   // the state build, materializer and readout on the caller's stream.  The
@@ -358,7 +384,13 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
     // cache's open state, written by window wi - 1's engine
     if (reuse && cudaStreamWaitEvent(sd, ax->ev[EV_DONE0 + pi], 0) != cudaSuccess)
       return DLA_ERR_CUDA;
-    { ProfScope ps(pf, DLA_K_SCORE, sd); e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, sd); }
+    if (info) {
+      ProfScope ps(pf, DLA_K_INFO_SCORE, sd);
+      e = launch_info_score(dm, pl, ca, sd);
+    } else {
+      ProfScope ps(pf, DLA_K_SCORE, sd);
+      e = launch_score(dm, pl, ca, DLA_POLICY_DYNAMIC, sd);
+    }
     if (e != cudaSuccess) return DLA_ERR_CUDA;
     { ProfScope ps(pf, DLA_K_SEGSCAN, sd); e = launch_segscan(dm, pl, ca, sd); }
     if (e != cudaSuccess || cudaEventRecord(ax->ev[EV_SCAN], sd) != cudaSuccess) return DLA_ERR_CUDA;
@@ -420,6 +452,25 @@ dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, cons
       return DLA_ERR_CUDA;
   }
   return DLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dla_status dla_prefill(const dla_config *cfg, const void *q, const void *k, const void *v,
+                       void *o, const dla_cache *cache, const dla_trace *trace, void *ws,
+                       size_t ws_bytes, int32_t *dev_status, void *stream) {
+  return prefill_impl(DLA_POLICY_DYNAMIC, cfg, q, k, v, o, cache, trace, ws, ws_bytes,
+                      dev_status, stream);
+}
+
+dla_status dla_info_policy_prefill(const dla_config *cfg, const void *q, const void *k,
+                                   const void *v, void *o, const dla_cache *cache,
+                                   const dla_trace *trace, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, void *stream) {
+  return prefill_impl(DLA_POLICY_INFO, cfg, q, k, v, o, cache, trace, ws, ws_bytes, dev_status,
+                      stream);
 }
 
 size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {

@@ -63,6 +63,7 @@ struct Dims {
   int32_t vbytes;  // bytes of one version's S
   int32_t pmax;    // max tensor-core pieces per head per window (0 = none)
   int32_t fenwick; // 1: fixed Fenwick policy (every token a piece; closed-form epochs)
+  int32_t info;    // 1: information policy (state score, density merges)
 };
 
 // Per-window plan, every array strided by head.
@@ -93,6 +94,10 @@ struct Plan {
   void *phi_k;         // [heads][tiles][2][128][64] bf16 phi(k) tiles, as in shared memory
   float *pre_w;        // [heads][tiles][amax][M] atom weights
   void *pre_o;         // [heads][tiles][M * D] intra-tile outputs (bf16)
+  // information policy: score sum of each window piece's state at the
+  // piece's end (the piece's own tokens plus, for a continued open state,
+  // its earlier ones)
+  double *seg_info;    // [heads][W]
 };
 
 struct CallArgs {
@@ -105,6 +110,10 @@ struct CallArgs {
   dla_cache cache;
   dla_trace trace;    // boundary == NULL when no trace
   int32_t *dev_status;
+  // information policy, carried across the call's windows (null otherwise)
+  double *info_S;     // [heads][D * D] fp64 open state, element j of thread i at j * 2D + i
+  double *info_aux;   // [heads][4]: |S|^2, the open state's score sum, has-open flag
+  double *info_slot;  // [heads][C] score sum of each cache slot's state
 };
 
 __device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
@@ -140,6 +149,7 @@ cudaError_t launch_score(const Dims &dm, const Plan &pl, const CallArgs &ca, int
                          cudaStream_t s);
 cudaError_t launch_segscan(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_segsum(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
+cudaError_t launch_info_score(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s);
 cudaError_t launch_materialize(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                cudaStream_t s, bool bf16_versions);

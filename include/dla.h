@@ -56,7 +56,7 @@ typedef enum {
 
 typedef enum { DLA_F32 = 0, DLA_BF16 = 1 } dla_dtype;
 
-typedef enum { DLA_POLICY_DYNAMIC = 0, DLA_POLICY_FENWICK = 1 } dla_policy;
+typedef enum { DLA_POLICY_DYNAMIC = 0, DLA_POLICY_FENWICK = 1, DLA_POLICY_INFO = 2 } dla_policy;
 
 /* Kernel kinds reported through dla_profile. */
 typedef enum {
@@ -70,7 +70,8 @@ typedef enum {
   DLA_K_DECODE_STREAM = 7,
   DLA_K_BUILD = 8,       /* tensor-core state-piece builder */
   DLA_K_READOUT_PRE = 9, /* tensor-core readout prologue (weights, intra-tile output) */
-  DLA_K_PHI = 10         /* phi(q) as the bf16 tensor-core operand */
+  DLA_K_PHI = 10,        /* phi(q) as the bf16 tensor-core operand */
+  DLA_K_INFO_SCORE = 11  /* information policy: state score + boundary */
 } dla_kernel_kind;
 
 /* Optional timing hook (host memory, caller-owned).  When non-NULL, the
@@ -147,8 +148,9 @@ size_t dla_cache_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v
 dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int32_t d_k,
                           int32_t d_v, void *dev_base, size_t bytes, void *stream);
 
-/* Workspace bytes for dla_prefill (policy = DLA_POLICY_DYNAMIC) or
- * dla_fixed_policy_prefill (DLA_POLICY_FENWICK) with this config. */
+/* Workspace bytes for dla_prefill (policy = DLA_POLICY_DYNAMIC),
+ * dla_fixed_policy_prefill (DLA_POLICY_FENWICK) or dla_info_policy_prefill
+ * (DLA_POLICY_INFO) with this config; 0 for an invalid config or policy. */
 size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy);
 
 /* DLA prefill of T tokens for B x H streams, continuing `cache` (required,
@@ -200,6 +202,30 @@ dla_status dla_decode_step_static(const dla_cache *cache, float tau, int32_t in_
 dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const void *k,
                                     const void *v, void *o, void *ws, size_t ws_bytes,
                                     int32_t *dev_status, void *stream);
+
+/* The pages' own decision and merge rule (Chlience section 5.1 and section
+ * 5.2) through the same windows, engine and readout as dla_prefill:
+ *   - token t's state v_t phi(k_t)^T is compared with the open state S after
+ *     RMSNorm over all d_v x d_k entries (no gain):
+ *       I_t = |N(v_t phi(k_t)^T) - N(S)|_F / (|N(S)|_F + 1e-6),
+ *       N(X) = X / sqrt(mean of X^2 + 1e-6);
+ *   - I_t >= tau opens a new state; the first token of a stream opens one
+ *     with I = 0;
+ *   - each state keeps the sum of its tokens' scores, and at capacity the
+ *     adjacent sealed pair with the least (sum_i + sum_i+1) / (n_i + n_i+1)
+ *     merges (leftmost on ties); the readout is dla_prefill's.
+ * Arguments as for dla_prefill; ws: at least dla_workspace_bytes(cfg,
+ * DLA_POLICY_INFO) bytes.  The decisions need the open state in fp64 and the
+ * states' score sums, which the cache does not hold, so every stream starts
+ * from an empty cache: a stream whose cache has t > 0 sets
+ * DLA_ERR_UNSUPPORTED in *dev_status and its outputs are unspecified.  After
+ * the call the cache holds the policy's states, counts and time order, and
+ * pair_loss the pair densities; dla_decode_step does not continue it (it
+ * applies the cosine score and Ward merges). */
+dla_status dla_info_policy_prefill(const dla_config *cfg, const void *q, const void *k,
+                                   const void *v, void *o, const dla_cache *cache,
+                                   const dla_trace *trace, void *ws, size_t ws_bytes,
+                                   int32_t *dev_status, void *stream);
 
 /* Static description of a status code. */
 const char *dla_status_string(dla_status status);

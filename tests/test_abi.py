@@ -48,6 +48,8 @@ def test_size_queries_and_argument_errors():
     good = dla.make_config(1, 1, 16, 32, 4, 0.5, dla.DLA_F32)
     assert dla.dla_workspace_bytes(good) > 0
     assert dla.dla_workspace_bytes(good, dla.DLA_POLICY_FENWICK) > 0
+    # the information policy carries its fp64 open states across windows
+    assert dla.dla_workspace_bytes(good, dla.DLA_POLICY_INFO) > dla.dla_workspace_bytes(good)
     assert dla.dla_workspace_bytes(good, 7) == 0
     lib = dla._lib
     cache = dla.dla_cache()
@@ -61,5 +63,12 @@ def test_size_queries_and_argument_errors():
     assert lib.dla_prefill(ctypes.byref(good), None, None, None, None, ctypes.byref(cache), None,
                            None, 0, None, None) == 1
     assert lib.dla_cache_init(ctypes.byref(cache), 1, 1, 4, 32, 32, None, 0, None) == 1
+    # the information policy's entry point checks the same way
+    assert lib.dla_info_policy_prefill(None, None, None, None, None, ctypes.byref(cache), None,
+                                       None, 0, None, None) == 1
+    assert lib.dla_info_policy_prefill(ctypes.byref(good), None, None, None, None,
+                                       ctypes.byref(cache), None, None, 0, None, None) == 1
+    assert lib.dla_info_policy_prefill(ctypes.byref(bad_c), None, None, None, None,
+                                       ctypes.byref(cache), None, None, 0, None, None) == 2
     for code in range(8):
         assert dla.status_string(code)
