@@ -33,6 +33,17 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "sm_max_mhz": 1965.0}
 SMS = 148
 FP32_LANES_PER_SM = 128
+FP64_LANES_PER_SM = 64
+
+
+def policy_of(workload):
+    """The decision policy a workload runs: the fixed Fenwick buckets, the
+    information policy or the dynamic (cosine score, Ward merge) one."""
+    if workload.startswith("fixed"):
+        return "fenwick"
+    if workload.startswith("info"):
+        return "info"
+    return "dla"
 
 
 def load_peaks():
@@ -172,6 +183,7 @@ class ClockSampler:
 TRAFFIC_SOURCES = {
     ("readout", "tc"): ("readout_tc", ["readout_tc.cu", "tc_ptx.cuh", "dla_internal.cuh"]),
     ("decode_stream", "-"): ("decode_stream", ["decode.cu", "dla_internal.cuh"]),
+    ("info_score", "tc"): ("info_score", ["info.cu", "dla_internal.cuh"]),
 }
 
 
@@ -303,7 +315,10 @@ def bench_prefill(args, wl, rank, world, local_rank):
     prof = dla.Profiler(cap=4096)
     dcode = dla.DLA_BF16 if dt == "bf16" else dla.DLA_F32
     cfg = dla.make_config(B, H, T, d, C, wl["tau"], dcode, args.window, prof.p)
-    ws = torch.empty(dla.dla_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    info = policy_of(args.workload) == "info"
+    policy_code = dla.DLA_POLICY_INFO if info else dla.DLA_POLICY_DYNAMIC
+    run = dla.dla_info_policy_prefill if info else dla.dla_prefill
+    ws = torch.empty(dla.dla_workspace_bytes(cfg, policy_code), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -311,7 +326,7 @@ def bench_prefill(args, wl, rank, world, local_rank):
     # one traced run (untimed) to count live states for the FLOP model
     tr = dla.Trace(B * H, T, T + 1, dev)
     dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
-    dla.dla_prefill(cfg, q, k, v, o, cache.c, tr.c, ws, st, stream)
+    run(cfg, q, k, v, o, cache.c, tr.c, ws, st, stream)
     torch.cuda.synchronize(dev)
     dla.check_device_status(st, "dla_prefill")
     bnd = tr.boundary.cpu().numpy()
@@ -331,7 +346,7 @@ def bench_prefill(args, wl, rank, world, local_rank):
 
     def step(qq=q, kk=k, vv=v, oo=o):
         dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
-        dla.dla_prefill(cfg, qq, kk, vv, oo, cache.c, None, ws, st, stream)
+        run(cfg, qq, kk, vv, oo, cache.c, None, ws, st, stream)
 
     fixed = args.workload.startswith("fixed")
     if fixed:
@@ -435,8 +450,13 @@ def bench_prefill(args, wl, rank, world, local_rank):
     # it waits for SMs: these are not the serialised shares of an ncu launch
     # list. The roofline is the readout's (the contraction), the largest
     # kernel of that serialised list on every prefill workload here.
+    # Under the information policy the sequential fp64 score dominates the
+    # step and carries the roofline instead.
     tot = {kname: sum(v_) for kname, v_ in kt.items()}
-    dom = "readout" if "readout" in kt else max(tot, key=tot.get)
+    if info:
+        dom = "info_score"
+    else:
+        dom = "readout" if "readout" in kt else max(tot, key=tot.get)
     per_launch_ms = statistics.mean(kt[dom])
     n_launch = len(kt[dom])
     steps_recorded = args.steps
@@ -455,6 +475,15 @@ def bench_prefill(args, wl, rank, world, local_rank):
             peak = peaks.get("bf16_tflops_sustained", 1371.4)
             peak_note = f"bf16 dense, {peaks_kind} sustained"
         achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
+    elif dom == "info_score":
+        # per token: x_t = v_t^T S u_t (2 d^2 FLOP) and the state update
+        # S += v_t u_t^T (2 d^2 FLOP), fp64; one CTA (one SM) per head
+        flops_per_launch = 4.0 * d * d * B * H * T / (n_launch / steps_recorded)
+        bound, unit = "alu", "TFLOP/s"
+        peak = SMS * FP64_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        peak_note = ("fp64 FMA: 148 SMs x 64 lanes x 2 FLOP x max SM clock (derived); the "
+                     "kernel runs one SM per head, %d of 148" % min(B * H, SMS))
+        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
     else:
         bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
         achieved = float("nan")
@@ -469,15 +498,22 @@ def bench_prefill(args, wl, rank, world, local_rank):
             "event_share_note": "CUDA-event time per kernel on its own stream; concurrent "
                                 "streams overlap, so these are not serialised shares"}
     cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(
-        wl, q_h, k_h, v_h, policy="fenwick" if fixed else "dla")
+        wl, q_h, k_h, v_h, policy=policy_of(args.workload))
     e2e_val = tokens / (e2e_ms * 1e-3) / 1e6
     extra = {}
+    if info and "readout" in kt:
+        # the readout is the dynamic policy's; its atom loop's rate beside
+        rl_ms = statistics.mean(kt["readout"])
+        ra = loop_flops / (len(kt["readout"]) / steps_recorded) / (rl_ms * 1e-3) / 1e12
+        rp = peaks.get("bf16_tflops_sustained", 1371.4)
+        extra["readout_atom_loop"] = {"achieved": round(ra, 3), "peak": rp, "unit": "TFLOP/s",
+                                      "frac": round(ra / rp, 4), "launch_ms": round(rl_ms, 4)}
     if fixed:
         extra = {"dla_same_inputs": {
             "C": C, "value": round(tokens / (dla_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
             "ms_per_step": round(dla_ms, 4), "mean_live_states": round(dla_live / (B * H * T), 2)}}
     return {
-        **({"policy": "fenwick"} if fixed else {}), **extra,
+        **({"policy": policy_of(args.workload)} if fixed or info else {}), **extra,
         "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -710,7 +746,7 @@ def bench_reference(args, wl):
     Ts = min(T, args.ref_tokens)
     times = []
     for i in range(args.warmup + args.steps):
-        orc = O.Oracle(H, d, d, wl["C"])
+        orc = O.Oracle(H, d, d, wl["C"], policy_of(args.workload))
         t0 = time.perf_counter()
         orc.run(k[0, :, :Ts], q[0, :, :Ts], v[0, :, :Ts], tau=wl["tau"], dtype=wl["dtype"],
                 nthreads=cores)

@@ -6,10 +6,11 @@
 // a state with I = 0.
 //
 // One CTA of 2D threads per head walks the window in blocks of INFO_K tokens.
-// Thread i keeps row i / 2, columns (i % 2) D/2 .. + D/2 of S in fp64
+// Thread i keeps row i % D, columns (i / D) D/2 .. + D/2 of S in fp64
 // registers.  Writing x_t = <s_t, S> = v_t^T S u_t,
 //   |N(s) - N(S)|^2 = |s|^2 / ra + |S|^2 / rb - 2 x_t / sqrt(ra rb)
-// (ra, rb: the two squared RMS denominators), so a block needs per token
+// (ra, rb: the two squared RMS denominators; with g = 1 / sqrt(rb) the
+// middle term is |S|^2 g^2 and |N(S)| = |S| g), so a block needs per token
 // v_t^T S0 u_t against the state S0 at the block's start (one pass over the
 // registers with INFO_K accumulators and one block reduction) and the Gram
 // terms (v_t . v_j)(u_t . u_j) of the block's earlier tokens j (staged per
@@ -41,9 +42,11 @@ struct InfoSmem {
   uint32_t raw[2][2][INFO_CHUNK * D];  // [buffer][k, v] input rows (room for fp32)
   double u[INFO_CHUNK][D];             // phi(k) in fp64
   double v[INFO_CHUNK][D];
-  double uu[INFO_CHUNK], vv[INFO_CHUNK];  // |u_t|^2, |v_t|^2
+  // per token: |s|^2, |s|^2 / ra and 1 / sqrt(ra), ra = |s|^2 / (d_k d_v) + eps
+  double ss[INFO_CHUNK], ssra[INFO_CHUNK], rsa[INFO_CHUNK];
   double H[INFO_CHUNK][INFO_K];           // (v_t . v_j)(u_t . u_j), j an earlier token of t's block
   double red[2][INFO_K][2 * D / 32];      // per-warp partials, by block parity
+  int jb;                                 // the block's last boundary (-1: none)
 };
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -81,8 +84,8 @@ __device__ void info_stage(InfoSmem<D> &sm, int buf, const Dims &dm, const CallA
   cp_commit();
 }
 
-// raw[buf] -> u = phi(k), v in fp64; then the squared norms and the in-block
-// Gram terms of the chunk.  Two barriers inside.
+// raw[buf] -> u = phi(k), v in fp64; then each token's norm terms and the
+// in-block Gram terms of the chunk.  Two barriers inside.
 template <int D>
 __device__ void info_prepare(InfoSmem<D> &sm, int buf, bool bf16) {
   for (int e = threadIdx.x; e < INFO_CHUNK * D; e += blockDim.x) {
@@ -111,8 +114,11 @@ __device__ void info_prepare(InfoSmem<D> &sm, int buf, bool bf16) {
     a = warp_sum(a);
     b = warp_sum(b);
     if (lane == 0) {
-      sm.uu[r] = a;
-      sm.vv[r] = b;
+      const double ss = a * b;  // |s_t|^2 = |v_t|^2 |u_t|^2
+      const double ra = fma(ss, 1.0 / (double)(D * D), INFO_EPS);
+      sm.ss[r] = ss;
+      sm.ssra[r] = ss / ra;
+      sm.rsa[r] = rsqrt(ra);
     }
   }
   // one thread per (token, earlier token of its block); each lane starts at
@@ -143,7 +149,9 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
   extern __shared__ __align__(16) unsigned char info_raw[];
   InfoSmem<D> &sm = *reinterpret_cast<InfoSmem<D> *>(info_raw);
   const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int a = tid >> 1, c0 = (tid & 1) * EPT;
+  // warp w holds rows 32 (w % (D / 32)) .. + 31, all in one column half, so
+  // the lanes of a warp read the same element of u: one broadcast per load
+  const int a = tid % D, c0 = (tid / D) * EPT;
   const bool bf16 = ca.in_dtype == DLA_BF16;
   const int esize = bf16 ? 2 : 4;
   const double tau = (double)ca.tau;
@@ -213,52 +221,60 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
         if (lane == 0) sm.red[rb][i][warp] = p;
       }
       __syncthreads();
-      double A[INFO_K];
+      // the block's decisions in token order, by warp 0 (its lanes agree);
+      // the other warps wait: the fp64 pipe is the kernel's bound, so they
+      // do not repeat this sequence
+      if (warp == 0) {
+        double A[INFO_K];
 #pragma unroll
-      for (int i = 0; i < INFO_K; i++) {
-        double s = 0.0;
+        for (int i = 0; i < INFO_K; i++) {
+          double s = 0.0;
 #pragma unroll
-        for (int w = 0; w < NW; w++) s += sm.red[rb][i][w];
-        A[i] = s;
-      }
-      // the block's decisions in token order (every thread, same values)
-      int jb = -1;  // the block's last boundary so far
+          for (int w = 0; w < NW; w++) s += sm.red[rb][i][w];
+          A[i] = s;
+        }
+        int jb = -1;  // the block's last boundary so far
 #pragma unroll
-      for (int i = 0; i < INFO_K; i++) {
-        if (i < nb) {
-          const int t = t0 + r0 + i;
-          const double ss = sm.uu[r0 + i] * sm.vv[r0 + i];
-          double I = 0.0, x = 0.0;
-          bool bnd = true;
-          if (has_open) {
-            x = jb < 0 ? A[i] : 0.0;
-            for (int j = jb < 0 ? 0 : jb; j < i; j++) x += sm.H[r0 + i][j];
-            const double ra = fma(ss, inv_d2, INFO_EPS), rq = fma(sS, inv_d2, INFO_EPS);
-            const double nS2 = sS / rq;
-            const double num2 = fmax(ss / ra + nS2 - 2.0 * x / sqrt(ra * rq), 0.0);
-            I = sqrt(num2) / (sqrt(nS2) + INFO_EPS);
-            bnd = !(I < tau);
-          }
-          if (tid == 0) {
-            r_out[t] = I;
-            b_out[t] = bnd ? 1 : 0;
-            if (tr_b) tr_b[t] = bnd ? 1 : 0;
-          }
-          if (bnd) {
-            if (t > 0) {
-              if (tid == 0) seg[sg] = iopen;
-              sg++;
+        for (int i = 0; i < INFO_K; i++) {
+          if (i < nb) {
+            const int t = t0 + r0 + i;
+            double I = 0.0, x = 0.0;
+            bool bnd = true;
+            if (has_open) {
+              x = jb < 0 ? A[i] : 0.0;
+              for (int j = jb < 0 ? 0 : jb; j < i; j++) x += sm.H[r0 + i][j];
+              // |N(s) - N(S)|^2 = |s|^2/ra + |S|^2 g^2 - 2 x g / sqrt(ra),
+              // g = 1 / sqrt(|S|^2 / (d_k d_v) + eps); |N(S)| = |S| g
+              const double g = rsqrt(fma(sS, inv_d2, INFO_EPS));
+              const double num2 = fmax(sm.ssra[r0 + i] + sS * g * g - 2.0 * x * sm.rsa[r0 + i] * g, 0.0);
+              I = sqrt(num2) / (sqrt(sS) * g + INFO_EPS);
+              bnd = !(I < tau);
             }
-            jb = i;
-            sS = ss;
-            iopen = I;
-            has_open = true;
-          } else {
-            sS = sS + 2.0 * x + ss;
-            iopen = iopen + I;
+            if (lane == 0) {
+              r_out[t] = I;
+              b_out[t] = bnd ? 1 : 0;
+              if (tr_b) tr_b[t] = bnd ? 1 : 0;
+            }
+            const double ssv = sm.ss[r0 + i];
+            if (bnd) {
+              if (t > 0) {
+                if (lane == 0) seg[sg] = iopen;
+                sg++;
+              }
+              jb = i;
+              sS = ssv;
+              iopen = I;
+              has_open = true;
+            } else {
+              sS = sS + 2.0 * x + ssv;
+              iopen = iopen + I;
+            }
           }
         }
+        if (lane == 0) sm.jb = jb;
       }
+      __syncthreads();
+      const int jb = sm.jb;
       // add the block's tokens from its last boundary on
       if (jb >= 0) {
 #pragma unroll
