@@ -153,3 +153,34 @@ def test_decode_full_size(gpu):
         got = np.stack([outs[s][n, h] for s in range(steps)])
         err = float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
         assert err <= TOL["bf16"], (n, h, err)
+
+
+def test_info_policy_full_size(gpu):
+    """The information policy on info_t8192 (every stream, the benchmark's
+    launch configuration).  Boundaries of every stream bit for bit; merges bit
+    for bit on every stream whose pair densities the oracle separates by more
+    than the kernel's rounding (a relative 1e-6), which must be at least 60 of
+    the 64, since a closer near-tie may resolve either way; two of those streams'
+    outputs at sampled tokens."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    wl = synth.WORKLOADS["info_t8192"]
+    q, k, v = gen_prefill_parallel(wl)
+    B, H, T, d = k.shape
+    cache = dla.Cache(B, H, wl["C"], d)
+    o, tr = dla.info_prefill(to_device(q, "bf16"), to_device(k, "bf16"), to_device(v, "bf16"),
+                             cache, wl["tau"])
+    torch.cuda.synchronize()
+    orc = O.Oracle(B * H, d, d, wl["C"], "info")
+    res = orc.run(k.reshape(B * H, T, d), None, v.reshape(B * H, T, d), tau=wl["tau"],
+                  dtype="bf16", want_out=False)
+    mg = res["margins"]
+    assert mg[:, 0].min() > 1e-6
+    assert np.array_equal(tr.boundary.cpu().numpy().reshape(B * H, T), res["boundary"])
+    got = tr.merges()
+    clear = [u for u in range(B * H) if mg[u, 1] > 1e-6 and mg[u, 2] == 0]
+    assert len(clear) >= 60, len(clear)
+    for u in clear:
+        assert got[u] == res["merges"][u], u
+    heads = [(u // H, u % H) for u in (clear[0], clear[-1])]
+    check_outputs(from_device(o), q, k, v, wl["C"], wl["tau"], "info", heads, wl["seed"])
