@@ -219,3 +219,24 @@ def all_info_pins(lib):
     check_info_invariants(lib)
     check_info_single_state(lib)
     check_info_all_singletons(lib)
+
+
+def test_value_regimes_leave_other_inputs_unchanged():
+    # the value-regime draws come after all others: q and k are those of the
+    # plain recipe, and v follows each token's regime (one value centre per
+    # key centre), within the noise
+    kw = dict(T=200, d=16, n_centres=5, lengths=("geometric", 12.0), sigma=0.05)
+    plain = synth.HeadStream(77, 0, 1, **kw)
+    vr = synth.HeadStream(77, 0, 1, value_regimes=True, **kw)
+    assert np.array_equal(plain.q, vr.q) and np.array_equal(plain.k, vr.k)
+    assert not np.array_equal(plain.v, vr.v)
+    # each v is nearest to its regime's value centre, whose key centre is
+    # nearest to k
+    kc = np.argmax(vr.k @ plain.centres.T, axis=1)
+    vc = np.argmax(vr.v @ vr.vcentres.T, axis=1)
+    assert (kc == vc).mean() > 0.95
+    # and the workloads without the option draw what they drew before
+    wl = dict(synth.WORKLOADS["tiny_f32"], T=64)
+    a = synth.make_prefill(wl)
+    b = synth.make_prefill(dict(wl, value_regimes=False))
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
