@@ -253,6 +253,16 @@ typedef struct {
   double *margins; /* [nrun][3]: min |score - tau|, min relative gap of the merge
                       criterion (Ward loss or density), #exact ties */
   double *score;   /* [nrun][T] decision score of each token (r_t or I_t), or NULL */
+  /* forced merges (NULL: argmin): each capacity merge of head r takes the
+   * next entry (t, i) of force_t / force_i [nrun][fcap] (force_count [nrun]
+   * entries) instead of the argmin; excess [nrun] receives the largest
+   * relative excess (l_i - l_min) / l_min of a forced pair's criterion over
+   * the minimum (0 for the minimum itself, +inf when the list does not match
+   * the capacity merges, i.e. a wrong token, an index out of range, or an
+   * entry left over or missing) */
+  const int32_t *force_t, *force_i, *force_count;
+  int fcap;
+  double *excess;
   int next;        /* work counter */
   pthread_mutex_t mu;
 } job;
@@ -264,6 +274,42 @@ static void record_merge(job *J, int r, int64_t t, int i) {
     J->merge_i[(size_t)r * J->cap + c] = i;
   }
   J->merge_count[r] = c + 1;
+}
+
+/* Forced mode: the pair the capacity merge at token t takes.  `best` is the
+ * argmin and `bl` its criterion; crit(i) gives pair i's criterion.  Updates
+ * the head's forced-list position *fk and largest excess *ex. */
+static int forced_pair(job *J, int r, int *fk, int64_t t, int best, double bl, int npairs,
+                       double (*crit)(const ohead *, int, int), const ohead *hd, int dk,
+                       double *ex) {
+  int k = (*fk)++;
+  const int32_t *ft = J->force_t + (size_t)r * J->fcap;
+  const int32_t *fi = J->force_i + (size_t)r * J->fcap;
+  if (k >= J->force_count[r] || k >= J->fcap || (int64_t)ft[k] != t || fi[k] < 0 ||
+      fi[k] >= npairs) {
+    *ex = INFINITY;
+    return best;
+  }
+  int i = fi[k];
+  double l = crit(hd, i, dk);
+  double e = l == bl ? 0.0 : (bl > 0.0 ? (l - bl) / bl : INFINITY);
+  if (e > *ex) *ex = e;
+  return i;
+}
+
+static double crit_ward(const ohead *hd, int i, int dk) {
+  return ward(&hd->sealed[i], &hd->sealed[i + 1], dk);
+}
+
+static double crit_density(const ohead *hd, int i, int dk) {
+  (void)dk;
+  return density(&hd->sealed[i], &hd->sealed[i + 1]);
+}
+
+/* Forced mode, at the end of a head's run: every forced entry was used. */
+static void forced_close(job *J, int r, int fk, double ex) {
+  if (fk != J->force_count[r]) ex = INFINITY;
+  if (ex > J->excess[r] || ex != ex) J->excess[r] = ex;
 }
 
 /* Readout: lambda = softmax(phi(q).mu/sqrt(dk)) over states; o = sum lambda S p. */
@@ -307,6 +353,8 @@ static void run_head_dla(job *J, int r) {
   double *vv = (double *)malloc(sizeof(double) * dv);
   ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(C + 1));
   double min_rm = INFINITY, min_gap = INFINITY, ties = 0.0;
+  int fk = 0;
+  double fex = 0.0;
   for (int tl = 0; tl < T; tl++) {
     size_t base = ((size_t)r * T + tl) * dk;
     for (int c = 0; c < dk; c++) kk[c] = widen(J->k, J->dtype, base + c);
@@ -340,6 +388,8 @@ static void run_head_dla(job *J, int r) {
         }
         if (second == bl) ties += 1.0;
         else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;
+        if (J->force_count)
+          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward, hd, dk, &fex);
         st_absorb(&hd->sealed[best], &hd->sealed[best + 1], dk, dv);
         /* drop best+1: rotate its buffers to the end of the list */
         ostate tmp = hd->sealed[best + 1];
@@ -379,6 +429,7 @@ static void run_head_dla(job *J, int r) {
     if (min_gap < mg[1]) mg[1] = min_gap;
     mg[2] += ties;
   }
+  if (J->force_count) forced_close(J, r, fk, fex);
   free(kk);
   free(u);
   free(p);
@@ -395,6 +446,8 @@ static void run_head_info(job *J, int r) {
   double *vv = (double *)malloc(sizeof(double) * dv);
   ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(C + 1));
   double min_im = INFINITY, min_gap = INFINITY, ties = 0.0;
+  int fk = 0;
+  double fex = 0.0;
   for (int tl = 0; tl < T; tl++) {
     size_t base = ((size_t)r * T + tl) * dk;
     size_t vb = ((size_t)r * T + tl) * dv;
@@ -431,6 +484,8 @@ static void run_head_info(job *J, int r) {
         }
         if (second == bl) ties += 1.0;
         else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;
+        if (J->force_count)
+          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_density, hd, dk, &fex);
         st_absorb(&hd->sealed[best], &hd->sealed[best + 1], dk, dv);
         ostate tmp = hd->sealed[best + 1];
         for (int i = best + 1; i < hd->nsealed - 1; i++) hd->sealed[i] = hd->sealed[i + 1];
@@ -465,6 +520,7 @@ static void run_head_info(job *J, int r) {
     if (min_gap < mg[1]) mg[1] = min_gap;
     mg[2] += ties;
   }
+  if (J->force_count) forced_close(J, r, fk, fex);
   free(u);
   free(p);
   free(vv);
@@ -540,16 +596,25 @@ static void *worker(void *arg) {
  * `out` needs the oracle created with want_S = 1; with `out_mask` the readout
  * runs only at tokens whose mask entry is set (states are updated at every
  * token either way); `score` receives each token's decision score.  The
- * information policy needs v even without outputs.  Returns 0 on success. */
-int dla_oracle_run_scored(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+ * information policy needs v even without outputs.  With force_count
+ * (dynamic and information policies) the capacity merges take the pairs of
+ * the given list instead of the argmin (see job.force_t); the decisions that
+ * open states do not depend on merges, so they are unchanged.  Returns 0 on
+ * success. */
+int dla_oracle_run_forced(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
                           const void *q, const void *k, const void *v, double *out,
                           const uint8_t *out_mask, uint8_t *boundary, int32_t *merge_t,
                           int32_t *merge_i, int32_t *merge_count, int cap, int32_t *live,
-                          double *margins, double *score, int nthreads) {
+                          double *margins, double *score, const int32_t *force_t,
+                          const int32_t *force_i, const int32_t *force_count, int fcap,
+                          double *excess, int nthreads) {
   if (!o || head_lo < 0 || head_hi > o->nheads || head_lo > head_hi || T < 0) return 1;
   if (out && (!o->want_S || !q || !v)) return 2;
   if (o->policy == OR_POLICY_INFO && !v) return 2;
   if (!k) return 3;
+  if (force_count && (!force_t || !force_i || !excess || fcap < 0 ||
+                      o->policy == OR_POLICY_FENWICK))
+    return 4;
   job J;
   memset(&J, 0, sizeof J);
   J.o = o;
@@ -571,6 +636,11 @@ int dla_oracle_run_scored(oracle *o, int head_lo, int head_hi, int T, double tau
   J.live = live;
   J.margins = margins;
   J.score = score;
+  J.force_t = force_t;
+  J.force_i = force_i;
+  J.force_count = force_count;
+  J.fcap = fcap;
+  J.excess = excess;
   int nrun = head_hi - head_lo;
   int32_t *mc_local = NULL;
   if (!merge_count) {
@@ -588,6 +658,17 @@ int dla_oracle_run_scored(oracle *o, int head_lo, int head_hi, int T, double tau
   pthread_mutex_destroy(&J.mu);
   free(mc_local);
   return 0;
+}
+
+/* Same, taking every capacity merge's pair from the argmin. */
+int dla_oracle_run_scored(oracle *o, int head_lo, int head_hi, int T, double tau, int dtype,
+                          const void *q, const void *k, const void *v, double *out,
+                          const uint8_t *out_mask, uint8_t *boundary, int32_t *merge_t,
+                          int32_t *merge_i, int32_t *merge_count, int cap, int32_t *live,
+                          double *margins, double *score, int nthreads) {
+  return dla_oracle_run_forced(o, head_lo, head_hi, T, tau, dtype, q, k, v, out, out_mask,
+                               boundary, merge_t, merge_i, merge_count, cap, live, margins, score,
+                               NULL, NULL, NULL, 0, NULL, nthreads);
 }
 
 /* Same, without the per-token scores. */

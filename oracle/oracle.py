@@ -52,6 +52,11 @@ def load_library(path: str):
     lib.dla_oracle_run_scored.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
                                           P, P, ctypes.c_int, P, P, P, ctypes.c_int]
+    lib.dla_oracle_run_forced.restype = ctypes.c_int
+    lib.dla_oracle_run_forced.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_double, ctypes.c_int, P, P, P, P, P, P, P,
+                                          P, P, ctypes.c_int, P, P, P, P, P, P, ctypes.c_int,
+                                          P, ctypes.c_int]
     lib.dla_oracle_state.restype = ctypes.c_int
     lib.dla_oracle_state.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
     lib.dla_oracle_state_info.restype = ctypes.c_int
@@ -95,7 +100,7 @@ class Oracle:
 
     def run(self, k, q=None, v=None, *, tau: float, dtype: str, head_lo: int = 0,
             want_out: bool = True, cap: int | None = None, nthreads: int | None = None,
-            out_mask=None):
+            out_mask=None, force_merges=None):
         """Run T tokens for heads [head_lo, head_lo + k.shape[0]).
 
         k, q, v: arrays [nrun, T, d] (float32, float64 or bf16 uint16 bits).
@@ -107,6 +112,13 @@ class Oracle:
         information policy) and margins [nrun, 3] (min |score - tau|, min
         relative gap of the merge criterion, exact ties).  The information
         policy needs v even without outputs.
+
+        ``force_merges`` (one list of (t, i) per run head) makes every
+        capacity merge take the listed pair instead of the argmin; the result
+        then has ``excess`` [nrun]: the largest relative excess of a forced
+        pair's merge criterion over the minimum at its merge (0 when every
+        forced pair was a minimum, inf when the list does not match the
+        capacity merges the decisions call for).
         """
         k = np.ascontiguousarray(k)
         nrun, T = k.shape[0], k.shape[1]
@@ -132,17 +144,31 @@ class Oracle:
             out_mask = np.ascontiguousarray(out_mask, dtype=np.uint8)
             if out_mask.shape != (T,):
                 raise ValueError("out_mask must have shape [T]")
-        rc = self.lib.dla_oracle_run_scored(self.h, head_lo, head_lo + nrun, T, float(tau),
+        ft = fi = fc = excess = None
+        fcap = 0
+        if force_merges is not None:
+            if len(force_merges) != nrun:
+                raise ValueError("force_merges needs one list per run head")
+            fcap = max(1, max(len(m) for m in force_merges))
+            ft = np.zeros((nrun, fcap), dtype=np.int32)
+            fi = np.zeros((nrun, fcap), dtype=np.int32)
+            fc = np.array([len(m) for m in force_merges], dtype=np.int32)
+            for r, m in enumerate(force_merges):
+                for j, (t_, i_) in enumerate(m):
+                    ft[r, j], fi[r, j] = t_, i_
+            excess = np.zeros(nrun, dtype=np.float64)
+        rc = self.lib.dla_oracle_run_forced(self.h, head_lo, head_lo + nrun, T, float(tau),
                                             DTYPES[dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                             _ptr(out_mask), _ptr(boundary), _ptr(mt), _ptr(mi),
                                             _ptr(mc), cap, _ptr(live), _ptr(margins),
-                                            _ptr(score), nthreads)
+                                            _ptr(score), _ptr(ft), _ptr(fi), _ptr(fc), fcap,
+                                            _ptr(excess), nthreads)
         if rc != 0:
             raise RuntimeError(f"dla_oracle_run failed with code {rc}")
         merges = [list(zip(mt[r, :min(mc[r], cap)].tolist(), mi[r, :min(mc[r], cap)].tolist()))
                   for r in range(nrun)]
         return dict(out=out, boundary=boundary, merges=merges, merge_count=mc, live=live,
-                    margins=margins, score=score)
+                    margins=margins, score=score, excess=excess)
 
     def state(self, head: int):
         """Live states of a head in time order: S, z, n, ts, info (score sums),

@@ -209,8 +209,80 @@ def test_info_trace_only_mode_matches():
     assert tr["merges"] == full["merges"]
 
 
+def _f(x):
+    return float("inf") if x == "inf" else float(x)
+
+
+def check_info_margins_hand(lib=None):
+    """min |I_t - tau|, the least relative gap between the best and the
+    second-best pair density over the merges and the count of exact ties,
+    derived by hand for the golden trace (tests/golden/info_hand_trace.json)."""
+    g = json.load(open(os.path.join(HERE, "golden", "info_hand_trace.json")))
+    v = np.array(g["v"], dtype=np.float64)[:, None]
+    z = np.zeros_like(v)
+    res, _ = run_info(z, z, v, g["C"], g["tau"], lib=lib)
+    got = res["margins"][0]
+    want = g["margins_approx"]
+    assert abs(got[0] - want[0]) < 1e-5 and abs(got[1] - want[1]) < 1e-5 and got[2] == want[2], got
+    T = g["zero_T"]
+    z = np.zeros((T, 1))
+    res, _ = run_info(z, z, z, g["zero_C"], g["zero_tau"], lib=lib)
+    got = res["margins"][0]
+    want = [_f(x) for x in g["zero_margins"]]
+    assert got[0] == want[0] and got[1] == want[1] and got[2] == want[2], got
+
+
+def test_info_margins_hand():
+    check_info_margins_hand()
+
+
+def check_info_forced_mode(seed, C, tau, lib=None):
+    """The information policy with merges taken from a list: its own list
+    reproduces the run (excess 0); the first merge forced onto another pair
+    gives brute-force outputs over the implied ranges and the relative excess
+    of that pair's density, recomputed from the ranges' score sums (Gram-form
+    scores), over the least one."""
+    T, d = 48, 6
+    q, k, v = info_case(seed, T, d)
+    res, _ = run_info(q, k, v, C, tau, lib=lib)
+    merges = res["merges"][0]
+
+    def forced(lst):
+        orc = O.Oracle(1, d, d, C, "info", lib=lib)
+        return orc.run(k[None], q[None], v[None], tau=tau, dtype="f64", nthreads=1,
+                       force_merges=[lst])
+
+    same = forced(merges)
+    assert np.array_equal(same["out"], res["out"]) and same["excess"][0] == 0.0
+    if not merges or C < 3:
+        return
+    t0, i0 = merges[0]
+    alt = (t0, (i0 + 1) % (C - 1))
+    lst = forced([alt])["merges"][0]
+    got = forced(lst)
+    assert got["merges"][0] == lst and lst[0] == alt
+    bnd, _, score = bf.info_simulate(k, v, C, tau)
+    assert res["boundary"][0].tolist() == bnd.tolist()
+    o = bf.outputs(q, k, v, bf.replay(bnd, lst, C))
+    assert np.allclose(got["out"][0], o, rtol=0, atol=1e-11 * np.abs(o).max())
+    sealed = bf.replay(bnd[:t0], [], C)[t0 - 1]
+    dens = np.array([(score[a0:b1 + 1].sum()) / (b1 - a0 + 1)
+                     for (a0, _), (_, b1) in zip(sealed[:-1], sealed[1:])])
+    best = dens.min()
+    want = (dens[alt[1]] - best) / best if best > 0 else (0.0 if dens[alt[1]] == 0 else np.inf)
+    assert abs(got["excess"][0] - want) <= 1e-6 * max(1.0, want), (got["excess"][0], want)
+
+
+@pytest.mark.parametrize("seed,C", [(s, C) for s in range(8) for C in (3, 5)])
+def test_info_forced_mode(seed, C):
+    check_info_forced_mode(seed, C, 0.5)
+
+
 def all_info_pins(lib):
     check_info_hand_trace(lib)
+    check_info_margins_hand(lib)
+    for seed in range(3):
+        check_info_forced_mode(seed, 3, 0.5, lib)
     check_info_score_closed_forms(lib)
     for seed in range(6):
         for C in (2, 3, 5):

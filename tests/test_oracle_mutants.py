@@ -35,6 +35,16 @@ MUTANTS = {
                              "  left->n = left->n + right->n;\n  left->ts = right->ts;"),
     "readout_before_write": ("    for (int c = 0; c < dk; c++) hd->open.z[c] = hd->open.z[c] + u[c];\n    hd->open.n = hd->open.n + 1;\n    int m = 0;",
                              "    int m = 0;"),
+    "margin_gap_over_second": ("else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward",
+                               "else if (bl > 0.0 && (second - bl) / second < min_gap) min_gap = (second - bl) / second;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward"),
+    "margin_ties_not_counted": ("        if (second == bl) ties += 1.0;\n        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward",
+                                "        if (second == bl) ties += 0.0;\n        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward"),
+    "margin_includes_first_token": ("    if (hd->t > 0) {\n      double mrg = fabs(rt - J->tau);",
+                                    "    {\n      double mrg = fabs(rt - J->tau);"),
+    "forced_index_ignored": ("  if (e > *ex) *ex = e;\n  return i;", "  if (e > *ex) *ex = e;\n  return best;"),
+    "forced_excess_over_second": ("double e = l == bl ? 0.0 : (bl > 0.0 ? (l - bl) / bl : INFINITY);",
+                                  "double e = l == bl ? 0.0 : (bl > 0.0 ? (l - bl) / l : INFINITY);"),
+    "forced_leftover_ignored": ("  if (fk != J->force_count[r]) ex = INFINITY;\n", ""),
     "fenwick_no_carry": ("while (hd->nsealed >= 2 && hd->sealed[hd->nsealed - 1].n == hd->sealed[hd->nsealed - 2].n) {",
                          "while (0) {"),
 }
@@ -55,6 +65,10 @@ INFO_MUTANTS = {
                                    "return a->info / (double)a->n + b->info / (double)b->n;"),
     "info_rightmost_tie": ("double l = density(&hd->sealed[i], &hd->sealed[i + 1]);\n          if (l < bl) {",
                            "double l = density(&hd->sealed[i], &hd->sealed[i + 1]);\n          if (l <= bl) {"),
+    "info_margin_ties_not_counted": ("        if (second == bl) ties += 1.0;\n        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_density",
+                                     "        if (second == bl) ties += 0.0;\n        else if (bl > 0.0 && (second - bl) / bl < min_gap) min_gap = (second - bl) / bl;\n        if (J->force_count)\n          best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_density"),
+    "info_forced_uses_ward": ("best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_density,",
+                              "best = forced_pair(J, r, &fk, hd->t, best, bl, C - 1, crit_ward,"),
     "info_sum_not_carried": ("  left->info = left->info + right->info;\n", ""),
 }
 
@@ -75,6 +89,10 @@ def build_mutant(name):
 
 def all_pins(lib):
     pins.check_hand_trace(lib)
+    pins.check_margins_hand(lib)
+    for seed in range(3):
+        for C in (3, 5):
+            pins.check_forced_mode(seed, C, 0.5, lib)
     for seed in range(6):
         for C in (2, 3, 5):
             for tau in (0.3, 0.5, 1.0):

@@ -238,3 +238,86 @@ def test_masked_readout_equals_full_readout(policy):
     assert not part["out"][0, ~sel].any()
     assert np.array_equal(part["boundary"], full["boundary"])
     assert part["merges"] == full["merges"]
+
+
+# ---- the margins diagnostic and the forced-merge mode -----------------------
+
+def _f(x):
+    return float("inf") if x == "inf" else float(x)
+
+
+def check_margins_hand(lib=None):
+    """min |r_t - tau|, the least relative gap between the best and the
+    second-best Ward loss over the merges and the count of exact ties, derived
+    by hand for the golden keys (tests/golden/hand_trace.json)."""
+    g = json.load(open(os.path.join(HERE, "golden", "hand_trace.json")))
+    for keys, tau, want in (("keys", "tau", "margins"), ("keys2", "tau", "margins2"),
+                            ("keys3", "tau3", "margins3"), ("keys4", "tau4", "margins4")):
+        k = np.array(g[keys], dtype=np.float64)
+        res, _ = run_one(np.ones_like(k), k, np.ones_like(k), g["C"], g[tau], lib=lib)
+        got = res["margins"][0]
+        exp = [_f(x) for x in g[want]]
+        assert abs(got[0] - exp[0]) < 1e-12, (keys, got)
+        assert (got[1] == exp[1]) if exp[1] == float("inf") else abs(got[1] - exp[1]) < 1e-12, (keys, got)
+        assert got[2] == exp[2], (keys, got)
+
+
+def test_margins_hand():
+    check_margins_hand()
+
+
+def check_forced_mode(seed, C, tau, lib=None):
+    """Merges taken from a given list instead of the argmin.
+
+    - The oracle's own merge list reproduces its run bit for bit, excess 0.
+    - Forcing the first merge onto another pair (the later merges are then the
+      argmin choices of that path) gives the outputs of brute force over the
+      ranges the list implies, and an excess equal to the relative excess of
+      the forced pair's scatter increase (Corollary 1) over the least one,
+      recomputed from the token ranges.
+    - A list whose token is not a capacity merge reports an infinite excess.
+    """
+    T, d = 48, 6
+    q, k, v = small_case(seed, T, d)
+    res, _ = run_one(q, k, v, C, tau, lib=lib)
+    merges = res["merges"][0]
+    b = res["boundary"][0]
+
+    def forced(lst, want_out=True):
+        orc = O.Oracle(1, d, d, C, lib=lib)
+        return orc.run(k[None], q[None] if want_out else None, v[None] if want_out else None,
+                       tau=tau, dtype="f64", nthreads=1, want_out=want_out,
+                       force_merges=[lst])
+
+    same = forced(merges)
+    assert np.array_equal(same["out"], res["out"]) and same["merges"] == res["merges"]
+    assert same["excess"][0] == 0.0
+    if not merges:
+        return
+    t0, i0 = merges[0]
+    assert forced([(t0 + 1, i0)] + merges[1:], want_out=False)["excess"][0] == np.inf
+    # an entry left over, or one missing, is a mismatch too
+    assert forced(merges + [(T + 5, 0)], want_out=False)["excess"][0] == np.inf
+    assert forced(merges[:-1], want_out=False)["excess"][0] == np.inf
+    if C < 3:
+        return
+    alt = (t0, (i0 + 1) % (C - 1))
+    lst = forced([alt], want_out=False)["merges"][0]  # alt, then the argmin path
+    assert lst[0] == alt
+    got = forced(lst)
+    assert got["merges"][0] == lst
+    ranges = bf.replay(b, lst, C)
+    o = bf.outputs(q, k, v, ranges)
+    assert np.allclose(got["out"][0], o, rtol=0, atol=1e-11 * np.abs(o).max())
+    # the sealed states just before the first merge: every state present at t0 - 1
+    sealed = bf.replay(b[:t0], [], C)[t0 - 1]
+    cost = bf.merge_costs_sse(k, sealed)
+    best = cost.min()
+    want = (cost[alt[1]] - best) / best if best > 0 else (0.0 if cost[alt[1]] == 0 else np.inf)
+    assert abs(got["excess"][0] - want) <= 1e-9 * max(1.0, want), (got["excess"][0], want)
+
+
+@pytest.mark.parametrize("seed,C,tau", [(s, C, tau) for s in range(8) for C in (2, 3, 5)
+                                        for tau in (0.3, 0.5)])
+def test_forced_mode(seed, C, tau):
+    check_forced_mode(seed, C, tau)
