@@ -6,12 +6,17 @@
 A step is one pass of the whole hot path over one batch of synthetic input:
   prefill workloads: dla_cache_init + dla_prefill of B x H x T tokens
   decode workload:   one dla_decode_step of N x H streams (cache pre-filled)
+The default run times prefill_t8192 (the line's value) and nests the metric's
+decode half (decode_n256, "decode") and the long-context and fixed-policy
+configurations ("configs") in the same line; --only times the named workload
+alone.
 Timing: CUDA events on the launching stream around exactly K steps after W
 warm-up steps, barrier + synchronize on both sides, max over ranks.  Inputs
 are larger than L2 (126 MB) so no flush is needed between steps.
 The kernel-level roofline uses events the library records around each of
 its launches in the timed region (dla_profile).
-Under torchrun every rank runs an independent replica (weak scaling).
+--gpus N runs N independent replicas (weak scaling), one process per GPU: under
+an outer torchrun, or relaunched under one when WORLD_SIZE is not set.
 """
 from __future__ import annotations
 
@@ -262,6 +267,27 @@ def to_torch(x, dtype, device):
     return torch.from_numpy(x).to(device)
 
 
+# ------------------------------------------------------------ roofline peaks ----
+
+def tensor_peak(peaks, peaks_kind, clocks):
+    """The bf16 tensor peak a kernel of this run is held to.
+
+    The measured burst figure (a GEMM timed alone at full clock) when the
+    timed region's SM clock stayed at its maximum with no power cap; the
+    sustained figure (seconds under the power cap) otherwise."""
+    burst = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    sust = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    if clocks is None:
+        return sust, f"bf16 dense, {peaks_kind} sustained (no clock record)"
+    mhz, mx = clocks.get("sm_mhz", 0.0), clocks.get("sm_max_mhz", 0.0)
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    if mx and mhz >= 0.98 * mx and not capped:
+        return burst, (f"bf16 dense, {peaks_kind} burst: the timed region ran at a median "
+                       f"{mhz:.0f} MHz (max {mx:.0f}) with no power cap")
+    return sust, (f"bf16 dense, {peaks_kind} sustained: the timed region ran at a median "
+                  f"{mhz:.0f} MHz (max {mx:.0f}){', power cap active' if capped else ''}")
+
+
 # ------------------------------------------------------------ prefill arm ----
 
 def prefill_flops(trace_live_sum, heads_tokens, d):
@@ -301,7 +327,7 @@ def _time_steps(step, steps, warmup, stream, world, dev):
     return reduce_max(e0.elapsed_time(e1), world, dev) / steps
 
 
-def bench_prefill(args, wl, rank, world, local_rank):
+def bench_prefill(args, wl, rank, world, local_rank, e2e=True):
     import torch
     from dynamic_state_memory_b200 import dla
     dev = torch.device(f"cuda:{local_rank}")
@@ -332,6 +358,7 @@ def bench_prefill(args, wl, rank, world, local_rank):
     bnd = tr.boundary.cpu().numpy()
     mt = tr.merge_t.cpu().numpy()
     mc = tr.merge_count.cpu().numpy()
+    del tr
     live_sum = 0
     m0_rows = 0
     for h in range(B * H):
@@ -389,10 +416,118 @@ def bench_prefill(args, wl, rank, world, local_rank):
     launches = prof.p.count
     kt = prof.times_ms()
 
-    # End to end through the public API with host buffers: every step copies
-    # its q, k, v in from pinned host memory and its o back out. Two device
-    # buffer sets and two copy streams let step i+1's upload and step i's
-    # download run while step i computes, as a stream of requests would.
+    in_bytes = sum(x.nbytes for x in (q_h, k_h, v_h))
+    e2e_ms = None
+    if e2e:
+        e2e_ms, out_bytes = _prefill_e2e(args, q_h, k_h, v_h, q, k, v, o, dt, step, stream, st,
+                                         world, dev)
+
+    if rank != 0:
+        return None
+    ms_step = ms_max / args.steps
+    tokens = B * T * world
+    value = tokens / (ms_step * 1e-3) / 1e6
+    # CUDA-event time of each kernel on its own stream. Kernels on concurrent
+    # streams overlap, so a low-priority kernel's event time includes the time
+    # it waits for SMs: these are not the serialised shares of an ncu launch
+    # list. The roofline is the readout's (the contraction), the largest
+    # kernel of that serialised list on every prefill workload here.
+    # Under the information policy the sequential fp64 score dominates the
+    # step and carries the roofline instead.
+    tot = {kname: sum(v_) for kname, v_ in kt.items()}
+    if info:
+        dom = "info_score"
+    else:
+        dom = "readout" if "readout" in kt else max(tot, key=tot.get)
+    per_launch_ms = statistics.mean(kt[dom])
+    n_launch = len(kt[dom])
+    steps_recorded = args.steps
+    step_flops = readout_flops + build_flops
+    step_frac = None
+    if dom == "readout":
+        # the tensor-core readout's timed kernel is its atom loop (the prologue,
+        # "readout_pre", runs beside the materializer); the SIMT readout is one
+        # kernel doing all of the readout's work
+        work = readout_flops if args.path == "simt" else loop_flops
+        flops_per_launch = work / (n_launch / steps_recorded)
+        if args.path == "simt":
+            bound, unit = "alu", "TFLOP/s"
+            peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock (derived)"
+        else:
+            bound, unit = "tensor", "TFLOP/s"
+            peak, peak_note = tensor_peak(peaks, peaks_kind, clocks)
+        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
+        # the whole step: every algorithmic FLOP of the readout and the state
+        # build over the step time, against the same peak
+        step_frac = round(step_flops / (ms_step * 1e-3) / 1e12 / peak, 4)
+    elif dom == "info_score":
+        # per token: x_t = v_t^T S u_t (2 d^2 FLOP) and the state update
+        # S += v_t u_t^T (2 d^2 FLOP), fp64; one CTA (one SM) per head
+        flops_per_launch = 4.0 * d * d * B * H * T / (n_launch / steps_recorded)
+        bound, unit = "alu", "TFLOP/s"
+        peak = SMS * FP64_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        peak_note = ("fp64 FMA: 148 SMs x 64 lanes x 2 FLOP x max SM clock (derived); the "
+                     "kernel runs one SM per head, %d of 148" % min(B * H, SMS))
+        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
+    else:
+        bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
+        achieved = float("nan")
+    traffic = None if args.B else ncu_traffic(dom, "simt" if args.path == "simt" else "tc",
+                                              args.workload)
+    roof = {"kernel": dom, "bound": bound,
+            "achieved": round(achieved, 3), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": peak_note, "launch_ms": round(per_launch_ms, 4),
+            "launches": n_launch,
+            "step_flops": step_flops, "step_frac": step_frac,
+            "step_frac_note": "flops_per_step / ms_per_step / peak (readout + state build)"
+                              if step_frac is not None else None,
+            "event_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()},
+            "event_share_note": "CUDA-event time per kernel on its own stream; concurrent "
+                                "streams overlap, so these are not serialised shares"}
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(
+        wl, q_h, k_h, v_h, policy=policy_of(args.workload), target_s=args.cpu_seconds)
+    extra = {}
+    if info and "readout" in kt:
+        # the readout is the dynamic policy's; its atom loop's rate beside
+        rl_ms = statistics.mean(kt["readout"])
+        ra = loop_flops / (len(kt["readout"]) / steps_recorded) / (rl_ms * 1e-3) / 1e12
+        rp, rnote = tensor_peak(peaks, peaks_kind, clocks)
+        extra["readout_atom_loop"] = {"achieved": round(ra, 3), "peak": rp, "unit": "TFLOP/s",
+                                      "frac": round(ra / rp, 4), "launch_ms": round(rl_ms, 4),
+                                      "peak_source": rnote}
+    if fixed:
+        extra = {"dla_same_inputs": {
+            "C": C, "value": round(tokens / (dla_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
+            "ms_per_step": round(dla_ms, 4), "mean_live_states": round(dla_live / (B * H * T), 2)}}
+    return {
+        **({"policy": policy_of(args.workload)} if fixed or info else {}), **extra,
+        "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if args.path == "simt" else "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "H": H, "T": T, "d": d, "C": C,
+                   "tau": wl["tau"], "input_dtype": dt, "path": args.path,
+                   "l2": "inputs larger than L2 (q+k+v %d MiB), no flush" % (in_bytes >> 20),
+                   "flops_per_step": step_flops,
+                   "mean_live_states": round(live_sum / (B * H * T), 2)},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": None if e2e_ms is None else {
+            "value": round(tokens / (e2e_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
+            "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+
+
+def _prefill_e2e(args, q_h, k_h, v_h, q, k, v, o, dt, step, stream, st, world, dev):
+    """End to end through the public API with host buffers: every step copies
+    its q, k, v in from pinned host memory and its o back out.  Two device
+    buffer sets and two copy streams let step i+1's upload and step i's
+    download run while step i computes, as a stream of requests would.
+    Returns (ms per step, max over ranks; output bytes per step)."""
+    import torch
+    from dynamic_state_memory_b200 import dla
     pin = [torch.from_numpy(x.view(np.int16) if dt == "bf16" else x).pin_memory()
            for x in (q_h, k_h, v_h)]
     o_host = torch.empty(o.shape, dtype=torch.int16 if dt == "bf16" else torch.float32).pin_memory()
@@ -436,106 +571,25 @@ def bench_prefill(args, wl, rank, world, local_rank):
     # the pipelined output is the device-timed step's output, bit for bit
     if not torch.equal(o_host, o.view(o_host.dtype).cpu()):
         raise RuntimeError("end-to-end output differs from the device-timed output")
-    del sets
-    in_bytes = sum(x.nbytes for x in (q_h, k_h, v_h))
-    out_bytes = o_host.numel() * o_host.element_size()
+    return e2e_ms, o_host.numel() * o_host.element_size()
 
-    if rank != 0:
-        return None
-    ms_step = ms_max / args.steps
-    tokens = B * T * world
-    value = tokens / (ms_step * 1e-3) / 1e6
-    # CUDA-event time of each kernel on its own stream. Kernels on concurrent
-    # streams overlap, so a low-priority kernel's event time includes the time
-    # it waits for SMs: these are not the serialised shares of an ncu launch
-    # list. The roofline is the readout's (the contraction), the largest
-    # kernel of that serialised list on every prefill workload here.
-    # Under the information policy the sequential fp64 score dominates the
-    # step and carries the roofline instead.
-    tot = {kname: sum(v_) for kname, v_ in kt.items()}
-    if info:
-        dom = "info_score"
-    else:
-        dom = "readout" if "readout" in kt else max(tot, key=tot.get)
-    per_launch_ms = statistics.mean(kt[dom])
-    n_launch = len(kt[dom])
-    steps_recorded = args.steps
-    if dom == "readout":
-        # the tensor-core readout's timed kernel is its atom loop (the prologue,
-        # "readout_pre", runs beside the materializer); the SIMT readout is one
-        # kernel doing all of the readout's work
-        work = readout_flops if args.path == "simt" else loop_flops
-        flops_per_launch = work / (n_launch / steps_recorded)
-        if args.path == "simt":
-            bound, unit = "alu", "TFLOP/s"
-            peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-            peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock (derived)"
-        else:
-            bound, unit = "tensor", "TFLOP/s"
-            peak = peaks.get("bf16_tflops_sustained", 1371.4)
-            peak_note = f"bf16 dense, {peaks_kind} sustained"
-        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
-    elif dom == "info_score":
-        # per token: x_t = v_t^T S u_t (2 d^2 FLOP) and the state update
-        # S += v_t u_t^T (2 d^2 FLOP), fp64; one CTA (one SM) per head
-        flops_per_launch = 4.0 * d * d * B * H * T / (n_launch / steps_recorded)
-        bound, unit = "alu", "TFLOP/s"
-        peak = SMS * FP64_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        peak_note = ("fp64 FMA: 148 SMs x 64 lanes x 2 FLOP x max SM clock (derived); the "
-                     "kernel runs one SM per head, %d of 148" % min(B * H, SMS))
-        achieved = flops_per_launch / (per_launch_ms * 1e-3) / 1e12
-    else:
-        bound, unit, peak, peak_note = "hbm", "GB/s", peaks.get("hbm_gbs", 6540.8), peaks_kind
-        achieved = float("nan")
-    traffic = None if args.B else ncu_traffic(dom, "simt" if args.path == "simt" else "tc",
-                                              args.workload)
-    roof = {"kernel": dom, "bound": bound,
-            "achieved": round(achieved, 3), "peak": peak,
-            "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-            "peak_source": peak_note, "launch_ms": round(per_launch_ms, 4),
-            "launches": n_launch,
-            "event_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()},
-            "event_share_note": "CUDA-event time per kernel on its own stream; concurrent "
-                                "streams overlap, so these are not serialised shares"}
-    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_prefill(
-        wl, q_h, k_h, v_h, policy=policy_of(args.workload))
-    e2e_val = tokens / (e2e_ms * 1e-3) / 1e6
-    extra = {}
-    if info and "readout" in kt:
-        # the readout is the dynamic policy's; its atom loop's rate beside
-        rl_ms = statistics.mean(kt["readout"])
-        ra = loop_flops / (len(kt["readout"]) / steps_recorded) / (rl_ms * 1e-3) / 1e12
-        rp = peaks.get("bf16_tflops_sustained", 1371.4)
-        extra["readout_atom_loop"] = {"achieved": round(ra, 3), "peak": rp, "unit": "TFLOP/s",
-                                      "frac": round(ra / rp, 4), "launch_ms": round(rl_ms, 4)}
-    if fixed:
-        extra = {"dla_same_inputs": {
-            "C": C, "value": round(tokens / (dla_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
-            "ms_per_step": round(dla_ms, 4), "mean_live_states": round(dla_live / (B * H * T), 2)}}
-    return {
-        **({"policy": policy_of(args.workload)} if fixed or info else {}), **extra,
-        "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32" if args.path == "simt" else "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "B": B, "H": H, "T": T, "d": d, "C": C,
-                   "tau": wl["tau"], "input_dtype": dt, "path": args.path,
-                   "l2": "inputs larger than L2 (q+k+v %d MiB), no flush" % (in_bytes >> 20),
-                   "flops_per_step": readout_flops + build_flops,
-                   "mean_live_states": round(live_sum / (B * H * T), 2)},
-        "roofline": roof, "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_val, 4), "unit": "Mtok/s", "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": out_bytes},
-        "gpu_launches": launches, "clocks": clocks,
-    }
+
+def oracle_heads(wl, cores):
+    """The streams the oracle runs as its bounded sample of a prefill
+    workload: the first min(B*H, cores) streams, full length."""
+    return min(wl["B"] * wl["H"], cores)
 
 
 def cpu_baseline_prefill(wl, q, k, v, target_s=15.0, policy="dla"):
-    """The oracle as it stands on a bounded sample of the same workload."""
+    """The oracle as it stands on a bounded sample of the same workload: the
+    first streams (one per host core), full per-token work, from the first
+    256 tokens up until one run takes a quarter of the target or covers the
+    whole sequence (each longer prefix sized from the last run's time, at
+    most x4)."""
     from oracle import oracle as O
     cores = O.cores()
     B, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
-    heads = min(B * H, cores)
+    heads = oracle_heads(wl, cores)
     Ts = min(T, 256)
     t_used = 0.0
     while True:
@@ -548,7 +602,10 @@ def cpu_baseline_prefill(wl, q, k, v, target_s=15.0, policy="dla"):
         t_used = time.perf_counter() - t0
         if t_used > target_s / 4 or Ts >= T:
             break
-        Ts = min(T, Ts * 4)
+        # a longer prefix costs more than in proportion (more live states),
+        # so aim at half the remaining factor
+        grow = min(4.0, 0.5 * (target_s / 4) / max(t_used, 1e-3) + 1.0)
+        Ts = min(T, max(Ts + 256, int(Ts * grow) // 256 * 256))
     head_tokens_s = heads * Ts / t_used
     return {"value": round(head_tokens_s / H / 1e6, 6), "unit": "Mtok/s", "cores": cores,
             "kind": "oracle",
@@ -674,6 +731,7 @@ def bench_decode(args, wl, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(f0.elapsed_time(f1) / e2e_steps, world, dev)
     dla.check_device_status(dec.status, "dla_decode_step")
+    del cache, dec, sq, sk, sv, dsets
     if rank != 0:
         return None
     ms_step = ms / args.steps
@@ -684,12 +742,15 @@ def bench_decode(args, wl, rank, world, local_rank):
     state_bytes = live * d * d * 4
     achieved = state_bytes / (stream_ms * 1e-3) / 1e9
     peak = peaks.get("hbm_gbs", 6540.8)
+    step_bytes_frac = state_bytes / (ms_step * 1e-3) / 1e9 / peak
     roof = {"kernel": "decode_stream", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": None if args.B else ncu_traffic("decode_stream", "-", args.workload),
+            "traffic": None if args.B else ncu_traffic("decode_stream", "-", "decode_n256"),
             "peak_source": f"{peaks_kind} copy bandwidth",
             "algorithmic_bytes_per_launch": state_bytes, "launch_ms": round(stream_ms, 4),
             "launches": len(kt["decode_stream"]),
+            "step_frac": round(step_bytes_frac, 4),
+            "step_frac_note": "state bytes per step / ms_per_step / peak (decision kernel included)",
             "kernel_share": {kk: round(vv / sum(tot.values()), 4) for kk, vv in tot.items()}}
     cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_decode(wl, pre_h, stp_h)
     return {
@@ -697,10 +758,10 @@ def bench_decode(args, wl, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "N": N, "H": H, "prefill_T": T, "d": d, "C": C,
+        "config": {"workload": "decode_n256", "N": N, "H": H, "prefill_T": T, "d": d, "C": C,
                    "tau": tau, "input_dtype": "bf16", "state_dtype": "f32",
                    "mean_live_states": round(live / (N * H), 2),
-                   "l2": "state cache %d GiB >> L2, no flush" % (cache.base.numel() >> 30)},
+                   "l2": "state cache %d GiB >> L2, no flush" % ((N * H * C * d * d * 4) >> 30)},
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": round(world * 1000.0 / e2e_ms, 3), "unit": "steps/s",
                 "h2d_bytes_per_step": 3 * N * H * d * 2, "d2h_bytes_per_step": N * H * d * 2},
@@ -708,65 +769,109 @@ def bench_decode(args, wl, rank, world, local_rank):
     }
 
 
-def cpu_baseline_decode(wl, pre, stp, prefill_tokens=4096, steps=8):
-    """Oracle: 16 streams pre-filled on the workload's tokens, then timed steps."""
+def oracle_decode(wl, pre, stp, steps, cores, streams=16, prefill_tokens=4096):
+    """Oracle decode on a bounded sample: `streams` streams pre-filled with
+    their workload tokens (untimed; states updated at every token, no
+    readout), then `steps` timed single-token steps with full per-token work.
+    Returns (seconds per step for the sample, sample description)."""
     from oracle import oracle as O
-    cores = O.cores()
     N, H, d = wl["B"], wl["H"], wl["d"]
-    U = min(16, N * H)
+    U = min(streams, N * H)
     Tp = min(prefill_tokens, wl["T"])
     k = pre[1].reshape(N * H, -1, d)[:U, :Tp]
     q = pre[0].reshape(N * H, -1, d)[:U, :Tp]
     v = pre[2].reshape(N * H, -1, d)[:U, :Tp]
     orc = O.Oracle(U, d, d, wl["C"])
-    orc.run(k, q, v, tau=wl["tau"], dtype="bf16", nthreads=cores)
+    orc.run(k, q, v, tau=wl["tau"], dtype="bf16", nthreads=cores,
+            out_mask=np.zeros(Tp, dtype=np.uint8))
     sk = stp[1].reshape(stp[1].shape[0], N * H, d)
     sq = stp[0].reshape(stp[0].shape[0], N * H, d)
     sv = stp[2].reshape(stp[2].shape[0], N * H, d)
-    t0 = time.perf_counter()
     n = min(steps, sk.shape[0])
+    t0 = time.perf_counter()
     for i in range(n):
         orc.run(np.ascontiguousarray(sk[i, :U, None]), np.ascontiguousarray(sq[i, :U, None]),
                 np.ascontiguousarray(sv[i, :U, None]), tau=wl["tau"], dtype="bf16",
                 nthreads=cores)
     dt = (time.perf_counter() - t0) / n
+    return dt, U, (f"{U} streams pre-filled with {Tp} tokens (untimed), {n} timed steps; "
+                   f"steps/s extrapolated to {N * H} streams")
+
+
+def cpu_baseline_decode(wl, pre, stp, steps=8):
+    """Oracle decode steps/s, extrapolated from its sample to every stream."""
+    from oracle import oracle as O
+    cores = O.cores()
+    dt, U, sample = oracle_decode(wl, pre, stp, steps, cores)
+    N, H = wl["B"], wl["H"]
     return {"value": round(1.0 / (dt * (N * H) / U), 6), "unit": "steps/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"{U} streams pre-filled with {Tp} tokens (untimed), {n} timed steps; "
-                      f"steps/s extrapolated to {N * H} streams"}
+            "kind": "oracle", "sample": sample}
 
 
 # ------------------------------------------------------------ reference arm ----
 
 def bench_reference(args, wl):
+    """The oracle as it stands, on the same bounded sample as our arm's
+    cpu_baseline: the first min(B*H, cores) streams at full length (or the
+    first --ref-tokens tokens), full per-token work, every step."""
     from oracle import oracle as O
+    from dynamic_state_memory_b200 import synth
     cores = O.cores()
-    q, k, v = make_inputs(dict(wl, B=1, H=min(wl["H"], cores)))
-    B, H, T, d = 1, q.shape[1], wl["T"], wl["d"]
-    Ts = min(T, args.ref_tokens)
+    B, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
+    heads = oracle_heads(wl, cores)
+    Ts = T if args.ref_tokens <= 0 else min(T, args.ref_tokens)
+    pol = policy_of(args.workload)
+    q, k, v = (np.empty((heads, Ts, d), dtype=np.uint16 if wl["dtype"] == "bf16" else np.float32)
+               for _ in range(3))
+    cast = synth.to_bf16_bits if wl["dtype"] == "bf16" else (lambda x: np.ascontiguousarray(x, np.float32))
+    for i in range(heads):
+        stv = synth.HeadStream(wl["seed"], i // H, i % H, **wl)
+        q[i], k[i], v[i] = cast(stv.q[:Ts]), cast(stv.k[:Ts]), cast(stv.v[:Ts])
     times = []
     for i in range(args.warmup + args.steps):
-        orc = O.Oracle(H, d, d, wl["C"], policy_of(args.workload))
+        orc = O.Oracle(heads, d, d, wl["C"], pol)
         t0 = time.perf_counter()
-        orc.run(k[0, :, :Ts], q[0, :, :Ts], v[0, :, :Ts], tau=wl["tau"], dtype=wl["dtype"],
-                nthreads=cores)
+        orc.run(k, q, v, tau=wl["tau"], dtype=wl["dtype"], nthreads=cores)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
     mean = sum(times) / len(times)
-    val = H * Ts / mean / wl["H"] / 1e6
-    return {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "Mtok/s",
+    val = heads * Ts / mean / H / 1e6
+    sample = (f"{pol} policy, {heads} heads x first {Ts} tokens of the workload per step, full "
+              f"per-token work (the sample of the GPU arm's cpu_baseline); Mtok/s = "
+              f"head-tokens/s / H")
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "Mtok/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(mean * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "B": wl["B"], "H": wl["H"], "T": wl["T"],
-                       "d": d, "C": wl["C"], "tau": wl["tau"]},
+            "config": {"workload": args.workload, "B": B, "H": H, "T": T, "d": d,
+                       "C": wl["C"], "tau": wl["tau"]},
             "cpu_baseline": {"value": round(val, 6), "unit": "Mtok/s", "cores": cores,
-                             "kind": "oracle",
-                             "sample": f"{H} heads x first {Ts} tokens per step; Mtok/s = "
-                                       "head-tokens/s / H"},
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": round(val, 6), "unit": "Mtok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    if args.workload == "prefill_t8192" and not args.only:
+        # the decode half of the metric, on the decode workload's sample
+        dwl = dict(synth.WORKLOADS["decode_n256"])
+        U = 16
+        pre = [np.empty((1, U, dwl["T"], d), dtype=np.uint16) for _ in range(3)]
+        nst = min(args.steps, 8)
+        stp = [np.empty((nst, 1, U, d), dtype=np.uint16) for _ in range(3)]
+        for i in range(U):
+            stv = synth.HeadStream(dwl["seed"], i // dwl["H"], i % dwl["H"], **dwl)
+            sq_, sk_, sv_ = stv.decode_steps(nst, dwl["switch_p"])
+            for j, (p_, s_) in enumerate(((stv.q, sq_), (stv.k, sk_), (stv.v, sv_))):
+                pre[j][0, i] = synth.to_bf16_bits(p_)
+                stp[j][:, 0, i] = synth.to_bf16_bits(s_)
+        dt, Us, dsample = oracle_decode(dict(dwl, B=1, H=U), pre, stp, nst, cores, streams=U)
+        dval = 1.0 / (dt * (dwl["B"] * dwl["H"]) / Us)
+        line["decode"] = {"value": round(dval, 6), "unit": "steps/s",
+                          "ms_per_step": round(1e3 / dval, 3),
+                          "config": {"workload": "decode_n256"},
+                          "cpu_baseline": {"value": round(dval, 6), "unit": "steps/s",
+                                           "cores": cores, "kind": "oracle",
+                                           "sample": dsample}}
+    return line
 
 
 # ------------------------------------------------------------------ plumbing ----
@@ -787,6 +892,45 @@ def reduce_max(x, world, dev):
     return float(t.item())
 
 
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(n):
+    """Run this command as n ranks under torchrun (one process per GPU) and
+    return its exit status: `--gpus N` without an outer launcher."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={_free_port()}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd, timeout=3 * 3600).returncode
+
+
+def sub_args(args, workload, steps=None, warmup=None):
+    """A copy of the command's arguments for another workload."""
+    from dynamic_state_memory_b200 import synth
+    a = argparse.Namespace(**vars(args))
+    a.workload = workload
+    a.steps = args.steps if steps is None else steps
+    a.warmup = args.warmup if warmup is None else warmup
+    wl = synth.WORKLOADS[workload]
+    a.path = "tc" if (wl["dtype"] == "bf16" and wl["d"] == 128) else "simt"
+    a.B = 0
+    a.window = 0
+    return a
+
+
+def guarded(fn, *a, **kw):
+    """A secondary measurement: its failure is reported in the line, it does
+    not lose the headline."""
+    try:
+        return fn(*a, **kw)
+    except Exception as exc:  # noqa: BLE001
+        return {"error": f"{type(exc).__name__}: {exc}"[:300]}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -796,11 +940,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--window", type=int, default=0)
     ap.add_argument("--path", default="auto", help="reported path; auto = tc for bf16 d=128")
-    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="reference arm: tokens per stream (0 = the whole sequence)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle's cpu_baseline sample")
+    ap.add_argument("--only", action="store_true",
+                    help="the named workload alone (no decode or other configurations nested)")
     ap.add_argument("--B", type=int, default=0, help="override the batch (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
     from dynamic_state_memory_b200 import synth
     wl = dict(synth.WORKLOADS[args.workload])
     if args.B:
@@ -808,6 +959,9 @@ def main():
     if args.path == "auto":
         args.path = "tc" if (wl["dtype"] == "bf16" and wl["d"] == 128) else "simt"
     rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        sys.exit(2)
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(bench_reference(args, wl)), flush=True)
@@ -822,6 +976,24 @@ def main():
         res = bench_decode(args, wl, rank, world, local_rank)
     else:
         res = bench_prefill(args, wl, rank, world, local_rank)
+        if args.workload == "prefill_t8192" and not args.only:
+            # the metric's other half and the other configurations, nested in
+            # the same line (every rank runs them: they hold barriers)
+            import torch
+            torch.cuda.empty_cache()
+            dec = guarded(bench_decode, sub_args(args, "decode_n256"),
+                          dict(synth.WORKLOADS["decode_n256"]), rank, world, local_rank)
+            torch.cuda.empty_cache()
+            others = {}
+            for name in ("prefill_t131072", "fixed_t32768"):
+                a = sub_args(args, name, steps=min(args.steps, 10), warmup=3)
+                a.cpu_seconds = min(args.cpu_seconds, 8.0)
+                others[name] = guarded(bench_prefill, a, dict(synth.WORKLOADS[name]), rank, world,
+                                       local_rank, e2e=False)
+                torch.cuda.empty_cache()
+            if rank == 0:
+                res["decode"] = dec
+                res["configs"] = others
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -535,6 +535,10 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   // ---- load the head's summaries ------------------------------------------
   int m = ca.cache.m[u];
   const int64_t t0 = ca.cache.t[u];
+  // the cosine / Ward policy does not continue a cache of the information
+  // policy (its pair entries are densities, its prev_r an information score)
+  if (!info && lane == 0 && c_loss[C - 1] == CACHE_INFO_MARK)
+    set_status(dev_status, DLA_ERR_UNSUPPORTED);
   if (lane < 4) sm->used[lane] = 0u;
   __syncwarp();
   for (int p = lane; p < C; p += 32) {
@@ -838,7 +842,9 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
     c_order[p] = sm->order[p];
     c_n[p] = sm->n[p];
     c_ts[p] = sm->ts[p];
-    c_loss[p] = sm->loss[p];
+    // pair_loss[C - 1] belongs to no pair: under the information policy it
+    // marks the cache as holding that policy's states (CACHE_INFO_MARK)
+    c_loss[p] = (info && p == C - 1) ? CACHE_INFO_MARK : sm->loss[p];
     if (info) c_info[p] = sm->info[p];
   }
   for (int i = lane; i < C * D; i += 32) c_z[i] = zs[i];

@@ -14,7 +14,9 @@
 //   loads, applies the merge / open-state update in registers, writes back the
 //   changed slots and accumulates o = sum_i lambda_i S_i phi(q).  Each CTA owns
 //   32 rows of d_v of one stream, so o needs no cross-CTA reduction.
-#include <atomic>
+#include <cuda.h>
+
+#include <mutex>
 
 #include "dla_internal.cuh"
 
@@ -68,6 +70,8 @@ __global__ void __launch_bounds__(128) k_decode_decide(dla_cache cc, float tau, 
   const int64_t t = cc.t[u];
   int m = cc.m[u];
   const size_t row = (size_t)u * D;
+  // a cache of the information policy is not continued here
+  if (lane == 0 && loss[C - 1] == CACHE_INFO_MARK) set_status(dev_status, DLA_ERR_UNSUPPORTED);
 
   // score in index order on lane 0 (same operation sequence as the oracle)
   double r = 0.0;
@@ -381,24 +385,66 @@ cudaError_t launch_decode_stream(const dla_cache &cc, int32_t dt, const void *q,
 // For callers that cannot allocate device memory themselves (see
 // dla_decode_step_static in dla.h).  The scratch is one file-scope device
 // array shared by every call on a device; the host resolves its device
-// address once per device with cudaGetSymbolAddress (the array's name is not
-// a device pointer in host code).
+// address with cudaGetSymbolAddress (the array's name is not a device pointer
+// in host code).  The address belongs to the CUDA context the module was
+// loaded in, so it is kept per device together with that context's id: after
+// a cudaDeviceReset (or any other teardown) the next call on the device runs
+// in a new context and looks the address up again.
 namespace {
 constexpr size_t STATIC_DECODE_BYTES = (size_t)8 << 20;
 __device__ __align__(256) unsigned char g_decode_scratch[STATIC_DECODE_BYTES];
 constexpr int MAX_DEVICES = 64;
-std::atomic<void *> g_scratch_addr[MAX_DEVICES];
+std::mutex g_scratch_mu;
+unsigned long long g_scratch_ctx[MAX_DEVICES];  // id of the context of g_scratch_addr
+void *g_scratch_addr[MAX_DEVICES];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current context (false when none is current or
+// the driver has no context ids).
+bool current_ctx_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked = true;
+  }
+  CUcontext ctx = nullptr;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 cudaError_t static_scratch(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
-  void *p = g_scratch_addr[dev].load();
-  if (!p) {
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev].store(p);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  unsigned long long id = 0;
+  if (current_ctx_id(&id) && g_scratch_addr[dev] && g_scratch_ctx[dev] == id) {
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+  }
+  // first call on this device, or its context changed: resolve the address
+  // (this also makes the device's primary context current)
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess) return e;
+  if (current_ctx_id(&id)) {
+    g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = id;
+  } else {
+    g_scratch_addr[dev] = nullptr;  // no context id: resolve on every call
   }
   *out = p;
   return cudaSuccess;

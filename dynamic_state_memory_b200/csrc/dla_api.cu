@@ -230,7 +230,9 @@ const char *dla_status_string(dla_status s) {
   switch (s) {
     case DLA_OK: return "ok";
     case DLA_ERR_INVALID_ARG: return "invalid argument";
-    case DLA_ERR_UNSUPPORTED: return "unsupported shape (need d_k == d_v in {32, 64, 128}, 2 <= C <= 128)";
+    case DLA_ERR_UNSUPPORTED:
+      return "unsupported shape (need d_k == d_v in {32, 64, 128}, 2 <= C <= 128) or a cache "
+             "this policy cannot continue";
     case DLA_ERR_CUDA: return "CUDA launch failed";
     case DLA_ERR_TRACE_OVERFLOW: return "more merges than the trace capacity";
     case DLA_ERR_WORKSPACE: return "workspace smaller than dla_workspace_bytes()";

@@ -44,6 +44,12 @@ constexpr int PIECE_MIN = 16;
 // flags and runs concurrently with the capacity-merge engine.
 constexpr int PIECES_PER_TILE = 128 / PIECE_MIN;
 
+// pair_loss[C - 1] of a stream belongs to no pair (C states have C - 1
+// adjacent pairs).  The information policy writes this value there: its pair
+// entries are densities, not Ward losses, so the cosine / Ward entry points
+// refuse such a cache (DLA_ERR_UNSUPPORTED) until dla_cache_init resets it.
+constexpr double CACHE_INFO_MARK = -1.0;
+
 // Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
 // pair at that time-order position, <= -2 merge the two newest sealed states
 // (-code - 1) times (binary-counter carries of the fixed policy).

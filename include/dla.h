@@ -46,7 +46,8 @@ extern "C" {
 typedef enum {
   DLA_OK = 0,
   DLA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, mismatched shapes */
-  DLA_ERR_UNSUPPORTED = 2,     /* d_k != d_v, d not in {32, 64, 128}, C < 2 */
+  DLA_ERR_UNSUPPORTED = 2,     /* d_k != d_v, d not in {32, 64, 128}, C < 2; on the device:
+                                  a cache the policy cannot continue */
   DLA_ERR_CUDA = 3,            /* a CUDA launch failed (see cudaGetLastError) */
   DLA_ERR_TRACE_OVERFLOW = 4,  /* device: more merges than dla_trace.cap */
   DLA_ERR_WORKSPACE = 5,       /* ws_bytes smaller than the size query */
@@ -106,7 +107,9 @@ typedef struct {
  *   S         float  [u][C][d_v][d_k]  slot states sum v phi(k)^T (fp32)
  *   z         double [u][C][d_k]       slot sums of phi(k) (fp64, decisions)
  *   n, ts     int64  [u][C]            token count and first token of a slot
- *   pair_loss double [u][C]            Ward loss of sealed pair (p, p+1)
+ *   pair_loss double [u][C]            Ward loss of sealed pair (p, p+1); entry
+ *                                      C-1 (no pair) is -1 after the
+ *                                      information policy, 0 otherwise
  *   order     int32  [u][C]            time-order position -> slot
  *   m         int32  [u]               live states (open one included)
  *   prev_k    float  [u][d_k]          last key, for the next score
@@ -184,7 +187,10 @@ dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype,
  * at most that size (about 30,000 streams at C = 64) and returns
  * DLA_ERR_WORKSPACE for larger ones.  It allocates nothing.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.  All
+ * that device current; make that first call before any stream capture.  The
+ * address is kept with the id of the context it was found in: after a
+ * cudaDeviceReset or any other context teardown, the next call on the device
+ * looks it up again, so that call too must come before any capture.  All
  * calls share the one array and it keeps the last call's contents (every call
  * rewrites what it reads, so nothing needs clearing); calls that overlap on
  * the GPU, from any stream or thread, race on it, so serialise them.  The
@@ -220,8 +226,11 @@ dla_status dla_fixed_policy_prefill(const dla_config *cfg, const void *q, const 
  * from an empty cache: a stream whose cache has t > 0 sets
  * DLA_ERR_UNSUPPORTED in *dev_status and its outputs are unspecified.  After
  * the call the cache holds the policy's states, counts and time order, and
- * pair_loss the pair densities; dla_decode_step does not continue it (it
- * applies the cosine score and Ward merges). */
+ * pair_loss the pair densities, with its unused last entry set to -1 to mark
+ * the cache as this policy's: dla_prefill, dla_decode_step and
+ * dla_decode_step_static (cosine score, Ward merges) set DLA_ERR_UNSUPPORTED
+ * in *dev_status on such a stream, and its results are unspecified, until
+ * dla_cache_init resets the cache. */
 dla_status dla_info_policy_prefill(const dla_config *cfg, const void *q, const void *k,
                                    const void *v, void *o, const dla_cache *cache,
                                    const dla_trace *trace, void *ws, size_t ws_bytes,

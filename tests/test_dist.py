@@ -77,7 +77,7 @@ def test_reference_arm_prints_on_rank0_only(rank):
                MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--workload", "tiny_f32", "--steps", "1", "--warmup", "3",
-                        "--ref-tokens", "32"],
+                        "--ref-tokens", "32", "--gpus", "2"],
                        env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
@@ -88,3 +88,43 @@ def test_reference_arm_prints_on_rank0_only(rank):
         assert line["e2e"]["h2d_bytes_per_step"] == 0
     else:
         assert lines == []
+
+
+def test_gpus_flag_must_match_world_size():
+    """Under an outer launcher, --gpus N must equal WORLD_SIZE (no silent
+    single replica)."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0",
+               MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_f32", "--steps", "1", "--gpus", "1"],
+                       env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 2 and "WORLD_SIZE=2" in r.stderr
+
+
+def test_gpus_flag_relaunches_under_torchrun():
+    """--gpus 2 without WORLD_SIZE relaunches itself as two ranks (torchrun
+    on 127.0.0.1); rank 0 alone prints the line."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_f32", "--steps", "1", "--warmup", "3",
+                        "--ref-tokens", "32", "--gpus", "2"],
+                       env=env, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference"
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """Burst peak when the timed region stayed at the max SM clock with no
+    power cap, sustained otherwise."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1656.2, "bf16_tflops_sustained": 1371.4}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.tensor_peak(peaks, "measured", at_max)[0] == 1656.2
+    capped = dict(at_max, reasons=["sw_power_cap"])
+    assert bench.tensor_peak(peaks, "measured", capped)[0] == 1371.4
+    slow = dict(at_max, sm_mhz=1400.0)
+    assert bench.tensor_peak(peaks, "measured", slow)[0] == 1371.4
+    assert bench.tensor_peak(peaks, "measured", None)[0] == 1371.4

@@ -112,3 +112,35 @@ def test_nonempty_cache_is_refused(gpu):
     with pytest.raises(dla.DlaError) as ei:
         dla.info_prefill(q, k, v, cache, 0.5)
     assert ei.value.code == 2
+
+
+def test_info_cache_is_refused_by_the_cosine_policy(gpu):
+    """After the information policy, the cache's pair entries are densities
+    and prev_r an information score: dla_prefill and both decode steps report
+    DLA_ERR_UNSUPPORTED on it until dla_cache_init resets it."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    q, k, v = (to_device(x, "f32") for x in info_case(1, 2, 40, 32, "f32", seed=3))
+    cache = dla.Cache(1, 2, 4, 32)
+    dla.info_prefill(q, k, v, cache, 0.5)
+    assert float(cache.views()["pair_loss"][0, 0, 3]) == -1.0
+    with pytest.raises(dla.DlaError) as ei:
+        dla.prefill(q, k, v, cache, 0.5)
+    assert ei.value.code == 2
+    cache2 = dla.Cache(1, 2, 4, 32)
+    dla.info_prefill(q, k, v, cache2, 0.5)
+    dec = dla.Decoder(cache2)
+    dec.step(q[:, :, 0].contiguous(), k[:, :, 0].contiguous(), v[:, :, 0].contiguous(), 0.5)
+    torch.cuda.synchronize()
+    assert int(dec.status.item()) == 2
+    cache3 = dla.Cache(1, 2, 4, 32)
+    dla.info_prefill(q, k, v, cache3, 0.5)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.empty(1, 2, 32, device="cuda")
+    dla.dla_decode_step_static(cache3.c, 0.5, dla.DLA_F32, q[:, :, 0].contiguous(),
+                               k[:, :, 0].contiguous(), v[:, :, 0].contiguous(), o, None, None, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 2
+    # a reset cache is the cosine policy's again
+    dla.dla_cache_init(cache.c, 1, 2, 4, 32, 32, cache.base)
+    dla.prefill(q, k, v, cache, 0.5)
