@@ -47,6 +47,11 @@
  *     (I-bar_i + I-bar_{i+1}) / (n_i + n_{i+1}) is merged (leftmost on ties)
  *     and the sums add.
  *
+ * The unbounded policy, DLA(I) (the ablation row "Mamba-2 + DLA(I)" of the
+ * Chlience page's ablation table: dynamic merging without the capacity-bounded
+ * memory), takes the same decisions and readout with no capacity at all:
+ * every segment stays a state of its own and nothing is ever merged.
+ *
  * The fixed-bucket policy (Chlience section 2 and section 5.4, Log-Linear
  * Attention's Fenwick buckets) keeps a binary-counter list of blocks over
  * [0, t-1]; token t reads the blocks plus {t} with the same softmax, then {t}
@@ -76,6 +81,7 @@
 #define OR_POLICY_DLA 0
 #define OR_POLICY_FENWICK 1
 #define OR_POLICY_INFO 2
+#define OR_POLICY_UNBOUNDED 3
 
 /* RMSNorm epsilon and the information score's denominator epsilon. */
 #define OR_INFO_EPS 1e-6
@@ -149,6 +155,15 @@ static void st_absorb(ostate *left, const ostate *right, int dk, int dv) {
   left->info = left->info + right->info;
 }
 
+/* Room for one more sealed state (the unbounded policy grows its list). */
+static void ensure_room(ohead *hd, int dk, int dv, int want_S) {
+  if (hd->nsealed < hd->cap_sealed) return;
+  int cap = hd->cap_sealed * 2;
+  hd->sealed = (ostate *)realloc(hd->sealed, sizeof(ostate) * (size_t)cap);
+  for (int i = hd->cap_sealed; i < cap; i++) st_alloc(&hd->sealed[i], dk, dv, want_S);
+  hd->cap_sealed = cap;
+}
+
 /* Ward loss n_a n_b / (n_a + n_b) * sum_i (z_a[i]/n_a - z_b[i]/n_b)^2. */
 static double ward(const ostate *a, const ostate *b, int dk) {
   double na = (double)a->n, nb = (double)b->n;
@@ -209,7 +224,7 @@ oracle *dla_oracle_new(int nheads, int dk, int dv, int C, int policy, int want_S
   o->want_S = policy == OR_POLICY_INFO ? 1 : want_S;
   want_S = o->want_S;
   o->heads = (ohead *)calloc((size_t)nheads, sizeof(ohead));
-  int cap = policy == OR_POLICY_FENWICK ? 64 : C;
+  int cap = policy == OR_POLICY_FENWICK ? 64 : (policy == OR_POLICY_UNBOUNDED ? 16 : C);
   for (int h = 0; h < nheads; h++) {
     ohead *hd = &o->heads[h];
     hd->cap_sealed = cap;
@@ -343,15 +358,18 @@ static void readout(const oracle *o, ostate *const *st, int m, const double *p, 
   free(a);
 }
 
+/* The dynamic policy, and without its capacity merges the unbounded one. */
 static void run_head_dla(job *J, int r) {
   oracle *o = J->o;
   int dk = o->dk, dv = o->dv, C = o->C, T = J->T;
+  const int unbounded = o->policy == OR_POLICY_UNBOUNDED;
   ohead *hd = &o->heads[J->head_lo + r];
+  int lst_cap = unbounded ? hd->cap_sealed : C;
   double *kk = (double *)malloc(sizeof(double) * dk);
   double *u = (double *)malloc(sizeof(double) * dk);
   double *p = (double *)malloc(sizeof(double) * dk);
   double *vv = (double *)malloc(sizeof(double) * dv);
-  ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(C + 1));
+  ostate **lst = (ostate **)malloc(sizeof(ostate *) * (size_t)(lst_cap + 1));
   double min_rm = INFINITY, min_gap = INFINITY, ties = 0.0;
   int fk = 0;
   double fex = 0.0;
@@ -369,10 +387,17 @@ static void run_head_dla(job *J, int r) {
     if (J->boundary) J->boundary[(size_t)r * T + tl] = (uint8_t)(!join);
     if (!join) {
       if (hd->has_open) {
+        if (unbounded) {
+          ensure_room(hd, dk, dv, o->want_S);
+          if (hd->cap_sealed > lst_cap) {
+            lst_cap = hd->cap_sealed;
+            lst = (ostate **)realloc(lst, sizeof(ostate *) * (size_t)(lst_cap + 1));
+          }
+        }
         st_copy(&hd->sealed[hd->nsealed], &hd->open, dk, dv);
         hd->nsealed++;
       }
-      if (hd->nsealed == C) {
+      if (!unbounded && hd->nsealed == C) {
         int best = 0;
         double bl = ward(&hd->sealed[0], &hd->sealed[1], dk);
         double second = INFINITY;
@@ -584,7 +609,7 @@ static void *worker(void *arg) {
     int r = J->next++;
     pthread_mutex_unlock(&J->mu);
     if (r >= J->head_hi - J->head_lo) break;
-    if (J->o->policy == OR_POLICY_DLA) run_head_dla(J, r);
+    if (J->o->policy == OR_POLICY_DLA || J->o->policy == OR_POLICY_UNBOUNDED) run_head_dla(J, r);
     else if (J->o->policy == OR_POLICY_INFO) run_head_info(J, r);
     else run_head_fenwick(J, r);
   }
@@ -613,7 +638,7 @@ int dla_oracle_run_forced(oracle *o, int head_lo, int head_hi, int T, double tau
   if (o->policy == OR_POLICY_INFO && !v) return 2;
   if (!k) return 3;
   if (force_count && (!force_t || !force_i || !excess || fcap < 0 ||
-                      o->policy == OR_POLICY_FENWICK))
+                      o->policy == OR_POLICY_FENWICK || o->policy == OR_POLICY_UNBOUNDED))
     return 4;
   job J;
   memset(&J, 0, sizeof J);

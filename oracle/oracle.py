@@ -17,7 +17,7 @@ _SRC = os.path.join(_HERE, "dla_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPES = {"f32": 0, "bf16": 1, "f64": 2}
-POLICIES = {"dla": 0, "fenwick": 1, "info": 2}
+POLICIES = {"dla": 0, "fenwick": 1, "info": 2, "unbounded": 3}
 
 
 def build(force: bool = False) -> str:
@@ -174,6 +174,9 @@ class Oracle:
         """Live states of a head in time order: S, z, n, ts, info (score sums),
         prev_r, t."""
         maxm = 64 if self.policy == "fenwick" else self.C
+        if self.policy == "unbounded":
+            maxm = self.lib.dla_oracle_state_info(self.h, head, 0, None, None, None, None, None,
+                                                  None, None)
         S = np.zeros((maxm, self.d_v, self.d_k)) if self.want_S else None
         z = np.zeros((maxm, self.d_k))
         n = np.zeros(maxm, dtype=np.int64)

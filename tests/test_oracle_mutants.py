@@ -24,7 +24,8 @@ MUTANTS = {
     "non_strict_threshold": ("int join = hd->t > 0 && rt < J->tau && hd->prev_r < J->tau;",
                              "int join = hd->t > 0 && rt <= J->tau && hd->prev_r <= J->tau;"),
     "rightmost_tie": ("          if (l < bl) {", "          if (l <= bl) {"),
-    "capacity_off_by_one": ("      if (hd->nsealed == C) {", "      if (hd->nsealed == C - 1) {"),
+    "capacity_off_by_one": ("      if (!unbounded && hd->nsealed == C) {",
+                            "      if (!unbounded && hd->nsealed == C - 1) {"),
     "phi_is_plain_elu": ("return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x) - 1.0;"),
     "transposed_state": ("acc = acc + st[i]->S[(size_t)r * dk + c] * p[c];",
                          "acc = acc + st[i]->S[(size_t)c * dk + r] * p[c];"),
@@ -45,6 +46,7 @@ MUTANTS = {
     "forced_excess_over_second": ("double e = l == bl ? 0.0 : (bl > 0.0 ? (l - bl) / bl : INFINITY);",
                                   "double e = l == bl ? 0.0 : (bl > 0.0 ? (l - bl) / l : INFINITY);"),
     "forced_leftover_ignored": ("  if (fk != J->force_count[r]) ex = INFINITY;\n", ""),
+    "unbounded_still_merges": ("      if (!unbounded && hd->nsealed == C) {", "      if (hd->nsealed == C) {"),
     "fenwick_no_carry": ("while (hd->nsealed >= 2 && hd->sealed[hd->nsealed - 1].n == hd->sealed[hd->nsealed - 2].n) {",
                          "while (0) {"),
 }
@@ -100,6 +102,8 @@ def all_pins(lib):
     pins.check_single_state(lib)
     pins.check_all_singletons(lib)
     pins.check_fenwick(lib)
+    for seed in range(3):
+        pins.check_unbounded(seed, 0.5, lib)
 
 
 def test_real_oracle_passes_pins():

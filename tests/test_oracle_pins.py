@@ -321,3 +321,47 @@ def check_forced_mode(seed, C, tau, lib=None):
                                         for tau in (0.3, 0.5)])
 def test_forced_mode(seed, C, tau):
     check_forced_mode(seed, C, tau)
+
+
+# ---- DLA(I): no capacity bound ------------------------------------------------
+
+def check_unbounded(seed, tau, lib=None):
+    """The unbounded policy (the ablation row "Mamba-2 + DLA(I)"): boundaries
+    from numpy scores, no merge ever, one state per segment, every output
+    rebuilt from explicit outer products over the segments' token ranges."""
+    T, d = 96, 6
+    q, k, v = small_case(seed, T, d, mean_len=3.0)
+    orc = O.Oracle(1, d, d, 2, "unbounded", lib=lib)
+    res = orc.run(k[None], q[None], v[None], tau=tau, dtype="f64", nthreads=1)
+    b = res["boundary"][0]
+    r = bf.scores(k)
+    join = np.zeros(T, dtype=bool)
+    join[1:] = (r[1:] < tau) & (r[:-1] < tau)
+    assert (b == (~join).astype(np.uint8)).all()
+    assert res["merges"][0] == []
+    ranges = bf.replay(b, [], policy="unbounded")
+    assert res["live"][0].tolist() == [len(x) for x in ranges]
+    assert res["live"][0].tolist() == np.cumsum(b).tolist()
+    o = bf.outputs(q, k, v, ranges)
+    assert np.allclose(res["out"][0], o, rtol=0, atol=1e-11 * np.abs(o).max())
+    st = orc.state(0)
+    assert st["m"] == int(b.sum()) and st["n"].sum() == T
+    assert st["ts"].tolist() == np.flatnonzero(b).tolist()
+
+
+@pytest.mark.parametrize("seed,tau", [(s, tau) for s in range(12) for tau in (0.3, 0.5, 1.0)])
+def test_unbounded(seed, tau):
+    check_unbounded(seed, tau)
+
+
+def test_unbounded_split_calls_equal_one_call():
+    T, d = 120, 5
+    q, k, v = small_case(3, T, d, mean_len=2.0)
+    one = O.Oracle(1, d, d, 2, "unbounded")
+    full = one.run(k[None], q[None], v[None], tau=0.5, dtype="f64", nthreads=1)
+    two = O.Oracle(1, d, d, 2, "unbounded")
+    a = two.run(k[None, :50], q[None, :50], v[None, :50], tau=0.5, dtype="f64", nthreads=1)
+    b = two.run(k[None, 50:], q[None, 50:], v[None, 50:], tau=0.5, dtype="f64", nthreads=1)
+    assert np.array_equal(np.concatenate([a["out"][0], b["out"][0]]), full["out"][0])
+    assert np.array_equal(np.concatenate([a["boundary"][0], b["boundary"][0]]), full["boundary"][0])
+    assert full["live"][0].max() > 40  # far past any small capacity
