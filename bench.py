@@ -48,6 +48,8 @@ def policy_of(workload):
         return "fenwick"
     if workload.startswith("info"):
         return "info"
+    if workload.startswith("unbounded"):
+        return "unbounded"
     return "dla"
 
 
@@ -341,9 +343,12 @@ def bench_prefill(args, wl, rank, world, local_rank, e2e=True):
     prof = dla.Profiler(cap=4096)
     dcode = dla.DLA_BF16 if dt == "bf16" else dla.DLA_F32
     cfg = dla.make_config(B, H, T, d, C, wl["tau"], dcode, args.window, prof.p)
-    info = policy_of(args.workload) == "info"
-    policy_code = dla.DLA_POLICY_INFO if info else dla.DLA_POLICY_DYNAMIC
-    run = dla.dla_info_policy_prefill if info else dla.dla_prefill
+    pol = policy_of(args.workload)
+    info = pol == "info"
+    policy_code = {"info": dla.DLA_POLICY_INFO, "unbounded": dla.DLA_POLICY_UNBOUNDED}.get(
+        pol, dla.DLA_POLICY_DYNAMIC)
+    run = {"info": dla.dla_info_policy_prefill, "unbounded": dla.dla_unbounded_prefill}.get(
+        pol, dla.dla_prefill)
     ws = torch.empty(dla.dla_workspace_bytes(cfg, policy_code), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -502,7 +507,7 @@ def bench_prefill(args, wl, rank, world, local_rank, e2e=True):
             "C": C, "value": round(tokens / (dla_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",
             "ms_per_step": round(dla_ms, 4), "mean_live_states": round(dla_live / (B * H * T), 2)}}
     return {
-        **({"policy": policy_of(args.workload)} if fixed or info else {}), **extra,
+        **({"policy": pol} if pol != "dla" else {}), **extra,
         "metric": METRIC, "value": round(value, 4), "unit": "Mtok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -985,7 +990,7 @@ def main():
                           dict(synth.WORKLOADS["decode_n256"]), rank, world, local_rank)
             torch.cuda.empty_cache()
             others = {}
-            for name in ("prefill_t131072", "fixed_t32768"):
+            for name in ("prefill_t131072", "fixed_t32768", "unbounded_t8192"):
                 a = sub_args(args, name, steps=min(args.steps, 10), warmup=3)
                 a.cpu_seconds = min(args.cpu_seconds, 8.0)
                 others[name] = guarded(bench_prefill, a, dict(synth.WORKLOADS[name]), rank, world,

@@ -537,8 +537,7 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   const int64_t t0 = ca.cache.t[u];
   // the cosine / Ward policy does not continue a cache of the information
   // policy (its pair entries are densities, its prev_r an information score)
-  if (!info && lane == 0 && c_loss[C - 1] == CACHE_INFO_MARK)
-    set_status(dev_status, DLA_ERR_UNSUPPORTED);
+  if (!info && lane == 0 && c_loss[C - 1] < 0.0) set_status(dev_status, DLA_ERR_UNSUPPORTED);
   if (lane < 4) sm->used[lane] = 0u;
   __syncwarp();
   for (int p = lane; p < C; p += 32) {
@@ -859,6 +858,290 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   for (int d2 = lane; d2 < D; d2 += 32) ca.cache.prev_k[(size_t)u * D + d2] = load_in(ca.k, ca.in_dtype, krow + d2);
 }
 
+// ------------------------------------------------------ unbounded engine ----
+// The unbounded policy, DLA(I) (the ablation row "Mamba-2 + DLA(I)" of the
+// Chlience page's ablation table): the same walk over tiles and segment
+// starts, with no capacity merge.  Every segment stays a state of its own, so
+// a sealed state never changes again: its version is written once, and its
+// fp64 z goes straight to the cache when it is sealed.  The cache's C slots
+// are storage only; a stream that needs more states than C sets
+// DLA_ERR_CAPACITY (its later boundaries are then not opened and its results
+// are unspecified).  Per-slot summaries (time order, version, last op, n, ts)
+// sit in shared memory for up to DLA_MAX_SLOTS slots; lane w keeps the
+// used-slot bits of slots 32w .. 32w + 31.
+template <int D>
+__global__ void __launch_bounds__(32) k_engine_unb(Dims dm, Plan pl, CallArgs ca) {
+  constexpr int QD = D / 32;
+  extern __shared__ __align__(16) unsigned char unb_raw[];
+  const int C = dm.C, M = dm.M, W = dm.W, tiles = dm.tiles, amax = dm.amax, vmax = dm.vmax;
+  const int opsmax = dm.opsmax, pmax = dm.pmax;
+  double(*zring)[128] = reinterpret_cast<double(*)[128]>(unb_raw);
+  double *zdump = reinterpret_cast<double *>(unb_raw + sizeof(double) * ZR * 128);
+  long long *s_n = reinterpret_cast<long long *>(zdump + 128);
+  long long *s_ts = s_n + C;
+  int32_t *s_order = reinterpret_cast<int32_t *>(s_ts + C);
+  int32_t *s_sver = s_order + C;
+  int32_t *s_lastmod = s_sver + C;
+  const int u = blockIdx.x, lane = threadIdx.x;
+  const int Tw = ca.Tw;
+  int32_t *const dev_status = ca.dev_status;
+  int32_t *const c_order = ca.cache.order + (size_t)u * C;
+  int64_t *const c_n = ca.cache.n + (size_t)u * C;
+  int64_t *const c_ts = ca.cache.ts + (size_t)u * C;
+  double *const c_loss = ca.cache.pair_loss + (size_t)u * C;
+  double *const c_z = ca.cache.z + (size_t)u * C * D;
+  const int nseg = pl.nseg[u];
+  const int32_t *const ss = pl.seg_start + (size_t)u * (W + 1);
+  const double *const zend = pl.z_end + (size_t)u * W * D;
+  const double *const ztile_g = pl.z_tile + (size_t)u * tiles * D;
+  int4 *const ops = pl.ops + (size_t)u * opsmax;
+  int32_t *const tm0 = pl.tile_m0 + (size_t)u * tiles;
+  int32_t *const tat = pl.tile_atoms + (size_t)u * tiles * amax;
+  int32_t *const tnev = pl.tile_nev + (size_t)u * tiles;
+  int32_t *const toff = pl.tile_ev_off + (size_t)u * tiles * M;
+  int32_t *const tmrg = pl.tile_ev_mrg + (size_t)u * tiles * M;
+  float *const ver_z = pl.ver_z + (size_t)u * vmax * D;
+  float *const ver_n = pl.ver_n + (size_t)u * vmax;
+
+  // only an empty cache or one of this policy is continued
+  if (lane == 0 && ca.cache.t[u] > 0 && c_loss[C - 1] != CACHE_UNBOUNDED_MARK)
+    set_status(dev_status, DLA_ERR_UNSUPPORTED);
+
+  // ---- segment-end sums: prefetch ring (as in k_engine) ----------------------
+  auto zfetch = [&](int g) {
+    if (g < nseg) {
+      double *dst = zring[g % ZR] + lane;
+      const double *src = zend + (size_t)g * D + lane;
+#pragma unroll
+      for (int q = 0; q < QD; q++) cp_async8(dst + 32 * q, src + 32 * q);
+    }
+    cp_async_commit();
+  };
+#pragma unroll 1
+  for (int g = 0; g < ZR; g++) zfetch(g);
+  int zcons = 0;
+  auto ztake = [&](double *dst) {
+    cp_async_wait<ZR - 1>();
+    const double *src = zring[zcons % ZR] + lane;
+#pragma unroll
+    for (int q = 0; q < QD; q++) dst[lane + 32 * q] = src[32 * q];
+    zfetch(zcons + ZR);
+    zcons++;
+  };
+
+  int m = ca.cache.m[u];
+  const int64_t t0 = ca.cache.t[u];
+  uint32_t uw = 0u;  // this lane's word of the used-slot bits
+  for (int p = lane; p < C; p += 32) {
+    s_order[p] = c_order[p];
+    s_n[p] = c_n[p];
+    s_ts[p] = c_ts[p];
+    s_sver[p] = -1;
+    s_lastmod[p] = -1;
+  }
+  __syncwarp();
+  for (int p = 0; p < m; p++) {
+    const int o = s_order[p];
+    if (lane == (o >> 5)) uw |= 1u << (o & 31);
+  }
+  const uint32_t valid_bits =
+      lane * 32 >= C ? 0u : (C - lane * 32 >= 32 ? ~0u : ((1u << (C - lane * 32)) - 1u));
+  auto alloc_slot = [&]() -> int {
+    const uint32_t fr = ~uw & valid_bits;
+    const unsigned bal = __ballot_sync(FULL, fr != 0u);
+    if (bal == 0u) {  // m < C with no free slot: an inconsistent cache
+      if (lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
+      return 0;
+    }
+    const int w = __ffs(bal) - 1;
+    const int bit = __ffs(__shfl_sync(FULL, fr, w)) - 1;
+    if (lane == w) uw |= 1u << bit;
+    return w * 32 + bit;
+  };
+
+  int nops = 0, nver = 0;
+  int ptile = -1, pk = 0;
+  auto emit = [&](int op, int a, int b, int c) {
+    if (lane == 0) {
+      if (nops < opsmax) ops[nops] = make_int4(op, a, b, c);
+      else set_status(dev_status, DLA_ERR_INVARIANT);
+    }
+    nops++;
+  };
+  auto emit_add = [&](int slot, int from, int cnt) {
+    if (pmax > 0 && cnt >= PIECE_MIN) {
+      const int tl = from / M;
+      if (tl != ptile) {
+        ptile = tl;
+        pk = 0;
+      }
+      const int id = tl * PIECES_PER_TILE + pk++;
+      if (id >= pmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
+      emit(OP_ADDP, slot, id, cnt);
+    } else {
+      emit(OP_ADD, slot, from, cnt);
+    }
+  };
+  if (m > 0) emit(OP_LOAD, s_order[m - 1], 0, 0);
+  const bool cont0 = nseg > 0 && pl.b[(size_t)u * W] == 0;
+  int sbase = 0;
+  int ssA = lane < nseg ? ss[lane] : 0x7fffffff;
+  int ssB = 32 + lane < nseg ? ss[32 + lane] : 0x7fffffff;
+  int j = 0;
+  int cur_from = 0;
+  double ztile[QD];
+#pragma unroll
+  for (int q = 0; q < QD; q++) ztile[q] = 0.0;
+#pragma unroll 1
+  for (int c = 0; c < tiles && c * M < Tw; c++) {
+    const int T0 = c * M;
+    const int Tend = min(T0 + M, Tw);
+    double ztile_cur[QD];
+#pragma unroll
+    for (int q = 0; q < QD; q++) {
+      ztile_cur[q] = ztile[q];
+      ztile[q] = (c + 1 < tiles && (c + 1) * M < Tw) ? ztile_g[(size_t)(c + 1) * D + lane + 32 * q] : 0.0;
+    }
+    if (m > 0 && T0 > cur_from) {
+      const int os = s_order[m - 1];
+      emit_add(os, cur_from, T0 - cur_from);
+      if (lane == 0) s_n[os] += T0 - cur_from;
+      cur_from = T0;
+    }
+    __syncwarp();
+    // ---- the states present before the tile: every live state --------------
+    const int m0 = m;
+#pragma unroll 1
+    for (int p0 = 0; p0 < m0; p0 += 32) {
+      const int p = p0 + lane;
+      const int slot = p < m0 ? s_order[p] : 0;
+      const int sv = p < m0 ? s_sver[slot] : 0;
+      const bool need = p < m0 && (p == m0 - 1 || sv < 0);
+      const int lm = (need && p != m0 - 1) ? s_lastmod[slot] : -1;
+      const bool patch = lm >= 0;
+      const unsigned bal = __ballot_sync(FULL, need);
+      const unsigned bal_emit = __ballot_sync(FULL, need && !patch);
+      const unsigned below = (1u << lane) - 1u;
+      const int rank = __popc(bal & below);
+      if (need) {
+        const int v = nver + rank;
+        if (patch) {
+          if (lm < opsmax) ops[lm].w = v + 1;
+          s_lastmod[slot] = -1;
+        } else {
+          const int erank = __popc(bal_emit & below);
+          if (nops + erank < opsmax) ops[nops + erank] = make_int4(OP_SHADOW, slot, v, 0);
+          else set_status(dev_status, DLA_ERR_INVARIANT);
+        }
+        if (p != m0 - 1) s_sver[slot] = v;
+        tat[(size_t)c * amax + p] = min(v, vmax - 1);  // (v >= vmax is flagged below)
+      } else if (p < m0) {
+        tat[(size_t)c * amax + p] = sv;
+      }
+      unsigned todo = bal;
+      while (todo) {
+        const int l = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int pv = p0 + l;
+        const int sl = __shfl_sync(FULL, slot, l);
+        const int v = nver + __popc(bal & ((1u << l) - 1u));
+        if (v < vmax) {
+          float *zv = ver_z + (size_t)v * D + lane;
+          if (pv == m0 - 1 && c > 0) {
+#pragma unroll
+            for (int q = 0; q < QD; q++) zv[32 * q] = (float)ztile_cur[q];
+          } else {
+            const double *zsrc = c_z + (size_t)sl * D + lane;
+#pragma unroll
+            for (int q = 0; q < QD; q++) zv[32 * q] = (float)zsrc[32 * q];
+          }
+          if (lane == 0) ver_n[v] = (float)s_n[sl];
+        }
+      }
+      nver += __popc(bal);
+      nops += __popc(bal_emit);
+      __syncwarp();
+    }
+    if (nver > vmax && lane == 0) set_status(dev_status, DLA_ERR_INVARIANT);
+    if (lane == 0) tm0[c] = m0;
+    // ---- boundaries inside the tile ----------------------------------------
+    int nev = 0;
+#pragma unroll 1
+    while (j < nseg) {
+      if (j - sbase == 32) {
+        sbase += 32;
+        ssA = ssB;
+        ssB = sbase + 32 + lane < nseg ? ss[sbase + 32 + lane] : 0x7fffffff;
+      }
+      const int s = __shfl_sync(FULL, ssA, j - sbase);
+      if (s >= Tend) break;
+      if (!(s == 0 && cont0)) {
+        if (m == C) {
+          // no slot left for a new state: report it; the token stays in the
+          // open state (the ring entry of the segment is consumed)
+          if (lane == 0) set_status(dev_status, DLA_ERR_CAPACITY);
+          if (j >= 1) ztake(zdump);
+          j++;
+          continue;
+        }
+        if (m > 0) {
+          const int os = s_order[m - 1];
+          if (s > cur_from) {
+            emit_add(os, cur_from, s - cur_from);
+            if (lane == 0) s_n[os] += s - cur_from;
+          }
+          if (j >= 1) ztake(c_z + (size_t)os * D);  // the sealed state's final z
+          if (lane == 0) s_lastmod[os] = nops;
+          emit(OP_STORE, os, 0, 0);
+        }
+        const int slot = alloc_slot();
+        emit(OP_ZERO, slot, 0, 0);
+        if (lane == 0) {
+          s_n[slot] = 0;
+          s_ts[slot] = t0 + s;
+          s_order[m] = slot;
+          s_sver[slot] = -1;
+          s_lastmod[slot] = -1;
+          toff[(size_t)c * M + nev] = s - T0;
+          tmrg[(size_t)c * M + nev] = EV_NO_MERGE;
+        }
+        __syncwarp();
+        m += 1;
+        cur_from = s;
+        nev++;
+      }
+      j++;
+    }
+    if (lane == 0) tnev[c] = nev;
+  }
+  // ---- window end ----------------------------------------------------------
+  if (m > 0) {
+    const int os = s_order[m - 1];
+    if (Tw > cur_from) {
+      emit_add(os, cur_from, Tw - cur_from);
+      if (lane == 0) s_n[os] += Tw - cur_from;
+    }
+    emit(OP_STORE, os, 0, 0);
+    if (nseg >= 1 && zcons < nseg) ztake(c_z + (size_t)os * D);
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+  for (int p = lane; p < C; p += 32) {
+    c_order[p] = s_order[p];
+    c_n[p] = s_n[p];
+    c_ts[p] = s_ts[p];
+  }
+  if (lane == 0) {
+    c_loss[C - 1] = CACHE_UNBOUNDED_MARK;
+    ca.cache.m[u] = m;
+    ca.cache.t[u] = t0 + Tw;
+    ca.cache.prev_r[u] = pl.r[(size_t)u * W + Tw - 1];
+    pl.nops[u] = min(nops, opsmax);
+  }
+  const size_t krow = ((size_t)u * dm.T + ca.w0 + Tw - 1) * D;
+  for (int d2 = lane; d2 < D; d2 += 32) ca.cache.prev_k[(size_t)u * D + d2] = load_in(ca.k, ca.in_dtype, krow + d2);
+}
+
 }  // namespace
 
 // The score kernel also forms the tile sums for bf16 keys with tiles of
@@ -930,7 +1213,26 @@ static cudaError_t launch_engine_d(const Dims &dm, const Plan &pl, const CallArg
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_engine_unb_d(const Dims &dm, const Plan &pl, const CallArgs &ca,
+                                       cudaStream_t s) {
+  size_t sb = sizeof(double) * (ZR * 128 + 128) + (size_t)dm.C * (2 * sizeof(long long) + 3 * sizeof(int32_t));
+  if (dm.heads <= sm_count() && sb < ENGINE_SM_RESERVE) sb = ENGINE_SM_RESERVE;
+  cudaError_t e = cudaFuncSetAttribute(k_engine_unb<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+  if (e != cudaSuccess) return e;
+  k_engine_unb<D><<<dm.heads, 32, sb, s>>>(dm, pl, ca);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_engine(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
+  if (dm.unb) {
+    switch (dm.D) {
+      case 32: return launch_engine_unb_d<32>(dm, pl, ca, s);
+      case 64: return launch_engine_unb_d<64>(dm, pl, ca, s);
+      case 128: return launch_engine_unb_d<128>(dm, pl, ca, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (dm.D) {
     case 32: return launch_engine_d<32>(dm, pl, ca, s);
     case 64: return launch_engine_d<64>(dm, pl, ca, s);

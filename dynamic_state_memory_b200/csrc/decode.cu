@@ -70,8 +70,8 @@ __global__ void __launch_bounds__(128) k_decode_decide(dla_cache cc, float tau, 
   const int64_t t = cc.t[u];
   int m = cc.m[u];
   const size_t row = (size_t)u * D;
-  // a cache of the information policy is not continued here
-  if (lane == 0 && loss[C - 1] == CACHE_INFO_MARK) set_status(dev_status, DLA_ERR_UNSUPPORTED);
+  // a cache of the information or unbounded policy is not continued here
+  if (lane == 0 && loss[C - 1] < 0.0) set_status(dev_status, DLA_ERR_UNSUPPORTED);
 
   // score in index order on lane 0 (same operation sequence as the oracle)
   double r = 0.0;

@@ -8,6 +8,7 @@ namespace dla {
 
 int simt_tile_rows();
 int tc_tile_rows();
+bool simt_fits(int D, int C);
 
 namespace {
 
@@ -56,6 +57,7 @@ Dims make_dims(const dla_config &cfg, int policy) {
   dm.D = cfg.d_k;
   dm.C = cfg.C;
   dm.info = policy == DLA_POLICY_INFO ? 1 : 0;
+  dm.unb = policy == DLA_POLICY_UNBOUNDED ? 1 : 0;
   int W = cfg.window > 0 ? cfg.window : (tc ? 8192 : 2048);
   W = (W + dm.M - 1) / dm.M * dm.M;
   const int Tr = (cfg.T + dm.M - 1) / dm.M * dm.M;
@@ -65,7 +67,9 @@ Dims make_dims(const dla_config &cfg, int policy) {
   dm.tiles = W / dm.M;
   dm.amax = dm.C;
   const int per_tile = dm.C < 2 * dm.M + 1 ? dm.C : 2 * dm.M + 1;
-  dm.vmax = dm.C + dm.tiles * per_tile;
+  // with no merges a state is frozen at most once, plus the open state at
+  // every tile start
+  dm.vmax = dm.unb ? dm.C + dm.tiles : dm.C + dm.tiles * per_tile;
   dm.opsmax = 4 * W + dm.tiles + 2 + dm.vmax + 8;
   dm.vbytes = dm.D * dm.D * (tc ? 2 : (int)sizeof(float));
   dm.pmax = tc ? dm.tiles * PIECES_PER_TILE : 0;
@@ -167,6 +171,11 @@ dla_status shape_ok(const dla_config *cfg, int policy) {
   if (cfg->d_k != cfg->d_v || !d_ok(cfg->d_k)) return DLA_ERR_UNSUPPORTED;
   if ((policy == DLA_POLICY_DYNAMIC || policy == DLA_POLICY_INFO) && (cfg->C < 2 || cfg->C > 128))
     return DLA_ERR_UNSUPPORTED;
+  if (policy == DLA_POLICY_UNBOUNDED) {
+    if (cfg->C < 2 || cfg->C > DLA_MAX_SLOTS) return DLA_ERR_UNSUPPORTED;
+    // the SIMT readout keeps every atom's logits of a tile in shared memory
+    if (!use_tc(*cfg) && !simt_fits(cfg->d_k, cfg->C)) return DLA_ERR_UNSUPPORTED;
+  }
   return DLA_OK;
 }
 
@@ -238,6 +247,7 @@ const char *dla_status_string(dla_status s) {
     case DLA_ERR_WORKSPACE: return "workspace smaller than dla_workspace_bytes()";
     case DLA_ERR_INVARIANT: return "device invariant violated";
     case DLA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case DLA_ERR_CAPACITY: return "the unbounded policy needs more states than the cache has slots";
   }
   return "unknown status";
 }
@@ -262,7 +272,7 @@ dla_status dla_cache_init(dla_cache *cache, int32_t N, int32_t H, int32_t C, int
   const size_t need = dla_cache_bytes(N, H, C, d_k, d_v);
   if (need == 0) return DLA_ERR_INVALID_ARG;
   if (bytes < need) return DLA_ERR_WORKSPACE;
-  if (d_k != d_v || !d_ok(d_k) || C < 2 || C > 128) return DLA_ERR_UNSUPPORTED;
+  if (d_k != d_v || !d_ok(d_k) || C < 2 || C > DLA_MAX_SLOTS) return DLA_ERR_UNSUPPORTED;
   dla_cache c{};
   c.N = N;
   c.H = H;
@@ -290,7 +300,8 @@ size_t dla_workspace_bytes(const dla_config *cfg, int32_t policy) {
     carve_fenwick(cv, dm, pl, &a, &b);
     return cv.off;
   }
-  if (policy != DLA_POLICY_DYNAMIC && policy != DLA_POLICY_INFO) return 0;
+  if (policy != DLA_POLICY_DYNAMIC && policy != DLA_POLICY_INFO && policy != DLA_POLICY_UNBOUNDED)
+    return 0;
   const Dims dm = make_dims(*cfg, policy);
   Plan pl{};
   Carver cv{nullptr};
@@ -473,6 +484,14 @@ dla_status dla_info_policy_prefill(const dla_config *cfg, const void *q, const v
                                    int32_t *dev_status, void *stream) {
   return prefill_impl(DLA_POLICY_INFO, cfg, q, k, v, o, cache, trace, ws, ws_bytes, dev_status,
                       stream);
+}
+
+dla_status dla_unbounded_prefill(const dla_config *cfg, const void *q, const void *k,
+                                 const void *v, void *o, const dla_cache *cache,
+                                 const dla_trace *trace, void *ws, size_t ws_bytes,
+                                 int32_t *dev_status, void *stream) {
+  return prefill_impl(DLA_POLICY_UNBOUNDED, cfg, q, k, v, o, cache, trace, ws, ws_bytes,
+                      dev_status, stream);
 }
 
 size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {

@@ -45,10 +45,13 @@ constexpr int PIECE_MIN = 16;
 constexpr int PIECES_PER_TILE = 128 / PIECE_MIN;
 
 // pair_loss[C - 1] of a stream belongs to no pair (C states have C - 1
-// adjacent pairs).  The information policy writes this value there: its pair
-// entries are densities, not Ward losses, so the cosine / Ward entry points
-// refuse such a cache (DLA_ERR_UNSUPPORTED) until dla_cache_init resets it.
+// adjacent pairs).  The information policy writes CACHE_INFO_MARK there (its
+// pair entries are densities, not Ward losses) and the unbounded policy
+// CACHE_UNBOUNDED_MARK (it keeps no pair losses); the capacity-bounded
+// cosine / Ward entry points refuse a cache with a negative entry
+// (DLA_ERR_UNSUPPORTED) until dla_cache_init resets it.
 constexpr double CACHE_INFO_MARK = -1.0;
+constexpr double CACHE_UNBOUNDED_MARK = -2.0;
 
 // Merge code of an in-tile boundary event: -1 none, >= 0 merge of the sealed
 // pair at that time-order position, <= -2 merge the two newest sealed states
@@ -70,6 +73,7 @@ struct Dims {
   int32_t pmax;    // max tensor-core pieces per head per window (0 = none)
   int32_t fenwick; // 1: fixed Fenwick policy (every token a piece; closed-form epochs)
   int32_t info;    // 1: information policy (state score, density merges)
+  int32_t unb;     // 1: unbounded policy (no capacity merges; C = storage slots)
 };
 
 // Per-window plan, every array strided by head.

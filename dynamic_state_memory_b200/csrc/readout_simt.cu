@@ -300,6 +300,20 @@ cudaError_t launch_d(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStr
 
 int simt_tile_rows() { return M; }
 
+// Whether a tile's atoms (up to C) fit the SIMT readout's shared memory and
+// its epoch bitmask.
+bool simt_fits(int D, int C) {
+  if (C + M > 16 * 32) return false;
+  size_t b = 0;
+  switch (D) {
+    case 32: b = smem_bytes<32>(C); break;
+    case 64: b = smem_bytes<64>(C); break;
+    case 128: b = smem_bytes<128>(C); break;
+    default: return false;
+  }
+  return b <= 227 * 1024;
+}
+
 cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                 cudaStream_t s) {
   if (dm.M != M || dm.C + M > 16 * 32) return cudaErrorInvalidValue;

@@ -79,10 +79,10 @@ struct PreSmem {
                            // K-half is 16 KB after the first, whatever the atom count)
                            // q and mu, once the first MMAs have read them, hold the
                            // values of pieces PREG.. (fp32 [piece][row], 128 pieces)
-  uint64_t bar_load, bar_mma, bar_v;
+  uint64_t bar_load, bar_mma, bar_v, bar_la;
   uint32_t tmem_base;
   int abort;
-  int m0, np, len;
+  int m0, np, len, cont;
   float nA[128];
   int atom[128];
   int pst[M + 1], pen[M + 1], pidx[M];
@@ -95,8 +95,8 @@ static_assert(offsetof(PreSmem, mu) == offsetof(PreSmem, q) + TILE_BYTES, "q, mu
 struct Smem {
   uint8_t q[TILE_BYTES];  // phi(Q) on its way to tensor memory, then version stage NST
   uint8_t st[NST][VER_BYTES];
-  float w[128 * M];       // W[atom][row]
-  uint64_t bar_load, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
+  float w[128 * M];       // W[atom][row] of 128 atoms at a time
+  uint64_t bar_load, bar_w, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
   uint32_t tmem_base;
   int abort;
   int atom[128];
@@ -169,17 +169,17 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     bulk_load(sm.kp, static_cast<const uint8_t *>(pl.phi_k) + g * TILE_BYTES, TILE_BYTES, &sm.bar_load);
   }
   const int m0 = pl.tile_m0[(size_t)u * dm.tiles + c];
-  {
-    const int32_t *atoms = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
-    for (int a = tid; a < m0; a += PRE_THREADS) {
-      const int at = atoms[a];
-      sm.atom[a] = at;
-      sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + at];
-    }
+  const int32_t *const atoms_g = pl.tile_atoms + ((size_t)u * dm.tiles + c) * dm.amax;
+  const int m0c = min(m0, 128);  // atoms of the first logit chunk (all of them unless unbounded)
+  for (int a = tid; a < m0c; a += PRE_THREADS) {
+    const int at = atoms_g[a];
+    sm.atom[a] = at;
+    sm.nA[a] = pl.ver_n[(size_t)u * dm.vmax + at];
   }
   if (tid == 0) {
     mbar_init(&sm.bar_mma, 1);
     mbar_init(&sm.bar_v, 1);
+    mbar_init(&sm.bar_la, 1);
     fence_mbar_init();
     sm.abort = 0;
   }
@@ -206,6 +206,10 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     for (int i = 0; i < nev; i++) sm.pst[np++] = evo[i];
     for (int p = 0; p < np; p++) sm.pen[p] = p + 1 < np ? sm.pst[p + 1] : len;
     sm.np = np;
+    sm.cont = cont ? 1 : 0;
+    // unbounded policy: no merges, so every atom and piece ends a state of
+    // its own except the last atom when piece 0 continues it (no bitmask)
+    if (!dm.unb) {
     uint32_t cur[BW];
     for (int w = 0; w < BW; w++)
       cur[w] = m0 >= 32 * (w + 1) ? ~0u : (m0 > 32 * w ? (1u << (m0 - 32 * w)) - 1u : 0u);
@@ -242,6 +246,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
       cur[beta >> 5] |= 1u << (beta & 31);
       for (int w = 0; w < BW; w++) sm.bits[p * BW + w] = cur[w];
     }
+    }
   }
   __syncthreads();
   tc_fence_after();
@@ -256,11 +261,11 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
   mbar_wait(&sm.bar_load, 0, abort);
 
   // ---- Mu (bf16 means of the atoms) -------------------------------------------
-  const int n_mu = (m0 + 15) & ~15;
+  const int n_mu = (m0c + 15) & ~15;
   for (int e = tid; e < n_mu * 16; e += PRE_THREADS) {
     const int a = e >> 4, ch = e & 15;
     uint4 x = make_uint4(0, 0, 0, 0);
-    if (a < m0) {
+    if (a < m0c) {
       const float4 *zz = reinterpret_cast<const float4 *>(pl.ver_z + ((size_t)u * dm.vmax + sm.atom[a]) * D + ch * 8);
       const float inv = 1.0f / sm.nA[a];
       const float4 z0 = zz[0], z1 = zz[1];
@@ -296,6 +301,89 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     mbar_expect_tx(&sm.bar_v, TILE_BYTES);
     for (int h = 0; h < 2; h++)
       tma_load_3d(sm.kp + h * (TILE_BYTES / 2), &tv, &sm.bar_v, h * 64, ca.w0 + T0, u);
+  }
+
+  // ---- unbounded policy: the atoms' logits, 128 at a time ----------------------
+  // With no merges every atom is a state of its own, except the last one
+  // when piece 0 continues it (the open state), so no segmented sums are
+  // needed.  Chunk 0's logits came with A; each further chunk's means replace
+  // Mu and its logits LA (all threads take part: shared Mu, one MMA thread).
+  // The row warps keep the softmax's running maximum and sum over the atoms
+  // that end a state and park each atom's scaled logit in the plan's weight
+  // array, rewritten as its weight once the maximum and sum are final.
+  float u_mx = -INFINITY, u_l = 0.f, u_lalast = 0.f;
+  if (dm.unb) {
+    const bool rw = warp >= 4 && warp < 8;
+    const int qd = warp & 3;
+    const int t = 32 * qd + lane;
+    const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
+    const bool last_joins = sm.cont && m0 > 0;
+    for (int a0 = 0; a0 < m0; a0 += 128) {
+      const int na = min(128, m0 - a0);
+      if (a0 > 0) {
+        const int nmu = (na + 15) & ~15;
+        for (int e = tid; e < nmu * 16; e += PRE_THREADS) {
+          const int a = e >> 4, ch = e & 15;
+          uint4 x = make_uint4(0, 0, 0, 0);
+          if (a < na) {
+            const int at = atoms_g[a0 + a];
+            const float4 *zz = reinterpret_cast<const float4 *>(pl.ver_z + ((size_t)u * dm.vmax + at) * D + ch * 8);
+            const float inv = 1.0f / pl.ver_n[(size_t)u * dm.vmax + at];
+            const float4 z0 = zz[0], z1 = zz[1];
+            x.x = pack_bf16(z0.x * inv, z0.y * inv);
+            x.y = pack_bf16(z0.z * inv, z0.w * inv);
+            x.z = pack_bf16(z1.x * inv, z1.y * inv);
+            x.w = pack_bf16(z1.z * inv, z1.w * inv);
+          }
+          *reinterpret_cast<uint4 *>(mu_buf + sw128_offset(a, ch * 8, 128)) = x;
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 1 && lane == 0) {
+          tc_fence_after();
+          const uint32_t q_s0 = smem_u32(sm.q);
+          for (int k = 0; k < 8; k++)
+            mma_bf16(tbase + PRE_LA, sdesc(q_s0 + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024),
+                     sdesc(smem_u32(mu_buf) + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024),
+                     idesc_bf16(M, nmu, 0, 0), k > 0);
+          mma_commit(&sm.bar_la);
+        }
+        mbar_wait(&sm.bar_la, ((a0 >> 7) - 1) & 1, abort);
+        tc_fence_after();
+      }
+      if (rw) {
+#pragma unroll 1
+        for (int b = 0; b * 32 < na; b++) {
+          uint32_t r[32];
+          DLA_TMEM_LD32(trow + PRE_LA + 32 * b, r);
+          tmem_wait_ld();
+          float x[32];
+#pragma unroll
+          for (int j = 0; j < 32; j++) {
+            const int a = a0 + 32 * b + j;
+            const bool joins = last_joins && a == m0 - 1;
+            u_lalast = joins ? __uint_as_float(r[j]) : u_lalast;
+            x[j] = (a < m0 && !joins) ? __uint_as_float(r[j]) * INV_SQRT_D : -INFINITY;
+          }
+          const float cmx = max32(x);
+          if (cmx > -INFINITY) {
+            float e[32];
+#pragma unroll
+            for (int j = 0; j < 32; j++) e[j] = __expf(x[j] - cmx);
+            const float cl = sum32(e);
+            const float nm = fmaxf(u_mx, cmx);
+            u_l = u_l * __expf(u_mx - nm) + cl * __expf(cmx - nm);
+            u_mx = nm;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; j++)
+            if (a0 + 32 * b + j < m0) preW[(size_t)(a0 + 32 * b + j) * M + t] = x[j];
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+    }
   }
 
   // ---- softmax weights per row (warps 4..7, row t = TMEM lane) ----------------
@@ -468,11 +556,23 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     }
     // pass A: each state's logit at its last atom / piece, online softmax max
     // and sum; atom columns keep exp(logit - block max) (0 for atoms that do
-    // not end a state), pieces keep their logits
+    // not end a state), pieces keep their logits.  Under the unbounded policy
+    // the atoms were done chunk by chunk above; the last atom joins piece 0
+    // when the tile continues the open state.
     float mx = -INFINITY, l = 0.f, sacc = 0.f, nacc = 0.f;
     float bmx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // block maxima
+    const bool unb = dm.unb != 0;
+    if (unb) {
+      mx = u_mx;
+      l = u_l;
+      if (sm.cont && m0 > 0) {
+        const float nn = pl.ver_n[(size_t)u * dm.vmax + atoms_g[m0 - 1]];
+        sacc = nn * u_lalast;
+        nacc = nn;
+      }
+    }
 #pragma unroll 1
-    for (int b = 0; b * 32 < m0; b++) {
+    for (int b = 0; !unb && b * 32 < m0; b++) {
       const int a0 = b * 32;
       uint32_t r[32];
       DLA_TMEM_LD32(trow + PRE_LA + a0, r);
@@ -526,7 +626,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
         const float nn = p < ep ? (float)(sm.pen[p] - sm.pst[p]) : (float)(t - sm.pst[p] + 1);
         sacc += y;
         nacc += nn;
-        if (bit_of(bits, m0 + p)) {
+        if (unb || bit_of(bits, m0 + p)) {
           const float a = __fdividef(sacc, nacc) * INV_SQRT_D;
           y = a;
           const float nm = fmaxf(mx, a);
@@ -546,13 +646,24 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
       const float a = piece_get(p);
       float w = 0.f;
       if (p <= ep) {
-        if (bit_of(bits, m0 + p)) cur = __expf(a - mx) * inv_l;
+        if (unb || bit_of(bits, m0 + p)) cur = __expf(a - mx) * inv_l;
         w = cur;
       }
       piece_put(p, w);
     }
+    if (unb) {
+      // every atom's weight from its parked logit; the last one shares
+      // piece 0's state when it continues into the tile
+      const float w0 = piece_get(0);
+      const bool last_joins = sm.cont && m0 > 0;
+#pragma unroll 4
+      for (int a = 0; a < m0; a++) {
+        float *pw = preW + (size_t)a * M + t;
+        *pw = (last_joins && a == m0 - 1) ? w0 : __expf(*pw - mx) * inv_l;
+      }
+    }
 #pragma unroll 1
-    for (int b = (m0 - 1) >> 5; m0 > 0 && b >= 0; b--) {
+    for (int b = (m0 - 1) >> 5; !unb && m0 > 0 && b >= 0; b--) {
       const int a0 = b * 32;
       uint32_t r[32];
       DLA_TMEM_LD32(trow + PRE_LA + a0, r);
@@ -690,6 +801,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
+    mbar_init(&sm.bar_w, 1);
     mbar_init(&sm.bar_qa, 8);
     for (int i = 0; i < NSV; i++) {
       mbar_init(&sm.full[i], 1);
@@ -701,23 +813,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     fence_mbar_init();
     sm.abort = 0;
-    const uint32_t wbytes = (uint32_t)m0 * M * 4;
+    const uint32_t wbytes = (uint32_t)min(m0, 128) * M * 4;  // the first 128 atoms' weights
     mbar_expect_tx(&sm.bar_load, TILE_BYTES + wbytes);
     for (int h = 0; h < 2; h++)
       tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, T0, u);
     if (m0 > 0) bulk_load(sm.w, pl.pre_w + g * dm.amax * M, wbytes, &sm.bar_load);
   }
-  {
-    const int32_t *atoms = pl.tile_atoms + g * dm.amax;
-    for (int a = tid; a < m0; a += THREADS) sm.atom[a] = atoms[a];
-  }
+  const int32_t *const atoms_g = pl.tile_atoms + g * dm.amax;
+  for (int a = tid; a < m0 && a < 128; a += THREADS) sm.atom[a] = atoms_g[a];
+  // the version of atom a (beyond 128 atoms, only the unbounded policy, read
+  // from the plan)
+  auto atom_at = [&](int a) -> int { return a < 128 ? sm.atom[a] : atoms_g[a]; };
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
   if (tid == 0) {
     for (int a = 0; a < m0 && a < NST; a++) {
       mbar_expect_tx(&sm.full[a], VER_BYTES);
-      bulk_load(sm.st[a], verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[a]);
+      bulk_load(sm.st[a], verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES, &sm.full[a]);
     }
   }
   auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
@@ -760,9 +873,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // written by the materializer, so a head's first tiles mostly miss L2
     constexpr int PF = 6;
     for (int a = NST; a < m0 && a < NST + PF; a++)
-      bulk_prefetch_l2(verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES);
+      bulk_prefetch_l2(verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES);
     for (int a = NST; a < m0; a++) {
-      if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)sm.atom[a + PF] * VER_BYTES, VER_BYTES);
+      if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)atom_at(a + PF) * VER_BYTES, VER_BYTES);
       const int s = a % NSV;
       // stage NST is the phi(Q) tile: free once every epilogue warp has put
       // its rows into tensor memory (bar_qa)
@@ -770,7 +883,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                : mbar_wait(&sm.bar_qa, 0, abort);
       if (!ok) break;
       mbar_expect_tx(&sm.full[s], VER_BYTES);
-      bulk_load(stage(s), verS + (size_t)sm.atom[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
+      bulk_load(stage(s), verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES, &sm.full[s]);
     }
   } else if (warp >= 4) {
     const int qd = warp & 3, hc = (warp - 4) >> 2;
@@ -816,7 +929,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
     for (int a = 0; a < m0; a++) {
       const int b = a % NPB;
-      const float w = sW[a * M + t];
+      if (a > 0 && (a & 127) == 0) {
+        // the next 128 atoms' weights replace the last ones (the epilogue
+        // warps alone read them: a named barrier over those 256 threads)
+        fence_proxy_async();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (warp == 4 && lane == 0) {
+          const uint32_t nb = (uint32_t)min(128, m0 - a) * M * 4;
+          mbar_expect_tx(&sm.bar_w, nb);
+          bulk_load(sm.w, pl.pre_w + g * dm.amax * M + (size_t)a * M, nb, &sm.bar_w);
+        }
+        mbar_wait(&sm.bar_w, ((a >> 7) - 1) & 1, abort);
+      }
+      const float w = sW[(a & 127) * M + t];
       mbar_wait(&sm.tfull[b], (a / NPB) & 1, abort);
       tc_fence_after();
       uint32_t pr[32];
@@ -907,7 +1032,7 @@ cudaError_t launch_phi_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
 
 cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs &ca,
                                   cudaStream_t s) {
-  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.phi_q)
+  if (dm.M != M || dm.D != D || (dm.C > 128 && !dm.unb) || ca.in_dtype != DLA_BF16 || !pl.phi_q)
     return cudaErrorInvalidValue;
   CUtensorMap tq, tv;
   if (!make_bf16_map_rows(&tq, pl.phi_q, ca.Tw, dm.W, dm.heads) ||
@@ -923,7 +1048,7 @@ cudaError_t launch_readout_pre_tc(const Dims &dm, const Plan &pl, const CallArgs
 }
 
 cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca, cudaStream_t s) {
-  if (dm.M != M || dm.D != D || dm.C > 128 || ca.in_dtype != DLA_BF16 || !pl.phi_q)
+  if (dm.M != M || dm.D != D || (dm.C > 128 && !dm.unb) || ca.in_dtype != DLA_BF16 || !pl.phi_q)
     return cudaErrorInvalidValue;
   CUtensorMap tq;
   if (!make_bf16_map_rows(&tq, pl.phi_q, ca.Tw, dm.W, dm.heads)) return cudaErrorInvalidValue;

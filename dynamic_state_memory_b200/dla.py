@@ -16,10 +16,11 @@ LIB_PATH = os.path.join(_HERE, "libdla.so")
 
 DLA_OK = 0
 DLA_F32, DLA_BF16 = 0, 1
-DLA_POLICY_DYNAMIC, DLA_POLICY_FENWICK, DLA_POLICY_INFO = 0, 1, 2
+DLA_POLICY_DYNAMIC, DLA_POLICY_FENWICK, DLA_POLICY_INFO, DLA_POLICY_UNBOUNDED = 0, 1, 2, 3
+DLA_MAX_SLOTS = 1024
 STATUS_NAMES = {0: "DLA_OK", 1: "DLA_ERR_INVALID_ARG", 2: "DLA_ERR_UNSUPPORTED", 3: "DLA_ERR_CUDA",
                 4: "DLA_ERR_TRACE_OVERFLOW", 5: "DLA_ERR_WORKSPACE", 6: "DLA_ERR_INVARIANT",
-                7: "DLA_ERR_TIMEOUT"}
+                7: "DLA_ERR_TIMEOUT", 8: "DLA_ERR_CAPACITY"}
 
 c_i32, c_f32, c_vp, c_size = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -71,6 +72,9 @@ _lib.dla_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_cach
 _lib.dla_info_policy_prefill.restype = c_i32
 _lib.dla_info_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_cache),
                                          _P(dla_trace), c_vp, c_size, c_vp, c_vp]
+_lib.dla_unbounded_prefill.restype = c_i32
+_lib.dla_unbounded_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_cache),
+                                       _P(dla_trace), c_vp, c_size, c_vp, c_vp]
 _lib.dla_decode_workspace_bytes.restype = c_size
 _lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
 _lib.dla_decode_step.restype = c_i32
@@ -85,7 +89,8 @@ _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp
 
 EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
            "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
-           "dla_decode_step_static", "dla_fixed_policy_prefill", "dla_info_policy_prefill"]
+           "dla_decode_step_static", "dla_fixed_policy_prefill", "dla_info_policy_prefill",
+           "dla_unbounded_prefill"]
 
 
 def status_string(code: int) -> str:
@@ -146,6 +151,15 @@ def dla_info_policy_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, strea
                                         0 if ws is None else ws.numel(), _ptr(dev_status),
                                         _stream(stream)),
            "dla_info_policy_prefill")
+
+
+def dla_unbounded_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, stream=None):
+    tr = ctypes.byref(trace) if trace is not None else None
+    _check(_lib.dla_unbounded_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                      ctypes.byref(cache), tr, _ptr(ws),
+                                      0 if ws is None else ws.numel(), _ptr(dev_status),
+                                      _stream(stream)),
+           "dla_unbounded_prefill")
 
 
 def dla_decode_workspace_bytes(N, H, C, d_k, d_v) -> int:
@@ -326,6 +340,27 @@ def info_prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, cap=N
     if sync:
         torch.cuda.synchronize()
         check_device_status(st, "dla_info_policy_prefill")
+    return o, tr
+
+
+def unbounded_prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, cap=None,
+                      window=0, stream=None, sync=True, profile=None):
+    """o = DLA(I) prefill (no capacity bound; cache.C is the slot storage) of
+    q, k, v [B, H, T, d]."""
+    B, H, T, d = k.shape
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    cfg = make_config(B, H, T, d, cache.C, tau, _dtype_code(k), window, profile)
+    ws = torch.empty(max(dla_workspace_bytes(cfg, DLA_POLICY_UNBOUNDED), 1), dtype=torch.uint8,
+                     device=k.device)
+    o = torch.empty_like(q)
+    tr = Trace(B * H, T, 1 if cap is None else cap, k.device) if trace else None
+    st = torch.zeros(1, dtype=torch.int32, device=k.device)
+    dla_unbounded_prefill(cfg, q, k, v, o, cache.c, None if tr is None else tr.c, ws, st, stream)
+    if sync:
+        torch.cuda.synchronize()
+        check_device_status(st, "dla_unbounded_prefill")
     return o, tr
 
 

@@ -54,6 +54,12 @@ WORKLOADS = {
     "fixed_t32768": dict(B=2, H=16, T=32768, d=128, C=16, tau=0.5,
                          dtype="bf16", n_centres=64,
                          lengths=("geometric", 96.0), sigma=0.05, seed=1005),
+    # DLA(I), no capacity bound, on the T=8192 prefill's sizes with shorter
+    # regimes (mean 32): about 460 states per stream by the end (230 live on
+    # average), in a cache of 1024 slots
+    "unbounded_t8192": dict(B=4, H=16, T=8192, d=128, C=1024, tau=0.5,
+                            dtype="bf16", n_centres=64,
+                            lengths=("geometric", 32.0), sigma=0.05, seed=1007),
     # the information policy on the T=8192 prefill's sizes; values follow the
     # regimes (recipe step 6) and tau sits between the within-regime score
     # (about 0.6 at d = 128) and the score of a regime switch (about 1.4)

@@ -52,12 +52,22 @@ typedef enum {
   DLA_ERR_TRACE_OVERFLOW = 4,  /* device: more merges than dla_trace.cap */
   DLA_ERR_WORKSPACE = 5,       /* ws_bytes smaller than the size query */
   DLA_ERR_INVARIANT = 6,       /* device: a cache invariant was violated */
-  DLA_ERR_TIMEOUT = 7          /* device: a bounded wait inside a kernel gave up */
+  DLA_ERR_TIMEOUT = 7,         /* device: a bounded wait inside a kernel gave up */
+  DLA_ERR_CAPACITY = 8         /* device: the unbounded policy ran out of cache slots */
 } dla_status;
+
+/* Most state slots a cache may have (the unbounded policy's storage; the
+ * capacity-bounded policies take 2 <= C <= 128). */
+#define DLA_MAX_SLOTS 1024
 
 typedef enum { DLA_F32 = 0, DLA_BF16 = 1 } dla_dtype;
 
-typedef enum { DLA_POLICY_DYNAMIC = 0, DLA_POLICY_FENWICK = 1, DLA_POLICY_INFO = 2 } dla_policy;
+typedef enum {
+  DLA_POLICY_DYNAMIC = 0,   /* cosine score, capacity C, Ward merges (dla_prefill) */
+  DLA_POLICY_FENWICK = 1,   /* fixed Fenwick buckets (dla_fixed_policy_prefill) */
+  DLA_POLICY_INFO = 2,      /* the pages' state score and density merges */
+  DLA_POLICY_UNBOUNDED = 3  /* DLA(I): cosine score, no capacity bound (dla_unbounded_prefill) */
+} dla_policy;
 
 /* Kernel kinds reported through dla_profile. */
 typedef enum {
@@ -109,7 +119,8 @@ typedef struct {
  *   n, ts     int64  [u][C]            token count and first token of a slot
  *   pair_loss double [u][C]            Ward loss of sealed pair (p, p+1); entry
  *                                      C-1 (no pair) is -1 after the
- *                                      information policy, 0 otherwise
+ *                                      information policy, -2 after the
+ *                                      unbounded one, 0 otherwise
  *   order     int32  [u][C]            time-order position -> slot
  *   m         int32  [u]               live states (open one included)
  *   prev_k    float  [u][d_k]          last key, for the next score
@@ -235,6 +246,27 @@ dla_status dla_info_policy_prefill(const dla_config *cfg, const void *q, const v
                                    const void *v, void *o, const dla_cache *cache,
                                    const dla_trace *trace, void *ws, size_t ws_bytes,
                                    int32_t *dev_status, void *stream);
+
+/* DLA(I), dynamic merging without the capacity bound (the ablation row
+ * "Mamba-2 + DLA(I)" of the Chlience page's ablation table): the decisions of
+ * dla_prefill (cosine score, two consecutive low scores join a token to the
+ * open state) with no capacity merge at all.  Every segment stays a state of
+ * its own and the readout's softmax runs over all of them, so the state count
+ * grows with the sequence.  cfg->C is the cache's number of slots (storage
+ * only, 2 <= C <= DLA_MAX_SLOTS; on the fp32 SIMT path, used for inputs
+ * other than bf16 at d = 128, a tile's C logits must also fit in shared
+ * memory, else DLA_ERR_UNSUPPORTED).  A stream that needs more states than C
+ * sets DLA_ERR_CAPACITY in *dev_status; its later boundaries are then not
+ * opened and its results are unspecified.  The cache must be empty or hold
+ * a stream of this policy (a call continues it); a stream of another policy
+ * sets DLA_ERR_UNSUPPORTED and its results are unspecified.  Afterwards pair_loss[C-1] is -2, which dla_prefill and the decode steps
+ * refuse (DLA_ERR_UNSUPPORTED) until dla_cache_init resets the cache.  The
+ * trace records boundaries and no merges.  Other arguments as for
+ * dla_prefill; ws: at least dla_workspace_bytes(cfg, DLA_POLICY_UNBOUNDED). */
+dla_status dla_unbounded_prefill(const dla_config *cfg, const void *q, const void *k,
+                                 const void *v, void *o, const dla_cache *cache,
+                                 const dla_trace *trace, void *ws, size_t ws_bytes,
+                                 int32_t *dev_status, void *stream);
 
 /* Static description of a status code. */
 const char *dla_status_string(dla_status status);
