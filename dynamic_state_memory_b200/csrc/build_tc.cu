@@ -57,10 +57,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        ~static_cast<uintptr_t>(1023));
   const int u = blockIdx.y, c = blockIdx.x;
   const int T0 = c * M;
-  if (T0 >= ca.Tw) return;
+  const int Tw = tw_of(ca, u);
+  if (T0 >= Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5;
   volatile int *abort = &sm.abort;
-  const int len = min(M, ca.Tw - T0);
+  const int len = min(M, Tw - T0);
   if (warp == 0) tmem_alloc(&sm.tmem_base, 128);
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);

@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
   const int tb = blockIdx.x * SCORE_TOK;
   const int tl = tb + threadIdx.x;
   const int D = dm.D;
+  const int Tw = tw_of(ca, u);  // this stream's tokens in the window
+  if (tb >= Tw) return;         // (a whole block: a ragged stream ends before it)
   const int wpr = BF16 ? D / 2 : D;  // 32-bit words per row
   const int ld = wpr + 1;
   // the stream's token count before the window (read only in a call's first
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
           const int rr = e / vpr, cv = e % vpr;
           const int t = tb - 2 + rr;
           xs[i] = make_uint4(0, 0, 0, 0);
-          if (b0 + i < MAXIT && e < (SCORE_TOK + 2) * vpr && ca.w0 + t >= 0 && t < ca.Tw)
+          if (b0 + i < MAXIT && e < (SCORE_TOK + 2) * vpr && ca.w0 + t >= 0 && t < Tw)
             xs[i] = kv[(ptrdiff_t)t * vpr + cv];
         }
 #pragma unroll
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
         const int t = tb - 2 + rr;
         if (t == -1 && ca.w0 == 0) continue;  // the cache's previous key, written below
         uint4 x = make_uint4(0, 0, 0, 0);
-        if (ca.w0 + t >= 0 && t < ca.Tw) x = kv[(ptrdiff_t)t * vpr + cv];
+        if (ca.w0 + t >= 0 && t < Tw) x = kv[(ptrdiff_t)t * vpr + cv];
         uint32_t *dst = srow + rr * ld + cv * 4;
         dst[0] = x.x;
         dst[1] = x.y;
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
     }
     __syncthreads();
     double dot = 0.0, na = 0.0;
-    if (tl < ca.Tw) dot_norm<BF16>(srow + (threadIdx.x + 2) * ld, srow + (threadIdx.x + 1) * ld, D, dot, na);
+    if (tl < Tw) dot_norm<BF16>(srow + (threadIdx.x + 2) * ld, srow + (threadIdx.x + 1) * ld, D, dot, na);
     nsq[threadIdx.x + 1] = na;
     if (threadIdx.x == 32) {  // a thread of the second warp: token tb-1
       const int tp = tb - 1;
@@ -203,12 +205,12 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
       }
     }
     __syncthreads();
-    if (tl < ca.Tw) r = (ca.w0 == 0 && t0 + tl == 0) ? 0.0 : score_of(dot, na, nsq[threadIdx.x]);
+    if (tl < Tw) r = (ca.w0 == 0 && t0 + tl == 0) ? 0.0 : score_of(dot, na, nsq[threadIdx.x]);
   }
   rs[threadIdx.x + 1] = r;
   __syncthreads();
   uint8_t b = 1;
-  if (tl < ca.Tw) {
+  if (tl < Tw) {
     if (policy == DLA_POLICY_DYNAMIC) {
       const double rp = rs[threadIdx.x];
       const double tau = (double)ca.tau;
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(SCORE_TOK, 6) k_score(Dims dm, Plan pl, CallAr
   // between boundaries, stored at the run's first token
   s_b[threadIdx.x] = b;
   __syncthreads();
-  const int len = min(SCORE_TOK, ca.Tw - tb);
+  const int len = min(SCORE_TOK, Tw - tb);
   for (int c = threadIdx.x; c < D; c += SCORE_TOK) {
     double *zp = pl.z_part + (size_t)u * dm.W * D + c;
     double z = 0.0;
@@ -258,9 +260,10 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int c0 = 0; c0 < ca.Tw; c0 += blockDim.x) {
+  const int Tw = tw_of(ca, u);
+  for (int c0 = 0; c0 < Tw; c0 += blockDim.x) {
     const int t = c0 + threadIdx.x;
-    const bool f = t > 0 && t < ca.Tw && b[t];
+    const bool f = t > 0 && t < Tw && b[t];
     const unsigned bal = __ballot_sync(FULL, f);
     if (lane == 0) warp_tot[warp] = __popc(bal);
     __syncthreads();
@@ -275,7 +278,7 @@ __global__ void k_segscan(Dims dm, Plan pl, CallArgs ca) {
     }
     __syncthreads();
   }
-  if (threadIdx.x == 0) pl.nseg[u] = base;
+  if (threadIdx.x == 0) pl.nseg[u] = Tw > 0 ? base : 0;  // no token, no piece
 }
 
 // z = sum of phi(k) of every window piece, in fp64, in two levels:
@@ -296,8 +299,9 @@ __global__ void k_tilesum_any(Dims dm, Plan pl, CallArgs ca) {
   const int c = threadIdx.x;  // dimension
   const int D = dm.D, M = dm.M;
   const int T0 = tile * M;
-  if (T0 >= ca.Tw) return;
-  const int T1 = min(T0 + M, ca.Tw);
+  const int Tw = tw_of(ca, u);
+  if (T0 >= Tw) return;
+  const int T1 = min(T0 + M, Tw);
   const uint8_t *b = pl.b + (size_t)u * dm.W;
   const size_t kb = ((size_t)u * dm.T + ca.w0) * D + c;
   double *zp = pl.z_part + (size_t)u * dm.W * D + c;
@@ -319,12 +323,13 @@ __global__ void k_segcombine(Dims dm, Plan pl, CallArgs ca) {
   const int c = threadIdx.x;  // dimension
   const int D = dm.D, M = dm.M;
   const int nseg = pl.nseg[u];
+  const int Tw = tw_of(ca, u);
   const int32_t *ss = pl.seg_start + (size_t)u * (dm.W + 1);
   const uint8_t *b = pl.b + (size_t)u * dm.W;
   const double *zp = pl.z_part + (size_t)u * dm.W * D + c;
   for (int j = blockIdx.x; j < nseg; j += gridDim.x) {
     const int s0 = ss[j];
-    const int s1 = j + 1 < nseg ? ss[j + 1] : ca.Tw;
+    const int s1 = j + 1 < nseg ? ss[j + 1] : Tw;
     double z = 0.0;
     if (j == 0 && b[0] == 0) {
       // continuation of the cache's open state
@@ -339,7 +344,7 @@ __global__ void k_segcombine(Dims dm, Plan pl, CallArgs ca) {
     }
     // the tile start right after the segment's end (if the segment ends at a
     // tile boundary the next tile's open state is this one, complete)
-    if (s1 % M == 0 && s1 < ca.Tw) pl.z_tile[((size_t)u * dm.tiles + s1 / M) * D + c] = z;
+    if (s1 % M == 0 && s1 < Tw) pl.z_tile[((size_t)u * dm.tiles + s1 / M) * D + c] = z;
     pl.z_end[((size_t)u * dm.W + j) * D + c] = z;
   }
 }
@@ -480,8 +485,12 @@ __global__ void __launch_bounds__(32) k_engine(Dims dm, Plan pl, CallArgs ca) {
   const int u = blockIdx.x, lane = threadIdx.x;
   const int C = dm.C, M = dm.M, W = dm.W, tiles = dm.tiles, amax = dm.amax, vmax = dm.vmax;
   const int opsmax = dm.opsmax, pmax = dm.pmax;
-  const int Tw = ca.Tw;
+  const int Tw = tw_of(ca, u);
   int32_t *const dev_status = ca.dev_status;
+  if (Tw == 0) {  // a ragged stream with no token in this window: nothing changes
+    if (lane == 0) pl.nops[u] = 0;
+    return;
+  }
   // the head's cache
   int32_t *const c_order = ca.cache.order + (size_t)u * C;
   int64_t *const c_n = ca.cache.n + (size_t)u * C;
@@ -883,8 +892,12 @@ __global__ void __launch_bounds__(32) k_engine_unb(Dims dm, Plan pl, CallArgs ca
   int32_t *s_sver = s_order + C;
   int32_t *s_lastmod = s_sver + C;
   const int u = blockIdx.x, lane = threadIdx.x;
-  const int Tw = ca.Tw;
+  const int Tw = tw_of(ca, u);
   int32_t *const dev_status = ca.dev_status;
+  if (Tw == 0) {  // a ragged stream with no token in this window: nothing changes
+    if (lane == 0) pl.nops[u] = 0;
+    return;
+  }
   int32_t *const c_order = ca.cache.order + (size_t)u * C;
   int64_t *const c_n = ca.cache.n + (size_t)u * C;
   int64_t *const c_ts = ca.cache.ts + (size_t)u * C;

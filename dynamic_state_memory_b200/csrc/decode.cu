@@ -55,11 +55,18 @@ __device__ double ward64(const double *za, const double *zb, double na, double n
 __global__ void __launch_bounds__(128) k_decode_decide(dla_cache cc, float tau, int32_t dt,
                                                        const void *q, const void *k,
                                                        DecodeWs w, uint8_t *boundary,
-                                                       int32_t *merge_i, int32_t *dev_status) {
+                                                       int32_t *merge_i, int32_t *dev_status,
+                                                       const uint8_t *active) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = blockIdx.x * 4 + warp;
   const int U = cc.N * cc.H;
   if (u >= U) return;
+  if (active && !active[u / cc.H]) {
+    // a sequence that takes no token this step: its cache is left alone and
+    // the streaming kernel skips it (open slot -1)
+    if (lane == 0) w.instr[u] = make_int4(-1, 0, -1, -1);
+    return;
+  }
   const int C = cc.C, D = cc.d_k;
   int32_t *order = cc.order + (size_t)u * C;
   int64_t *n = cc.n + (size_t)u * C;
@@ -260,6 +267,7 @@ __global__ void __launch_bounds__(WARPS * 32) k_decode_stream(dla_cache cc, int3
   const int C = cc.C;
   const size_t row = (size_t)u * D;
   const int4 ins = w.instr[u];
+  if (ins.x < 0) return;  // an inactive sequence (masked step)
   const float *lam = w.lam + (size_t)u * C;
   const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
   float pq[4], pk[4], vr[ROWS_PER_WARP];
@@ -359,11 +367,11 @@ size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C) {
 
 cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,
                                  const void *k, void *ws, uint8_t *boundary, int32_t *merge_i,
-                                 int32_t *dev_status, cudaStream_t s) {
+                                 int32_t *dev_status, cudaStream_t s, const uint8_t *active) {
   const int U = cc.N * cc.H;
   DecodeWs w = carve_ws(ws, U, cc.C);
   k_decode_decide<<<(U + 3) / 4, 128, 0, s>>>(cc, tau, dt, q, k, w, boundary, merge_i,
-                                              dev_status);
+                                              dev_status, active);
   return cudaGetLastError();
 }
 

@@ -322,7 +322,8 @@ namespace {
 // streams and kernels but the score and the engine's pair criterion.
 dla_status prefill_impl(int policy, const dla_config *cfg, const void *q, const void *k,
                         const void *v, void *o, const dla_cache *cache, const dla_trace *trace,
-                        void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+                        void *ws, size_t ws_bytes, int32_t *dev_status, void *stream,
+                        const int32_t *lens = nullptr) {
   if (!cfg_ok(cfg, policy) || !cache) return DLA_ERR_INVALID_ARG;
   const dla_status sh = shape_ok(cfg, policy);
   if (sh != DLA_OK) return sh;
@@ -362,6 +363,8 @@ dla_status prefill_impl(int policy, const dla_config *cfg, const void *q, const 
   ca.in_dtype = cfg->in_dtype;
   ca.tau = cfg->tau;
   ca.cache = *cache;
+  ca.lens = lens;
+  ca.H = cfg->H;
   if (trace) {
     ca.trace = *trace;
     if (cudaMemsetAsync(trace->merge_count, 0, sizeof(int32_t) * dm.heads, s) != cudaSuccess)
@@ -467,6 +470,34 @@ dla_status prefill_impl(int policy, const dla_config *cfg, const void *q, const 
   return DLA_OK;
 }
 
+dla_status decode_impl(const dla_cache *cache, float tau, int32_t in_dtype, const uint8_t *active,
+                       const void *q, const void *k, const void *v, void *o, uint8_t *boundary,
+                       int32_t *merge_i, void *ws, size_t ws_bytes, int32_t *dev_status,
+                       void *stream, dla_profile *profile) {
+  if (!cache || !q || !k || !v || !o || !ws) return DLA_ERR_INVALID_ARG;
+  if (in_dtype != DLA_F32 && in_dtype != DLA_BF16) return DLA_ERR_INVALID_ARG;
+  if (!cache->S || !cache->z || !cache->order || !cache->m) return DLA_ERR_INVALID_ARG;
+  const size_t need = dla_decode_workspace_bytes(cache->N, cache->H, cache->C, cache->d_k,
+                                                 cache->d_v);
+  if (need == 0) return DLA_ERR_UNSUPPORTED;
+  if (ws_bytes < need) return DLA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    ProfScope ps(profile, DLA_K_DECODE_DECIDE, s);
+    e = launch_decode_decide(*cache, tau, in_dtype, q, k, ws, boundary, merge_i, dev_status, s,
+                             active);
+  }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  {
+    ProfScope ps(profile, DLA_K_DECODE_STREAM, s);
+    e = launch_decode_stream(*cache, in_dtype, q, k, v, o, ws, s);
+  }
+  if (e != cudaSuccess) return DLA_ERR_CUDA;
+  return DLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -494,37 +525,39 @@ dla_status dla_unbounded_prefill(const dla_config *cfg, const void *q, const voi
                       dev_status, stream);
 }
 
+dla_status dla_prefill_varlen(const dla_config *cfg, int32_t policy, const int32_t *lens,
+                              const void *q, const void *k, const void *v, void *o,
+                              const dla_cache *cache, const dla_trace *trace, void *ws,
+                              size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!lens) return DLA_ERR_INVALID_ARG;
+  if (policy != DLA_POLICY_DYNAMIC && policy != DLA_POLICY_INFO && policy != DLA_POLICY_UNBOUNDED)
+    return DLA_ERR_INVALID_ARG;
+  return prefill_impl(policy, cfg, q, k, v, o, cache, trace, ws, ws_bytes, dev_status, stream,
+                      lens);
+}
+
 size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {
   if (N <= 0 || H <= 0 || C < 2 || C > 128 || d_k != d_v || !d_ok(d_k)) return 0;
   return decode_ws_bytes(N, H, C);
+}
+
+dla_status dla_decode_step_masked(const dla_cache *cache, float tau, int32_t in_dtype,
+                                  const uint8_t *active, const void *q, const void *k,
+                                  const void *v, void *o, uint8_t *boundary, int32_t *merge_i,
+                                  void *ws, size_t ws_bytes, int32_t *dev_status, void *stream) {
+  if (!active) return DLA_ERR_INVALID_ARG;
+  return decode_impl(cache, tau, in_dtype, active, q, k, v, o, boundary, merge_i, ws, ws_bytes,
+                     dev_status, stream, nullptr);
 }
 
 dla_status dla_decode_step(const dla_cache *cache, float tau, int32_t in_dtype, const void *q,
                            const void *k, const void *v, void *o, uint8_t *boundary,
                            int32_t *merge_i, void *ws, size_t ws_bytes, int32_t *dev_status,
                            void *stream, dla_profile *profile) {
-  if (!cache || !q || !k || !v || !o || !ws) return DLA_ERR_INVALID_ARG;
-  if (in_dtype != DLA_F32 && in_dtype != DLA_BF16) return DLA_ERR_INVALID_ARG;
-  if (!cache->S || !cache->z || !cache->order || !cache->m) return DLA_ERR_INVALID_ARG;
-  const size_t need = dla_decode_workspace_bytes(cache->N, cache->H, cache->C, cache->d_k,
-                                                 cache->d_v);
-  if (need == 0) return DLA_ERR_UNSUPPORTED;
-  if (ws_bytes < need) return DLA_ERR_WORKSPACE;
-  if (reinterpret_cast<uintptr_t>(ws) % ALIGN != 0) return DLA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  {
-    ProfScope ps(profile, DLA_K_DECODE_DECIDE, s);
-    e = launch_decode_decide(*cache, tau, in_dtype, q, k, ws, boundary, merge_i, dev_status, s);
-  }
-  if (e != cudaSuccess) return DLA_ERR_CUDA;
-  {
-    ProfScope ps(profile, DLA_K_DECODE_STREAM, s);
-    e = launch_decode_stream(*cache, in_dtype, q, k, v, o, ws, s);
-  }
-  if (e != cudaSuccess) return DLA_ERR_CUDA;
-  return DLA_OK;
+  return decode_impl(cache, tau, in_dtype, nullptr, q, k, v, o, boundary, merge_i, ws, ws_bytes,
+                     dev_status, stream, profile);
 }
+
 
 dla_status dla_decode_step_static(const dla_cache *cache, float tau, int32_t in_dtype,
                                   const void *q, const void *k, const void *v, void *o,

@@ -115,7 +115,9 @@ struct CallArgs {
   void *o;
   int32_t in_dtype;
   int32_t w0;         // first token of the window inside the call
-  int32_t Tw;         // tokens in this window
+  int32_t Tw;         // tokens in this window (of the longest stream when ragged)
+  const int32_t *lens;  // ragged call: tokens of each sequence [B] (null: all T)
+  int32_t H;          // heads per sequence (stream u is sequence u / H)
   float tau;
   dla_cache cache;
   dla_trace trace;    // boundary == NULL when no trace
@@ -125,6 +127,14 @@ struct CallArgs {
   double *info_aux;   // [heads][4]: |S|^2, the open state's score sum, has-open flag
   double *info_slot;  // [heads][C] score sum of each cache slot's state
 };
+
+// Tokens of stream u in this window: the window's length, cut at the
+// stream's own sequence length in a ragged call (lens[b], clamped to [0, T]).
+__device__ __forceinline__ int tw_of(const CallArgs &ca, int u) {
+  if (!ca.lens) return ca.Tw;
+  const int L = ca.lens[u / ca.H] - ca.w0;
+  return L <= 0 ? 0 : (L < ca.Tw ? L : ca.Tw);
+}
 
 __device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
   if (st) atomicCAS(st, 0, code);
@@ -179,7 +189,8 @@ cudaError_t launch_readout_simt(const Dims &dm, const Plan &pl, const CallArgs &
                                 cudaStream_t s);
 cudaError_t launch_decode_decide(const dla_cache &cc, float tau, int32_t dt, const void *q,
                                  const void *k, void *ws, uint8_t *boundary, int32_t *merge_i,
-                                 int32_t *dev_status, cudaStream_t s);
+                                 int32_t *dev_status, cudaStream_t s,
+                                 const uint8_t *active = nullptr);
 cudaError_t launch_decode_stream(const dla_cache &cc, int32_t dt, const void *q, const void *k,
                                  const void *v, void *o, void *ws, cudaStream_t s);
 size_t decode_ws_bytes(int32_t N, int32_t H, int32_t C);

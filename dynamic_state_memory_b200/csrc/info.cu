@@ -68,8 +68,8 @@ __device__ __forceinline__ double warp_sum(double s) {
 // rows past the window are zero-filled instead of loaded.
 template <int D>
 __device__ void info_stage(InfoSmem<D> &sm, int buf, const Dims &dm, const CallArgs &ca, int u,
-                           int t0, int esize) {
-  const int nrow = min(INFO_CHUNK, ca.Tw - t0);
+                           int t0, int esize, int Tw) {
+  const int nrow = min(INFO_CHUNK, Tw - t0);
   const int rowbytes = D * esize;
   const int n16 = INFO_CHUNK * rowbytes / 16;
   for (int which = 0; which < 2; which++) {
@@ -183,15 +183,15 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
   uint8_t *const tr_b = ca.trace.boundary ? ca.trace.boundary + (size_t)u * dm.T + ca.w0 : nullptr;
   double *const seg = pl.seg_info + (size_t)u * dm.W;
   int sg = 0;  // current window piece
-  const int Tw = ca.Tw;
+  const int Tw = tw_of(ca, u);
   const int nchunk = (Tw + INFO_CHUNK - 1) / INFO_CHUNK;
-  info_stage<D>(sm, 0, dm, ca, u, 0, esize);
+  info_stage<D>(sm, 0, dm, ca, u, 0, esize, Tw);
   int blk = 0;
 #pragma unroll 1
   for (int ch = 0; ch < nchunk; ch++) {
     const int t0 = ch * INFO_CHUNK;
     __syncthreads();  // the previous chunk's passes are done with u, v, H
-    if (ch + 1 < nchunk) info_stage<D>(sm, (ch + 1) & 1, dm, ca, u, t0 + INFO_CHUNK, esize);
+    if (ch + 1 < nchunk) info_stage<D>(sm, (ch + 1) & 1, dm, ca, u, t0 + INFO_CHUNK, esize, Tw);
     else cp_commit();  // an empty group keeps the wait count uniform
     cp_wait1();
     __syncthreads();

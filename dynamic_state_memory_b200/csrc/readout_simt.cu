@@ -37,8 +37,9 @@ __global__ void __launch_bounds__(THREADS) k_readout(Dims dm, Plan pl, CallArgs 
   extern __shared__ __align__(16) float smem[];
   const int u = blockIdx.y, c = blockIdx.x;
   const int T0 = c * M;
-  if (T0 >= ca.Tw) return;
-  const int len = min(M, ca.Tw - T0);
+  const int Tw = tw_of(ca, u);
+  if (T0 >= Tw) return;
+  const int len = min(M, Tw - T0);
   const int tid = threadIdx.x;
   const int C = dm.C;
   const int BW = (C + M + 31) / 32;

@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
                                              ~static_cast<uintptr_t>(1023));
   const int u = blockIdx.y, c = blockIdx.x;
   const int T0 = c * M;
-  if (T0 >= ca.Tw) return;
+  const int Tw = tw_of(ca, u);
+  if (T0 >= Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
   const size_t g = (size_t)u * dm.tiles + c;  // tile index in the plan
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     // bit of o) and {T0 + o}; the weight pass derives them from o directly
     if (tid == 0) {
       sm.m0 = m0;
-      sm.len = min(M, ca.Tw - T0);
+      sm.len = min(M, Tw - T0);
       sm.np = 0;
     }
   } else if (warp == 2 && lane == 0) {
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
     const int nev = pl.tile_nev[(size_t)u * dm.tiles + c];
     const int32_t *evo = pl.tile_ev_off + ((size_t)u * dm.tiles + c) * M;
     const int32_t *evm = pl.tile_ev_mrg + ((size_t)u * dm.tiles + c) * M;
-    const int len = min(M, ca.Tw - T0);
+    const int len = min(M, Tw - T0);
     sm.m0 = m0;
     sm.len = len;
     const bool cont = !(nev > 0 && evo[0] == 0);
@@ -786,7 +787,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        ~static_cast<uintptr_t>(1023));
   const int u = blockIdx.y, c = blockIdx.x;
   const int T0 = c * M;
-  if (T0 >= ca.Tw) return;
+  const int Tw = tw_of(ca, u);
+  if (T0 >= Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
   auto stage = [&](int s) -> uint8_t * {
@@ -795,7 +797,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
   const size_t g = (size_t)u * dm.tiles + c;
   const int m0 = pl.tile_m0[g];
-  const int len = min(M, ca.Tw - T0);
+  const int len = min(M, Tw - T0);
 
   // ---- setup: TMEM, barriers, the phi(Q) tile and the prologue's weights ----
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);

@@ -75,6 +75,12 @@ _lib.dla_info_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp,
 _lib.dla_unbounded_prefill.restype = c_i32
 _lib.dla_unbounded_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_cache),
                                        _P(dla_trace), c_vp, c_size, c_vp, c_vp]
+_lib.dla_prefill_varlen.restype = c_i32
+_lib.dla_prefill_varlen.argtypes = [_P(dla_config), c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                    _P(dla_cache), _P(dla_trace), c_vp, c_size, c_vp, c_vp]
+_lib.dla_decode_step_masked.restype = c_i32
+_lib.dla_decode_step_masked.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                        c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
 _lib.dla_decode_workspace_bytes.restype = c_size
 _lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
 _lib.dla_decode_step.restype = c_i32
@@ -90,7 +96,7 @@ _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp
 EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
            "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
            "dla_decode_step_static", "dla_fixed_policy_prefill", "dla_info_policy_prefill",
-           "dla_unbounded_prefill"]
+           "dla_unbounded_prefill", "dla_prefill_varlen", "dla_decode_step_masked"]
 
 
 def status_string(code: int) -> str:
@@ -160,6 +166,25 @@ def dla_unbounded_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, stream=
                                       0 if ws is None else ws.numel(), _ptr(dev_status),
                                       _stream(stream)),
            "dla_unbounded_prefill")
+
+
+def dla_prefill_varlen(cfg, policy, lens, q, k, v, o, cache, trace, ws, dev_status, stream=None):
+    tr = ctypes.byref(trace) if trace is not None else None
+    _check(_lib.dla_prefill_varlen(ctypes.byref(cfg), int(policy), _ptr(lens), _ptr(q), _ptr(k),
+                                   _ptr(v), _ptr(o), ctypes.byref(cache), tr, _ptr(ws),
+                                   0 if ws is None else ws.numel(), _ptr(dev_status),
+                                   _stream(stream)),
+           "dla_prefill_varlen")
+
+
+def dla_decode_step_masked(cache, tau, in_dtype, active, q, k, v, o, boundary, merge_i, ws,
+                           dev_status, stream=None):
+    _check(_lib.dla_decode_step_masked(ctypes.byref(cache), float(tau), int(in_dtype),
+                                       _ptr(active), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                       _ptr(boundary), _ptr(merge_i), _ptr(ws),
+                                       0 if ws is None else ws.numel(), _ptr(dev_status),
+                                       _stream(stream)),
+           "dla_decode_step_masked")
 
 
 def dla_decode_workspace_bytes(N, H, C, d_k, d_v) -> int:
@@ -364,6 +389,30 @@ def unbounded_prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, 
     return o, tr
 
 
+def prefill_varlen(q, k, v, lens, cache: Cache, tau: float, *, policy=DLA_POLICY_DYNAMIC,
+                   trace: bool = True, window=0, stream=None, sync=True, o=None):
+    """Ragged prefill: sequence b uses the first lens[b] of its T rows of
+    q, k, v [B, H, T, d]; lens is a CUDA int32 tensor [B].  Rows past a
+    sequence's length of o (and of the trace's boundaries) are left as given."""
+    B, H, T, d = k.shape
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one shape and dtype")
+    if lens.dtype != torch.int32 or not lens.is_cuda or lens.shape != (B,):
+        raise ValueError("lens must be a CUDA int32 tensor [B]")
+    cfg = make_config(B, H, T, d, cache.C, tau, _dtype_code(k), window)
+    ws = torch.empty(max(dla_workspace_bytes(cfg, policy), 1), dtype=torch.uint8, device=k.device)
+    o = torch.zeros_like(q) if o is None else o
+    tr = Trace(B * H, T, T + 1, k.device) if trace else None
+    st = torch.zeros(1, dtype=torch.int32, device=k.device)
+    dla_prefill_varlen(cfg, policy, lens, q, k, v, o, cache.c, None if tr is None else tr.c, ws,
+                       st, stream)
+    if sync:
+        torch.cuda.synchronize()
+        check_device_status(st, "dla_prefill_varlen")
+    return o, tr
+
+
 class Decoder:
     """Reusable buffers for dla_decode_step on one cache."""
 
@@ -384,6 +433,13 @@ class Decoder:
             o = torch.empty_like(q)
         dla_decode_step(self.cache.c, tau, _dtype_code(k), q, k, v, o, self.boundary,
                         self.merge_i, self.ws, self.status, stream, profile)
+        return o
+
+    def step_masked(self, active, q, k, v, tau, o, stream=None):
+        """One token for the sequences with active[n] != 0 (CUDA uint8 [N]);
+        the others' caches and rows of o, boundary and merge_i are untouched."""
+        dla_decode_step_masked(self.cache.c, tau, _dtype_code(k), active, q, k, v, o,
+                               self.boundary, self.merge_i, self.ws, self.status, stream)
         return o
 
 

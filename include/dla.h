@@ -268,6 +268,35 @@ dla_status dla_unbounded_prefill(const dla_config *cfg, const void *q, const voi
                                  const dla_trace *trace, void *ws, size_t ws_bytes,
                                  int32_t *dev_status, void *stream);
 
+/* A ragged batch: sequence b of the call has lens[b] tokens (a device int32
+ * array [B]; values are clamped to [0, T]), stored in the first lens[b]
+ * rows of its [T] rows of q, k, v, as in a padded batch.  Each stream (b, h)
+ * runs exactly as a call of its own with T = lens[b] would: its cache
+ * advances by lens[b] tokens (lens[b] = 0 leaves it unchanged), rows
+ * t >= lens[b] of o and of trace->boundary are not written, and the trace's
+ * merges are its own.  The serving case the pages point to: requests of
+ * different lengths prefilled in one call into their own caches.
+ * `policy` is DLA_POLICY_DYNAMIC (as dla_prefill), DLA_POLICY_UNBOUNDED (as
+ * dla_unbounded_prefill) or DLA_POLICY_INFO (as dla_info_policy_prefill); the
+ * workspace is dla_workspace_bytes(cfg, policy) and the work is that of the
+ * longest sequence per window.  Other arguments and errors as for that
+ * policy's entry point. */
+dla_status dla_prefill_varlen(const dla_config *cfg, int32_t policy, const int32_t *lens,
+                              const void *q, const void *k, const void *v, void *o,
+                              const dla_cache *cache, const dla_trace *trace, void *ws,
+                              size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* dla_decode_step for a subset of the cache's sequences (continuous
+ * batching: requests that have no token this step, or have finished, stay in
+ * the cache untouched).  active: device uint8 [N]; sequence n takes the step
+ * when active[n] != 0.  For an inactive sequence nothing is read from q, k,
+ * v and nothing is written to its cache, o, boundary or merge_i rows.  Other
+ * arguments as for dla_decode_step. */
+dla_status dla_decode_step_masked(const dla_cache *cache, float tau, int32_t in_dtype,
+                                  const uint8_t *active, const void *q, const void *k,
+                                  const void *v, void *o, uint8_t *boundary, int32_t *merge_i,
+                                  void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
 /* Static description of a status code. */
 const char *dla_status_string(dla_status status);
 
