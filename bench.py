@@ -305,15 +305,6 @@ def atom_flops(m0_rows_sum, d):
     return 2.0 * m0_rows_sum * d * d
 
 
-def tile_atoms_rows(m, T, M=128):
-    """sum over tiles of (rows in the tile) x (states live just before it), for
-    one head with m[t] = states live after token t."""
-    tot = 0
-    for c in range(1, (T + M - 1) // M):
-        tot += min(M, T - c * M) * int(m[c * M - 1])
-    return tot
-
-
 def _time_steps(step, steps, warmup, stream, world, dev):
     import torch
     for _ in range(warmup):
@@ -354,25 +345,22 @@ def bench_prefill(args, wl, rank, world, local_rank, e2e=True):
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    # one traced run (untimed) to count live states for the FLOP model
+    # one traced run (untimed) whose trace the library reduces on the device
+    # (dla_trace_stats) to the live-state counts of the FLOP model
     tr = dla.Trace(B * H, T, T + 1, dev)
     dla.dla_cache_init(cache.c, B, H, C, d, d, cache.base, stream)
     run(cfg, q, k, v, o, cache.c, tr.c, ws, st, stream)
+    stats = dla.Stats(B * H, dev)
+    sst = stats.reduce(tr, T, tile=128, stream=stream)
     torch.cuda.synchronize(dev)
     dla.check_device_status(st, "dla_prefill")
-    bnd = tr.boundary.cpu().numpy()
-    mt = tr.merge_t.cpu().numpy()
-    mc = tr.merge_count.cpu().numpy()
+    dla.check_device_status(sst, "dla_trace_stats")
     del tr
-    live_sum = 0
-    m0_rows = 0
-    for h in range(B * H):
-        m = np.cumsum(bnd[h].astype(np.int64))
-        merges_at = np.zeros(T, dtype=np.int64)
-        np.add.at(merges_at, mt[h, :mc[h]], 1)
-        m = m - np.cumsum(merges_at)
-        live_sum += int(m.sum())
-        m0_rows += tile_atoms_rows(m, T)
+    live_sum = int(stats.live_sum.sum())
+    m0_rows = int(stats.atom_rows.sum())
+    trace_stats = {"boundaries_per_stream": round(float(stats.boundaries.float().mean()), 2),
+                   "merges_per_stream": round(float(stats.merges.float().mean()), 2),
+                   "live_max": int(stats.live_max.max())}
     readout_flops, build_flops = prefill_flops(live_sum, B * H * T, d)
     loop_flops = atom_flops(m0_rows, d)
 
@@ -516,7 +504,8 @@ def bench_prefill(args, wl, rank, world, local_rank, e2e=True):
                    "tau": wl["tau"], "input_dtype": dt, "path": args.path,
                    "l2": "inputs larger than L2 (q+k+v %d MiB), no flush" % (in_bytes >> 20),
                    "flops_per_step": step_flops,
-                   "mean_live_states": round(live_sum / (B * H * T), 2)},
+                   "mean_live_states": round(live_sum / (B * H * T), 2),
+                   "trace_stats": trace_stats},
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": None if e2e_ms is None else {
             "value": round(tokens / (e2e_ms * 1e-3) / 1e6, 4), "unit": "Mtok/s",

@@ -9,6 +9,9 @@ namespace dla {
 int simt_tile_rows();
 int tc_tile_rows();
 bool simt_fits(int D, int C);
+cudaError_t launch_trace_stats(const dla_trace &tr, int heads, int T, const int32_t *m_before,
+                               const int64_t *t_before, int tile, const dla_stats &out,
+                               int32_t *dev_status, cudaStream_t s);
 
 namespace {
 
@@ -534,6 +537,20 @@ dla_status dla_prefill_varlen(const dla_config *cfg, int32_t policy, const int32
     return DLA_ERR_INVALID_ARG;
   return prefill_impl(policy, cfg, q, k, v, o, cache, trace, ws, ws_bytes, dev_status, stream,
                       lens);
+}
+
+dla_status dla_trace_stats(const dla_trace *trace, int32_t heads, int32_t T,
+                           const int32_t *m_before, const int64_t *t_before, int32_t tile,
+                           const dla_stats *out, int32_t *dev_status, void *stream) {
+  if (!trace || !out || heads <= 0 || T < 0 || tile < 0) return DLA_ERR_INVALID_ARG;
+  if (!trace->boundary || !trace->merge_count || (trace->cap > 0 && !trace->merge_t) ||
+      trace->cap < 0)
+    return DLA_ERR_INVALID_ARG;
+  if (T == 0) return DLA_OK;
+  if (launch_trace_stats(*trace, heads, T, m_before, t_before, tile, *out, dev_status,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DLA_ERR_CUDA;
+  return DLA_OK;
 }
 
 size_t dla_decode_workspace_bytes(int32_t N, int32_t H, int32_t C, int32_t d_k, int32_t d_v) {

@@ -47,6 +47,11 @@ class dla_trace(ctypes.Structure):
                 ("merge_count", c_vp), ("cap", c_i32)]
 
 
+class dla_stats(ctypes.Structure):
+    _fields_ = [("boundaries", c_vp), ("merges", c_vp), ("live_sum", c_vp), ("live_max", c_vp),
+                ("atom_rows", c_vp)]
+
+
 class DlaError(RuntimeError):
     def __init__(self, code, where=""):
         self.code = code
@@ -81,6 +86,9 @@ _lib.dla_prefill_varlen.argtypes = [_P(dla_config), c_i32, c_vp, c_vp, c_vp, c_v
 _lib.dla_decode_step_masked.restype = c_i32
 _lib.dla_decode_step_masked.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                         c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
+_lib.dla_trace_stats.restype = c_i32
+_lib.dla_trace_stats.argtypes = [_P(dla_trace), c_i32, c_i32, c_vp, c_vp, c_i32, _P(dla_stats),
+                                 c_vp, c_vp]
 _lib.dla_decode_workspace_bytes.restype = c_size
 _lib.dla_decode_workspace_bytes.argtypes = [c_i32] * 5
 _lib.dla_decode_step.restype = c_i32
@@ -96,7 +104,8 @@ _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp
 EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
            "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
            "dla_decode_step_static", "dla_fixed_policy_prefill", "dla_info_policy_prefill",
-           "dla_unbounded_prefill", "dla_prefill_varlen", "dla_decode_step_masked"]
+           "dla_unbounded_prefill", "dla_prefill_varlen", "dla_decode_step_masked",
+           "dla_trace_stats"]
 
 
 def status_string(code: int) -> str:
@@ -185,6 +194,13 @@ def dla_decode_step_masked(cache, tau, in_dtype, active, q, k, v, o, boundary, m
                                        0 if ws is None else ws.numel(), _ptr(dev_status),
                                        _stream(stream)),
            "dla_decode_step_masked")
+
+
+def dla_trace_stats(trace, heads, T, m_before, t_before, tile, out, dev_status, stream=None):
+    _check(_lib.dla_trace_stats(ctypes.byref(trace), int(heads), int(T), _ptr(m_before),
+                                _ptr(t_before), int(tile), ctypes.byref(out), _ptr(dev_status),
+                                _stream(stream)),
+           "dla_trace_stats")
 
 
 def dla_decode_workspace_bytes(N, H, C, d_k, d_v) -> int:
@@ -302,6 +318,27 @@ class Profiler:
             b, e = self.events[i]
             out.setdefault(self.KINDS[self._k[i]], []).append(b.elapsed_time(e))
         return out
+
+
+class Stats:
+    """Device summary of a trace (dla_trace_stats): boundaries, merges,
+    live_sum, live_max and atom_rows per stream."""
+
+    def __init__(self, heads, device="cuda"):
+        self.boundaries = torch.zeros(heads, dtype=torch.int32, device=device)
+        self.merges = torch.zeros(heads, dtype=torch.int32, device=device)
+        self.live_sum = torch.zeros(heads, dtype=torch.int64, device=device)
+        self.live_max = torch.zeros(heads, dtype=torch.int32, device=device)
+        self.atom_rows = torch.zeros(heads, dtype=torch.int64, device=device)
+        self.c = dla_stats(self.boundaries.data_ptr(), self.merges.data_ptr(),
+                           self.live_sum.data_ptr(), self.live_max.data_ptr(),
+                           self.atom_rows.data_ptr())
+
+    def reduce(self, trace, T, m_before=None, t_before=None, tile=128, stream=None):
+        st = torch.zeros(1, dtype=torch.int32, device=self.boundaries.device)
+        dla_trace_stats(trace.c, self.boundaries.numel(), T, m_before, t_before, tile, self.c, st,
+                        stream)
+        return st
 
 
 class Trace:

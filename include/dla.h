@@ -297,6 +297,38 @@ dla_status dla_decode_step_masked(const dla_cache *cache, float tau, int32_t in_
                                   const void *v, void *o, uint8_t *boundary, int32_t *merge_i,
                                   void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* Per-stream summary of one prefill's decision trace (device arrays [B*H],
+ * caller-owned; a NULL member is not written):
+ *   boundaries  states the call opened (boundary flags set)
+ *   merges      capacity merges of the call (the trace's merge_count)
+ *   live_sum    sum over the call's tokens of the states each token read
+ *               (mean live states = live_sum / T)
+ *   live_max    most states a token of the call read
+ *   atom_rows   sum over tiles c >= 1 of `tile` tokens of (rows of the tile) x
+ *               (states live after token c * tile - 1): the states a tiled
+ *               readout reads before each tile, the readout's FLOP count over
+ *               2 d^2 (tile 128 for the tensor-core readout)                 */
+typedef struct {
+  int32_t *boundaries, *merges;
+  int64_t *live_sum;
+  int32_t *live_max;
+  int64_t *atom_rows;
+} dla_stats;
+
+/* Reduce `trace` (as written by a prefill of T tokens for `heads` streams)
+ * on `stream`, without copying it to the host: the observables the pages
+ * list for a DLA memory (the Chlience page's list of what to observe:
+ * boundary counts, merge frequency, live states).  The live count read by
+ * token t is m_before + (boundaries at s <= t) - (merges at s <= t);
+ * m_before [heads] (int32) and t_before [heads] (int64) are the streams'
+ * live states and tokens seen before the call (device arrays saved from the
+ * cache before it; NULL = an empty cache).  A trace whose merge_count exceeds
+ * its cap sets DLA_ERR_TRACE_OVERFLOW in *dev_status (the counts then miss
+ * the lost merges).  The fixed policy writes no trace. */
+dla_status dla_trace_stats(const dla_trace *trace, int32_t heads, int32_t T,
+                           const int32_t *m_before, const int64_t *t_before, int32_t tile,
+                           const dla_stats *out, int32_t *dev_status, void *stream);
+
 /* Static description of a status code. */
 const char *dla_status_string(dla_status status);
 
