@@ -5,9 +5,13 @@
 // with eps = 1e-6; b_t = [I_t >= tau], and the first token of a stream opens
 // a state with I = 0.
 //
-// One CTA of 2D threads per head walks the window in blocks of INFO_K tokens.
-// Thread i keeps row i % D, columns (i / D) D/2 .. + D/2 of S in fp64
-// registers.  Writing x_t = <s_t, S> = v_t^T S u_t,
+// A cluster of two CTAs of 2D threads per head walks the window in blocks of
+// INFO_K tokens.  CTA r of the pair keeps rows r D/2 .. + D/2 of S in fp64
+// registers: thread i holds row r D/2 + i % (D/2), columns (i / (D/2)) D/4
+// .. + D/4.  Each warp's partial sums of the block's inner products go to
+// both CTAs' shared memory (distributed shared memory), one cluster barrier
+// later both CTAs add them in the same order and take the same decisions;
+// rank 0 alone writes the outputs.  Writing x_t = <s_t, S> = v_t^T S u_t,
 //   |N(s) - N(S)|^2 = |s|^2 / ra + |S|^2 / rb - 2 x_t / sqrt(ra rb)
 // (ra, rb: the two squared RMS denominators; with g = 1 / sqrt(rb) the
 // middle term is |S|^2 g^2 and |N(S)| = |S| g), so a block needs per token
@@ -27,7 +31,11 @@
 // (pieces as numbered by the segment scan: piece 0 starts at the window's
 // first token, piece j > 0 at the j-th later boundary).  S, |S|^2, the open
 // state's score sum and the has-open flag carry to the call's next window.
+#include <cooperative_groups.h>
+
 #include "dla_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace dla {
 namespace {
@@ -45,7 +53,7 @@ struct InfoSmem {
   // per token: |s|^2, |s|^2 / ra and 1 / sqrt(ra), ra = |s|^2 / (d_k d_v) + eps
   double ss[INFO_CHUNK], ssra[INFO_CHUNK], rsa[INFO_CHUNK];
   double H[INFO_CHUNK][INFO_K];           // (v_t . v_j)(u_t . u_j), j an earlier token of t's block
-  double red[2][INFO_K][2 * D / 32];      // per-warp partials, by block parity
+  double red[2][INFO_K][2 * (2 * D / 32)];  // per-warp partials of both CTAs, by block parity
   int jb;                                 // the block's last boundary (-1: none)
 };
 
@@ -144,19 +152,24 @@ __device__ void info_prepare(InfoSmem<D> &sm, int buf, bool bf16) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallArgs ca) {
-  constexpr int NT = 2 * D, EPT = D / 2, NW = NT / 32;
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(2 * D, 1)
+    k_info_score(Dims dm, Plan pl, CallArgs ca) {
+  constexpr int NT = 2 * D, HR = D / 2, EPT = D / 4, NW = NT / 32;
   extern __shared__ __align__(16) unsigned char info_raw[];
   InfoSmem<D> &sm = *reinterpret_cast<InfoSmem<D> *>(info_raw);
-  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // warp w holds rows 32 (w % (D / 32)) .. + 31, all in one column half, so
-  // the lanes of a warp read the same element of u: one broadcast per load
-  const int a = tid % D, c0 = (tid / D) * EPT;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int u = blockIdx.x / 2, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the lanes of a warp hold consecutive rows of one column quarter (for
+  // D >= 64), so they read the same element of u: one broadcast per load
+  const int a = rank * HR + tid % HR, c0 = (tid / HR) * EPT;
+  // this warp's partials go to slot rank * NW + warp of both CTAs
+  double(*const red_peer)[INFO_K][2 * NW] = cl.map_shared_rank(sm.red, rank ^ 1);
   const bool bf16 = ca.in_dtype == DLA_BF16;
   const int esize = bf16 ? 2 : 4;
   const double tau = (double)ca.tau;
   const double inv_d2 = 1.0 / (double)(D * D);  // a power of two: exact
-  double *const carry = ca.info_S + (size_t)u * D * D;
+  double *const carry = ca.info_S + (size_t)u * D * D + (size_t)rank * HR * D;
   double *const aux = ca.info_aux + (size_t)u * 4;
   double S[EPT];
   double sS, iopen;
@@ -164,7 +177,7 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
   if (ca.w0 == 0) {
     // the decisions need the open state in fp64, which a cache does not
     // hold: this policy starts every stream from an empty cache
-    if (tid == 0 && (ca.cache.t[u] != 0 || ca.cache.m[u] != 0))
+    if (rank == 0 && tid == 0 && (ca.cache.t[u] != 0 || ca.cache.m[u] != 0))
       set_status(ca.dev_status, DLA_ERR_UNSUPPORTED);
 #pragma unroll
     for (int j = 0; j < EPT; j++) S[j] = 0.0;
@@ -218,9 +231,14 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
 #pragma unroll
       for (int i = 0; i < INFO_K; i++) {
         const double p = warp_sum(sm.v[r0 + i][a] * acc[i]);
-        if (lane == 0) sm.red[rb][i][warp] = p;
+        if (lane == 0) {
+          sm.red[rb][i][rank * NW + warp] = p;
+          red_peer[rb][i][rank * NW + warp] = p;
+        }
       }
-      __syncthreads();
+      // both CTAs' partials of this block are in place (the peer can be at
+      // most one block ahead, so the other parity is never overwritten early)
+      cl.sync();
       // the block's decisions in token order, by warp 0 (its lanes agree);
       // the other warps wait: the fp64 pipe is the kernel's bound, so they
       // do not repeat this sequence
@@ -230,7 +248,7 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
         for (int i = 0; i < INFO_K; i++) {
           double s = 0.0;
 #pragma unroll
-          for (int w = 0; w < NW; w++) s += sm.red[rb][i][w];
+          for (int w = 0; w < 2 * NW; w++) s += sm.red[rb][i][w];
           A[i] = s;
         }
         int jb = -1;  // the block's last boundary so far
@@ -250,7 +268,7 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
               I = sqrt(num2) / (sqrt(sS) * g + INFO_EPS);
               bnd = !(I < tau);
             }
-            if (lane == 0) {
+            if (lane == 0 && rank == 0) {
               r_out[t] = I;
               b_out[t] = bnd ? 1 : 0;
               if (tr_b) tr_b[t] = bnd ? 1 : 0;
@@ -258,7 +276,7 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
             const double ssv = sm.ss[r0 + i];
             if (bnd) {
               if (t > 0) {
-                if (lane == 0) seg[sg] = iopen;
+                if (lane == 0 && rank == 0) seg[sg] = iopen;
                 sg++;
               }
               jb = i;
@@ -292,7 +310,7 @@ __global__ void __launch_bounds__(2 * D, 1) k_info_score(Dims dm, Plan pl, CallA
       }
     }
   }
-  if (tid == 0) {
+  if (tid == 0 && rank == 0) {
     seg[sg] = iopen;
     aux[0] = sS;
     aux[1] = iopen;
@@ -307,7 +325,7 @@ cudaError_t launch_info_d(const Dims &dm, const Plan &pl, const CallArgs &ca, cu
   const size_t sb = sizeof(InfoSmem<D>);
   cudaError_t e = cudaFuncSetAttribute(k_info_score<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
   if (e != cudaSuccess) return e;
-  k_info_score<D><<<dm.heads, 2 * D, sb, s>>>(dm, pl, ca);
+  k_info_score<D><<<2 * dm.heads, 2 * D, sb, s>>>(dm, pl, ca);  // a cluster of two CTAs per head
   return cudaGetLastError();
 }
 
