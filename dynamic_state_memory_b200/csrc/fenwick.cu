@@ -11,11 +11,15 @@
 //   - k_fen_means: every node's phi(k) sum and count (children added level by
 //   level, one block per head), so the readout's prologue can start while the
 //   states are still being summed;
-//   - k_fen_level: node state = left child + right child, level by level;
-//   even-indexed nodes are also written as frozen versions (fp32 or the bf16
-//   UMMA layout).  A block of size 2^b in a prefix [0, T0) starts at a
-//   multiple of 2^(b+1), so only even-indexed nodes are ever atoms; odd ones
-//   only build their parents;
+//   - k_fen_sub: node states four levels at a time.  A CTA takes 16 nodes of
+//   the pass's base level and a slice of their elements, and adds them in
+//   order with a binary counter of partial sums in registers, so every node
+//   of the four levels above is formed once (left child + right child) and
+//   only the subtree roots, the next pass's base, are stored in fp32;
+//   even-indexed nodes are written as frozen versions (fp32 or the bf16 UMMA
+//   layout).  A block of size 2^b in a prefix [0, T0) starts at a multiple
+//   of 2^(b+1), so only even-indexed nodes are ever atoms; odd ones only
+//   build their parents;
 //   - k_fen_plan: per tile, the atoms (tree nodes, oldest first) and the
 //     in-tile events: every token is a boundary, and at offset o >= 1 the
 //     binary-counter carry merges the two newest blocks (trailing ones of
@@ -132,25 +136,76 @@ __global__ void __launch_bounds__(THREADS) k_fen_means(Dims dm, Plan pl, FenTree
   }
 }
 
-// One tree level: node (level, i) = (level-1, 2i) + (level-1, 2i+1).
+// Levels base + 1 .. base + SUBL of the tree, from the (stored) nodes of level
+// `base`: block (x, head) takes subtree x / nslice (SUBN consecutive base
+// nodes) and element slice x % nslice of SUB_EPT * SUB_THREADS elements;
+// thread i holds SUB_EPT consecutive elements of one row of each state.
+constexpr int SUBL = 4, SUBN = 1 << SUBL;
+constexpr int SUB_THREADS = 256, SUB_EPT = 8;
+
 template <int D>
-__global__ void __launch_bounds__(THREADS) k_fen_level(Dims dm, Plan pl, FenTree tr, int level,
-                                                       int count, bool bf16) {
-  const int u = blockIdx.y, i = blockIdx.x;
-  if (i >= count) return;
-  const int a = node_id(tr, level - 1, 2 * i), b = node_id(tr, level - 1, 2 * i + 1);
-  const int nid = node_id(tr, level, i);
-  const float *Sa = tr.S + ((size_t)u * tr.nodes + a) * D * D;
-  const float *Sb = tr.S + ((size_t)u * tr.nodes + b) * D * D;
-  float *S = tr.S + ((size_t)u * tr.nodes + nid) * D * D;
-  for (int e = threadIdx.x * 4; e < D * D; e += THREADS * 4) {
-    const float4 x = *reinterpret_cast<const float4 *>(Sa + e);
-    const float4 y = *reinterpret_cast<const float4 *>(Sb + e);
-    *reinterpret_cast<float4 *>(S + e) = make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+__global__ void __launch_bounds__(SUB_THREADS) k_fen_sub(Dims dm, Plan pl, FenTree tr, int base,
+                                                         int nbase, int nslice, bool bf16) {
+  const int u = blockIdx.y;
+  const int sub = blockIdx.x / nslice, slice = blockIdx.x % nslice;
+  const int e0 = (slice * SUB_THREADS + threadIdx.x) * SUB_EPT;  // first element of the thread
+  if (e0 >= D * D) return;
+  const int r = e0 / D, c0 = e0 % D;
+  float acc[SUBL][SUB_EPT];  // pending left child of each level above the base
+  const int first = sub * SUBN;
+  const int last = min(first + SUBN, nbase);
+  for (int j = first; j < last; j++) {
+    float x[SUB_EPT];
+    const float *src = tr.S + ((size_t)u * tr.nodes + node_id(tr, base, j)) * D * D + e0;
+#pragma unroll
+    for (int i = 0; i < SUB_EPT; i += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + i);
+      x[i] = v.x;
+      x[i + 1] = v.y;
+      x[i + 2] = v.z;
+      x[i + 3] = v.w;
+    }
+    // carry: node j closes the node above it at every level where its index
+    // (relative to the subtree) is odd, up to the first even one, where it
+    // waits as a left child
+    const int rel = j - first;
+    bool carry = true;
+#pragma unroll
+    for (int l = 0; l < SUBL; l++) {
+      if (carry) {
+        if ((rel >> l) & 1) {
+#pragma unroll
+          for (int i = 0; i < SUB_EPT; i++) x[i] = acc[l][i] + x[i];
+          const int level = base + l + 1;
+          const int index = j >> (l + 1);  // the node's index at that level
+          const int nid = node_id(tr, level, index);
+          if (l + 1 == SUBL) {  // a subtree root: the next pass's base, in fp32
+            float *dst = tr.S + ((size_t)u * tr.nodes + nid) * D * D + e0;
+#pragma unroll
+            for (int i = 0; i < SUB_EPT; i += 4)
+              *reinterpret_cast<float4 *>(dst + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+          }
+          if ((index & 1) == 0) {  // an atom: its frozen version
+            if (bf16) {
+              uint8_t *Vd = static_cast<uint8_t *>(pl.ver_S) + ((size_t)u * dm.vmax + nid) * D * D * 2;
+              *reinterpret_cast<uint4 *>(Vd + tc::sw128_offset(r, c0, D)) =
+                  make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                             tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+            } else {
+              float *Vd = static_cast<float *>(pl.ver_S) + ((size_t)u * dm.vmax + nid) * D * D + e0;
+#pragma unroll
+              for (int i = 0; i < SUB_EPT; i += 4)
+                *reinterpret_cast<float4 *>(Vd + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < SUB_EPT; i++) acc[l][i] = x[i];
+          carry = false;
+        }
+      }
+    }
   }
-  if (i & 1) return;  // never an atom
-  __syncthreads();
-  write_version<D>(dm, pl, u, nid, S, nullptr, 0.f, bf16, false);
 }
 
 // Per (head, tile): atoms = tree nodes of the blocks of [0, T0-1], events.
@@ -188,10 +243,14 @@ template <int D>
 cudaError_t run_d(const Dims &dm, const Plan &pl, const CallArgs &ca, const FenTree &tr,
                   int ntiles, bool bf16, bool levels, cudaStream_t s) {
   if (levels) {
-    for (int l = 1; l < tr.levels; l++) {
-      const int count = ntiles >> l;
-      if (count <= 0) break;
-      k_fen_level<D><<<dim3(count, dm.heads), THREADS, 0, s>>>(dm, pl, tr, l, count, bf16);
+    // four levels per launch, from the leaves up
+    const int nslice = (D * D + SUB_THREADS * SUB_EPT - 1) / (SUB_THREADS * SUB_EPT);
+    for (int base = 0; base + 1 < tr.levels; base += SUBL) {
+      const int nbase = ntiles >> base;
+      if (nbase < 2) break;
+      const int nsub = (nbase + SUBN - 1) / SUBN;
+      k_fen_sub<D><<<dim3(nsub * nslice, dm.heads), SUB_THREADS, 0, s>>>(dm, pl, tr, base, nbase,
+                                                                        nslice, bf16);
     }
     return cudaGetLastError();
   }
