@@ -21,11 +21,11 @@
 //   P = W o A (causal) as the bf16 A operand of
 //     O_intra = P V                                    TMEM cols [256, 384)
 //   It stores the atom weights W[atom][row] and O_intra (fp32) to the plan.
-// k_readout_tc then runs the pipelined loop over atoms: the epilogue warps
-// start from O_intra and put phi(Q) into tensor memory; per atom alpha, a
-// bulk copy brings the frozen bf16 state version (already in the UMMA K-major
-// swizzled layout) into one of 4 shared stages (3 of their own, then the
-// phi(Q) tile), two threads issue P_alpha = phi(Q) S_alpha^T (even / odd
+// k_readout_tc then runs the pipelined loop over atoms, over a run of
+// consecutive tiles per CTA: the epilogue warps start from O_intra and put
+// phi(Q) into tensor memory; per atom alpha, a bulk copy brings the frozen
+// bf16 state version (already in the UMMA K-major swizzled layout) into one
+// of 5 shared stages, two threads issue P_alpha = phi(Q) S_alpha^T (even / odd
 // atoms) into three TMEM buffers with phi(Q) read from tensor memory, and 8
 // epilogue warps accumulate W_alpha(t) * P_alpha in registers while the next
 // MMAs run.
@@ -39,8 +39,7 @@ using namespace tc;
 
 constexpr int M = 128;
 constexpr int D = 128;
-constexpr int NST = 3;   // version stages of their own
-constexpr int NSV = 4;   // + the phi(Q) tile once it is in tensor memory
+constexpr int NSV = 5;   // version stages of the atom loop
 constexpr int THREADS = 384;      // atom loop
 constexpr int PRE_THREADS = 256;  // per-tile prologue
 constexpr int TILE_BYTES = M * D * 2;
@@ -49,10 +48,11 @@ constexpr int BW = 8;  // epoch bitmask words: atoms + pieces <= 256
 constexpr uint32_t COL_AI = 256;  // phi(Q) of the atom loop
 constexpr int NPB = 3;  // TMEM P buffers: cols [0,128), [128,256) and [384,512)
 __device__ __forceinline__ uint32_t pbuf_col(int b) { return b == 2 ? 384u : (uint32_t)b * 128u; }
-// phi(Q) as the A operand of the atom MMAs, in tensor memory: elements
-// [64h, 64h + 64) of a row in cols COL_AI + 64h + [0, 32), two per column
-__device__ __forceinline__ uint32_t qa_col(int kstep) {
-  return COL_AI + (kstep < 4 ? 8 * kstep : 64 + 8 * (kstep - 4));
+// phi(Q) as the A operand of the atom MMAs, in tensor memory, in one of two
+// regions (par, alternating by tile): elements [64h, 64h + 64) of a row in
+// cols COL_AI + 32 par + 64h + [0, 32), two per column
+__device__ __forceinline__ uint32_t qa_col(int kstep, int par) {
+  return COL_AI + 32 * par + (kstep < 4 ? 8 * kstep : 64 + 8 * (kstep - 4));
 }
 constexpr float INV_SQRT_D = 0.08838834764831845f;
 // Tensor memory of the prologue (256 columns, two CTAs per SM): A, then P in
@@ -92,15 +92,19 @@ struct PreSmem {
 
 static_assert(offsetof(PreSmem, mu) == offsetof(PreSmem, q) + TILE_BYTES, "q, mu adjacent");
 
+// Shared memory of the persistent atom loop: the phi(Q) landing buffer, NSV
+// version stages and a ring of NWC weight chunks of WCH atoms.
+constexpr int NWC = 2, WCH = 32;
 struct Smem {
-  uint8_t q[TILE_BYTES];  // phi(Q) on its way to tensor memory, then version stage NST
-  uint8_t st[NST][VER_BYTES];
-  float w[128 * M];       // W[atom][row] of 128 atoms at a time
-  uint64_t bar_load, bar_w, bar_qa, full[NSV], empty[NSV], tfull[NPB], tempty[NPB];
+  uint8_t q[TILE_BYTES];  // phi(Q) of a tile, on its way to tensor memory
+  uint8_t st[NSV][VER_BYTES];
+  float w[NWC][WCH * M];  // W[atom][row] of WCH atoms per chunk
+  uint64_t bar_load, bar_qa, bar_qs, full[NSV], empty[NSV], tfull[NPB], tempty[NPB], wfull[NWC],
+      wempty[NWC];
   uint32_t tmem_base;
   int abort;
-  int atom[128];
 };
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "atom loop shared memory");
 
 __device__ __forceinline__ bool bit_of(const uint32_t *b, int i) { return (b[i >> 5] >> (i & 31)) & 1u; }
 
@@ -780,31 +784,44 @@ __global__ void __launch_bounds__(PRE_THREADS, 2)
   if (tid == 0 && sm.abort) set_status(ca.dev_status, DLA_ERR_TIMEOUT);
 }
 
+// The atom loop: each CTA walks a run of consecutive tiles of one head.
+// Tensor memory is allocated and the barriers set up once per run; stage,
+// product-buffer and weight-chunk phases follow cumulative counters over the
+// run's tiles, so each role runs ahead into the next tile as far as its
+// barriers let it.  phi(Q) has a landing buffer of its own and two
+// tensor-memory regions (by tile parity): the next tile's phi(Q) loads while
+// this tile's MMAs run, and the epilogue moves it into tensor memory as soon
+// as it starts that tile.  The prologue's weights stream through a ring of
+// WCH-atom chunks; its intra-tile output is the accumulator's start.  The
+// producer also prefetches the run's next tile (weights, intra-tile output,
+// first versions) into L2.
 __global__ void __launch_bounds__(THREADS, 1)
-    k_readout_tc(const __grid_constant__ CUtensorMap tq, Dims dm, Plan pl, CallArgs ca) {
+    k_readout_tc(const __grid_constant__ CUtensorMap tq, Dims dm, Plan pl, CallArgs ca, int run) {
   extern __shared__ uint8_t raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                        ~static_cast<uintptr_t>(1023));
-  const int u = blockIdx.y, c = blockIdx.x;
-  const int T0 = c * M;
-  const int Tw = tw_of(ca, u);
-  if (T0 >= Tw) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int *abort = &sm.abort;
-  auto stage = [&](int s) -> uint8_t * {
-    return s < NST ? sm.st[s] : sm.q;
+  // this CTA's run: tiles [c0, c0 + run) of head u (flat index gi = u tiles + c)
+  const int runs = (dm.tiles + run - 1) / run;
+  const int u = blockIdx.x / runs, c0 = (blockIdx.x % runs) * run;
+  const int G = u * dm.tiles + min(dm.tiles, c0 + run);  // one past the run
+  const int Tw = tw_of(ca, u);
+  // the run's next tile from gi on; a tile at or past the stream's length has
+  // no rows, nor has any later one
+  auto next_tile = [&](int gi) -> int {
+    return gi < G && (gi - u * dm.tiles) * M < Tw ? gi : G;
   };
-  const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
-  const size_t g = (size_t)u * dm.tiles + c;
-  const int m0 = pl.tile_m0[g];
-  const int len = min(M, Tw - T0);
 
-  // ---- setup: TMEM, barriers, the phi(Q) tile and the prologue's weights ----
+  const int first = next_tile(u * dm.tiles + c0);
+  if (first >= G) return;  // the whole run lies past the stream's length
+
+  // ---- setup (once): TMEM, barriers, the first tile's phi(Q) ----------------
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
   if (tid == 0) {
     mbar_init(&sm.bar_load, 1);
-    mbar_init(&sm.bar_w, 1);
     mbar_init(&sm.bar_qa, 8);
+    mbar_init(&sm.bar_qs, 2);
     for (int i = 0; i < NSV; i++) {
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
@@ -813,161 +830,207 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.tfull[i], 1);
       mbar_init(&sm.tempty[i], 8);
     }
+    for (int i = 0; i < NWC; i++) {
+      mbar_init(&sm.wfull[i], 1);
+      mbar_init(&sm.wempty[i], 8);
+    }
     fence_mbar_init();
     sm.abort = 0;
-    const uint32_t wbytes = (uint32_t)min(m0, 128) * M * 4;  // the first 128 atoms' weights
-    mbar_expect_tx(&sm.bar_load, TILE_BYTES + wbytes);
+    mbar_expect_tx(&sm.bar_load, TILE_BYTES);
     for (int h = 0; h < 2; h++)
-      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, T0, u);
-    if (m0 > 0) bulk_load(sm.w, pl.pre_w + g * dm.amax * M, wbytes, &sm.bar_load);
+      tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, (first - u * dm.tiles) * M, u);
   }
-  const int32_t *const atoms_g = pl.tile_atoms + g * dm.amax;
-  for (int a = tid; a < m0 && a < 128; a += THREADS) sm.atom[a] = atoms_g[a];
-  // the version of atom a (beyond 128 atoms, only the unbounded policy, read
-  // from the plan)
-  auto atom_at = [&](int a) -> int { return a < 128 ? sm.atom[a] : atoms_g[a]; };
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  if (tid == 0) {
-    for (int a = 0; a < m0 && a < NST; a++) {
-      mbar_expect_tx(&sm.full[a], VER_BYTES);
-      bulk_load(sm.st[a], verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES, &sm.full[a]);
-    }
-  }
   auto kdesc = [](uint32_t base, int k) {  // K-major SW128, 128 rows per half
     return sdesc(base + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 32, 16, 1024);
   };
 
-  // ---- the pipelined readout over atoms --------------------------------------
-  // Two issuing threads (warp 1: even atoms, warp 2: odd atoms); an issuing
-  // thread is held for about the duration of its MMAs, so with one issuer
-  // every barrier wait left the tensor pipe idle.  The atom MMAs read phi(Q)
-  // from tensor memory: with both operands in shared memory, their reads plus
-  // the version copies exceeded its bandwidth.  Atom a goes to product buffer
-  // a % 3: three buffers cover a buffer's round trip (MMAs, commit, epilogue
-  // drain, release) at the MMA rate.
-  auto issue_atoms = [&](int first) {
-    bool ok_qa = first < m0 ? mbar_wait(&sm.bar_qa, 0, abort) : true;
-    for (int a = first; a < m0; a += 2) {
-      const int s = a % NSV, b = a % NPB;
-      bool ok = mbar_wait(&sm.full[s], (a / NSV) & 1, abort) && ok_qa;
-      if (a >= NPB) ok = mbar_wait(&sm.tempty[b], ((a / NPB) - 1) & 1, abort) && ok;
-      tc_fence_after();
-      if (ok) {
-        const uint32_t st_s = smem_u32(stage(s));
-        for (int k = 0; k < 8; k++)
-          mma_bf16_ta(tbase + pbuf_col(b), tbase + qa_col(k), kdesc(st_s, k),
-                      idesc_bf16(M, 128, 0, 0), k > 0);
-      }
-      mma_commit(&sm.empty[s]);
-      mma_commit(&sm.tfull[b]);
-    }
-  };
-  if (warp == 1 && lane == 0) {
-    tc_fence_after();
-    issue_atoms(0);
-  } else if (warp == 2 && lane == 0) {
-    tc_fence_after();
-    issue_atoms(1);
-  } else if (warp == 0 && lane == 0) {
-    // L2 prefetch PF atoms ahead of the stage loads: versions were just
-    // written by the materializer, so a head's first tiles mostly miss L2
+  if (warp == 0 && lane == 0) {
+    // ---- producer: versions (L2 prefetch PF atoms ahead), weight chunks,
+    // and the next tile's phi(Q) once this tile's is in tensor memory -------
     constexpr int PF = 6;
-    for (int a = NST; a < m0 && a < NST + PF; a++)
-      bulk_prefetch_l2(verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES);
-    for (int a = NST; a < m0; a++) {
-      if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)atom_at(a + PF) * VER_BYTES, VER_BYTES);
-      const int s = a % NSV;
-      // stage NST is the phi(Q) tile: free once every epilogue warp has put
-      // its rows into tensor memory (bar_qa)
-      const bool ok = a >= NSV ? mbar_wait(&sm.empty[s], ((a / NSV) - 1) & 1, abort)
-                               : mbar_wait(&sm.bar_qa, 0, abort);
-      if (!ok) break;
-      mbar_expect_tx(&sm.full[s], VER_BYTES);
-      bulk_load(stage(s), verS + (size_t)atom_at(a) * VER_BYTES, VER_BYTES, &sm.full[s]);
+    // a tile's weights, intra-tile output and first versions, into L2 a tile
+    // ahead of their loads
+    auto prefetch_tile = [&](int gp) {
+      if (gp >= G) return;
+      const int mp = pl.tile_m0[gp];
+      if (mp > 0) bulk_prefetch_l2(pl.pre_w + (size_t)gp * dm.amax * M, (uint32_t)mp * M * 4);
+      bulk_prefetch_l2(static_cast<const uint8_t *>(pl.pre_o) + (size_t)gp * M * D * 2, M * D * 2);
+      const int32_t *ap = pl.tile_atoms + (size_t)gp * dm.amax;
+      const uint8_t *vp = static_cast<const uint8_t *>(pl.ver_S) +
+                          (size_t)u * dm.vmax * VER_BYTES;
+      for (int a = 0; a < mp && a < PF; a++) bulk_prefetch_l2(vp + (size_t)ap[a] * VER_BYTES, VER_BYTES);
+    };
+    uint32_t A0 = 0, W0 = 0;
+    int it = 0;
+    for (int gi = first; gi < G; gi = next_tile(gi + 1), it++) {
+      const int m0 = pl.tile_m0[gi];
+      const int32_t *atoms = pl.tile_atoms + (size_t)gi * dm.amax;
+      const uint8_t *verS = static_cast<const uint8_t *>(pl.ver_S) + (size_t)u * dm.vmax * VER_BYTES;
+      const float *wsrc = pl.pre_w + (size_t)gi * dm.amax * M;
+      if (it == 0) prefetch_tile(gi);
+      prefetch_tile(next_tile(gi + 1));
+      bool qdone = false;
+      auto next_q = [&]() {  // the next tile's phi(Q), once this one's is moved
+        qdone = true;
+        const int gn = next_tile(gi + 1);
+        if (gn >= G) return;
+        // the landing buffer is free once this tile's phi(Q) is in tensor
+        // memory, and both issuers must have seen that before the barrier
+        // can complete again (an issuer with no atoms in a tile still takes
+        // its phase, so its parity waits never fall two phases behind)
+        if (!mbar_wait(&sm.bar_qa, it & 1, abort) || !mbar_wait(&sm.bar_qs, it & 1, abort)) return;
+        mbar_expect_tx(&sm.bar_load, TILE_BYTES);
+        for (int h = 0; h < 2; h++)
+          tma_load_3d(sm.q + h * (TILE_BYTES / 2), &tq, &sm.bar_load, h * 64, (gn - u * dm.tiles) * M, u);
+      };
+      for (int a = 0; a < m0; a++) {
+        if (a % WCH == 0) {
+          const uint32_t k = W0 + a / WCH;
+          const int w = (int)(k % NWC);
+          if (k >= NWC && !mbar_wait(&sm.wempty[w], (int)((k / NWC) - 1) & 1, abort)) break;
+          const uint32_t nb = (uint32_t)min(WCH, m0 - a) * M * 4;
+          mbar_expect_tx(&sm.wfull[w], nb);
+          bulk_load(sm.w[w], wsrc + (size_t)a * M, nb, &sm.wfull[w]);
+        }
+        if (a + PF < m0) bulk_prefetch_l2(verS + (size_t)atoms[a + PF] * VER_BYTES, VER_BYTES);
+        const uint32_t x = A0 + a;
+        const int s = (int)(x % NSV);
+        if (x >= NSV && !mbar_wait(&sm.empty[s], (int)((x / NSV) - 1) & 1, abort)) break;
+        mbar_expect_tx(&sm.full[s], VER_BYTES);
+        bulk_load(sm.st[s], verS + (size_t)atoms[a] * VER_BYTES, VER_BYTES, &sm.full[s]);
+        if (a == NSV - 1) next_q();
+      }
+      if (!qdone) next_q();
+      A0 += m0;
+      W0 += (m0 + WCH - 1) / WCH;
+    }
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // ---- two MMA issuers: even / odd atoms of the CTA's running count ------
+    // (an issuing thread is held for about the duration of its MMAs, so with
+    // one issuer every barrier wait left the tensor pipe idle).  Atom x goes
+    // to product buffer x % 3: three buffers cover a buffer's round trip
+    // (MMAs, commit, epilogue drain, release) at the MMA rate.
+    tc_fence_after();
+    const int par_i = warp - 1;
+    uint32_t A0 = 0;
+    int it = 0;
+    for (int gi = first; gi < G; gi = next_tile(gi + 1), it++) {
+      const int m0 = pl.tile_m0[gi];
+      // every tile's phi(Q) phase is taken, atoms or not, and acknowledged
+      const bool ok_qa = mbar_wait(&sm.bar_qa, it & 1, abort);
+      mbar_arrive(&sm.bar_qs);
+      {
+        int a = (int)((par_i - (A0 & 1) + 2) & 1);  // first atom of this issuer's parity
+        for (; a < m0; a += 2) {
+          const uint32_t x = A0 + a;
+          const int s = (int)(x % NSV), b = (int)(x % NPB);
+          bool ok = mbar_wait(&sm.full[s], (int)(x / NSV) & 1, abort) && ok_qa;
+          if (x >= NPB) ok = mbar_wait(&sm.tempty[b], (int)((x / NPB) - 1) & 1, abort) && ok;
+          tc_fence_after();
+          if (ok) {
+            const uint32_t st_s = smem_u32(sm.st[s]);
+            for (int k = 0; k < 8; k++)
+              mma_bf16_ta(tbase + pbuf_col(b), tbase + qa_col(k, it & 1), kdesc(st_s, k),
+                          idesc_bf16(M, 128, 0, 0), k > 0);
+          }
+          mma_commit(&sm.empty[s]);
+          mma_commit(&sm.tfull[b]);
+        }
+      }
+      A0 += m0;
     }
   } else if (warp >= 4) {
+    // ---- 8 epilogue warps: row t = 32 qd + lane, columns [64 hc, 64 hc + 64)
     const int qd = warp & 3, hc = (warp - 4) >> 2;
     const int t = 32 * qd + lane;
     const uint32_t trow = tbase + ((uint32_t)(32 * qd) << 16);
-    float acc[64];
-    {  // start from the intra-tile output
-      const uint4 *src = reinterpret_cast<const uint4 *>(pl.pre_o) + g * (M * D / 8);
+    uint32_t A0 = 0, W0 = 0;
+    int it = 0;
+    for (int gi = first; gi < G; gi = next_tile(gi + 1), it++) {
+      const int c = gi - u * dm.tiles;
+      const int T0 = c * M;
+      const int len = min(M, tw_of(ca, u) - T0);
+      const int m0 = pl.tile_m0[gi];
+      // the intra-tile output, the accumulator's start (in flight during the
+      // phi(Q) move)
+      const uint4 *src = reinterpret_cast<const uint4 *>(pl.pre_o) + (size_t)gi * (M * D / 8);
+      uint4 po[8];
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint4 x = src[pre_o_chunk(t, hc, i)];
-        acc[8 * i] = bf16_lo(x.x);
-        acc[8 * i + 1] = bf16_hi(x.x);
-        acc[8 * i + 2] = bf16_lo(x.y);
-        acc[8 * i + 3] = bf16_hi(x.y);
-        acc[8 * i + 4] = bf16_lo(x.z);
-        acc[8 * i + 5] = bf16_hi(x.z);
-        acc[8 * i + 6] = bf16_lo(x.w);
-        acc[8 * i + 7] = bf16_hi(x.w);
-      }
-    }
-    mbar_wait(&sm.bar_load, 0, abort);
-    {
-      // row t, elements [64 hc, 64 hc + 64) of phi(q_t), from the swizzled tile
-      uint32_t qw[32];
+      for (int i = 0; i < 8; i++) po[i] = src[pre_o_chunk(t, hc, i)];
+      // this tile's phi(Q) rows into its tensor-memory region (the region's
+      // last reader, tile it - 2, is done: this warp drained all its products)
+      mbar_wait(&sm.bar_load, it & 1, abort);
+      {
+        uint32_t qw[32];
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(sm.q + sw128_offset(t, 64 * hc + 8 * i, M));
-        qw[4 * i] = x.x;
-        qw[4 * i + 1] = x.y;
-        qw[4 * i + 2] = x.z;
-        qw[4 * i + 3] = x.w;
-      }
-      DLA_TMEM_ST32(trow + COL_AI + 64 * hc, qw);
-      tmem_wait_st();
-    }
-    // the tile's shared copy is read (it becomes a version stage)
-    fence_proxy_async();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.bar_qa);
-    const float *sW = sm.w;
-#pragma unroll 1
-    for (int a = 0; a < m0; a++) {
-      const int b = a % NPB;
-      if (a > 0 && (a & 127) == 0) {
-        // the next 128 atoms' weights replace the last ones (the epilogue
-        // warps alone read them: a named barrier over those 256 threads)
-        fence_proxy_async();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (warp == 4 && lane == 0) {
-          const uint32_t nb = (uint32_t)min(128, m0 - a) * M * 4;
-          mbar_expect_tx(&sm.bar_w, nb);
-          bulk_load(sm.w, pl.pre_w + g * dm.amax * M + (size_t)a * M, nb, &sm.bar_w);
+        for (int i = 0; i < 8; i++) {
+          const uint4 x = *reinterpret_cast<const uint4 *>(sm.q + sw128_offset(t, 64 * hc + 8 * i, M));
+          qw[4 * i] = x.x;
+          qw[4 * i + 1] = x.y;
+          qw[4 * i + 2] = x.z;
+          qw[4 * i + 3] = x.w;
         }
-        mbar_wait(&sm.bar_w, ((a >> 7) - 1) & 1, abort);
+        DLA_TMEM_ST32(trow + COL_AI + 32 * (it & 1) + 64 * hc, qw);
+        tmem_wait_st();
       }
-      const float w = sW[(a & 127) * M + t];
-      mbar_wait(&sm.tfull[b], (a / NPB) & 1, abort);
-      tc_fence_after();
-      uint32_t pr[32];
-      DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64, pr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i++) acc[i] = fmaf(w, __uint_as_float(pr[i]), acc[i]);
-      DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64 + 32, pr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(w, __uint_as_float(pr[i]), acc[32 + i]);
+      // the landing buffer is read (the next tile's phi(Q) may overwrite it)
+      fence_proxy_async();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.tempty[b]);
-    }
-    if (t < len) {
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(ca.o) +
-                                             ((size_t)u * dm.T + ca.w0 + T0 + t) * D + hc * 64);
+      if (lane == 0) mbar_arrive(&sm.bar_qa);
+      float acc[64];
 #pragma unroll
-      for (int ch = 0; ch < 8; ch++)
-        dst[ch] = make_uint4(pack_bf16(acc[8 * ch], acc[8 * ch + 1]),
-                             pack_bf16(acc[8 * ch + 2], acc[8 * ch + 3]),
-                             pack_bf16(acc[8 * ch + 4], acc[8 * ch + 5]),
-                             pack_bf16(acc[8 * ch + 6], acc[8 * ch + 7]));
+      for (int i = 0; i < 8; i++) {
+        acc[8 * i] = bf16_lo(po[i].x);
+        acc[8 * i + 1] = bf16_hi(po[i].x);
+        acc[8 * i + 2] = bf16_lo(po[i].y);
+        acc[8 * i + 3] = bf16_hi(po[i].y);
+        acc[8 * i + 4] = bf16_lo(po[i].z);
+        acc[8 * i + 5] = bf16_hi(po[i].z);
+        acc[8 * i + 6] = bf16_lo(po[i].w);
+        acc[8 * i + 7] = bf16_hi(po[i].w);
+      }
+#pragma unroll 1
+      for (int a = 0; a < m0; a++) {
+        const uint32_t k = W0 + a / WCH;
+        const int w = (int)(k % NWC);
+        if (a % WCH == 0) mbar_wait(&sm.wfull[w], (int)(k / NWC) & 1, abort);
+        const float wt = sm.w[w][(a % WCH) * M + t];
+        const uint32_t x = A0 + a;
+        const int b = (int)(x % NPB);
+        mbar_wait(&sm.tfull[b], (int)(x / NPB) & 1, abort);
+        tc_fence_after();
+        uint32_t pr[32];
+        DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64, pr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i++) acc[i] = fmaf(wt, __uint_as_float(pr[i]), acc[i]);
+        DLA_TMEM_LD32(trow + pbuf_col(b) + hc * 64 + 32, pr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i++) acc[32 + i] = fmaf(wt, __uint_as_float(pr[i]), acc[32 + i]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&sm.tempty[b]);
+          if (a % WCH == WCH - 1 || a == m0 - 1) mbar_arrive(&sm.wempty[w]);
+        }
+      }
+      // the tile's rows
+      if (t < len) {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(ca.o) +
+                                               ((size_t)u * dm.T + ca.w0 + T0 + t) * D + hc * 64);
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+          dst[i] = make_uint4(pack_bf16(acc[8 * i], acc[8 * i + 1]), pack_bf16(acc[8 * i + 2], acc[8 * i + 3]),
+                              pack_bf16(acc[8 * i + 4], acc[8 * i + 5]),
+                              pack_bf16(acc[8 * i + 6], acc[8 * i + 7]));
+      }
+      A0 += m0;
+      W0 += (m0 + WCH - 1) / WCH;
     }
   }
   tc_fence_before();
@@ -1058,8 +1121,16 @@ cudaError_t launch_readout_tc(const Dims &dm, const Plan &pl, const CallArgs &ca
   cudaError_t e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sb);
   if (e != cudaSuccess) return e;
-  dim3 g(dm.tiles, dm.heads);
-  k_readout_tc<<<g, THREADS, sb, s>>>(tq, dm, pl, ca);
+  // tiles per CTA: the CTAs in flight then cover run x (SM count) tiles, and
+  // the versions those tiles read must stay in L2.  A dynamic-policy head
+  // holds thousands of versions and one tile per CTA keeps the working set
+  // to about two heads' tiles in flight (longer runs measured slower: 0.67
+  // of the tensor peak at 1 tile per CTA, 0.63 at 4, 0.57 at 8 on the
+  // T = 8192 prefill); the fixed policy's few versions per head leave room
+  // for runs of 4, which save the per-CTA setup (0.21 -> 0.24)
+  const int run = dm.fenwick ? 4 : 1;
+  const int runs = (dm.tiles + run - 1) / run;
+  k_readout_tc<<<dm.heads * runs, THREADS, sb, s>>>(tq, dm, pl, ca, run);
   return cudaGetLastError();
 }
 

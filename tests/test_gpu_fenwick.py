@@ -28,3 +28,13 @@ def test_fenwick_simt(gpu, d, dtype):
     q, k, v = case(2, 2, 777, d, dtype, seed=d)
     ref = oracle_run(q, k, v, 2, 0.5, dtype, policy="fenwick")
     assert rel_err(run(q, k, v, dtype), ref["out"]) <= TOL[dtype]
+
+
+def test_fenwick_more_tiles_than_sms(gpu):
+    """160 streams x 8 tiles: the atom loop's CTAs each walk about nine tiles
+    whose atom counts (the popcounts of the tile indices) run 0, 1, 1, 2, ...
+    so a CTA often meets a tile with no atom or one between busier ones."""
+    q, k, v = case(4, 40, 1024, 128, "bf16", seed=5)
+    ref = oracle_run(q, k, v, 2, 0.5, "bf16", policy="fenwick")
+    assert rel_err(run(q, k, v, "bf16"), ref["out"]) <= TOL["bf16"]
+

@@ -115,3 +115,12 @@ def test_cuda_graph_capture_and_replay(gpu, window):
     ref = oracle_run(q, k, v, C, tau, "bf16")
     assert tr.merges() == ref["merges"]
     assert rel_err(from_device(o), ref["out"]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("mean_len", [3.0, 40.0])
+def test_more_tiles_than_sms(gpu, mean_len):
+    """160 streams x 5 tiles: the atom loop's CTAs each walk several tiles,
+    many of them with no atom or one (the first tile of every stream)."""
+    q, k, v = case(4, 40, 640, 128, "bf16", seed=int(mean_len) + 90, mean_len=mean_len)
+    check(q, k, v, 4, 0.5)
+

@@ -177,3 +177,13 @@ def test_masked_decode_steps(gpu):
                 want.append(r["out"][0, 0])
             pos[n] += 1
     assert rel_err(np.stack(got), np.stack(want)) <= TOL["bf16"]
+
+
+def test_ragged_more_tiles_than_sms(gpu):
+    """40 sequences of 0 to 1000 tokens x 8 heads (over 148 tiles in all, with
+    empty and partial ones): the atom loop skips every tile past a length."""
+    rng = np.random.default_rng(5)
+    lens = [0, 1000, 129, 1] + [int(x) for x in rng.integers(0, 1001, size=36)]
+    q, k, v = case(len(lens), 8, 1000, 128, "bf16", seed=57, mean_len=12.0)
+    check(q, k, v, lens, 8, 0.5, "bf16", "dla")
+
