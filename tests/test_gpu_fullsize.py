@@ -68,16 +68,35 @@ def gpu_prefill(q, k, v, C, tau):
     return from_device(o), tr
 
 
-@pytest.mark.parametrize("name,heads", [
-    ("prefill_t8192", [(0, 0), (3, 15)]),
-    ("prefill_t131072", [(0, 0), (0, 11)]),
-])
-def test_prefill_full_size(gpu, name, heads):
+@pytest.mark.parametrize("name", ["prefill_t8192", "prefill_t131072"])
+def test_prefill_full_size(gpu, name):
+    """Every stream: the trace bit for bit, and the outputs at the sampled
+    tokens (one threaded oracle run gives both).  The error distribution over
+    all compared elements (|o - ref| / max|ref| of the stream) is printed; at
+    T = 131072 and C = 128 the readout sums the most terms."""
     wl = synth.WORKLOADS[name]
     q, k, v = gen_prefill_parallel(wl)
-    o, tr = gpu_prefill(q, k, v, wl["C"], wl["tau"])
-    check_trace(tr, k, wl["C"], wl["tau"])
-    check_outputs(o, q, k, v, wl["C"], wl["tau"], "dla", heads, wl["seed"])
+    B, H, T, d = k.shape
+    C, tau = wl["C"], wl["tau"]
+    o, tr = gpu_prefill(q, k, v, C, tau)
+    mask = sample_mask(T, wl["seed"])
+    orc = O.Oracle(B * H, d, d, C)
+    res = orc.run(k.reshape(B * H, T, d), q.reshape(B * H, T, d), v.reshape(B * H, T, d),
+                  tau=tau, dtype="bf16", out_mask=mask)
+    gap = float(res["margins"][:, 1].min())
+    assert np.array_equal(tr.boundary.cpu().numpy().reshape(B * H, T), res["boundary"]), gap
+    assert tr.merges() == res["merges"], gap
+    sel = mask.astype(bool)
+    ref = res["out"][:, sel]
+    got = o.reshape(B * H, T, d)[:, sel]
+    rel = np.abs(got - ref) / np.abs(ref).max(axis=(1, 2))[:, None, None]
+    per_stream = rel.max(axis=(1, 2))
+    qs = np.quantile(rel, [0.5, 0.99, 0.999])
+    summary = (f"{name}: {B * H} streams x {int(sel.sum())} tokens; |o - ref| / max|ref|: median "
+               f"{qs[0]:.2e}, p99 {qs[1]:.2e}, p99.9 {qs[2]:.2e}, max {per_stream.max():.2e} "
+               f"(stream {int(per_stream.argmax())})")
+    print(summary)
+    assert per_stream.max() <= TOL["bf16"], summary
 
 
 def test_fixed_policy_full_size(gpu):
