@@ -763,11 +763,13 @@ def bench_decode(args, wl, rank, world, local_rank):
     }
 
 
-def oracle_decode(wl, pre, stp, steps, cores, streams=16, prefill_tokens=4096):
+def oracle_decode(wl, pre, stp, steps, cores, streams=16, prefill_tokens=4096, total=None):
     """Oracle decode on a bounded sample: `streams` streams pre-filled with
     their workload tokens (untimed; states updated at every token, no
     readout), then `steps` timed single-token steps with full per-token work.
-    Returns (seconds per step for the sample, sample description)."""
+    Returns (seconds per step for the sample, sample description); the
+    description names `total` streams (default: all of `wl`'s) as the
+    extrapolation target."""
     from oracle import oracle as O
     N, H, d = wl["B"], wl["H"], wl["d"]
     U = min(streams, N * H)
@@ -788,8 +790,9 @@ def oracle_decode(wl, pre, stp, steps, cores, streams=16, prefill_tokens=4096):
                 np.ascontiguousarray(sv[i, :U, None]), tau=wl["tau"], dtype="bf16",
                 nthreads=cores)
     dt = (time.perf_counter() - t0) / n
+    total = N * H if total is None else total
     return dt, U, (f"{U} streams pre-filled with {Tp} tokens (untimed), {n} timed steps; "
-                   f"steps/s extrapolated to {N * H} streams")
+                   f"steps/s extrapolated to {total} streams")
 
 
 def cpu_baseline_decode(wl, pre, stp, steps=8):
@@ -857,7 +860,8 @@ def bench_reference(args, wl):
             for j, (p_, s_) in enumerate(((stv.q, sq_), (stv.k, sk_), (stv.v, sv_))):
                 pre[j][0, i] = synth.to_bf16_bits(p_)
                 stp[j][:, 0, i] = synth.to_bf16_bits(s_)
-        dt, Us, dsample = oracle_decode(dict(dwl, B=1, H=U), pre, stp, nst, cores, streams=U)
+        dt, Us, dsample = oracle_decode(dict(dwl, B=1, H=U), pre, stp, nst, cores, streams=U,
+                                        total=dwl["B"] * dwl["H"])
         dval = 1.0 / (dt * (dwl["B"] * dwl["H"]) / Us)
         line["decode"] = {"value": round(dval, 6), "unit": "steps/s",
                           "ms_per_step": round(1e3 / dval, 3),
