@@ -90,6 +90,27 @@ def test_reference_arm_prints_on_rank0_only(rank):
         assert lines == []
 
 
+def test_reference_arm_decode_half():
+    """On the headline workload the reference arm also times the metric's
+    decode half: a 16-stream sample of decode_n256, extrapolated to its 4096
+    streams (value and description agree)."""
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "prefill_t8192", "--steps", "1", "--warmup", "3",
+                        "--ref-tokens", "32"],
+                       env=env, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    dec = json.loads(lines[0])["decode"]
+    assert dec["unit"] == "steps/s" and dec["value"] > 0
+    assert abs(dec["ms_per_step"] - 1e3 / dec["value"]) <= 1e-3 * dec["ms_per_step"] + 1e-3
+    assert "16 streams" in dec["cpu_baseline"]["sample"]
+    assert "extrapolated to 4096 streams" in dec["cpu_baseline"]["sample"]
+
+
 def test_gpus_flag_must_match_world_size():
     """Under an outer launcher, --gpus N must equal WORLD_SIZE (no silent
     single replica)."""
