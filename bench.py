@@ -608,6 +608,114 @@ def cpu_baseline_prefill(wl, q, k, v, target_s=15.0, policy="dla"):
                       f"Mtok/s = head-tokens/s / H ({t_used:.1f} s)"}
 
 
+# ----------------------------------------------------------- backward arm ----
+
+def backward_flops(T, d, heads):
+    """The masked form's products per stream: every (t, s <= t) pair takes
+    phi(q_t).phi(k_s), dO_t.v_s and dphi(q_t)'s term in the row pass, and the
+    two dot products again plus dv_s's and dphi(k_s)'s terms in the column
+    pass: 7 d T (T + 1) FLOP (2 per multiply-add)."""
+    return 7.0 * d * T * (T + 1) * heads
+
+
+def bench_backward(args, wl, rank, world, local_rank):
+    """dla_prefill_backward at the decisions of one traced dla_prefill
+    (untimed): each step is one call (its three kernels) over the batch."""
+    import torch
+    from dynamic_state_memory_b200 import dla
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    peaks, peaks_kind = load_peaks()
+    B, H, T, d, C = wl["B"], wl["H"], wl["T"], wl["d"], wl["C"]
+    dt = wl["dtype"]
+    q_h, k_h, v_h = make_inputs(wl, rank)
+    do32 = np.random.default_rng([wl["seed"], 7, rank]).standard_normal(q_h.shape).astype(np.float32)
+    from dynamic_state_memory_b200 import synth
+    do_h = synth.to_bf16_bits(do32) if dt == "bf16" else do32
+    q, k, v, d_o = (to_torch(x, dt, dev) for x in (q_h, k_h, v_h, do_h))
+    cache = dla.Cache(B, H, C, d, device=dev)
+    _, tr = dla.prefill(q, k, v, cache, wl["tau"])
+    dcode = dla.DLA_BF16 if dt == "bf16" else dla.DLA_F32
+    cfg = dla.make_config(B, H, T, d, C, wl["tau"], dcode)
+    ws = torch.empty(dla.dla_backward_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    dq, dk, dv = (torch.empty(B, H, T, d, dtype=torch.float32, device=dev) for _ in range(3))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dla.dla_prefill_backward(cfg, q, k, v, d_o, tr.c, dq, dk, dv, ws, st, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(local_rank)
+    if rank == 0:
+        clk.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = clk.stop() if rank == 0 else None
+    dla.check_device_status(st, "dla_prefill_backward")
+    ms_step = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+    if rank != 0:
+        return None
+    flops = backward_flops(T, d, B * H)
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline_backward(
+        wl, q_h, k_h, v_h, do_h, target_s=min(args.cpu_seconds, 8.0))
+    return {
+        "metric": METRIC, "value": round(B * T * world / (ms_step * 1e-3) / 1e6, 4),
+        "unit": "Mtok/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "H": H, "T": T, "d": d, "C": C,
+                   "tau": wl["tau"], "input_dtype": dt, "path": "simt",
+                   "l2": "q, k, v, dO %d MiB; the kernels re-read them from L2" %
+                         (4 * q_h.nbytes >> 20),
+                   "flops_per_step": flops},
+        "roofline": {"kernel": "backward (3 kernels)", "bound": "alu",
+                     "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock "
+                                    "(derived)"},
+        "cpu_baseline": cpu, "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks,
+    }
+
+
+def cpu_baseline_backward(wl, q, k, v, d_o, target_s=8.0):
+    """The oracle's gradient (oracle/backward.py, BLAS held to one thread) on
+    the first streams of the workload, full length, until target_s of work;
+    the C oracle's forward gives each stream's trace (untimed)."""
+    from threadpoolctl import threadpool_limits
+    from dynamic_state_memory_b200 import synth
+    from oracle import backward as BW
+    from oracle import oracle as O
+    B, H, T, d = wl["B"], wl["H"], wl["T"], wl["d"]
+    w = lambda x: synth.widen(x, wl["dtype"])
+    used, heads = 0.0, 0
+    with threadpool_limits(1):
+        while heads < B * H and used < target_s:
+            b, h = divmod(heads, H)
+            ref = O.prefill(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1],
+                            C=wl["C"], tau=wl["tau"], dtype=wl["dtype"], want_out=False)
+            t0 = time.perf_counter()
+            BW.backward_head(w(q[b, h]), w(k[b, h]), w(v[b, h]), w(d_o[b, h]),
+                             ref["boundary"][0, 0], ref["merges"][0])
+            used += time.perf_counter() - t0
+            heads += 1
+    return {"value": round(heads * T / used / H / 1e6, 6), "unit": "Mtok/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"oracle gradient, {heads} streams x {T} tokens, one thread; "
+                      f"Mtok/s = stream-tokens/s / H ({used:.1f} s)"}
+
+
 # ------------------------------------------------------------- decode arm ----
 
 def _gen_decode_head(args):
@@ -972,6 +1080,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     if args.workload.startswith("decode"):
         res = bench_decode(args, wl, rank, world, local_rank)
+    elif args.workload.startswith("backward"):
+        res = bench_backward(args, wl, rank, world, local_rank)
     else:
         res = bench_prefill(args, wl, rank, world, local_rank)
         if args.workload == "prefill_t8192" and not args.only:
@@ -989,6 +1099,12 @@ def main():
                 others[name] = guarded(bench_prefill, a, dict(synth.WORKLOADS[name]), rank, world,
                                        local_rank, e2e=False)
                 torch.cuda.empty_cache()
+            a = sub_args(args, "backward_t2048", steps=min(args.steps, 10), warmup=3)
+            a.cpu_seconds = min(args.cpu_seconds, 8.0)
+            others["backward_t2048"] = guarded(bench_backward, a,
+                                               dict(synth.WORKLOADS["backward_t2048"]), rank,
+                                               world, local_rank)
+            torch.cuda.empty_cache()
             if rank == 0:
                 res["decode"] = dec
                 res["configs"] = others

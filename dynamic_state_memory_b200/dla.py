@@ -100,12 +100,17 @@ _lib.dla_decode_step_static.argtypes = [_P(dla_cache), c_f32, c_i32, c_vp, c_vp,
 _lib.dla_fixed_policy_prefill.restype = c_i32
 _lib.dla_fixed_policy_prefill.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, c_vp, c_size,
                                           c_vp, c_vp]
+_lib.dla_backward_workspace_bytes.restype = c_size
+_lib.dla_backward_workspace_bytes.argtypes = [_P(dla_config)]
+_lib.dla_prefill_backward.restype = c_i32
+_lib.dla_prefill_backward.argtypes = [_P(dla_config), c_vp, c_vp, c_vp, c_vp, _P(dla_trace), c_vp,
+                                      c_vp, c_vp, c_vp, c_size, c_vp, c_vp]
 
 EXPORTS = ["dla_status_string", "dla_cache_bytes", "dla_cache_init", "dla_workspace_bytes",
            "dla_prefill", "dla_decode_workspace_bytes", "dla_decode_step",
            "dla_decode_step_static", "dla_fixed_policy_prefill", "dla_info_policy_prefill",
            "dla_unbounded_prefill", "dla_prefill_varlen", "dla_decode_step_masked",
-           "dla_trace_stats"]
+           "dla_trace_stats", "dla_backward_workspace_bytes", "dla_prefill_backward"]
 
 
 def status_string(code: int) -> str:
@@ -166,6 +171,18 @@ def dla_info_policy_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, strea
                                         0 if ws is None else ws.numel(), _ptr(dev_status),
                                         _stream(stream)),
            "dla_info_policy_prefill")
+
+
+def dla_backward_workspace_bytes(cfg: dla_config) -> int:
+    return int(_lib.dla_backward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def dla_prefill_backward(cfg, q, k, v, d_o, trace, dq, dk, dv, ws, dev_status, stream=None):
+    _check(_lib.dla_prefill_backward(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(d_o),
+                                     ctypes.byref(trace), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                                     0 if ws is None else ws.numel(), _ptr(dev_status),
+                                     _stream(stream)),
+           "dla_prefill_backward")
 
 
 def dla_unbounded_prefill(cfg, q, k, v, o, cache, trace, ws, dev_status, stream=None):
@@ -424,6 +441,28 @@ def unbounded_prefill(q, k, v, cache: Cache, tau: float, *, trace: bool = True, 
         torch.cuda.synchronize()
         check_device_status(st, "dla_unbounded_prefill")
     return o, tr
+
+
+def prefill_backward(q, k, v, d_o, trace: Trace, C: int, *, stream=None, sync=True):
+    """dq, dk, dv (fp32, [B, H, T, d]) of a dla_prefill of q, k, v [B, H, T, d]
+    from empty caches of capacity C, at the decisions its `trace` recorded;
+    d_o = dL/do in the inputs' dtype."""
+    B, H, T, d = k.shape
+    for t in (q, k, v, d_o):
+        if not t.is_cuda or not t.is_contiguous() or t.shape != k.shape or t.dtype != k.dtype:
+            raise ValueError("q, k, v, d_o must be contiguous CUDA tensors of one shape and dtype")
+    cfg = make_config(B, H, T, d, C, 0.0, _dtype_code(k), 0, None)
+    need = dla_backward_workspace_bytes(cfg)
+    if need == 0:
+        raise DlaError(2, "dla_prefill_backward (shape)")  # DLA_ERR_UNSUPPORTED
+    ws = torch.empty(need, dtype=torch.uint8, device=k.device)
+    dq, dk, dv = (torch.empty(B, H, T, d, dtype=torch.float32, device=k.device) for _ in range(3))
+    st = torch.zeros(1, dtype=torch.int32, device=k.device)
+    dla_prefill_backward(cfg, q, k, v, d_o, trace.c, dq, dk, dv, ws, st, stream)
+    if sync:
+        torch.cuda.synchronize()
+        check_device_status(st, "dla_prefill_backward")
+    return dq, dk, dv
 
 
 def prefill_varlen(q, k, v, lens, cache: Cache, tau: float, *, policy=DLA_POLICY_DYNAMIC,

@@ -60,6 +60,10 @@ WORKLOADS = {
     "unbounded_t8192": dict(B=4, H=16, T=8192, d=128, C=1024, tau=0.5,
                             dtype="bf16", n_centres=64,
                             lengths=("geometric", 32.0), sigma=0.05, seed=1007),
+    # the gradient at a forward's decisions (dla_prefill_backward, quadratic
+    # in T): the T=8192 prefill's distribution on 16 streams of 2048 tokens
+    "backward_t2048": dict(B=1, H=16, T=2048, d=128, C=64, tau=0.5, dtype="bf16",
+                           n_centres=64, lengths=("geometric", 96.0), sigma=0.05, seed=1008),
     # the information policy on the T=8192 prefill's sizes; values follow the
     # regimes (recipe step 6) and tau sits between the within-regime score
     # (about 0.6 at d = 128) and the score of a regime switch (about 1.4)

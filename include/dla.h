@@ -329,6 +329,39 @@ dla_status dla_trace_stats(const dla_trace *trace, int32_t heads, int32_t T,
                            const int32_t *m_before, const int64_t *t_before, int32_t tile,
                            const dla_stats *out, int32_t *dev_status, void *stream);
 
+/* Workspace bytes for dla_prefill_backward with this config; 0 when the
+ * config is outside its limits (d_k == d_v in {32, 64, 128}, 2 <= C <= 128,
+ * T <= 4096, in_dtype DLA_F32 or DLA_BF16). */
+size_t dla_backward_workspace_bytes(const dla_config *cfg);
+
+/* Gradient of dla_prefill's output with respect to q, k and v, at the
+ * decisions that prefill took (Chlience section 5.1 states, 5.2 merges, 5.3
+ * readout).  The boundaries and merges are piecewise constant in the keys,
+ * so wherever the forward is differentiable this is its exact gradient: the
+ * decision trace is an input and is held fixed.  (The page's section 5.1 says
+ * training uses a soft gate through the decisions and gives no form for it;
+ * no such term is added.)
+ *   cfg    the forward's config (B, H, T, d_k = d_v, C, in_dtype; tau and
+ *          window unused), within dla_backward_workspace_bytes' limits;
+ *   q, k, v, d_o  [B][H][T][d] in cfg->in_dtype (device): the forward's
+ *          inputs and dL/do;
+ *   trace  the forward's decision trace (boundary, merge_t, merge_i,
+ *          merge_count, cap), from a dla_prefill that started every stream
+ *          from an empty cache (merge_t then counts from 0);
+ *   dq, dk, dv  [B][H][T][d] fp32 outputs (device, caller-owned);
+ *   ws     device workspace of dla_backward_workspace_bytes(cfg) bytes,
+ *          256-byte aligned.
+ * Three kernels on `stream` (SIMT, quadratic in T).  Argument errors return
+ * at once (DLA_ERR_INVALID_ARG, DLA_ERR_UNSUPPORTED, DLA_ERR_WORKSPACE); a
+ * trace that does not describe such a forward (a merge off a boundary, a
+ * merge index out of range, more than C live states, token 0 not a
+ * boundary) sets DLA_ERR_INVALID_ARG in *dev_status, a merge_count above cap
+ * DLA_ERR_TRACE_OVERFLOW, and the gradients are then unspecified. */
+dla_status dla_prefill_backward(const dla_config *cfg, const void *q, const void *k, const void *v,
+                                const void *d_o, const dla_trace *trace, float *dq, float *dk,
+                                float *dv, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                void *stream);
+
 /* Static description of a status code. */
 const char *dla_status_string(dla_status status);
 

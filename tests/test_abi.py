@@ -70,5 +70,14 @@ def test_size_queries_and_argument_errors():
                                        ctypes.byref(cache), None, None, 0, None, None) == 1
     assert lib.dla_info_policy_prefill(ctypes.byref(bad_c), None, None, None, None,
                                        ctypes.byref(cache), None, None, 0, None, None) == 2
+    # the backward's limits and its argument checks (returned before any launch)
+    assert dla.dla_backward_workspace_bytes(good) > 0
+    assert dla.dla_backward_workspace_bytes(dla.make_config(1, 1, 4097, 32, 4, 0.5, dla.DLA_F32)) == 0
+    assert dla.dla_backward_workspace_bytes(dla.make_config(1, 1, 16, 32, 129, 0.5, dla.DLA_F32)) == 0
+    assert dla.dla_backward_workspace_bytes(bad) == 0
+    assert lib.dla_prefill_backward(ctypes.byref(bad), None, None, None, None, None, None, None,
+                                    None, None, 0, None, None) == 2
+    assert lib.dla_prefill_backward(ctypes.byref(good), None, None, None, None, None, None, None,
+                                    None, None, 0, None, None) == 1
     for code in range(8):
         assert dla.status_string(code)
