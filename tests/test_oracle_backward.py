@@ -9,7 +9,10 @@ itself (CPU only).
 - one token: the closed form;
 - tau > 2 (every token joins, one state): plain causal linear attention,
   differentiated by torch's fp64 autograd;
-- a hand-written live-state list.
+- a hand-written live-state list;
+- planted mistakes (the means term dropped, the state weight taken as 1, the
+  softmax gradient uncentred, phi' dropped, the mask's owner off by one
+  state) each fail the central-difference comparison.
 """
 import numpy as np
 import pytest
@@ -105,3 +108,42 @@ def test_one_state_is_causal_linear_attention():
     gq, gk, gv = BW.backward_head(q, k, v, dO, b, merges)
     for g, t in ((gq, tq), (gk, tk), (gv, tv)):
         np.testing.assert_allclose(g, t.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
+MUTANTS = {
+    "no_means_term": ("c = dA * Lam + (da * rs / n)[owner]", "c = dA * Lam"),
+    "state_weight_one": ("c = dA * Lam + (da * rs / n)[owner]", "c = dA + (da * rs / n)[owner]"),
+    "softmax_uncentred": ("da = lam * (dlam - np.dot(lam, dlam))", "da = lam * dlam"),
+    "no_dphi": ("return dfq * dphi(q), dfk * dphi(k), dv", "return dfq, dfk, dv"),
+    "owner_shifted": ("Lam = lam[owner]", "Lam = lam[np.minimum(owner + 1, len(lam) - 1)]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistakes_fail_the_difference_check(name):
+    import inspect
+    src = inspect.getsource(BW)
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1
+    ns = {}
+    exec(compile(src.replace(old, new), "mutant", "exec"), ns)
+    T, d, C, tau, eps = 48, 6, 3, 0.5, 1e-6
+    q, k, v = stream(12, T, d)
+    o, b, merges, _ = oracle_fwd(q, k, v, C, tau)
+    dO = np.random.default_rng(12).standard_normal(o.shape)
+    grads = dict(zip("qkv", ns["backward_head"](q, k, v, dO, b, merges)))
+    rng = np.random.default_rng(5)
+    worst = 0.0
+    for name_x in "qkv":
+        x = {"q": q, "k": k, "v": v}[name_x]
+        g = grads[name_x]
+        for _ in range(15):
+            t, c = int(rng.integers(T)), int(rng.integers(d))
+            xp, xm = x.copy(), x.copy()
+            xp[t, c] += eps
+            xm[t, c] -= eps
+            args = {"q": q, "k": k, "v": v}
+            lp = _loss(**{**args, name_x: xp}, dO=dO, C=C, tau=tau, ref_trace=(b, merges))
+            lm = _loss(**{**args, name_x: xm}, dO=dO, C=C, tau=tau, ref_trace=(b, merges))
+            worst = max(worst, abs((lp - lm) / (2 * eps) - g[t, c]) / max(np.abs(g).max(), 1e-30))
+    assert worst > 1e-6, (name, worst)
